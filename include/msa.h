@@ -1,0 +1,238 @@
+/*
+ * msa.h — C ABI of the B200 (sm_100a) hot path of Memory Sparse Attention (MSA).
+ *
+ * MSA routes a query over a memory bank of up to 100M tokens: each memory document is
+ * encoded once (document-wise RoPE, chunk-mean pooling of K, V and the router key K^R),
+ * the pooled router keys stay in GPU memory, the query's router vectors score every chunk
+ * by cosine similarity, the top-k documents are selected, their compressed K/V are fetched
+ * from host memory and the query attends over them together with its own local K/V. The
+ * Memory Interleave loop repeats route -> attend -> append -> re-route.
+ *
+ * Sources (web pages about the MSA paper, Chen et al., "MSA: Memory Sparse Attention for
+ * Efficient End-to-End Memory Model Scaling to 100M Tokens"), cited by tag:
+ *   [P1] Lighthouse AI-research news digest of the paper (2026-03-27)
+ *   [P2] hotdry blog "EverMind MSA router sparse attention architecture" (2026-03-24)
+ *   [P5] wiselychen blog "MSA: 4B 模型打贏 235B RAG 系統"
+ *
+ * Conventions
+ *   - Every call returns msa_status. On failure msa_last_error() gives a thread-local message.
+ *   - Validation happens before anything is enqueued: a call that fails validation launches
+ *     nothing and copies nothing.
+ *   - The caller owns all memory. Device pointers come from the caller's allocator (PyTorch),
+ *     pinned host buffers from cudaHostAlloc (torch pin_memory). The library allocates no
+ *     device or host memory; scratch space is a caller workspace whose size the matching
+ *     *_workspace_size call returns. Tensor memory (TMEM) is allocated and freed inside kernels.
+ *   - All calls are asynchronous on the given stream (a cudaStream_t; NULL = legacy default)
+ *     unless stated otherwise; outputs are valid once the stream has reached the call.
+ *   - Tensors are contiguous and row-major; the layout of each is given with the call.
+ *     Device pointers must be 16-byte aligned.
+ *   - Kernels that detect a bad value at run time (a position past the RoPE table, a wait
+ *     that ran out of time) skip the offending work and record a code in a device-side error
+ *     word, read and cleared by msa_device_status(). No kernel traps.
+ */
+#ifndef MSA_H_
+#define MSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t msa_status;
+enum {
+    MSA_OK = 0,
+    MSA_ERR_INVALID_ARG = 1, /* null or misaligned pointer, bad size, k > n_docs, dtype mismatch */
+    MSA_ERR_UNSUPPORTED = 2, /* a shape the kernels do not handle (e.g. head_dim != 128 in attention) */
+    MSA_ERR_CUDA = 3,        /* a CUDA runtime or launch error; message in msa_last_error() */
+    MSA_ERR_TIMEOUT = 4,     /* a host-side wait passed its deadline */
+    MSA_ERR_WORKSPACE = 5,   /* the workspace is smaller than the *_workspace_size answer */
+    MSA_ERR_DEVICE = 6       /* a kernel recorded a run-time error (msa_device_status) */
+};
+
+typedef int32_t msa_dtype;
+enum { MSA_F32 = 0, MSA_BF16 = 1 };
+
+/* Device-side error codes recorded by kernels (first one wins). */
+enum {
+    MSA_DEV_OK = 0,
+    MSA_DEV_ROPE_POSITION = 1, /* a RoPE position was >= max_pos; that row was not rotated/pooled */
+    MSA_DEV_WAIT_TIMEOUT = 2,  /* an mbarrier wait in the tensor-core router ran out of time */
+    MSA_DEV_BAD_INDEX = 3      /* a doc index outside [0, n_docs) reached a kernel */
+};
+
+/* Thread-local text of the last error on this host thread ("" if none). */
+const char* msa_last_error(void);
+
+/* Library version string. */
+const char* msa_version(void);
+
+/* Synchronises `stream`, then reads and clears the device-side error word of the current
+ * device into *code (MSA_DEV_*). Returns MSA_OK, or MSA_ERR_CUDA if the read failed. */
+msa_status msa_device_status(int32_t* code, void* stream);
+
+/* Host-only: fills the RoPE table used by every rotating call.
+ * out_host is [max_pos][d/2][2] float (cos, sin) of the angle p * base^(-2i/d), computed in
+ * double precision by the C math library and rounded once to float. d must be even.
+ * ([P1] §组件 2 Document-wise RoPE; rotate-half pairing i <-> i + d/2 with base 1e6 is the
+ * reading taken for the Qwen3-like backbone the pages name.) */
+msa_status msa_rope_table(int64_t max_pos, int d, double base, float* out_host);
+
+/* Fills chunk_doc[c] = index of the document that owns chunk c, from the CSR offsets
+ * doc_chunk_off[n_docs + 1] (device, int64, non-decreasing, doc_chunk_off[n_docs] == n_chunks).
+ * chunk_doc is device int32 [n_chunks]. The map is part of the pooled bank's metadata. */
+msa_status msa_chunk_doc_map(const int64_t* doc_chunk_off, int64_t n_docs, int64_t n_chunks, int32_t* chunk_doc,
+                             void* stream);
+
+/* Rotary position embedding of x [n_tok][n_heads][head_dim] (dt = MSA_F32 or MSA_BF16) into
+ * out (same layout; out may equal x for in-place). Token t of segment s (segments given by the
+ * device CSR offsets seg_tok_off[n_seg + 1]) gets position pos_offset + (t - seg_tok_off[s]).
+ *   Document-wise RoPE of memory keys: one segment per document, pos_offset = 0 — positions
+ *   restart at 0 in every document ([P1] §组件 2; [P2] §工程实现的关键细节).
+ *   Global RoPE of the active context: one segment per query, pos_offset = k + first local
+ *   index — the active context starts at position k, the top-k count ([P1] §组件 2).
+ * cos_sin is the device copy of msa_rope_table(max_pos, head_dim, ...). A position >= max_pos
+ * leaves that row unrotated in out and records MSA_DEV_ROPE_POSITION.
+ * Requires head_dim even, head_dim/VEC a power of two <= 32 (VEC = 4 for fp32, 8 for bf16). */
+msa_status msa_rope_doc(const void* x, void* out, msa_dtype dt, int64_t n_tok, int n_heads, int head_dim,
+                        const int64_t* seg_tok_off, int64_t n_seg, int64_t pos_offset, const float* cos_sin,
+                        int64_t max_pos, void* stream);
+
+/* Offline memory encoding ([P5] §3 inference stage 1; [P2] §可学习记忆路由层的核心架构):
+ * chunk-mean pooling of each document's token-level K, V and router key K^R into K-bar, V-bar
+ * and K-bar^R. Chunks have `chunk` tokens and never cross a document; a document's last chunk
+ * is the mean of its remaining tokens.
+ *   k, v: device [n_tok][hkv][d]; kr: device [n_tok][hr][d]; all of dtype in_dt. Any of
+ *     (k and v together) or kr may be NULL to skip that part.
+ *   doc_tok_off [n_docs+1], doc_chunk_off [n_docs+1]: device int64 CSR offsets (tokens, chunks).
+ *   chunk_doc [n_chunks]: device int32 (msa_chunk_doc_map).
+ *   fuse_doc_rope: rotate K with document-wise positions (p = token - doc start) before the
+ *     mean, using cos_sin [max_pos][d/2][2] (device); K-bar is then the mean of rotated keys.
+ *   kvbar: device [n_chunks][2][hkv][d] of out_dt — K-bar at [c][0], V-bar at [c][1] (the
+ *     layout of the host content bank, so one document is one contiguous byte run).
+ *   kr_index: device [n_chunks][hr][d] of out_dt — K-bar^R; when normalize_router != 0 each
+ *     head vector is divided by its L2 norm (a zero vector stays zero): the "index form" that
+ *     msa_route_scores reads. Pre-pooled router keys are put into index form by calling this
+ *     with chunk = 1, one document per chunk run, k = v = NULL.
+ * Arithmetic is fp32; outputs are rounded once to out_dt. */
+msa_status msa_pool_chunks(const void* k, const void* v, const void* kr, msa_dtype in_dt, int64_t n_tok, int hkv,
+                           int hr, int d, const int64_t* doc_tok_off, const int64_t* doc_chunk_off,
+                           const int32_t* chunk_doc, int64_t n_docs, int64_t n_chunks, int chunk, int fuse_doc_rope,
+                           const float* cos_sin, int64_t max_pos, void* kvbar, void* kr_index, msa_dtype out_dt,
+                           int normalize_router, void* stream);
+
+/* Router scoring ([P1] §组件 1 key formula; [P2] §可学习记忆路由层的核心架构):
+ *   S_{q,c} = max over tokens t of mean over heads h of cos(Q^R_{q,t,h}, K-bar^R_{c,h})
+ *   doc_scores[q][i] = max over the chunks c of document i of S_{q,c}
+ * (the document score as the max over its chunks is this library's stated reading.)
+ *   kr_index: device [n_chunks][H*d] in index form (per-head unit vectors), dtype dt.
+ *   qr: device [n_q][T][H][d] raw router queries, dtype dt.
+ *   chunk_doc: device int32 [n_chunks]; doc_scores: device float [n_q][n_docs] (output, every
+ *   entry written; a document without chunks gets -inf); chunk_scores: device float
+ *   [n_q][n_chunks] or NULL.
+ * The mean of the per-head cosines is computed as one dot product: each query head vector is
+ * divided by its norm and by H, the heads are concatenated, and the dot product with the
+ * concatenated unit-vector index row is the mean of the cosines. bf16 runs on the tcgen05
+ * tensor cores (fp32 accumulation in TMEM) when H*d % 64 == 0; fp32 runs on CUDA cores in
+ * fp32. ws: device workspace of msa_route_workspace_size bytes (256-byte aligned). */
+msa_status msa_route_scores(const void* kr_index, msa_dtype dt, int64_t n_chunks, const int32_t* chunk_doc,
+                            int64_t n_docs, const void* qr, int n_q, int T, int H, int d, float* doc_scores,
+                            float* chunk_scores, void* ws, size_t ws_bytes, void* stream);
+msa_status msa_route_workspace_size(int n_q, int T, int H, int d, msa_dtype dt, size_t* bytes);
+
+/* Selects the router kernel for testing: 0 = automatic, 1 = CUDA-core kernel, 2 = tensor-core
+ * kernel (bf16 only). Process-wide. */
+msa_status msa_route_set_impl(int impl);
+
+/* Top-k document selection ([P1] §组件 1; [P2] Top-k 选择机制): for every query the k documents
+ * with the largest doc_scores, in descending score order, ties broken by the lower document
+ * index. doc_scores: device float [n_q][n_docs]; idx: device int32 [n_q][k]; score: device
+ * float [n_q][k] (may be NULL). 1 <= k <= min(64, n_docs). ws: msa_topk_workspace_size bytes. */
+msa_status msa_topk_docs(const float* doc_scores, int n_q, int64_t n_docs, int k, int32_t* idx, float* score,
+                         void* ws, size_t ws_bytes, void* stream);
+msa_status msa_topk_workspace_size(int n_q, int64_t n_docs, int k, size_t* bytes);
+
+/* Fetch of the selected documents' compressed K-bar/V-bar from host memory
+ * ([P2] §工程实现的关键细节: K-bar^R stays in GPU memory, K-bar/V-bar live in host DRAM and are
+ * loaded asynchronously once routing has chosen the documents; [P5] §3 async prefetch).
+ *   host_bank: pinned host [n_chunks][2][hkv][d] of dt (the kvbar layout of msa_pool_chunks).
+ *   doc_chunk_off_host: host int64 [n_docs+1]; idx_host: host int32 [n_q][k] (msa_topk_docs
+ *   output copied to the host).
+ *   dev_mem_kv: device [n_q][max_mem][2][hkv][d]: query q's selected documents' chunk rows,
+ *   concatenated in rank order from row 0; mem_len_host[q] (host int32, written before the
+ *   call returns) is the number of rows filled.
+ * One cudaMemcpyAsync per selected document on copy_stream (the copy engines over the host
+ * link); the call returns once they are enqueued. Fails with MSA_ERR_INVALID_ARG, copying
+ * nothing, if an index is out of range or a query's rows exceed max_mem. */
+msa_status msa_gather_kv(const void* host_bank, msa_dtype dt, int64_t n_chunks, const int64_t* doc_chunk_off_host,
+                         int64_t n_docs, const int32_t* idx_host, int n_q, int k, int hkv, int d, int max_mem,
+                         void* dev_mem_kv, int32_t* mem_len_host, void* copy_stream);
+
+/* Sparse attention ([P1] §组件 1 稀疏注意力机制; [P2] concatenation of the selected compressed
+ * K/V with the query's local K/V): for query q, token t, head h (kv head g = h / (hq/hkv)):
+ *   out = softmax(scale * q . [mem K-bar ; local K_j, j <= q_start + t, j < L]) [mem V-bar ; local V]
+ *   q: device [n_q][T][hq][d], already rotated (global positions);
+ *   mem_kv: device [n_q][max_mem][2][hkv][d] (msa_gather_kv), mem_len: device int32 [n_q];
+ *   local_k, local_v: device [n_q][L_max][hkv][d], rotated keys of the active context;
+ *   out: device [n_q][T][hq][d]. All of dtype dt; arithmetic and softmax in fp32.
+ * Memory rows are all visible; local keys are causal. A row with no visible key is 0.
+ * Requires d == 128 and hq/hkv in {1, 2, 4, 8}. */
+msa_status msa_sparse_attn(const void* q, const void* mem_kv, const int32_t* mem_len, int max_mem,
+                           const void* local_k, const void* local_v, int L_max, int L, int q_start, int n_q, int T,
+                           int hq, int hkv, int d, float scale, void* out, msa_dtype dt, void* stream);
+
+/* One routed layer of one Memory Interleave round (see msa_interleave_step). */
+typedef struct msa_layer_args {
+    const void* kr_index;       /* device [n_chunks][H*d], index form */
+    const void* host_bank;      /* pinned host [n_chunks][2][hkv][d] */
+    const void* qr;             /* device [n_q][T_act][H][d]: router queries of every active token */
+    const void* q_new;          /* device: raw queries of the tokens appended this round,
+                                   element (q, t, h, i) at ((q * new_q_stride + t) * hq + h) * d + i */
+    const void* k_new;          /* device: raw keys of the appended tokens, same indexing with hkv */
+    const void* v_new;          /* device: values of the appended tokens, same indexing with hkv */
+    void* local_k;              /* device [n_q][L_max][hkv][d]: rotated local keys (appended here) */
+    void* local_v;              /* device [n_q][L_max][hkv][d] */
+    void* out;                  /* device [n_q][T_new][hq][d]: attention output of the appended tokens */
+    int32_t* topk_idx_host;     /* pinned host [n_q][k]: documents selected for this layer (output) */
+} msa_layer_args;
+
+typedef struct msa_interleave_args {
+    int n_layers;
+    const msa_layer_args* layers;   /* host array [n_layers] */
+    msa_dtype dt;                   /* MSA_BF16 or MSA_F32, for every tensor */
+    int64_t n_chunks, n_docs;
+    const int64_t* doc_chunk_off;   /* device int64 [n_docs+1] */
+    const int64_t* doc_chunk_off_host; /* host int64 [n_docs+1] */
+    const int32_t* chunk_doc;       /* device int32 [n_chunks] */
+    int n_q, H, d, hq, hkv, k;
+    int L_prev;                     /* tokens each query held before this round */
+    int T_new;                      /* tokens appended this round (T_act = L_prev + T_new) */
+    int new_q_stride;               /* tokens per query in the q_new/k_new/v_new buffers */
+    int L_max;                      /* capacity of local_k/local_v per query */
+    int max_mem;                    /* capacity of the gathered memory per query (rows) */
+    const float* rope_cos_sin;      /* device table of msa_rope_table(rope_max_pos, d, base) */
+    int64_t rope_max_pos;
+    float scale;                    /* attention scale, normally 1/sqrt(d) */
+    void* ws;                       /* device workspace of msa_interleave_workspace_size bytes */
+    size_t ws_bytes;
+} msa_interleave_args;
+
+/* One Memory Interleave round over every routed layer ([P1] §组件 3 Memory Interleaving;
+ * [P2] re-route with the updated context each round; [P5] §4 生成式檢索 -> 上下文擴展 -> 生成 ->
+ * 再檢索). Per layer: append the round's T_new tokens to the local cache (keys rotated to
+ * global positions k + L_prev + t, values copied), rotate their queries likewise, score the
+ * memory with the router queries of all T_act = L_prev + T_new active tokens, select the top-k
+ * documents, copy their indices to topk_idx_host, fetch their K-bar/V-bar from the host bank on
+ * `copy` and attend. The routing of every layer is enqueued on `compute` first; the host then
+ * waits for each layer's selection (polling with a deadline of host_wait_timeout_us, giving
+ * MSA_ERR_TIMEOUT) and enqueues its fetch on `copy`, so fetches overlap the routing of later
+ * layers; attention waits on its own fetch. Returns after everything is enqueued. */
+msa_status msa_interleave_step(const msa_interleave_args* a, void* compute, void* copy, int64_t host_wait_timeout_us);
+msa_status msa_interleave_workspace_size(const msa_interleave_args* a, size_t* bytes);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MSA_H_ */

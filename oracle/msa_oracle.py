@@ -148,7 +148,10 @@ def chunk_scores_one_query(krbar: np.ndarray, qr: np.ndarray) -> np.ndarray:
     """
     kn = unit(krbar)                                   # [C, H, d]
     qn = unit(qr)                                      # [T, H, d]
-    cos = np.einsum("thd,chd->tch", qn, kn)            # [T, C, H]
+    H = krbar.shape[1]
+    cos = np.empty((qr.shape[0], krbar.shape[0], H), dtype=F64)    # [T, C, H]
+    for h in range(H):                                 # cos of unit vectors = their dot product
+        cos[:, :, h] = qn[:, h, :] @ kn[:, h, :].T
     mean_h = cos.mean(axis=2)                          # [T, C]
     return mean_h.max(axis=0)                          # [C]
 

@@ -1,0 +1,221 @@
+"""Python binding of the MSA C ABI. Same names as the C entry points; argument marshalling only.
+
+PyTorch supplies device memory, pinned host memory and streams; every step of the hot path runs
+in the CUDA kernels of libmsa.so. Outputs that the caller does not pass are allocated with torch.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+
+import numpy as np
+import torch
+
+from . import _lib
+from ._lib import MSA_BF16, MSA_F32, check, lib
+
+_DT = {torch.float32: MSA_F32, torch.bfloat16: MSA_BF16}
+
+
+def _dt(t: torch.Tensor) -> int:
+    try:
+        return _DT[t.dtype]
+    except KeyError:
+        raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)") from None
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _ws(nbytes: int, device) -> torch.Tensor:
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def version() -> str:
+    return lib.msa_version().decode()
+
+
+def device_status(stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the device-side error word (0 = none)."""
+    code = ctypes.c_int32(0)
+    check(lib.msa_device_status(ctypes.byref(code), _stream(stream)), "msa_device_status")
+    return code.value
+
+
+def rope_table(max_pos: int, d: int, base: float = 1.0e6, device="cuda") -> torch.Tensor:
+    """[max_pos, d/2, 2] float32 (cos, sin) table, computed by the library on the host, then copied."""
+    host = np.empty((max_pos, d // 2, 2), dtype=np.float32)
+    check(lib.msa_rope_table(max_pos, d, base, host.ctypes.data), "msa_rope_table")
+    return torch.from_numpy(host).to(device)
+
+
+def chunk_doc_map(doc_chunk_off: torch.Tensor, n_chunks: int, stream=None) -> torch.Tensor:
+    out = torch.empty(n_chunks, dtype=torch.int32, device=doc_chunk_off.device)
+    check(lib.msa_chunk_doc_map(_ptr(doc_chunk_off), doc_chunk_off.numel() - 1, n_chunks, _ptr(out), _stream(stream)),
+          "msa_chunk_doc_map")
+    return out
+
+
+def msa_rope_doc(x: torch.Tensor, seg_tok_off: torch.Tensor, pos_offset: int, cos_sin: torch.Tensor,
+                 out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Rotate x [n_tok, heads, d]; token t of segment s gets position pos_offset + t - seg_tok_off[s]."""
+    out = x if out is None else out
+    n_tok, heads, d = x.shape
+    check(lib.msa_rope_doc(_ptr(x), _ptr(out), _dt(x), n_tok, heads, d, _ptr(seg_tok_off), seg_tok_off.numel() - 1,
+                           pos_offset, _ptr(cos_sin), cos_sin.shape[0], _stream(stream)), "msa_rope_doc")
+    return out
+
+
+def msa_pool_chunks(k, v, kr, doc_tok_off, doc_chunk_off, chunk_doc, chunk: int, cos_sin=None,
+                    fuse_doc_rope: bool = True, out_dtype=None, normalize_router: bool = True, kvbar=None,
+                    kr_index=None, stream=None):
+    """Chunk-mean pooling -> (kvbar [C, 2, hkv, d] or None, kr_index [C, hr, d] or None)."""
+    ref = k if k is not None else kr
+    n_tok, _, d = ref.shape
+    hkv = k.shape[1] if k is not None else 0
+    hr = kr.shape[1] if kr is not None else 0
+    C = chunk_doc.numel()
+    out_dtype = out_dtype or ref.dtype
+    if k is not None and kvbar is None:
+        kvbar = torch.empty((C, 2, hkv, d), dtype=out_dtype, device=ref.device)
+    if kr is not None and kr_index is None:
+        kr_index = torch.empty((C, hr, d), dtype=out_dtype, device=ref.device)
+    fuse = bool(fuse_doc_rope and k is not None)
+    check(lib.msa_pool_chunks(_ptr(k), _ptr(v), _ptr(kr), _dt(ref), n_tok, hkv, hr, d, _ptr(doc_tok_off),
+                              _ptr(doc_chunk_off), _ptr(chunk_doc), doc_tok_off.numel() - 1, C, chunk, int(fuse),
+                              _ptr(cos_sin) if fuse else None, cos_sin.shape[0] if fuse else 0,
+                              _ptr(kvbar) if k is not None else None, _ptr(kr_index) if kr is not None else None,
+                              _DT[out_dtype], int(normalize_router), _stream(stream)), "msa_pool_chunks")
+    return (kvbar if k is not None else None), (kr_index if kr is not None else None)
+
+
+def route_workspace_size(n_q: int, T: int, H: int, d: int, dtype) -> int:
+    n = ctypes.c_size_t(0)
+    check(lib.msa_route_workspace_size(n_q, T, H, d, _DT[dtype], ctypes.byref(n)), "msa_route_workspace_size")
+    return n.value
+
+
+def route_set_impl(impl: int) -> None:
+    """0 = automatic, 1 = CUDA-core kernel, 2 = tensor-core kernel."""
+    check(lib.msa_route_set_impl(impl), "msa_route_set_impl")
+
+
+def msa_route_scores(kr_index, chunk_doc, n_docs: int, qr, doc_scores=None, chunk_scores=None,
+                     want_chunk_scores: bool = False, ws=None, stream=None):
+    """Router scores: kr_index [C, H, d] (index form), qr [n_q, T, H, d] -> doc_scores [n_q, n_docs]
+    (and chunk_scores [n_q, C] when requested)."""
+    C = kr_index.shape[0]
+    n_q, T, H, d = qr.shape
+    dev = qr.device
+    if doc_scores is None:
+        doc_scores = torch.empty((n_q, n_docs), dtype=torch.float32, device=dev)
+    if want_chunk_scores and chunk_scores is None:
+        chunk_scores = torch.empty((n_q, C), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = _ws(route_workspace_size(n_q, T, H, d, qr.dtype), dev)
+    check(lib.msa_route_scores(_ptr(kr_index), _dt(kr_index), C, _ptr(chunk_doc), n_docs, _ptr(qr), n_q, T, H, d,
+                               _ptr(doc_scores), _ptr(chunk_scores), _ptr(ws), ws.numel(), _stream(stream)),
+          "msa_route_scores")
+    return (doc_scores, chunk_scores) if chunk_scores is not None else doc_scores
+
+
+def topk_workspace_size(n_q: int, n_docs: int, k: int) -> int:
+    n = ctypes.c_size_t(0)
+    check(lib.msa_topk_workspace_size(n_q, n_docs, k, ctypes.byref(n)), "msa_topk_workspace_size")
+    return n.value
+
+
+def msa_topk_docs(doc_scores, k: int, idx=None, score=None, ws=None, stream=None):
+    """-> (idx int32 [n_q, k], score float32 [n_q, k]) by descending score, ties to the lower index."""
+    n_q, n_docs = doc_scores.shape
+    dev = doc_scores.device
+    idx = torch.empty((n_q, k), dtype=torch.int32, device=dev) if idx is None else idx
+    score = torch.empty((n_q, k), dtype=torch.float32, device=dev) if score is None else score
+    if ws is None:
+        ws = _ws(topk_workspace_size(n_q, n_docs, k), dev)
+    check(lib.msa_topk_docs(_ptr(doc_scores), n_q, n_docs, k, _ptr(idx), _ptr(score), _ptr(ws), ws.numel(),
+                            _stream(stream)), "msa_topk_docs")
+    return idx, score
+
+
+def msa_gather_kv(host_bank, doc_chunk_off_host, idx_host, max_mem: int, dev_mem_kv=None, device="cuda",
+                  copy_stream=None):
+    """Copy the selected docs' rows [*, 2, hkv, d] from the pinned host bank into
+    dev_mem_kv [n_q, max_mem, 2, hkv, d]; returns (dev_mem_kv, mem_len int32 host tensor [n_q])."""
+    C, _, hkv, d = host_bank.shape
+    n_q, k = idx_host.shape
+    if dev_mem_kv is None:
+        dev_mem_kv = torch.zeros((n_q, max_mem, 2, hkv, d), dtype=host_bank.dtype, device=device)
+    off = torch.as_tensor(np.ascontiguousarray(doc_chunk_off_host, dtype=np.int64))
+    idx_c = idx_host.to(torch.int32).contiguous()
+    mem_len = torch.empty(n_q, dtype=torch.int32)
+    check(lib.msa_gather_kv(_ptr(host_bank), _dt(host_bank), C, _ptr(off), off.numel() - 1, _ptr(idx_c), n_q, k,
+                            hkv, d, max_mem, _ptr(dev_mem_kv), _ptr(mem_len), _stream(copy_stream)), "msa_gather_kv")
+    return dev_mem_kv, mem_len
+
+
+def msa_sparse_attn(q, mem_kv, mem_len, local_k, local_v, L: int, q_start: int, scale: float | None = None,
+                    out=None, stream=None):
+    """q [n_q, T, hq, d] (rotated), mem_kv [n_q, max_mem, 2, hkv, d], mem_len int32 [n_q] (device),
+    local_k/local_v [n_q, L_max, hkv, d] -> out [n_q, T, hq, d]."""
+    n_q, T, hq, d = q.shape
+    max_mem = mem_kv.shape[1]
+    hkv = mem_kv.shape[3]
+    L_max = local_k.shape[1]
+    out = torch.empty_like(q) if out is None else out
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    check(lib.msa_sparse_attn(_ptr(q), _ptr(mem_kv), _ptr(mem_len), max_mem, _ptr(local_k), _ptr(local_v), L_max, L,
+                              q_start, n_q, T, hq, hkv, d, scale, _ptr(out), _dt(q), _stream(stream)),
+          "msa_sparse_attn")
+    return out
+
+
+class InterleaveRound:
+    """Marshals msa_interleave_args for one round; holds the ctypes structures alive."""
+
+    def __init__(self, layers, *, n_chunks, n_docs, doc_chunk_off, doc_chunk_off_host, chunk_doc, n_q, H, d, hq, hkv,
+                 k, L_prev, T_new, new_q_stride, L_max, max_mem, cos_sin, scale=None, dtype=torch.bfloat16, ws=None):
+        self.layer_structs = (_lib.LayerArgs * len(layers))()
+        for i, y in enumerate(layers):
+            s = self.layer_structs[i]
+            for f in ("kr_index", "host_bank", "qr", "q_new", "k_new", "v_new", "local_k", "local_v", "out",
+                      "topk_idx_host"):
+                setattr(s, f, y[f].data_ptr())
+        self._off_host = torch.as_tensor(np.ascontiguousarray(doc_chunk_off_host, dtype=np.int64))
+        a = _lib.InterleaveArgs()
+        a.n_layers = len(layers)
+        a.layers = self.layer_structs
+        a.dt = _DT[dtype]
+        a.n_chunks, a.n_docs = n_chunks, n_docs
+        a.doc_chunk_off = doc_chunk_off.data_ptr()
+        a.doc_chunk_off_host = self._off_host.data_ptr()
+        a.chunk_doc = chunk_doc.data_ptr()
+        a.n_q, a.H, a.d, a.hq, a.hkv, a.k = n_q, H, d, hq, hkv, k
+        a.L_prev, a.T_new, a.new_q_stride, a.L_max, a.max_mem = L_prev, T_new, new_q_stride, L_max, max_mem
+        a.rope_cos_sin = cos_sin.data_ptr()
+        a.rope_max_pos = cos_sin.shape[0]
+        a.scale = 1.0 / math.sqrt(d) if scale is None else scale
+        self.args = a
+        need = ctypes.c_size_t(0)
+        a.ws, a.ws_bytes = None, 0
+        check(lib.msa_interleave_workspace_size(ctypes.byref(a), ctypes.byref(need)), "msa_interleave_workspace_size")
+        self.ws = _ws(need.value, doc_chunk_off.device) if ws is None else ws
+        a.ws, a.ws_bytes = self.ws.data_ptr(), self.ws.numel()
+
+    def run(self, compute=None, copy=None, timeout_us: int = 30_000_000) -> None:
+        check(lib.msa_interleave_step(ctypes.byref(self.args), _stream(compute), _stream(copy), timeout_us),
+              "msa_interleave_step")
+
+
+def msa_interleave_step(layers, compute=None, copy=None, timeout_us: int = 30_000_000, **kw) -> InterleaveRound:
+    """One Memory Interleave round over every routed layer (see include/msa.h). Returns the marshalled
+    round so it can be re-run."""
+    r = InterleaveRound(layers, **kw)
+    r.run(compute, copy, timeout_us)
+    return r

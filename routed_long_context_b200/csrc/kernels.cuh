@@ -1,0 +1,51 @@
+// Internal launchers shared between translation units of the library.
+#pragma once
+
+#include "common.cuh"
+
+namespace msa {
+
+// Rotates rows of [*, heads, d] vectors. Row r of the launch belongs to segment s at offset u:
+//   uniform_len > 0: s = r / uniform_len, u = r % uniform_len,
+//                    input row s*in_stride + u, output row s*out_stride + out_off + u;
+//   otherwise      : s from the CSR offsets seg_off[n_seg + 1], input row = output row = r.
+// Position = pos_offset + u.
+struct RopeRowsArgs {
+    const void* in;
+    void* out;
+    int64_t n_rows;
+    int heads;
+    int d;
+    const int64_t* seg_off;
+    int64_t n_seg;
+    int64_t uniform_len;
+    int64_t in_stride, out_stride, out_off;
+    int64_t pos_offset;
+    const float2* cs;
+    int64_t max_pos;
+    int* err;
+};
+msa_status launch_rope_rows(const RopeRowsArgs& a, msa_dtype dt, cudaStream_t s);
+bool rope_layout_ok(msa_dtype dt, int d);
+
+// Tensor-core router (tcgen05 + TMA + TMEM) over a bf16 index in unit-vector form.
+//   index [n_chunks][K] bf16; qhat [n_pad][K] bf16 (rows >= N are zero); N = n_q * T columns.
+//   doc_scores / chunk_scores pre-filled with -inf; results combined with float atomic max.
+struct RouteTcArgs {
+    const void* index;
+    const void* qhat;
+    int64_t n_chunks;
+    int K;
+    int N, n_pad, T;
+    const int32_t* chunk_doc;
+    int64_t n_docs;
+    float* doc_scores;
+    float* chunk_scores;
+    int* err;
+};
+// Returns MSA_ERR_UNSUPPORTED (without launching) when the shape does not fit the kernel.
+msa_status launch_route_tc(const RouteTcArgs& a, cudaStream_t s);
+// Rows the tensor-core path needs in qhat for N columns (0 if unsupported).
+int route_tc_pad_rows(int N, int K);
+
+}  // namespace msa

@@ -1,0 +1,502 @@
+// Tensor-core router for sm_100a: tcgen05.mma (kind::f16, bf16 in, fp32 accumulate in TMEM),
+// operands staged in shared memory by TMA with the 128-byte swizzle, persistent CTAs.
+//
+// GEMM view (swap-AB: chunks on M because the query side is narrow):
+//   D[m][n] = sum_k index[m][k] * qhat[n][k],  m = chunk, n = query token column, k = head*d + i.
+// Epilogue: per chunk (TMEM lane), max over each query's token columns, then a segmented max
+// over the document runs of the warp's 32 consecutive chunks, then one float atomic max per
+// (document, query) run into doc_scores (and per chunk into chunk_scores when requested).
+//
+// Roles (192 threads): warp 0 = TMA producer, warp 1 = TMEM owner and MMA issuer,
+// warps 2..5 = epilogue (warp w reads TMEM lanes 32*(w%4) .. 32*(w%4)+31).
+// Two TMEM accumulators let the epilogue of tile i overlap the main loop of tile i+1.
+// Modes: RESIDENT keeps all of qhat (<= 64 columns) in shared memory, loaded once per CTA,
+// so only the index streams from HBM; otherwise qhat tiles of BN <= 256 columns stream with A.
+// Every mbarrier wait is bounded (about 2 s of %globaltimer); on expiry the CTA records
+// MSA_DEV_WAIT_TIMEOUT, all roles leave their loops, in-flight copies and MMAs are waited for
+// (again bounded) and TMEM is freed before the kernel returns.
+#include <cuda.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace msa {
+namespace {
+
+constexpr int BM = 128;               // chunks per tile = MMA M = TMEM lanes
+constexpr int BK = 64;                // bf16 elements per 128-byte swizzled row
+constexpr int kThreads = 192;
+constexpr int kMaxStages = 8;
+constexpr int kSmemLimit = 232448;    // max dynamic shared memory per block on sm_100
+constexpr int kStageA = BM * BK * 2;  // 16 KB
+constexpr uint64_t kWaitNs = 2000000000ull;
+
+struct TcParams {
+    int64_t n_chunks;
+    int K, N, T, n_pad, BN, n_tiles_n;
+    int acc_stride;        // TMEM columns between the two accumulators: BN rounded up to 32
+    int64_t n_tiles;
+    int stages;
+    uint32_t tmem_cols;
+    uint32_t idesc;
+    const int32_t* chunk_doc;
+    int64_t n_docs;
+    float* doc_scores;
+    float* chunk_scores;
+    int* err;
+};
+
+// ---------------------------------------------------------------------------------- PTX helpers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t globaltimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Waits for phase `parity` of the barrier; gives up (returning false and raising the CTA's
+// abort flag) after kWaitNs, or as soon as another role of the CTA has given up.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    for (uint32_t n = 1;; ++n) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((n & 63) == 0) {
+            if (*abort_flag) return false;
+            if (globaltimer() - t0 > kWaitNs) {
+                *abort_flag = 1;
+                return false;
+            }
+        }
+    }
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_2d_evict_first(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                                        uint32_t bar, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(policy)
+        : "memory");
+}
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Shared-memory matrix descriptor of a K-major operand in the 128-byte swizzle layout:
+// 8-row x 128-byte atoms stacked along M/N (stride 1024 bytes), descriptor version 1.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4)   // start address
+           | ((uint64_t)1 << 16)                 // leading byte offset (unused for this layout)
+           | ((uint64_t)(1024 >> 4) << 32)       // stride byte offset: 8 rows * 128 B
+           | ((uint64_t)1 << 46)                 // descriptor version for tcgen05
+           | ((uint64_t)2 << 61);                // layout: 128-byte swizzle
+}
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// ------------------------------------------------------------------------------------- kernel
+template <bool RESIDENT>
+__global__ void __launch_bounds__(kThreads, 1)
+    route_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const TcParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int kblocks = p.K / BK;
+    const int stage_b = p.BN * BK * 2;                               // bytes of one qhat k-block
+    const int b_bytes = RESIDENT ? kblocks * stage_b : p.stages * stage_b;
+    uint8_t* smem_b = base;
+    uint8_t* smem_a = base + b_bytes;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem_a + p.stages * kStageA);
+    uint64_t* full = bars;                    // [kMaxStages]
+    uint64_t* empty = bars + kMaxStages;      // [kMaxStages]
+    uint64_t* tfull = bars + 2 * kMaxStages;  // [2]
+    uint64_t* tempty = tfull + 2;             // [2]
+    uint64_t* bfull = tempty + 2;             // [1]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bfull + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < p.stages; ++s) {
+            mbar_init(smem_u32(&full[s]), 1);
+            mbar_init(smem_u32(&empty[s]), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(smem_u32(&tfull[a]), 1);
+            mbar_init(smem_u32(&tempty[a]), 4);
+        }
+        mbar_init(smem_u32(bfull), 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 0 && lane == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(p.tmem_cols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            const uint64_t pol = policy_evict_first();
+            uint32_t issued_phase[kMaxStages];
+            bool issued[kMaxStages];
+            for (int s = 0; s < kMaxStages; ++s) issued[s] = false, issued_phase[s] = 0;
+            bool ok = true;
+            bool b_issued = false;
+            if (RESIDENT) {
+                mbar_expect_tx(smem_u32(bfull), (uint32_t)(kblocks * stage_b));
+                for (int kb = 0; kb < kblocks; ++kb)
+                    tma_load_2d(smem_u32(smem_b + kb * stage_b), &tmB, kb * BK, 0, smem_u32(bfull));
+                b_issued = true;
+            }
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int64_t tile = blockIdx.x; ok && tile < p.n_tiles; tile += gridDim.x) {
+                const int m0 = (int)(tile / p.n_tiles_n) * BM;
+                const int n0 = (int)(tile % p.n_tiles_n) * p.BN;
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = smem_u32(&full[stage]);
+                    mbar_expect_tx(fb, (uint32_t)(RESIDENT ? kStageA : kStageA + stage_b));
+                    tma_load_2d_evict_first(smem_u32(smem_a + stage * kStageA), &tmA, kb * BK, m0, fb, pol);
+                    if (!RESIDENT) tma_load_2d(smem_u32(smem_b + stage * stage_b), &tmB, kb * BK, n0, fb);
+                    issued[stage] = true;
+                    issued_phase[stage] = phase;
+                    if (++stage == p.stages) stage = 0, phase ^= 1;
+                }
+            }
+            if (!ok) {
+                // drain: wait (bounded, ignoring the abort flag) for copies this thread issued
+                const uint64_t t0 = globaltimer();
+                for (int s = 0; s < p.stages; ++s)
+                    while (issued[s] && !mbar_try_wait(smem_u32(&full[s]), issued_phase[s]) &&
+                           globaltimer() - t0 < kWaitNs) {
+                    }
+                if (b_issued)
+                    while (!mbar_try_wait(smem_u32(bfull), 0) && globaltimer() - t0 < kWaitNs) {
+                    }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            bool ok = true;
+            if (RESIDENT) ok = mbar_wait(smem_u32(bfull), 0, abort_flag);
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool mma_pending = false;
+            for (int64_t tile = blockIdx.x; ok && tile < p.n_tiles; tile += gridDim.x) {
+                if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * p.acc_stride);
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(smem_a + stage * kStageA);
+                    const uint32_t b_addr = RESIDENT ? smem_u32(smem_b + kb * stage_b) : smem_u32(smem_b + stage * stage_b);
+                    const uint64_t adesc = sw128_desc(a_addr);
+                    const uint64_t bdesc = sw128_desc(b_addr);
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        // +32 bytes per 16-element step inside the swizzle atom (encoded >> 4)
+                        umma_bf16(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), p.idesc,
+                                  (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    mma_pending = true;
+                    umma_commit(smem_u32(&empty[stage]));
+                    if (++stage == p.stages) stage = 0, phase ^= 1;
+                }
+                if (!ok) break;
+                umma_commit(smem_u32(&tfull[acc]));
+                mma_pending = false;
+                if (++acc == 2) acc = 0, acc_phase ^= 1;
+            }
+            if (!ok && mma_pending) {
+                // drain: commit to a free barrier and wait (bounded) for the issued MMAs
+                umma_commit(smem_u32(&tfull[acc]));
+                const uint64_t t0 = globaltimer();
+                while (!mbar_try_wait(smem_u32(&tfull[acc]), acc_phase) && globaltimer() - t0 < kWaitNs) {
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------------------- epilogue
+        const int quarter = warp & 3;
+        const float ninf = -__int_as_float(0x7f800000);
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int64_t tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x) {
+            bool ok = true;
+            if (lane == 0) ok = mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag);
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) break;
+            tc_fence_after();
+            const int64_t m0 = (tile / p.n_tiles_n) * BM;
+            const int n0 = (int)(tile % p.n_tiles_n) * p.BN;
+            const int64_t c = m0 + quarter * 32 + lane;
+            const bool valid = c < p.n_chunks;
+            int doc = valid ? p.chunk_doc[c] : -1;
+            if (valid && (doc < 0 || doc >= p.n_docs)) {
+                record_device_error(p.err, MSA_DEV_BAD_INDEX);
+                doc = -1;
+            }
+            const int col_end = min(n0 + p.BN, p.N);   // columns of this tile that are real tokens
+            // 32-column reads stay inside this accumulator's acc_stride columns
+            const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * p.acc_stride);
+
+            auto flush = [&](int q, float m) {
+                // segmented max over runs of equal doc among the warp's 32 consecutive chunks
+                float v = doc >= 0 ? m : ninf;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float ov = __shfl_down_sync(0xffffffffu, v, off);
+                    const int od = __shfl_down_sync(0xffffffffu, doc, off);
+                    if (lane + off < 32 && od == doc) v = fmaxf(v, ov);
+                }
+                const int prev = __shfl_up_sync(0xffffffffu, doc, 1);
+                if (doc >= 0 && (lane == 0 || prev != doc)) atomic_max_f32(p.doc_scores + (int64_t)q * p.n_docs + doc, v);
+                if (p.chunk_scores && doc >= 0) atomic_max_f32(p.chunk_scores + (int64_t)q * p.n_chunks + c, m);
+            };
+
+            int run_q = -1;
+            float run_max = ninf;
+            const int pieces = (max(col_end - n0, 0) + 31) / 32;
+            for (int pc = 0; pc < pieces; ++pc) {
+                float v[32];
+                tmem_ld32(trow + (uint32_t)(pc * 32), v);
+                if (pc == pieces - 1) {
+                    // every TMEM read of this accumulator is done: hand it back to the MMA warp
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));
+                }
+                const int base_col = n0 + pc * 32;
+                const int hi_col = min(base_col + 32, col_end);
+                for (int q = base_col / p.T; q * p.T < hi_col; ++q) {
+                    const int lo_j = max(q * p.T - base_col, 0);
+                    const int hi_j = min((q + 1) * p.T, hi_col) - base_col;
+                    float m = (q == run_q) ? run_max : ninf;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (j >= lo_j && j < hi_j) m = fmaxf(m, v[j]);
+                    // the query's columns in this tile are complete once they end inside this
+                    // piece or the tile's real columns end here; otherwise carry the running max
+                    if ((q + 1) * p.T <= hi_col || hi_col == col_end) {
+                        flush(q, m);
+                        run_q = -1;
+                    } else {
+                        run_q = q;
+                        run_max = m;
+                    }
+                }
+            }
+            if (pieces == 0) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));
+            }
+            if (run_q >= 0) flush(run_q, run_max);
+            if (++acc == 2) acc = 0, acc_phase ^= 1;
+        }
+    }
+
+    __syncthreads();
+    if (threadIdx.x == 0 && *abort_flag) record_device_error(p.err, MSA_DEV_WAIT_TIMEOUT);
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(p.tmem_cols)
+                     : "memory");
+    }
+}
+
+// ------------------------------------------------------------------------------------- host side
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    });
+    return fn;
+}
+
+msa_status make_map(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t rows, uint32_t box_rows, bool l2_256) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return set_error(MSA_ERR_CUDA, "route (tensor cores): cuTensorMapEncodeTiled unavailable");
+    const cuuint64_t dims[2] = {inner, rows};
+    const cuuint64_t strides[1] = {inner * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    l2_256 ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B : CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return set_error(MSA_ERR_CUDA, "route (tensor cores): tensor map encode failed (%d)", (int)r);
+    return MSA_OK;
+}
+
+struct Plan {
+    bool resident;
+    int BN, n_pad, n_tiles_n, stages;
+    size_t smem;
+};
+
+bool make_plan(int N, int K, Plan* pl) {
+    if (N <= 0 || K <= 0 || K % BK != 0 || K > 8192) return false;
+    const int kblocks = K / BK;
+    const int n16 = (N + 15) / 16 * 16;
+    const size_t fixed = 1024 + 256;
+    // resident: all of qhat stays in shared memory, only the index streams
+    if (n16 <= 64) {
+        const size_t b = (size_t)kblocks * n16 * BK * 2;
+        if (fixed + b + 4 * kStageA <= (size_t)kSmemLimit) {
+            int st = (int)((kSmemLimit - fixed - b) / kStageA);
+            if (st > kMaxStages) st = kMaxStages;
+            *pl = Plan{true, n16, n16, 1, st, fixed + b + (size_t)st * kStageA};
+            return true;
+        }
+    }
+    const int BN = n16 <= 256 ? n16 : 256;
+    const int n_tiles_n = (N + BN - 1) / BN;
+    const size_t stage = (size_t)kStageA + (size_t)BN * BK * 2;
+    int st = (int)((kSmemLimit - fixed) / stage);
+    if (st > kMaxStages) st = kMaxStages;
+    if (st < 2) return false;
+    *pl = Plan{false, BN, n_tiles_n * BN, n_tiles_n, st, fixed + (size_t)st * stage};
+    return true;
+}
+
+}  // namespace
+
+int route_tc_pad_rows(int N, int K) {
+    Plan pl;
+    return make_plan(N, K, &pl) ? pl.n_pad : 0;
+}
+
+msa_status launch_route_tc(const RouteTcArgs& a, cudaStream_t s) {
+    Plan pl;
+    if (!make_plan(a.N, a.K, &pl) || pl.n_pad != a.n_pad)
+        return set_error(MSA_ERR_UNSUPPORTED, "route (tensor cores): unsupported shape N=%d K=%d", a.N, a.K);
+    CUtensorMap tmA, tmB;
+    MSA_RETURN_IF(make_map(&tmA, a.index, (uint64_t)a.K, (uint64_t)a.n_chunks, BM, true));
+    MSA_RETURN_IF(make_map(&tmB, a.qhat, (uint64_t)a.K, (uint64_t)pl.n_pad, (uint32_t)pl.BN, false));
+    TcParams p{};
+    p.n_chunks = a.n_chunks;
+    p.K = a.K; p.N = a.N; p.T = a.T; p.n_pad = pl.n_pad; p.BN = pl.BN; p.n_tiles_n = pl.n_tiles_n;
+    const int64_t m_tiles = (a.n_chunks + BM - 1) / BM;
+    p.n_tiles = m_tiles * pl.n_tiles_n;
+    p.stages = pl.stages;
+    p.acc_stride = (pl.BN + 31) / 32 * 32;
+    uint32_t cols = 32;
+    while (cols < (uint32_t)(2 * p.acc_stride)) cols <<= 1;
+    if (cols > 512) return set_error(MSA_ERR_UNSUPPORTED, "route (tensor cores): %u TMEM columns needed", cols);
+    p.tmem_cols = cols;
+    p.idesc = (1u << 4)                      // D format: f32
+              | (1u << 7)                    // A format: bf16
+              | (1u << 10)                   // B format: bf16
+              | ((uint32_t)(pl.BN >> 3) << 17)   // N / 8
+              | ((uint32_t)(BM >> 4) << 24);     // M / 16 ; A and B K-major (bits 15, 16 = 0)
+    p.chunk_doc = a.chunk_doc; p.n_docs = a.n_docs; p.doc_scores = a.doc_scores; p.chunk_scores = a.chunk_scores;
+    p.err = a.err;
+    int64_t grid = p.n_tiles < (int64_t)sm_count() ? p.n_tiles : (int64_t)sm_count();
+    if (pl.resident) {
+        auto kern = route_tc_kernel<true>;
+        MSA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem));
+        kern<<<(unsigned)grid, kThreads, pl.smem, s>>>(tmA, tmB, p);
+    } else {
+        auto kern = route_tc_kernel<false>;
+        MSA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem));
+        kern<<<(unsigned)grid, kThreads, pl.smem, s>>>(tmA, tmB, p);
+    }
+    MSA_LAUNCH_CHECK();
+    return MSA_OK;
+}
+
+}  // namespace msa

@@ -1,0 +1,182 @@
+// Top-k document selection over doc_scores [n_q][n_docs].
+//
+// Order: descending score, ties to the lower document index (a strict total order, so the
+// result is unique). One launch: P blocks per query each keep a per-thread sorted list of the
+// KT >= k best candidates of a strided slice, merge them per warp and per block by a tournament
+// (warp arg-max over list heads, the winner's lane pops its head), and write their KT best to
+// the workspace. The last block of a query to finish (an atomic ticket, no spinning) merges the
+// P lists and writes the first k. Reading the partial lists goes through L2 (__ldcg).
+#include <climits>
+
+#include "common.cuh"
+
+namespace msa {
+namespace {
+
+constexpr int kTopkThreads = 256;
+constexpr int kTopkWarps = kTopkThreads / 32;
+
+__device__ __forceinline__ bool better(float a, int ia, float b, int ib) { return a > b || (a == b && ia < ib); }
+
+template <int KT>
+struct List {
+    float s[KT];
+    int i[KT];
+    __device__ __forceinline__ void clear() {
+#pragma unroll
+        for (int j = 0; j < KT; ++j) s[j] = -__int_as_float(0x7f800000), i[j] = INT_MAX;
+    }
+    // Inserts (v, id) if it beats the current last entry; keeps the list sorted best-first.
+    __device__ __forceinline__ bool insert(float v, int id) {
+        if (!better(v, id, s[KT - 1], i[KT - 1])) return false;
+        s[KT - 1] = v;
+        i[KT - 1] = id;
+#pragma unroll
+        for (int j = KT - 1; j > 0; --j) {
+            if (better(s[j], i[j], s[j - 1], i[j - 1])) {
+                const float ts = s[j]; s[j] = s[j - 1]; s[j - 1] = ts;
+                const int ti = i[j]; i[j] = i[j - 1]; i[j - 1] = ti;
+            }
+        }
+        return true;
+    }
+    __device__ __forceinline__ void pop() {
+#pragma unroll
+        for (int j = 0; j < KT - 1; ++j) s[j] = s[j + 1], i[j] = i[j + 1];
+        s[KT - 1] = -__int_as_float(0x7f800000);
+        i[KT - 1] = INT_MAX;
+    }
+};
+
+// The warp's KT best entries (over all lanes' sorted lists), written best-first by lane 0.
+template <int KT>
+__device__ __forceinline__ void warp_tournament(List<KT>& L, float* out_s, int* out_i) {
+    const int lane = threadIdx.x & 31;
+    for (int r = 0; r < KT; ++r) {
+        float bs = L.s[0];
+        int bi = L.i[0];
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) {
+            const float os = __shfl_xor_sync(0xffffffffu, bs, off);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+            if (better(os, oi, bs, bi)) bs = os, bi = oi;
+        }
+        if (lane == 0) out_s[r] = bs, out_i[r] = bi;
+        if (L.i[0] == bi && L.s[0] == bs) L.pop();
+    }
+}
+
+// Block-wide merge of every thread's list; the result lands in res_s/res_i [KT] (shared).
+template <int KT>
+__device__ void block_merge(List<KT>& L, float (*ws)[KT], int (*wi)[KT], float* res_s, int* res_i) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    warp_tournament<KT>(L, ws[warp], wi[warp]);
+    __syncthreads();
+    if (warp == 0) {
+        L.clear();
+        if (lane < kTopkWarps) {
+#pragma unroll
+            for (int j = 0; j < KT; ++j) L.s[j] = ws[lane][j], L.i[j] = wi[lane][j];
+        }
+        warp_tournament<KT>(L, res_s, res_i);
+    }
+    __syncthreads();
+}
+
+template <int KT>
+__global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restrict__ scores, int64_t n_docs, int k,
+                                                            int P, float* part_s, int* part_i, int* counters,
+                                                            int32_t* out_idx, float* out_score) {
+    __shared__ float ws[kTopkWarps][KT];
+    __shared__ int wi[kTopkWarps][KT];
+    __shared__ float res_s[KT];
+    __shared__ int res_i[KT];
+    __shared__ int is_last;
+    const int q = blockIdx.y;
+    const float* row = scores + (int64_t)q * n_docs;
+
+    List<KT> L;
+    L.clear();
+    for (int64_t i = (int64_t)blockIdx.x * kTopkThreads + threadIdx.x; i < n_docs; i += (int64_t)P * kTopkThreads)
+        L.insert(row[i], (int)i);
+    block_merge<KT>(L, ws, wi, res_s, res_i);
+
+    float* my_s = part_s + ((int64_t)q * P + blockIdx.x) * KT;
+    int* my_i = part_i + ((int64_t)q * P + blockIdx.x) * KT;
+    if (threadIdx.x < KT) my_s[threadIdx.x] = res_s[threadIdx.x], my_i[threadIdx.x] = res_i[threadIdx.x];
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) is_last = (atomicAdd(counters + q, 1) == P - 1);
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+
+    L.clear();
+    for (int l = threadIdx.x; l < P; l += kTopkThreads) {
+        const float* ps = part_s + ((int64_t)q * P + l) * KT;
+        const int* pi = part_i + ((int64_t)q * P + l) * KT;
+        for (int j = 0; j < KT; ++j)
+            if (!L.insert(__ldcg(ps + j), __ldcg(pi + j))) break;   // lists are sorted best-first
+    }
+    block_merge<KT>(L, ws, wi, res_s, res_i);
+    if (threadIdx.x < k) {
+        out_idx[(int64_t)q * k + threadIdx.x] = res_i[threadIdx.x];
+        if (out_score) out_score[(int64_t)q * k + threadIdx.x] = res_s[threadIdx.x];
+    }
+}
+
+int pick_kt(int k) { return k <= 8 ? 8 : k <= 16 ? 16 : k <= 32 ? 32 : 64; }
+
+int pick_blocks(int64_t n_docs) {
+    int64_t p = (n_docs + kTopkThreads * 4 - 1) / (kTopkThreads * 4);
+    const int64_t cap = (int64_t)sm_count() * 2;
+    if (p > cap) p = cap;
+    if (p < 1) p = 1;
+    return (int)p;
+}
+
+}  // namespace
+}  // namespace msa
+
+using namespace msa;
+
+extern "C" {
+
+msa_status msa_topk_workspace_size(int n_q, int64_t n_docs, int k, size_t* bytes) {
+    MSA_REQUIRE(bytes, "msa_topk_workspace_size: bytes is NULL");
+    MSA_REQUIRE(n_q > 0 && n_docs > 0 && k > 0 && k <= 64, "msa_topk_workspace_size: bad sizes");
+    const int P = pick_blocks(n_docs), KT = pick_kt(k);
+    const size_t lists = (size_t)n_q * P * KT;
+    *bytes = align_up(lists * 4, 256) * 2 + align_up((size_t)n_q * 4, 256);
+    return MSA_OK;
+}
+
+msa_status msa_topk_docs(const float* doc_scores, int n_q, int64_t n_docs, int k, int32_t* idx, float* score,
+                         void* ws, size_t ws_bytes, void* stream) {
+    MSA_REQUIRE(doc_scores && idx && ws, "msa_topk_docs: NULL pointer");
+    MSA_REQUIRE(n_q > 0 && n_docs > 0 && n_docs < (int64_t)INT_MAX, "msa_topk_docs: bad sizes");
+    MSA_REQUIRE(k >= 1 && k <= 64 && k <= n_docs, "msa_topk_docs: need 1 <= k <= min(64, n_docs), got k=%d", k);
+    MSA_REQUIRE(n_q <= 65535, "msa_topk_docs: at most 65535 queries");
+    size_t need = 0;
+    MSA_RETURN_IF(msa_topk_workspace_size(n_q, n_docs, k, &need));
+    if (ws_bytes < need) return set_error(MSA_ERR_WORKSPACE, "msa_topk_docs: workspace %zu < %zu", ws_bytes, need);
+    const int P = pick_blocks(n_docs), KT = pick_kt(k);
+    const size_t lists = (size_t)n_q * P * KT;
+    char* w = static_cast<char*>(ws);
+    float* part_s = reinterpret_cast<float*>(w);
+    int* part_i = reinterpret_cast<int*>(w + align_up(lists * 4, 256));
+    int* counters = reinterpret_cast<int*>(w + 2 * align_up(lists * 4, 256));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    MSA_CUDA_TRY(cudaMemsetAsync(counters, 0, (size_t)n_q * sizeof(int), s));
+    dim3 grid(P, n_q);
+    switch (KT) {
+        case 8: topk_kernel<8><<<grid, kTopkThreads, 0, s>>>(doc_scores, n_docs, k, P, part_s, part_i, counters, idx, score); break;
+        case 16: topk_kernel<16><<<grid, kTopkThreads, 0, s>>>(doc_scores, n_docs, k, P, part_s, part_i, counters, idx, score); break;
+        case 32: topk_kernel<32><<<grid, kTopkThreads, 0, s>>>(doc_scores, n_docs, k, P, part_s, part_i, counters, idx, score); break;
+        default: topk_kernel<64><<<grid, kTopkThreads, 0, s>>>(doc_scores, n_docs, k, P, part_s, part_i, counters, idx, score); break;
+    }
+    MSA_LAUNCH_CHECK();
+    return MSA_OK;
+}
+
+}  // extern "C"

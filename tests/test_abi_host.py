@@ -1,0 +1,126 @@
+"""The C-ABI library loads, exports every entry point include/msa.h declares, and rejects bad
+arguments on the host before touching the GPU. No test here launches a kernel."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from routed_long_context_b200 import build
+
+    build.build()
+    from routed_long_context_b200 import _lib
+
+    return _lib.lib
+
+
+def _declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", fn)).read()
+            txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+            names |= set(re.findall(r"\b(msa_\w+)\s*\(", txt))
+    return sorted(names)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared_symbols()
+    assert "msa_route_scores" in names and "msa_interleave_step" in names
+    for n in names:
+        assert hasattr(lib, n), n
+    from routed_long_context_b200 import _lib
+
+    assert set(_lib.SIGNATURES) <= set(names) | {"msa_last_error", "msa_version"}
+
+
+def test_the_seven_hot_path_calls_are_declared():
+    names = _declared_symbols()
+    for n in ("msa_rope_doc", "msa_pool_chunks", "msa_route_scores", "msa_topk_docs", "msa_gather_kv",
+              "msa_sparse_attn", "msa_interleave_step"):
+        assert n in names
+
+
+def test_rope_table_is_the_rotation_angle_table(lib):
+    max_pos, d, base = 40, 8, 1.0e4
+    out = np.empty((max_pos, d // 2, 2), dtype=np.float32)
+    assert lib.msa_rope_table(max_pos, d, base, out.ctypes.data) == 0
+    p = np.arange(max_pos)[:, None]
+    w = base ** (-2.0 * np.arange(d // 2) / d)
+    np.testing.assert_array_equal(out[..., 0], np.cos(p * w).astype(np.float32))
+    np.testing.assert_array_equal(out[..., 1], np.sin(p * w).astype(np.float32))
+    assert lib.msa_rope_table(4, 7, base, out.ctypes.data) == 1          # odd d
+    assert lib.msa_rope_table(4, 8, base, None) == 1
+
+
+def test_topk_rejects_k_larger_than_docs_without_launching(lib):
+    ws = ctypes.c_size_t(0)
+    assert lib.msa_topk_workspace_size(1, 10, 4, ctypes.byref(ws)) == 0 and ws.value > 0
+    st = lib.msa_topk_docs(ctypes.c_void_p(16), 1, 10, 11, ctypes.c_void_p(16), None, ctypes.c_void_p(16), 1 << 20,
+                           None)
+    assert st == 1
+    assert b"k" in lib.msa_last_error()
+    assert lib.msa_topk_workspace_size(1, 10, 65, ctypes.byref(ws)) == 1
+
+
+def test_gather_validates_indices_and_capacity_on_host(lib):
+    C, hkv, d = 10, 1, 8
+    bank = np.zeros((C, 2, hkv, d), dtype=np.float32)
+    off = np.array([0, 3, 5, 10], dtype=np.int64)
+    mem_len = np.zeros(1, dtype=np.int32)
+    bad_idx = np.array([[0, 7]], dtype=np.int32)        # doc 7 does not exist
+    st = lib.msa_gather_kv(bank.ctypes.data, 0, C, off.ctypes.data, 3, bad_idx.ctypes.data, 1, 2, hkv, d, 16,
+                           ctypes.c_void_p(256), mem_len.ctypes.data, None)
+    assert st == 1 and b"out of range" in lib.msa_last_error()
+    idx = np.array([[2, 0]], dtype=np.int32)            # 5 + 3 rows > max_mem 6
+    st = lib.msa_gather_kv(bank.ctypes.data, 0, C, off.ctypes.data, 3, idx.ctypes.data, 1, 2, hkv, d, 6,
+                           ctypes.c_void_p(256), mem_len.ctypes.data, None)
+    assert st == 1 and b"max_mem" in lib.msa_last_error()
+
+
+def test_route_and_attention_reject_bad_shapes(lib):
+    ws = ctypes.c_size_t(0)
+    assert lib.msa_route_workspace_size(2, 16, 8, 128, 1, ctypes.byref(ws)) == 0
+    assert lib.msa_route_workspace_size(0, 16, 8, 128, 1, ctypes.byref(ws)) == 1
+    # head_dim 64 is not supported by the attention kernel
+    st = lib.msa_sparse_attn(ctypes.c_void_p(256), ctypes.c_void_p(256), ctypes.c_void_p(256), 4,
+                             ctypes.c_void_p(256), ctypes.c_void_p(256), 8, 8, 0, 1, 4, 8, 2, 64, 0.125,
+                             ctypes.c_void_p(256), 0, None)
+    assert st == 2
+    # misaligned query pointer
+    st = lib.msa_sparse_attn(ctypes.c_void_p(258), ctypes.c_void_p(256), ctypes.c_void_p(256), 4,
+                             ctypes.c_void_p(256), ctypes.c_void_p(256), 8, 8, 0, 1, 4, 8, 2, 128, 0.125,
+                             ctypes.c_void_p(256), 0, None)
+    assert st == 1
+    # causal window larger than the cache
+    st = lib.msa_sparse_attn(ctypes.c_void_p(256), ctypes.c_void_p(256), ctypes.c_void_p(256), 4,
+                             ctypes.c_void_p(256), ctypes.c_void_p(256), 8, 9, 0, 1, 4, 8, 2, 128, 0.125,
+                             ctypes.c_void_p(256), 0, None)
+    assert st == 1
+    assert lib.msa_route_set_impl(3) == 1 and lib.msa_route_set_impl(0) == 0
+
+
+def test_interleave_rejects_local_cache_overflow(lib):
+    from routed_long_context_b200 import _lib
+
+    layers = (_lib.LayerArgs * 1)()
+    for f, _ in _lib.LayerArgs._fields_:
+        setattr(layers[0], f, 256)
+    a = _lib.InterleaveArgs()
+    a.n_layers, a.layers, a.dt = 1, layers, 1
+    a.n_chunks, a.n_docs = 10, 2
+    a.doc_chunk_off = a.doc_chunk_off_host = a.chunk_doc = a.rope_cos_sin = 256
+    a.n_q, a.H, a.d, a.hq, a.hkv, a.k = 1, 8, 128, 32, 8, 1
+    a.L_prev, a.T_new, a.new_q_stride, a.L_max, a.max_mem = 60, 8, 8, 64, 16
+    a.rope_max_pos, a.scale, a.ws, a.ws_bytes = 4096, 0.1, 256, 1 << 30
+    n = ctypes.c_size_t(0)
+    assert lib.msa_interleave_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 1
+    assert b"overflow" in lib.msa_last_error()
+    a.L_prev = 56
+    assert lib.msa_interleave_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0 and n.value > 0

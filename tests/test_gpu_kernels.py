@@ -1,0 +1,263 @@
+"""Kernel-level parity of the CUDA path (through the C ABI) against the fp64 oracle, on seeded
+inputs sized to span several tiles with ragged tails, plus the edge cases of each step."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from msa_inputs import rng
+from msa_inputs.device import upload
+
+pytestmark = pytest.mark.gpu
+
+SEED = 0x5EED
+
+
+@pytest.fixture(scope="module")
+def m():
+    import routed_long_context_b200 as m
+
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return m
+
+
+def _gen(tid, shape, dtype="f32", sigma=1.0):
+    return rng.normal(SEED, tid, 0, int(np.prod(shape)), sigma, dtype).reshape(shape)
+
+
+def _np(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def _close(got, ref, dtype, what):
+    """fp32: |err| <= 1e-5 (values are O(1)); bf16 outputs: one rounding of 2^-9 relative plus fp32 error."""
+    got, ref = np.asarray(got, np.float64), np.asarray(ref, np.float64)
+    if dtype == "f32":
+        tol = 1e-5 + 1e-6 * np.abs(ref)
+    else:
+        tol = 2.0 ** -8 * np.abs(ref) + 1e-5
+    bad = np.abs(got - ref) > tol
+    assert not bad.any(), f"{what}: {bad.sum()} of {bad.size} outside tolerance, max err {np.abs(got - ref).max():.3g}"
+
+
+def _status(m):
+    assert m.device_status() == 0
+
+
+# -------------------------------------------------------------------------------------- generator
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_device_generator_matches_host_bitwise(m, dtype):
+    n, start = 1_000_003, 12345
+    t = torch.empty(n, dtype=torch.float32 if dtype == "f32" else torch.bfloat16, device="cuda")
+    rng.fill_device(t, 99, 7, start=start, sigma=0.5)
+    host = rng.normal(99, 7, start, n, 0.5, dtype)
+    np.testing.assert_array_equal(t.float().cpu().numpy(), host)
+
+
+# -------------------------------------------------------------------------------------- RoPE
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_rope_doc_segments_and_offset(m, dtype):
+    off = np.array([0, 300, 300, 555, 1000], dtype=np.int64)        # includes an empty segment
+    x = _gen(1, (1000, 8, 128), dtype)
+    cs = m.rope_table(2048, 128, 1e6)
+    for pos_offset in (0, 12):
+        xd = upload(x, dtype)
+        out = torch.empty_like(xd)
+        m.msa_rope_doc(xd, torch.from_numpy(off).cuda(), pos_offset, cs, out=out)
+        ref = O.apply_rope(x, O.doc_positions(off) + pos_offset, 1e6)
+        _close(_np(out), ref, dtype, f"rope offset {pos_offset}")
+    # in place gives the same bits
+    xd = upload(x, dtype)
+    m.msa_rope_doc(xd, torch.from_numpy(off).cuda(), 12, cs)
+    assert torch.equal(xd, out)
+    _status(m)
+
+
+def test_rope_position_past_table_is_flagged_not_faulted(m):
+    x = upload(_gen(2, (10, 1, 128)), "f32")
+    cs = m.rope_table(8, 128, 1e6)
+    m.msa_rope_doc(x, torch.tensor([0, 10], device="cuda"), 0, cs)
+    assert m.device_status() == 1          # MSA_DEV_ROPE_POSITION, rows 8 and 9 left unrotated
+    assert m.device_status() == 0          # the word is cleared by the read
+
+
+# -------------------------------------------------------------------------------------- pooling
+RAGGED = [300, 128, 1, 129, 0, 257, 1024, 77]
+
+
+@pytest.mark.parametrize("in_dt,out_dt", [("f32", "f32"), ("bf16", "bf16"), ("f32", "bf16"), ("bf16", "f32")])
+def test_pool_chunks_ragged_documents(m, in_dt, out_dt):
+    from routed_long_context_b200.bank import BankLayout
+
+    chunk = 128
+    lay = BankLayout.from_doc_lengths(RAGGED, chunk)
+    n_tok = sum(RAGGED)
+    k, v, kr = (_gen(10 + i, (n_tok, 8, 128), in_dt) for i in range(3))
+    cs = m.rope_table(2048, 128, 1e6)
+    odt = torch.float32 if out_dt == "f32" else torch.bfloat16
+    kvbar, idx = m.msa_pool_chunks(upload(k, in_dt), upload(v, in_dt), upload(kr, in_dt), lay.doc_tok_off,
+                                   lay.doc_chunk_off, lay.chunk_doc, chunk, cos_sin=cs, out_dtype=odt)
+    kb, vb, krb = O.encode_memory(k, v, kr, lay.doc_tok_off_host, chunk, 1e6)
+    dco, _ = O.chunk_layout(lay.doc_tok_off_host, chunk)
+    np.testing.assert_array_equal(dco, lay.doc_chunk_off_host)
+    np.testing.assert_array_equal(lay.chunk_doc.cpu().numpy(), np.repeat(np.arange(len(RAGGED)), np.diff(dco)))
+    _close(_np(kvbar[:, 0]), kb, out_dt, "K-bar")
+    _close(_np(kvbar[:, 1]), vb, out_dt, "V-bar")
+    _close(_np(idx), O.unit(krb), out_dt, "router index")
+    _status(m)
+
+
+def test_pool_document_translation_invariance_bitwise(m):
+    """Document-wise positions: a document's pooled, rotated K-bar is bit-identical wherever it sits."""
+    from routed_long_context_b200.bank import BankLayout
+
+    lens = [200, 300, 130]
+    docs = [_gen(20 + i, (n, 8, 128), "bf16") for i, n in enumerate(lens)]
+    cs = m.rope_table(2048, 128, 1e6)
+    got = []
+    for order in ([0, 1, 2], [2, 0, 1]):
+        lay = BankLayout.from_doc_lengths([lens[i] for i in order], 64)
+        k = upload(np.concatenate([docs[i] for i in order]), "bf16")
+        kvbar, _ = m.msa_pool_chunks(k, k, None, lay.doc_tok_off, lay.doc_chunk_off, lay.chunk_doc, 64, cos_sin=cs)
+        w = order.index(1)
+        got.append(kvbar[lay.doc_chunk_off_host[w]:lay.doc_chunk_off_host[w + 1], 0].clone())
+    assert torch.equal(got[0], got[1])
+
+
+# -------------------------------------------------------------------------------------- routing
+def _route_case(C_docs_seed, n_q, T, dtype, n_docs=140):
+    counts = 1 + rng.uniform_int(SEED, 900 + C_docs_seed, n_docs, 12).astype(np.int64)   # 1..12 chunks per doc
+    C = int(counts.sum())
+    raw = _gen(30 + C_docs_seed, (C, 8, 128))
+    index = rng.round_to(O.unit(raw).astype(np.float32), dtype).reshape(C, 8, 128)
+    qr = _gen(40 + C_docs_seed, (n_q, T, 8, 128), dtype)
+    # plant: the first chunk of doc 3 equals query 0 token T-1 (so a score of ~1 exists)
+    off = np.zeros(n_docs + 1, dtype=np.int64)
+    np.cumsum(counts, out=off[1:])
+    index[off[3]] = rng.round_to(O.unit(qr[0, T - 1]).astype(np.float32), dtype)
+    return counts, off, index, qr
+
+
+@pytest.mark.parametrize("n_q,T", [(1, 5), (3, 5), (2, 16), (1, 33)])
+def test_route_fp32_cuda_cores(m, n_q, T):
+    from routed_long_context_b200.bank import BankLayout
+
+    counts, off, index, qr = _route_case(n_q * 100 + T, n_q, T, "f32")
+    lay = BankLayout(counts)
+    ds, cs_ = m.msa_route_scores(upload(index, "f32"), lay.chunk_doc, lay.n_docs, upload(qr, "f32"),
+                                 want_chunk_scores=True)
+    ref_ds, ref_cs = O.route(index, off, qr)
+    assert np.abs(_np(ds) - ref_ds).max() <= 1e-5
+    assert np.abs(_np(cs_) - ref_cs).max() <= 1e-5
+    assert np.all(_np(ds) <= 1 + 1e-5) and np.all(_np(ds) >= -1 - 1e-5)
+    assert abs(_np(ds)[0, 3] - 1.0) < 1e-5
+    _status(m)
+
+
+@pytest.mark.parametrize("n_q,T", [(1, 16), (1, 64), (2, 48), (3, 100), (32, 1), (8, 128), (1, 3)])
+@pytest.mark.parametrize("impl", [0, 1])
+def test_route_bf16_tensor_cores_and_cuda_cores(m, n_q, T, impl):
+    from routed_long_context_b200.bank import BankLayout
+
+    counts, off, index, qr = _route_case(n_q * 1000 + T, n_q, T, "bf16")
+    lay = BankLayout(counts)
+    m.route_set_impl(2 if impl == 0 else 1)
+    try:
+        ds, cs_ = m.msa_route_scores(upload(index, "bf16"), lay.chunk_doc, lay.n_docs, upload(qr, "bf16"),
+                                     want_chunk_scores=True)
+    finally:
+        m.route_set_impl(0)
+    ref_ds, ref_cs = O.route(index, off, qr)
+    err_d, err_c = np.abs(_np(ds) - ref_ds).max(), np.abs(_np(cs_) - ref_cs).max()
+    assert err_d <= 2e-3 and err_c <= 2e-3, (err_d, err_c)
+    assert abs(_np(ds)[0, 3] - 1.0) < 2e-3
+    _status(m)
+
+
+def test_route_many_tiles_with_ragged_tail(m):
+    """13,001 chunks (101 full 128-row tiles plus a 73-row tail) through the tensor-core path."""
+    from routed_long_context_b200.bank import BankLayout
+
+    counts = np.full(1625, 8, dtype=np.int64)
+    counts[-1] = 1
+    C = int(counts.sum())
+    assert C % 128 == 73
+    lay = BankLayout(counts)
+    index = rng.round_to(O.unit(_gen(50, (C, 8, 128))).astype(np.float32), "bf16").reshape(C, 8, 128)
+    qr = _gen(51, (1, 64, 8, 128), "bf16")
+    index[C - 1] = rng.round_to(O.unit(qr[0, 7]).astype(np.float32), "bf16")     # plant in the tail row
+    ds = m.msa_route_scores(upload(index, "bf16"), lay.chunk_doc, lay.n_docs, upload(qr, "bf16"))
+    ref, _ = O.route(index, lay.doc_chunk_off_host, qr)
+    assert np.abs(_np(ds) - ref).max() <= 2e-3
+    assert _np(ds)[0, -1] > 0.99
+    _status(m)
+
+
+# -------------------------------------------------------------------------------------- top-k
+@pytest.mark.parametrize("n_q,D,k", [(1, 1, 1), (1, 7, 7), (3, 1000, 4), (32, 9766, 16), (1, 97657, 16),
+                                     (2, 5000, 33), (2, 5000, 64), (8, 2000, 12)])
+def test_topk_exact_with_ties(m, n_q, D, k):
+    s = np.round(_gen(60 + D + k, (n_q, D)) * 4) / 4                 # coarse grid: many exact ties
+    s[:, ::17] = -np.inf
+    idx, val = m.msa_topk_docs(torch.from_numpy(s.astype(np.float32)).cuda(), k)
+    ref_i, ref_v = O.topk_docs(s.astype(np.float32), k)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ref_i)
+    np.testing.assert_array_equal(val.cpu().numpy(), ref_v.astype(np.float32))
+
+
+def test_topk_repeatable(m):
+    s = torch.from_numpy((np.round(_gen(70, (4, 50000)) * 8) / 8).astype(np.float32)).cuda()
+    a, _ = m.msa_topk_docs(s, 16)
+    b, _ = m.msa_topk_docs(s, 16)
+    assert torch.equal(a, b)
+
+
+# -------------------------------------------------------------------------------------- gather
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_gather_is_exact(m, dtype):
+    counts = np.array([3, 1, 4, 0, 2, 5], dtype=np.int64)
+    off = np.concatenate([[0], np.cumsum(counts)])
+    bank = torch.from_numpy(_gen(80, (int(off[-1]), 2, 8, 128), dtype)).to(
+        torch.float32 if dtype == "f32" else torch.bfloat16).pin_memory()
+    idx = torch.tensor([[2, 0, 5], [3, 1, 4]], dtype=torch.int32)
+    dev, mem_len = m.msa_gather_kv(bank, off, idx, max_mem=12)
+    torch.cuda.synchronize()
+    assert mem_len.tolist() == [12, 3]
+    ref = O.gather_memory(bank.float().numpy(), off, [2, 0, 5])
+    np.testing.assert_array_equal(dev[0, :12].float().cpu().numpy(), ref)
+    np.testing.assert_array_equal(dev[1, :3].float().cpu().numpy(), O.gather_memory(bank.float().numpy(), off, [3, 1, 4]))
+
+
+# -------------------------------------------------------------------------------------- attention
+def _row_rel_err(got, ref):
+    num = np.linalg.norm(got - ref, axis=-1)
+    den = np.maximum(np.linalg.norm(ref, axis=-1), 1e-30)
+    return (num / den).max()
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("hq,hkv", [(32, 8), (8, 8), (16, 8), (32, 4)])
+def test_sparse_attention(m, dtype, hq, hkv):
+    n_q, T, d, max_mem, q_start = 3, 13, 128, 40, 7
+    L = q_start + T
+    q = _gen(90, (n_q, T, hq, d), dtype)
+    mem = _gen(91, (n_q, max_mem, 2, hkv, d), dtype)
+    lk, lv = _gen(92, (n_q, L + 3, hkv, d), dtype), _gen(93, (n_q, L + 3, hkv, d), dtype)
+    mem_len = np.array([0, 5, 37], dtype=np.int32)
+    out = m.msa_sparse_attn(upload(q, dtype), upload(mem, dtype), torch.from_numpy(mem_len).cuda(), upload(lk, dtype),
+                            upload(lv, dtype), L, q_start)
+    got = _np(out)
+    tol = 1e-5 if dtype == "f32" else 2e-2
+    for qi in range(n_q):
+        ml = mem_len[qi]
+        ref = O.sparse_attention(q[qi], mem[qi, :ml, 0], mem[qi, :ml, 1], lk[qi, :L], lv[qi, :L], q_start,
+                                 1 / np.sqrt(d))
+        assert _row_rel_err(got[qi], ref) <= tol
+
+
+def test_sparse_attention_no_keys_gives_zero(m):
+    q = upload(_gen(94, (1, 4, 32, 128)), "f32")
+    mem = torch.zeros((1, 4, 2, 8, 128), device="cuda")
+    lk = torch.zeros((1, 4, 8, 128), device="cuda")
+    out = m.msa_sparse_attn(q, mem, torch.zeros(1, dtype=torch.int32, device="cuda"), lk, lk, 0, 0)
+    assert torch.count_nonzero(out) == 0
