@@ -178,7 +178,7 @@ def test_route_many_tiles_with_ragged_tail(m):
     """13,001 chunks (101 full 128-row tiles plus a 73-row tail) through the tensor-core path."""
     from routed_long_context_b200.bank import BankLayout
 
-    counts = np.full(1625, 8, dtype=np.int64)
+    counts = np.full(1626, 8, dtype=np.int64)
     counts[-1] = 1
     C = int(counts.sum())
     assert C % 128 == 73
