@@ -35,6 +35,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--layers", type=int, default=18)
     ap.add_argument("--host-banks", type=int, default=2)
+    ap.add_argument("--n-docs", type=int, default=97657, help="shorter bank for small profiling cases only")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -184,7 +185,7 @@ def main():
         if world > 1:
             dist.barrier()
 
-    w = workloads.mem_100m(layers=args.layers, n_host_banks=args.host_banks)
+    w = workloads.mem_100m(layers=args.layers, n_host_banks=args.host_banks, n_docs=args.n_docs)
     lay = BankLayout(w.doc_chunks)
     cs = m.rope_table(4096, w.d, w.rope_base)
     dt = torch.bfloat16

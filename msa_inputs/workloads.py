@@ -290,9 +290,10 @@ def mem_10m() -> Workload:
                     plant_kind="per_query", plant_args={"per_query": 4})
 
 
-def mem_100m(layers: int = 18, n_host_banks: int = 2) -> Workload:
-    """781,250 pre-pooled chunks (chunk 128; 97,656 docs of 1024 tokens + one of 256); 18 routed layers."""
-    lens = np.full(97657, 1024)
+def mem_100m(layers: int = 18, n_host_banks: int = 2, n_docs: int = 97657) -> Workload:
+    """781,250 pre-pooled chunks (chunk 128; 97,656 docs of 1024 tokens + one of 256); 18 routed layers.
+    A smaller n_docs keeps the same shapes with a shorter bank (profiling of a small case)."""
+    lens = np.full(n_docs, 1024)
     lens[-1] = 256
     return Workload("100m", SEED_BASE + 3, lens, 128, "bf16", n_q=1, T0=64, k=16, prepooled=True,
                     layers=layers, n_host_banks=n_host_banks, plant_kind="single", plant_args={"n": 16})
