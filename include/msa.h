@@ -153,6 +153,24 @@ msa_status msa_topk_docs(const float* doc_scores, int n_q, int64_t n_docs, int k
                          void* ws, size_t ws_bytes, void* stream);
 msa_status msa_topk_workspace_size(int n_q, int64_t n_docs, int k, size_t* bytes);
 
+/* Allocation-free variant of msa_topk_docs. The pages have no counterpart: this is a library
+ * addition for callers that cannot allocate device memory when they select documents — a host
+ * application that loads this library as a plugin and hands it only its own input and output
+ * buffers, a serving loop whose device memory is reserved up front by its own pool, or a
+ * latency-bound loop that cannot take cudaMalloc's implicit device synchronisation.
+ * Same arguments and results as msa_topk_docs without the workspace: the scratch (partial lists
+ * and ticket counters) is a fixed array of msa_topk_noalloc_max_scratch() bytes (1 MiB) in the
+ * library's device memory, held by every GPU that loads the library until the process exits.
+ * A size whose scratch (msa_topk_workspace_size) exceeds it fails with MSA_ERR_INVALID_ARG and
+ * launches nothing. The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream capture. Every call
+ * shares the array: calls whose work overlaps on the GPU (other streams, other host threads on
+ * the same device) race and corrupt each other's results, so order them on one stream. Calls no
+ * cudaMalloc, cudaFree or allocating library routine. */
+msa_status msa_topk_docs_noalloc(const float* doc_scores, int n_q, int64_t n_docs, int k, int32_t* idx, float* score,
+                                 void* stream);
+size_t msa_topk_noalloc_max_scratch(void);
+
 /* Fetch of the selected documents' compressed K-bar/V-bar from host memory
  * ([P2] §工程实现的关键细节: K-bar^R stays in GPU memory, K-bar/V-bar live in host DRAM and are
  * loaded asynchronously once routing has chosen the documents; [P5] §3 async prefetch).

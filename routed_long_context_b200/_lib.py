@@ -49,6 +49,8 @@ SIGNATURES = {
     "msa_route_set_impl": (i32, [ctypes.c_int]),
     "msa_topk_docs": (i32, [vp, ctypes.c_int, i64, ctypes.c_int, vp, vp, vp, sz, vp]),
     "msa_topk_workspace_size": (i32, [ctypes.c_int, i64, ctypes.c_int, ctypes.POINTER(sz)]),
+    "msa_topk_docs_noalloc": (i32, [vp, ctypes.c_int, i64, ctypes.c_int, vp, vp, vp]),
+    "msa_topk_noalloc_max_scratch": (sz, []),
     "msa_gather_kv": (i32, [vp, i32, i64, vp, i64, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                             ctypes.c_int, vp, vp, vp]),
     "msa_sparse_attn": (i32, [vp, vp, vp, ctypes.c_int, vp, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int,

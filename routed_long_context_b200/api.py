@@ -144,6 +144,18 @@ def msa_topk_docs(doc_scores, k: int, idx=None, score=None, ws=None, stream=None
     return idx, score
 
 
+def msa_topk_docs_noalloc(doc_scores, k: int, idx=None, score=None, stream=None):
+    """msa_topk_docs without a workspace: for callers that cannot allocate device memory at selection
+    time. Scratch is the library's fixed device array; calls that overlap on the GPU race."""
+    n_q, n_docs = doc_scores.shape
+    dev = doc_scores.device
+    idx = torch.empty((n_q, k), dtype=torch.int32, device=dev) if idx is None else idx
+    score = torch.empty((n_q, k), dtype=torch.float32, device=dev) if score is None else score
+    check(lib.msa_topk_docs_noalloc(_ptr(doc_scores), n_q, n_docs, k, _ptr(idx), _ptr(score), _stream(stream)),
+          "msa_topk_docs_noalloc")
+    return idx, score
+
+
 def msa_gather_kv(host_bank, doc_chunk_off_host, idx_host, max_mem: int, dev_mem_kv=None, device="cuda",
                   copy_stream=None):
     """Copy the selected docs' rows [*, 2, hkv, d] from the pinned host bank into

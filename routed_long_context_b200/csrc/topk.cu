@@ -7,6 +7,7 @@
 // the workspace. The last block of a query to finish (an atomic ticket, no spinning) merges the
 // P lists and writes the first k. Reading the partial lists goes through L2 (__ldcg).
 #include <climits>
+#include <mutex>
 
 #include "common.cuh"
 
@@ -167,6 +168,90 @@ msa_status msa_topk_docs(const float* doc_scores, int n_q, int64_t n_docs, int k
     int* part_i = reinterpret_cast<int*>(w + align_up(lists * 4, 256));
     int* counters = reinterpret_cast<int*>(w + 2 * align_up(lists * 4, 256));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    MSA_CUDA_TRY(cudaMemsetAsync(counters, 0, (size_t)n_q * sizeof(int), s));
+    dim3 grid(P, n_q);
+    switch (KT) {
+        case 8: topk_kernel<8><<<grid, kTopkThreads, 0, s>>>(doc_scores, n_docs, k, P, part_s, part_i, counters, idx, score); break;
+        case 16: topk_kernel<16><<<grid, kTopkThreads, 0, s>>>(doc_scores, n_docs, k, P, part_s, part_i, counters, idx, score); break;
+        case 32: topk_kernel<32><<<grid, kTopkThreads, 0, s>>>(doc_scores, n_docs, k, P, part_s, part_i, counters, idx, score); break;
+        default: topk_kernel<64><<<grid, kTopkThreads, 0, s>>>(doc_scores, n_docs, k, P, part_s, part_i, counters, idx, score); break;
+    }
+    MSA_LAUNCH_CHECK();
+    return MSA_OK;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------------------------------------
+// Allocation-free variant of msa_topk_docs.
+//
+// Some callers cannot allocate device memory at the point where they select documents: a C host
+// application that loads this library as a plugin and hands it only its input and output buffers,
+// a serving loop whose device memory is fully reserved up front by its own pool, or a latency-bound
+// loop where cudaMalloc's implicit device synchronisation is not acceptable. For them the partial
+// lists and ticket counters live in this fixed, file-scope device array instead of a caller
+// workspace. Every GPU that loads the library holds the array until the process exits.
+// ------------------------------------------------------------------------------------------------
+namespace msa {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;   // 1 MiB per device
+static __device__ __align__(256) unsigned char g_topk_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxNoAllocDevices = 64;
+void* g_scratch_ptr[kMaxNoAllocDevices] = {nullptr};
+std::mutex g_scratch_mu;
+
+// Device address of g_topk_scratch on the current device, looked up once per device. In host code
+// the array's name is only a host-side stand-in, so its address must come from the runtime.
+msa_status scratch_address(void** out) {
+    int dev = 0;
+    MSA_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxNoAllocDevices)
+        return set_error(MSA_ERR_UNSUPPORTED, "msa_topk_docs_noalloc: device %d out of range", dev);
+    std::lock_guard<std::mutex> lk(g_scratch_mu);
+    if (!g_scratch_ptr[dev]) {
+        void* p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_topk_scratch);
+        if (e != cudaSuccess || p == nullptr)
+            return set_error(MSA_ERR_CUDA, "msa_topk_docs_noalloc: cudaGetSymbolAddress failed: %s",
+                             cudaGetErrorString(e));
+        g_scratch_ptr[dev] = p;
+    }
+    *out = g_scratch_ptr[dev];
+    return MSA_OK;
+}
+
+}  // namespace
+}  // namespace msa
+
+extern "C" {
+
+size_t msa_topk_noalloc_max_scratch(void) { return kNoAllocScratchBytes; }
+
+msa_status msa_topk_docs_noalloc(const float* doc_scores, int n_q, int64_t n_docs, int k, int32_t* idx, float* score,
+                                 void* stream) {
+    MSA_REQUIRE(doc_scores && idx, "msa_topk_docs_noalloc: NULL pointer");
+    MSA_REQUIRE(n_q > 0 && n_docs > 0 && n_docs < (int64_t)INT_MAX, "msa_topk_docs_noalloc: bad sizes");
+    MSA_REQUIRE(k >= 1 && k <= 64 && k <= n_docs, "msa_topk_docs_noalloc: need 1 <= k <= min(64, n_docs), got k=%d", k);
+    MSA_REQUIRE(n_q <= 65535, "msa_topk_docs_noalloc: at most 65535 queries");
+    size_t need = 0;
+    MSA_RETURN_IF(msa_topk_workspace_size(n_q, n_docs, k, &need));
+    if (need > kNoAllocScratchBytes)
+        return set_error(MSA_ERR_INVALID_ARG,
+                         "msa_topk_docs_noalloc: n_q=%d, n_docs=%lld, k=%d need %zu bytes of scratch, above the fixed "
+                         "%zu-byte array; use msa_topk_docs with a workspace",
+                         n_q, (long long)n_docs, k, need, kNoAllocScratchBytes);
+    void* ws = nullptr;
+    MSA_RETURN_IF(scratch_address(&ws));
+    const int P = pick_blocks(n_docs), KT = pick_kt(k);
+    const size_t lists = (size_t)n_q * P * KT;
+    char* w = static_cast<char*>(ws);
+    float* part_s = reinterpret_cast<float*>(w);
+    int* part_i = reinterpret_cast<int*>(w + align_up(lists * 4, 256));
+    int* counters = reinterpret_cast<int*>(w + 2 * align_up(lists * 4, 256));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // the array keeps the previous call's contents: the tickets must start at zero
     MSA_CUDA_TRY(cudaMemsetAsync(counters, 0, (size_t)n_q * sizeof(int), s));
     dim3 grid(P, n_q);
     switch (KT) {
