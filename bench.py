@@ -36,8 +36,13 @@ def parse():
     ap.add_argument("--layers", type=int, default=18)
     ap.add_argument("--host-banks", type=int, default=2)
     ap.add_argument("--n-docs", type=int, default=97657, help="shorter bank for small profiling cases only")
+    ap.add_argument("--reserved-sms", type=int, default=8,
+                    help="SMs the routers leave free for the overlapped selection and attention")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default="100m", choices=["100m", "encode10m"],
+                    help="100m: the routing step (the reported metric); encode10m: offline encoding of the "
+                         "10M-token bank (document-wise RoPE + chunk-mean pooling), reported separately")
     return ap.parse_args()
 
 
@@ -157,6 +162,53 @@ def reference_arm(args, rank):
     }))
 
 
+# ---------------------------------------------------------------------------------------------- encode
+def encode_bench(args, rank, world, local_rank):
+    """Offline encoding of the 10M-token configuration: 9,766 docs x 1024 tokens, chunk 256, bf16 token-level
+    K, V, K^R [10,000,384 x 8 x 128] (61.4 GB read) -> pooled K-bar/V-bar and unit-vector router index."""
+    import torch
+
+    import routed_long_context_b200 as m
+    from msa_inputs import workloads
+    from msa_inputs.device import memory_tensor
+    from routed_long_context_b200.bank import BankLayout, encode_tokens
+
+    torch.cuda.set_device(local_rank)
+    w = workloads.mem_10m()
+    lay = BankLayout.from_doc_lengths(w.doc_len, w.chunk)
+    cs = m.rope_table(4096, w.d, w.rope_base)
+    k, v, kr = (memory_tensor(w, 0, n) for n in ("k", "v", "kr"))
+    kvbar = torch.empty((lay.n_chunks, 2, w.hkv, w.d), dtype=torch.bfloat16, device="cuda")
+    index = torch.empty((lay.n_chunks, w.H, w.d), dtype=torch.bfloat16, device="cuda")
+    s = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        m.msa_pool_chunks(k, v, kr, lay.doc_tok_off, lay.doc_chunk_off, lay.chunk_doc, w.chunk, cos_sin=cs,
+                          kvbar=kvbar, kr_index=index)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        e0.record(s)
+        for _ in range(args.steps):
+            m.msa_pool_chunks(k, v, kr, lay.doc_tok_off, lay.doc_chunk_off, lay.chunk_doc, w.chunk, cos_sin=cs,
+                              kvbar=kvbar, kr_index=index)
+        e1.record(s)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    read = 3 * w.n_tok * w.H * w.d * 2
+    write = lay.n_chunks * 3 * w.H * w.d * 2
+    gbs = (read + write) / (ms / 1e3) / 1e9
+    peak, kind = peaks()
+    if rank == 0:
+        print(json.dumps({
+            "metric": "10M-token offline encode (doc-wise RoPE + chunk-mean pooling) throughput", "value": w.n_tok / (ms / 1e3),
+            "unit": "memory tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "encode10m: 9,766 docs x 1024 tokens, chunk 256, K/V/K^R bf16 [10,000,384 x 8 x 128]"},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                         "traffic": None, "kernel": "pool_kernel", "peak_kind": kind},
+            "clocks": clk.summary(), "device_status": m.device_status()}))
+
+
 # ---------------------------------------------------------------------------------------------- ours
 def main():
     args = parse()
@@ -165,6 +217,8 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
     if args.impl == "reference":
         return reference_arm(args, rank)
+    if args.workload == "encode10m":
+        return encode_bench(args, rank, world, local_rank)
 
     import numpy as np
     import torch
@@ -218,7 +272,7 @@ def main():
     rnd = m.InterleaveRound(layer_args, n_chunks=lay.n_chunks, n_docs=lay.n_docs, doc_chunk_off=lay.doc_chunk_off,
                             doc_chunk_off_host=lay.doc_chunk_off_host, chunk_doc=lay.chunk_doc, n_q=1, H=w.H, d=w.d,
                             hq=w.hq, hkv=w.hkv, k=w.k, L_prev=0, T_new=w.T0, new_q_stride=w.T0, L_max=w.T0,
-                            max_mem=w.max_mem, cos_sin=cs, dtype=dt)
+                            max_mem=w.max_mem, cos_sin=cs, dtype=dt, reserved_sms=args.reserved_sms)
 
     # ---- warm-up, then K timed steps (inputs are 1.6 GB per layer: larger than L2, no flush needed)
     for _ in range(args.warmup):
@@ -311,6 +365,7 @@ def main():
                        "l2": "inputs larger than L2 (1.6 GB index per layer); no flush",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
             "route_ms_per_layer": route_ms,
+            "reserved_sms": args.reserved_sms,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": None,
                          "kernel": "route_tc_kernel (+ its query-normalisation prepass)",

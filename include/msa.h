@@ -232,6 +232,8 @@ typedef struct msa_interleave_args {
     const float* rope_cos_sin;      /* device table of msa_rope_table(rope_max_pos, d, base) */
     int64_t rope_max_pos;
     float scale;                    /* attention scale, normally 1/sqrt(d) */
+    int reserved_sms;               /* SMs the router kernels leave free for the overlapped selection
+                                       and attention of earlier layers (0 = routers use every SM) */
     void* ws;                       /* device workspace of msa_interleave_workspace_size bytes */
     size_t ws_bytes;
 } msa_interleave_args;
@@ -242,10 +244,12 @@ typedef struct msa_interleave_args {
  * global positions k + L_prev + t, values copied), rotate their queries likewise, score the
  * memory with the router queries of all T_act = L_prev + T_new active tokens, select the top-k
  * documents, copy their indices to topk_idx_host, fetch their K-bar/V-bar from the host bank on
- * `copy` and attend. The routing of every layer is enqueued on `compute` first; the host then
- * waits for each layer's selection (polling with a deadline of host_wait_timeout_us, giving
- * MSA_ERR_TIMEOUT) and enqueues its fetch on `copy`, so fetches overlap the routing of later
- * layers; attention waits on its own fetch. Returns after everything is enqueued. */
+ * `copy` and attend. The router kernels run back to back on `compute`; selection and attention
+ * run on two library-owned streams (created once per device) that fork from and join back into
+ * `compute`, so a layer's selection, fetch and attention overlap the routing of later layers.
+ * The host waits for each layer's selection (polling with a deadline of host_wait_timeout_us,
+ * giving MSA_ERR_TIMEOUT) before enqueueing its fetch. When the call returns, everything is
+ * enqueued and `compute` is ordered after all of it. */
 msa_status msa_interleave_step(const msa_interleave_args* a, void* compute, void* copy, int64_t host_wait_timeout_us);
 msa_status msa_interleave_workspace_size(const msa_interleave_args* a, size_t* bytes);
 

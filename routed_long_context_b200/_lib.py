@@ -29,7 +29,7 @@ class InterleaveArgs(ctypes.Structure):
                 ("hq", ctypes.c_int), ("hkv", ctypes.c_int), ("k", ctypes.c_int), ("L_prev", ctypes.c_int),
                 ("T_new", ctypes.c_int), ("new_q_stride", ctypes.c_int), ("L_max", ctypes.c_int),
                 ("max_mem", ctypes.c_int), ("rope_cos_sin", vp), ("rope_max_pos", i64), ("scale", f32),
-                ("ws", vp), ("ws_bytes", sz)]
+                ("reserved_sms", ctypes.c_int), ("ws", vp), ("ws_bytes", sz)]
 
 
 # name -> (restype, argtypes)

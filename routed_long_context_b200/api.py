@@ -192,7 +192,8 @@ class InterleaveRound:
     """Marshals msa_interleave_args for one round; holds the ctypes structures alive."""
 
     def __init__(self, layers, *, n_chunks, n_docs, doc_chunk_off, doc_chunk_off_host, chunk_doc, n_q, H, d, hq, hkv,
-                 k, L_prev, T_new, new_q_stride, L_max, max_mem, cos_sin, scale=None, dtype=torch.bfloat16, ws=None):
+                 k, L_prev, T_new, new_q_stride, L_max, max_mem, cos_sin, scale=None, dtype=torch.bfloat16, ws=None,
+                 reserved_sms: int = 0):
         self.layer_structs = (_lib.LayerArgs * len(layers))()
         for i, y in enumerate(layers):
             s = self.layer_structs[i]
@@ -213,6 +214,7 @@ class InterleaveRound:
         a.rope_cos_sin = cos_sin.data_ptr()
         a.rope_max_pos = cos_sin.shape[0]
         a.scale = 1.0 / math.sqrt(d) if scale is None else scale
+        a.reserved_sms = reserved_sms
         self.args = a
         need = ctypes.c_size_t(0)
         a.ws, a.ws_bytes = None, 0

@@ -42,10 +42,28 @@ struct RouteTcArgs {
     float* doc_scores;
     float* chunk_scores;
     int* err;
+    int grid_cap;          // > 0: at most this many CTAs (SMs left free for concurrent work)
+    int* tile_counter;     // zero at launch (route_prepare zeroes it)
 };
 // Returns MSA_ERR_UNSUPPORTED (without launching) when the shape does not fit the kernel.
 msa_status launch_route_tc(const RouteTcArgs& a, cudaStream_t s);
 // Rows the tensor-core path needs in qhat for N columns (0 if unsupported).
 int route_tc_pad_rows(int N, int K);
+
+// Router scoring split in two launches so a caller can hoist the (tiny) query prepass off the
+// router's stream: route_prepare normalises the queries into qhat and fills the score outputs with
+// -inf and zeroes the tile counter; route_launch runs the scorer. The workspace holds the tile
+// counter in its first 256 bytes and qhat after it. grid_cap > 0 limits the scorer's CTAs.
+struct RoutePlan {
+    msa_dtype dt;
+    int n_q, T, H, d, K, N, n_pad;
+    bool use_tc;
+};
+msa_status route_plan(msa_dtype dt, int64_t n_chunks, int n_q, int T, int H, int d, RoutePlan* plan);
+msa_status route_prepare(const RoutePlan& p, const void* qr, void* ws, float* doc_scores, int64_t n_docs,
+                         float* chunk_scores, int64_t n_chunks, cudaStream_t s);
+msa_status route_launch(const RoutePlan& p, const void* kr_index, int64_t n_chunks, const int32_t* chunk_doc,
+                        int64_t n_docs, void* ws, float* doc_scores, float* chunk_scores, int grid_cap,
+                        cudaStream_t s);
 
 }  // namespace msa

@@ -19,7 +19,8 @@ std::atomic<int> g_route_impl{0};   // 0 auto, 1 CUDA cores, 2 tensor cores
 template <typename T, typename TQ>
 __global__ void __launch_bounds__(128) route_prep_kernel(const T* __restrict__ qr, int N, int n_pad, int H, int d,
                                                          TQ* __restrict__ qhat, float* doc_scores, int64_t n_doc_fill,
-                                                         float* chunk_scores, int64_t n_chunk_fill) {
+                                                         float* chunk_scores, int64_t n_chunk_fill, int* tile_counter) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) *tile_counter = 0;
     constexpr int VEC = 16 / sizeof(T);
     const int K = H * d;
     const int lanes_per_head = d / VEC;
@@ -158,12 +159,84 @@ bool simt_supported(msa_dtype dt, int K) {
     return K % (32 * VEC) == 0 && (kpl == 8 || kpl == 16 || kpl == 32 || kpl == 64);
 }
 
+constexpr size_t kCounterBytes = 256;   // the tile counter sits in the first 256 bytes of the workspace
+
 size_t qhat_bytes(int N, int K) {
     const int rows = (N + 255) / 256 * 256;
-    return align_up((size_t)rows * K * sizeof(float), 256);
+    return kCounterBytes + align_up((size_t)rows * K * sizeof(float), 256);
 }
 
 }  // namespace
+
+msa_status route_plan(msa_dtype dt, int64_t n_chunks, int n_q, int T, int H, int d, RoutePlan* plan) {
+    MSA_REQUIRE(dtype_ok(dt), "msa_route_scores: bad dtype %d", dt);
+    MSA_REQUIRE(n_q > 0 && T > 0 && H > 0 && d > 0, "msa_route_scores: bad sizes");
+    MSA_REQUIRE((int64_t)n_q * T <= (1 << 20), "msa_route_scores: too many query tokens");
+    if (!rope_layout_ok(dt, d))
+        return set_error(MSA_ERR_UNSUPPORTED, "msa_route_scores: head_dim %d unsupported for this dtype", d);
+    RoutePlan p{};
+    p.dt = dt; p.n_q = n_q; p.T = T; p.H = H; p.d = d; p.K = H * d; p.N = n_q * T;
+    const int impl = g_route_impl.load();
+    const int tc_rows = dt == MSA_BF16 ? route_tc_pad_rows(p.N, p.K) : 0;
+    p.use_tc = dt == MSA_BF16 && impl != 1 && tc_rows > 0 && n_chunks > 0;
+    if (impl == 2 && !p.use_tc)
+        return set_error(MSA_ERR_UNSUPPORTED, "msa_route_scores: tensor-core path unavailable for this shape");
+    if (!p.use_tc && !simt_supported(dt, p.K))
+        return set_error(MSA_ERR_UNSUPPORTED, "msa_route_scores: H*d = %d unsupported", p.K);
+    p.n_pad = p.use_tc ? tc_rows : p.N;
+    *plan = p;
+    return MSA_OK;
+}
+
+msa_status route_prepare(const RoutePlan& p, const void* qr, void* ws, float* doc_scores, int64_t n_docs,
+                         float* chunk_scores, int64_t n_chunks, cudaStream_t s) {
+    int* counter = static_cast<int*>(ws);
+    void* qhat = static_cast<char*>(ws) + kCounterBytes;
+    const int64_t fill = (int64_t)p.n_q * n_docs;
+    const int64_t cfill = chunk_scores ? (int64_t)p.n_q * n_chunks : 0;
+    int64_t pblocks = p.n_pad;
+    const int64_t want_fill = (fill + cfill + 127) / 128;
+    if (pblocks < want_fill) pblocks = want_fill;
+    const int64_t cap = (int64_t)sm_count() * 16;
+    if (pblocks > cap) pblocks = cap;
+    if (pblocks < 1) pblocks = 1;
+    if (p.use_tc) {
+        route_prep_kernel<__nv_bfloat16, __nv_bfloat16><<<(unsigned)pblocks, 128, 0, s>>>(
+            static_cast<const __nv_bfloat16*>(qr), p.N, p.n_pad, p.H, p.d, static_cast<__nv_bfloat16*>(qhat),
+            doc_scores, fill, chunk_scores, cfill, counter);
+    } else if (p.dt == MSA_BF16) {
+        route_prep_kernel<__nv_bfloat16, float><<<(unsigned)pblocks, 128, 0, s>>>(
+            static_cast<const __nv_bfloat16*>(qr), p.N, p.n_pad, p.H, p.d, static_cast<float*>(qhat), doc_scores,
+            fill, chunk_scores, cfill, counter);
+    } else {
+        route_prep_kernel<float, float><<<(unsigned)pblocks, 128, 0, s>>>(
+            static_cast<const float*>(qr), p.N, p.n_pad, p.H, p.d, static_cast<float*>(qhat), doc_scores, fill,
+            chunk_scores, cfill, counter);
+    }
+    MSA_LAUNCH_CHECK();
+    return MSA_OK;
+}
+
+msa_status route_launch(const RoutePlan& p, const void* kr_index, int64_t n_chunks, const int32_t* chunk_doc,
+                        int64_t n_docs, void* ws, float* doc_scores, float* chunk_scores, int grid_cap,
+                        cudaStream_t s) {
+    if (n_chunks == 0) return MSA_OK;
+    int* err = device_error_word();
+    const void* qhat = static_cast<char*>(ws) + kCounterBytes;
+    if (p.use_tc) {
+        RouteTcArgs a{};
+        a.index = kr_index; a.qhat = qhat; a.n_chunks = n_chunks; a.K = p.K; a.N = p.N; a.n_pad = p.n_pad;
+        a.T = p.T; a.chunk_doc = chunk_doc; a.n_docs = n_docs; a.doc_scores = doc_scores;
+        a.chunk_scores = chunk_scores; a.err = err; a.grid_cap = grid_cap; a.tile_counter = static_cast<int*>(ws);
+        return launch_route_tc(a, s);
+    }
+    if (p.dt == MSA_BF16)
+        return launch_simt<__nv_bfloat16>(kr_index, n_chunks, p.K, static_cast<const float*>(qhat), p.N, p.T,
+                                          chunk_doc, n_docs, doc_scores, chunk_scores, err, s);
+    return launch_simt<float>(kr_index, n_chunks, p.K, static_cast<const float*>(qhat), p.N, p.T, chunk_doc, n_docs,
+                              doc_scores, chunk_scores, err, s);
+}
+
 }  // namespace msa
 
 using namespace msa;
@@ -186,69 +259,20 @@ msa_status msa_route_workspace_size(int n_q, int T, int H, int d, msa_dtype dt, 
 msa_status msa_route_scores(const void* kr_index, msa_dtype dt, int64_t n_chunks, const int32_t* chunk_doc,
                             int64_t n_docs, const void* qr, int n_q, int T, int H, int d, float* doc_scores,
                             float* chunk_scores, void* ws, size_t ws_bytes, void* stream) {
-    MSA_REQUIRE(dtype_ok(dt), "msa_route_scores: bad dtype %d", dt);
-    MSA_REQUIRE(n_chunks >= 0 && n_docs > 0 && n_q > 0 && T > 0 && H > 0 && d > 0, "msa_route_scores: bad sizes");
-    MSA_REQUIRE((int64_t)n_q * T <= (1 << 20), "msa_route_scores: too many query tokens");
+    MSA_REQUIRE(n_chunks >= 0 && n_docs > 0, "msa_route_scores: bad sizes");
     MSA_REQUIRE(qr && doc_scores && ws, "msa_route_scores: NULL pointer");
     MSA_REQUIRE(n_chunks == 0 || (kr_index && chunk_doc), "msa_route_scores: NULL index");
     MSA_REQUIRE(aligned16(qr) && aligned16(ws) && (n_chunks == 0 || aligned16(kr_index)),
                 "msa_route_scores: pointers must be 16-byte aligned");
-    const int K = H * d;
-    const int N = n_q * T;
+    RoutePlan plan;
+    MSA_RETURN_IF(route_plan(dt, n_chunks, n_q, T, H, d, &plan));
     size_t need = 0;
     MSA_RETURN_IF(msa_route_workspace_size(n_q, T, H, d, dt, &need));
     if (ws_bytes < need) return set_error(MSA_ERR_WORKSPACE, "msa_route_scores: workspace %zu < %zu", ws_bytes, need);
-    if (!rope_layout_ok(dt, d))
-        return set_error(MSA_ERR_UNSUPPORTED, "msa_route_scores: head_dim %d unsupported for this dtype", d);
-
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    int* err = device_error_word();
-    const int impl = g_route_impl.load();
-    const int tc_rows = dt == MSA_BF16 ? route_tc_pad_rows(N, K) : 0;
-    const bool use_tc = dt == MSA_BF16 && impl != 1 && tc_rows > 0 && n_chunks > 0;
-    if (impl == 2 && !use_tc)
-        return set_error(MSA_ERR_UNSUPPORTED, "msa_route_scores: tensor-core path unavailable for this shape");
-    if (!use_tc && !simt_supported(dt, K))
-        return set_error(MSA_ERR_UNSUPPORTED, "msa_route_scores: H*d = %d unsupported", K);
-
-    const int n_pad = use_tc ? tc_rows : N;
-    const int64_t fill = (int64_t)n_q * n_docs;
-    const int64_t cfill = chunk_scores ? (int64_t)n_q * n_chunks : 0;
-    int64_t pblocks = n_pad;
-    const int64_t want_fill = (fill + cfill + 127) / 128;
-    if (pblocks < want_fill) pblocks = want_fill;
-    const int64_t cap = (int64_t)sm_count() * 16;
-    if (pblocks > cap) pblocks = cap;
-    if (pblocks < 1) pblocks = 1;
-    if (use_tc) {
-        if (dt == MSA_BF16)
-            route_prep_kernel<__nv_bfloat16, __nv_bfloat16><<<(unsigned)pblocks, 128, 0, s>>>(
-                static_cast<const __nv_bfloat16*>(qr), N, n_pad, H, d, static_cast<__nv_bfloat16*>(ws), doc_scores,
-                fill, chunk_scores, cfill);
-    } else if (dt == MSA_BF16) {
-        route_prep_kernel<__nv_bfloat16, float><<<(unsigned)pblocks, 128, 0, s>>>(
-            static_cast<const __nv_bfloat16*>(qr), N, n_pad, H, d, static_cast<float*>(ws), doc_scores, fill,
-            chunk_scores, cfill);
-    } else {
-        route_prep_kernel<float, float><<<(unsigned)pblocks, 128, 0, s>>>(
-            static_cast<const float*>(qr), N, n_pad, H, d, static_cast<float*>(ws), doc_scores, fill, chunk_scores,
-            cfill);
-    }
-    MSA_LAUNCH_CHECK();
+    MSA_RETURN_IF(route_prepare(plan, qr, ws, doc_scores, n_docs, chunk_scores, n_chunks, s));
     if (n_chunks == 0) return MSA_OK;
-
-    if (use_tc) {
-        RouteTcArgs a{};
-        a.index = kr_index; a.qhat = ws; a.n_chunks = n_chunks; a.K = K; a.N = N; a.n_pad = n_pad; a.T = T;
-        a.chunk_doc = chunk_doc; a.n_docs = n_docs; a.doc_scores = doc_scores; a.chunk_scores = chunk_scores;
-        a.err = err;
-        return launch_route_tc(a, s);
-    }
-    if (dt == MSA_BF16)
-        return launch_simt<__nv_bfloat16>(kr_index, n_chunks, K, static_cast<const float*>(ws), N, T, chunk_doc,
-                                          n_docs, doc_scores, chunk_scores, err, s);
-    return launch_simt<float>(kr_index, n_chunks, K, static_cast<const float*>(ws), N, T, chunk_doc, n_docs,
-                              doc_scores, chunk_scores, err, s);
+    return route_launch(plan, kr_index, n_chunks, chunk_doc, n_docs, ws, doc_scores, chunk_scores, 0, s);
 }
 
 }  // extern "C"

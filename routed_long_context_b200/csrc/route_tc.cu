@@ -10,6 +10,9 @@
 // Roles (192 threads): warp 0 = TMA producer, warp 1 = TMEM owner and MMA issuer,
 // warps 2..5 = epilogue (warp w reads TMEM lanes 32*(w%4) .. 32*(w%4)+31).
 // Two TMEM accumulators let the epilogue of tile i overlap the main loop of tile i+1.
+// Tiles are handed out dynamically: the producer takes the next tile index from a launch-wide
+// atomic counter and publishes it to the MMA and epilogue warps through a 2-entry shared-memory
+// queue, so CTAs that start late (SMs still busy with concurrent kernels) simply take fewer tiles.
 // Modes: RESIDENT keeps all of qhat (<= 64 columns) in shared memory, loaded once per CTA,
 // so only the index streams from HBM; otherwise qhat tiles of BN <= 256 columns stream with A.
 // Every mbarrier wait is bounded (about 2 s of %globaltimer); on expiry the CTA records
@@ -46,6 +49,7 @@ struct TcParams {
     float* doc_scores;
     float* chunk_scores;
     int* err;
+    int* tile_counter;     // zero at launch; tiles are handed out in order by atomicAdd
 };
 
 // ---------------------------------------------------------------------------------- PTX helpers
@@ -169,8 +173,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* tfull = bars + 2 * kMaxStages;  // [2]
     uint64_t* tempty = tfull + 2;             // [2]
     uint64_t* bfull = tempty + 2;             // [1]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bfull + 1);
+    uint64_t* tqf = bfull + 1;                // [2] tile queue: entry written
+    uint64_t* tqe = tqf + 2;                  // [2] tile queue: entry read by the MMA and 4 epilogue warps
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tqe + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile int* tile_q = abort_flag + 1;    // [2] tile index per queue entry, -1 = no more tiles
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -184,6 +191,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(smem_u32(&tempty[a]), 4);
         }
         mbar_init(smem_u32(bfull), 1);
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(smem_u32(&tqf[a]), 1);
+            mbar_init(smem_u32(&tqe[a]), 5);
+        }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -220,9 +231,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             int stage = 0;
             uint32_t phase = 0;
-            for (int64_t tile = blockIdx.x; ok && tile < p.n_tiles; tile += gridDim.x) {
-                const int m0 = (int)(tile / p.n_tiles_n) * BM;
-                const int n0 = (int)(tile % p.n_tiles_n) * p.BN;
+            for (int seq = 0; ok; ++seq) {
+                // next tile from the launch-wide counter, published through the 2-entry tile queue
+                const int tslot = seq & 1;
+                if (!mbar_wait(smem_u32(&tqe[tslot]), (((uint32_t)seq >> 1) & 1u) ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const int t = atomicAdd(p.tile_counter, 1);
+                const int tile = (int64_t)t < p.n_tiles ? t : -1;
+                tile_q[tslot] = tile;
+                mbar_arrive(smem_u32(&tqf[tslot]));
+                if (tile < 0) break;
+                const int m0 = (tile / p.n_tiles_n) * BM;
+                const int n0 = (tile % p.n_tiles_n) * p.BN;
                 for (int kb = 0; kb < kblocks; ++kb) {
                     if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1, abort_flag)) {
                         ok = false;
@@ -259,7 +281,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             int acc = 0;
             uint32_t acc_phase = 0;
             bool mma_pending = false;
-            for (int64_t tile = blockIdx.x; ok && tile < p.n_tiles; tile += gridDim.x) {
+            for (int seq = 0; ok; ++seq) {
+                const int tslot = seq & 1;
+                if (!mbar_wait(smem_u32(&tqf[tslot]), ((uint32_t)seq >> 1) & 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const int tile = tile_q[tslot];
+                mbar_arrive(smem_u32(&tqe[tslot]));
+                if (tile < 0) break;
+                acc = seq & 1;
+                acc_phase = ((uint32_t)seq >> 1) & 1u;
                 if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1, abort_flag)) {
                     ok = false;
                     break;
@@ -289,7 +321,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 umma_commit(smem_u32(&tfull[acc]));
                 mma_pending = false;
-                if (++acc == 2) acc = 0, acc_phase ^= 1;
             }
             if (!ok && mma_pending) {
                 // drain: commit to a free barrier and wait (bounded) for the issued MMAs
@@ -303,10 +334,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------- epilogue
         const int quarter = warp & 3;
         const float ninf = -__int_as_float(0x7f800000);
-        int acc = 0;
-        uint32_t acc_phase = 0;
-        for (int64_t tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x) {
+        for (int seq = 0;; ++seq) {
+            const int tslot = seq & 1;
             bool ok = true;
+            int tile = -1;
+            if (lane == 0) {
+                ok = mbar_wait(smem_u32(&tqf[tslot]), ((uint32_t)seq >> 1) & 1u, abort_flag);
+                if (ok) {
+                    tile = tile_q[tslot];
+                    mbar_arrive(smem_u32(&tqe[tslot]));
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            tile = __shfl_sync(0xffffffffu, tile, 0);
+            if (!ok || tile < 0) break;
+            const int acc = seq & 1;
+            const uint32_t acc_phase = ((uint32_t)seq >> 1) & 1u;
             if (lane == 0) ok = mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag);
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
             if (!ok) break;
@@ -376,7 +419,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));
             }
             if (run_q >= 0) flush(run_q, run_max);
-            if (++acc == 2) acc = 0, acc_phase ^= 1;
         }
     }
 
@@ -485,7 +527,10 @@ msa_status launch_route_tc(const RouteTcArgs& a, cudaStream_t s) {
               | ((uint32_t)(BM >> 4) << 24);     // M / 16 ; A and B K-major (bits 15, 16 = 0)
     p.chunk_doc = a.chunk_doc; p.n_docs = a.n_docs; p.doc_scores = a.doc_scores; p.chunk_scores = a.chunk_scores;
     p.err = a.err;
+    p.tile_counter = a.tile_counter;
+    if (!p.tile_counter) return set_error(MSA_ERR_INVALID_ARG, "route (tensor cores): no tile counter");
     int64_t grid = p.n_tiles < (int64_t)sm_count() ? p.n_tiles : (int64_t)sm_count();
+    if (a.grid_cap > 0 && grid > a.grid_cap) grid = a.grid_cap;
     if (pl.resident) {
         auto kern = route_tc_kernel<true>;
         MSA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem));

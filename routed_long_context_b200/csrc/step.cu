@@ -1,13 +1,19 @@
 // One Memory Interleave round over all routed layers: append -> route -> top-k -> fetch -> attend.
 //
-// Stream schedule (compute = S0, copy = S1):
-//   S0: for every layer: rotate+append the new tokens' K/V, rotate their queries, route, top-k,
-//       copy the selected indices to pinned host memory, derive per-query memory lengths, record E_l.
-//   host: for every layer: wait for E_l (bounded poll), enqueue the layer's document fetches on S1,
-//       record G_l; S0 waits for G_l and runs the layer's attention.
-// Every layer's routing is enqueued before the host blocks on the first selection, so the host-link
-// fetches of layer l overlap the routing of layers l+1.. on the GPU.
+// Streams: R = the caller's compute stream (routers only), C = the caller's copy stream (fetches),
+// S = select (library-owned: top-k, index copy to the host, memory lengths),
+// A = attend (library-owned: query prepasses, appends, attention).
+//   A: every layer's router prepass (record P_l), then every layer's append + query rotation.
+//   R: for every layer: wait P_l, router kernel (optionally on fewer SMs than the GPU has), record R_l.
+//   S: for every layer: wait R_l, top-k, indices -> pinned host, memory lengths, record E_l.
+//   host: for every layer: wait E_l (bounded poll), enqueue the document fetches on C, record G_l;
+//         A waits G_l and runs the layer's attention.
+//   join: R waits for the last work of S and A.
+// The routers run back to back; selection, fetch and attention of layer l overlap the routing of
+// layers l+1.. (on SMs the routers leave free and in the copy engines).
+#include <algorithm>
 #include <chrono>
+#include <mutex>
 #include <thread>
 #include <vector>
 
@@ -38,8 +44,9 @@ __global__ void mem_len_kernel(const int32_t* __restrict__ idx, int n_q, int k, 
 }
 
 struct StepLayout {
-    size_t route_ws, scores, topk_ws, idx, mem_len, q_rot, mem_kv;   // per-layer sizes for the last four
-    size_t off_route, off_scores, off_topk, off_layers, per_layer, total;
+    size_t route_ws, scores, topk_ws, idx, mem_len, q_rot, mem_kv;   // all per layer except topk_ws
+    size_t off_topk, off_layers, per_layer, total;
+    size_t o_route, o_scores, o_idx, o_len, o_qrot, o_mem;           // offsets inside a layer's slot
 };
 
 msa_status layout(const msa_interleave_args* a, StepLayout* L) {
@@ -52,11 +59,16 @@ msa_status layout(const msa_interleave_args* a, StepLayout* L) {
     L->mem_len = align_up((size_t)a->n_q * sizeof(int32_t), 256);
     L->q_rot = align_up((size_t)a->n_q * a->T_new * a->hq * a->d * es, 256);
     L->mem_kv = align_up((size_t)a->n_q * a->max_mem * 2 * a->hkv * a->d * es, 256);
-    L->off_route = 0;
-    L->off_scores = align_up(L->route_ws, 256);
-    L->off_topk = L->off_scores + L->scores;
-    L->off_layers = L->off_topk + align_up(L->topk_ws, 256);
-    L->per_layer = L->idx + L->mem_len + L->q_rot + L->mem_kv;
+    L->route_ws = align_up(L->route_ws, 256);
+    L->off_topk = 0;
+    L->off_layers = align_up(L->topk_ws, 256);
+    L->o_route = 0;
+    L->o_scores = L->o_route + L->route_ws;
+    L->o_idx = L->o_scores + L->scores;
+    L->o_len = L->o_idx + L->idx;
+    L->o_qrot = L->o_len + L->mem_len;
+    L->o_mem = L->o_qrot + L->q_rot;
+    L->per_layer = L->o_mem + L->mem_kv;
     L->total = L->off_layers + L->per_layer * (size_t)a->n_layers;
     return MSA_OK;
 }
@@ -66,7 +78,7 @@ msa_status validate(const msa_interleave_args* a, bool need_ws) {
     MSA_REQUIRE(dtype_ok(a->dt), "msa_interleave_step: bad dtype");
     MSA_REQUIRE(a->n_layers > 0 && a->layers, "msa_interleave_step: no layers");
     MSA_REQUIRE(a->n_q > 0 && a->H > 0 && a->d > 0 && a->hq > 0 && a->hkv > 0 && a->k > 0 && a->T_new > 0 &&
-                    a->L_prev >= 0 && a->n_docs > 0 && a->n_chunks > 0 && a->max_mem > 0,
+                    a->L_prev >= 0 && a->n_docs > 0 && a->n_chunks > 0 && a->max_mem > 0 && a->reserved_sms >= 0,
                 "msa_interleave_step: bad sizes");
     MSA_REQUIRE(a->L_prev + a->T_new <= a->L_max, "msa_interleave_step: local cache overflow (%d + %d > %d)", a->L_prev,
                 a->T_new, a->L_max);
@@ -106,6 +118,23 @@ struct Events {
     }
 };
 
+// Library-owned auxiliary streams (select, attend), created once per device.
+constexpr int kMaxDev = 64;
+cudaStream_t g_aux[kMaxDev][2] = {{nullptr}};
+std::mutex g_aux_mu;
+
+msa_status aux_streams(cudaStream_t* sel, cudaStream_t* att) {
+    int dev = 0;
+    MSA_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDev) return set_error(MSA_ERR_UNSUPPORTED, "msa_interleave_step: device %d", dev);
+    std::lock_guard<std::mutex> lk(g_aux_mu);
+    for (int i = 0; i < 2; ++i)
+        if (!g_aux[dev][i]) MSA_CUDA_TRY(cudaStreamCreateWithFlags(&g_aux[dev][i], cudaStreamNonBlocking));
+    *sel = g_aux[dev][0];
+    *att = g_aux[dev][1];
+    return MSA_OK;
+}
+
 }  // namespace
 }  // namespace msa
 
@@ -132,65 +161,96 @@ msa_status msa_interleave_step(const msa_interleave_args* a, void* compute, void
     if (!rope_layout_ok(a->dt, a->d))
         return set_error(MSA_ERR_UNSUPPORTED, "msa_interleave_step: head_dim %d unsupported", a->d);
 
-    cudaStream_t s0 = static_cast<cudaStream_t>(compute);
-    cudaStream_t s1 = static_cast<cudaStream_t>(copy);
+    cudaStream_t sR = static_cast<cudaStream_t>(compute);
+    cudaStream_t sC = static_cast<cudaStream_t>(copy);
+    cudaStream_t sS = nullptr, sA = nullptr;
+    MSA_RETURN_IF(aux_streams(&sS, &sA));
     char* ws = static_cast<char*>(a->ws);
     const size_t es = dtype_size(a->dt);
     const int T_act = a->L_prev + a->T_new;
+    const int L = a->n_layers;
     int* err = device_error_word();
     const float2* cs = reinterpret_cast<const float2*>(a->rope_cos_sin);
+    RoutePlan plan;
+    MSA_RETURN_IF(route_plan(a->dt, a->n_chunks, a->n_q, T_act, a->H, a->d, &plan));
+    const int grid_cap = a->reserved_sms > 0 ? std::max(1, sm_count() - a->reserved_sms) : 0;
 
+    // events: fork, P_l, R_l, E_l, G_l, join x2
     Events evs;
-    evs.ev.resize(2 * (size_t)a->n_layers, nullptr);
+    evs.ev.resize(4 * (size_t)L + 3, nullptr);
     for (auto& e : evs.ev) MSA_CUDA_TRY(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+    cudaEvent_t ev_fork = evs.ev[4 * L], ev_join_s = evs.ev[4 * L + 1], ev_join_a = evs.ev[4 * L + 2];
+    auto P = [&](int l) { return evs.ev[l]; };
+    auto R = [&](int l) { return evs.ev[L + l]; };
+    auto E = [&](int l) { return evs.ev[2 * L + l]; };
+    auto G = [&](int l) { return evs.ev[3 * L + l]; };
+    auto slot = [&](int l, size_t off) { return ws + Lo.off_layers + Lo.per_layer * (size_t)l + off; };
 
-    auto layer_ws = [&](int l, size_t part) { return ws + Lo.off_layers + Lo.per_layer * (size_t)l + part; };
-    const size_t o_idx = 0, o_len = Lo.idx, o_qrot = Lo.idx + Lo.mem_len, o_mem = o_qrot + Lo.q_rot;
+    MSA_CUDA_TRY(cudaEventRecord(ev_fork, sR));
+    MSA_CUDA_TRY(cudaStreamWaitEvent(sS, ev_fork, 0));
+    MSA_CUDA_TRY(cudaStreamWaitEvent(sA, ev_fork, 0));
 
-    // ---- phase 1: append, rotate, route and select for every layer (all on S0)
-    for (int l = 0; l < a->n_layers; ++l) {
+    // ---- A: router prepasses of every layer, then appends and query rotations
+    for (int l = 0; l < L; ++l) {
+        MSA_RETURN_IF(route_prepare(plan, a->layers[l].qr, slot(l, Lo.o_route),
+                                    reinterpret_cast<float*>(slot(l, Lo.o_scores)), a->n_docs, nullptr, a->n_chunks, sA));
+        MSA_CUDA_TRY(cudaEventRecord(P(l), sA));
+    }
+    for (int l = 0; l < L; ++l) {
         const msa_layer_args& y = a->layers[l];
         RopeRowsArgs r{};
         r.heads = a->hkv; r.d = a->d; r.n_rows = (int64_t)a->n_q * a->T_new; r.uniform_len = a->T_new;
         r.in = y.k_new; r.out = y.local_k; r.in_stride = a->new_q_stride; r.out_stride = a->L_max; r.out_off = a->L_prev;
         r.pos_offset = (int64_t)a->k + a->L_prev; r.cs = cs; r.max_pos = a->rope_max_pos; r.err = err;
-        MSA_RETURN_IF(launch_rope_rows(r, a->dt, s0));
+        MSA_RETURN_IF(launch_rope_rows(r, a->dt, sA));
         const size_t vrow = (size_t)a->hkv * a->d * es;
         MSA_CUDA_TRY(cudaMemcpy2DAsync(static_cast<char*>(y.local_v) + (size_t)a->L_prev * vrow, (size_t)a->L_max * vrow,
                                        y.v_new, (size_t)a->new_q_stride * vrow, (size_t)a->T_new * vrow, a->n_q,
-                                       cudaMemcpyDeviceToDevice, s0));
+                                       cudaMemcpyDeviceToDevice, sA));
         RopeRowsArgs rq = r;
-        rq.heads = a->hq; rq.in = y.q_new; rq.out = layer_ws(l, o_qrot); rq.out_stride = a->T_new; rq.out_off = 0;
-        MSA_RETURN_IF(launch_rope_rows(rq, a->dt, s0));
-
-        float* scores = reinterpret_cast<float*>(ws + Lo.off_scores);
-        MSA_RETURN_IF(msa_route_scores(y.kr_index, a->dt, a->n_chunks, a->chunk_doc, a->n_docs, y.qr, a->n_q, T_act, a->H,
-                                       a->d, scores, nullptr, ws + Lo.off_route, Lo.route_ws, s0));
-        int32_t* idx = reinterpret_cast<int32_t*>(layer_ws(l, o_idx));
-        MSA_RETURN_IF(msa_topk_docs(scores, a->n_q, a->n_docs, a->k, idx, nullptr, ws + Lo.off_topk, Lo.topk_ws, s0));
-        MSA_CUDA_TRY(cudaMemcpyAsync(y.topk_idx_host, idx, (size_t)a->n_q * a->k * sizeof(int32_t),
-                                     cudaMemcpyDeviceToHost, s0));
-        mem_len_kernel<<<(a->n_q + 127) / 128, 128, 0, s0>>>(idx, a->n_q, a->k, a->doc_chunk_off, a->n_docs, a->max_mem,
-                                                            reinterpret_cast<int32_t*>(layer_ws(l, o_len)), err);
-        MSA_LAUNCH_CHECK();
-        MSA_CUDA_TRY(cudaEventRecord(evs.ev[2 * l], s0));
+        rq.heads = a->hq; rq.in = y.q_new; rq.out = slot(l, Lo.o_qrot); rq.out_stride = a->T_new; rq.out_off = 0;
+        MSA_RETURN_IF(launch_rope_rows(rq, a->dt, sA));
     }
 
-    // ---- phase 2: per layer, wait for its selection, fetch on S1, attend on S0
+    // ---- R: routers back to back; S: selection as each router finishes
+    for (int l = 0; l < L; ++l) {
+        const msa_layer_args& y = a->layers[l];
+        float* scores = reinterpret_cast<float*>(slot(l, Lo.o_scores));
+        MSA_CUDA_TRY(cudaStreamWaitEvent(sR, P(l), 0));
+        MSA_RETURN_IF(route_launch(plan, y.kr_index, a->n_chunks, a->chunk_doc, a->n_docs, slot(l, Lo.o_route), scores,
+                                   nullptr, grid_cap, sR));
+        MSA_CUDA_TRY(cudaEventRecord(R(l), sR));
+
+        MSA_CUDA_TRY(cudaStreamWaitEvent(sS, R(l), 0));
+        int32_t* idx = reinterpret_cast<int32_t*>(slot(l, Lo.o_idx));
+        MSA_RETURN_IF(msa_topk_docs(scores, a->n_q, a->n_docs, a->k, idx, nullptr, ws + Lo.off_topk, Lo.topk_ws, sS));
+        MSA_CUDA_TRY(cudaMemcpyAsync(y.topk_idx_host, idx, (size_t)a->n_q * a->k * sizeof(int32_t),
+                                     cudaMemcpyDeviceToHost, sS));
+        mem_len_kernel<<<(a->n_q + 127) / 128, 128, 0, sS>>>(idx, a->n_q, a->k, a->doc_chunk_off, a->n_docs, a->max_mem,
+                                                            reinterpret_cast<int32_t*>(slot(l, Lo.o_len)), err);
+        MSA_LAUNCH_CHECK();
+        MSA_CUDA_TRY(cudaEventRecord(E(l), sS));
+    }
+
+    // ---- host: per layer, wait for its selection, fetch on C, attend on A
     const auto deadline = std::chrono::steady_clock::now() + std::chrono::microseconds(host_wait_timeout_us);
     std::vector<int32_t> mem_len_host((size_t)a->n_q);
-    for (int l = 0; l < a->n_layers; ++l) {
+    for (int l = 0; l < L; ++l) {
         const msa_layer_args& y = a->layers[l];
-        MSA_RETURN_IF(wait_event(evs.ev[2 * l], deadline));
+        MSA_RETURN_IF(wait_event(E(l), deadline));
         MSA_RETURN_IF(msa_gather_kv(y.host_bank, a->dt, a->n_chunks, a->doc_chunk_off_host, a->n_docs, y.topk_idx_host,
-                                    a->n_q, a->k, a->hkv, a->d, a->max_mem, layer_ws(l, o_mem), mem_len_host.data(), s1));
-        MSA_CUDA_TRY(cudaEventRecord(evs.ev[2 * l + 1], s1));
-        MSA_CUDA_TRY(cudaStreamWaitEvent(s0, evs.ev[2 * l + 1], 0));
-        MSA_RETURN_IF(msa_sparse_attn(layer_ws(l, o_qrot), layer_ws(l, o_mem),
-                                      reinterpret_cast<const int32_t*>(layer_ws(l, o_len)), a->max_mem, y.local_k,
+                                    a->n_q, a->k, a->hkv, a->d, a->max_mem, slot(l, Lo.o_mem), mem_len_host.data(), sC));
+        MSA_CUDA_TRY(cudaEventRecord(G(l), sC));
+        MSA_CUDA_TRY(cudaStreamWaitEvent(sA, G(l), 0));
+        MSA_RETURN_IF(msa_sparse_attn(slot(l, Lo.o_qrot), slot(l, Lo.o_mem),
+                                      reinterpret_cast<const int32_t*>(slot(l, Lo.o_len)), a->max_mem, y.local_k,
                                       y.local_v, a->L_max, T_act, a->L_prev, a->n_q, a->T_new, a->hq, a->hkv, a->d,
-                                      a->scale, y.out, a->dt, s0));
+                                      a->scale, y.out, a->dt, sA));
     }
+    MSA_CUDA_TRY(cudaEventRecord(ev_join_s, sS));
+    MSA_CUDA_TRY(cudaEventRecord(ev_join_a, sA));
+    MSA_CUDA_TRY(cudaStreamWaitEvent(sR, ev_join_s, 0));
+    MSA_CUDA_TRY(cudaStreamWaitEvent(sR, ev_join_a, 0));
     return MSA_OK;
 }
 

@@ -24,16 +24,20 @@ def _np(t):
 
 
 def assert_topk_matches(gpu_idx, ref_scores_row, k, tol=2e-3):
-    """Exact match of the selected indices, excused only where the oracle's k-th and (k+1)-th scores
-    lie within tol; then every GPU pick must still score within tol of the oracle's k-th score."""
+    """The selected set equals the oracle's, excused only where the oracle's k-th and (k+1)-th scores
+    lie within tol (then every GPU pick must score within tol of the oracle's k-th score). The order
+    inside the set is unique only up to score differences the precision resolves: along the GPU's
+    ranking the oracle scores may never rise by more than 2 * tol."""
     ref_idx, ref_val = O.topk_docs(ref_scores_row[None], min(k + 1, len(ref_scores_row)))
     ref_idx, ref_val = ref_idx[0], ref_val[0]
     gpu_idx = np.asarray(gpu_idx)
-    if np.array_equal(gpu_idx, ref_idx[:k]):
-        return
-    assert len(ref_val) > k and ref_val[k - 1] - ref_val[k] <= tol, (gpu_idx, ref_idx[:k], ref_val[:k + 1])
     assert len(set(gpu_idx.tolist())) == k
-    assert np.all(ref_scores_row[gpu_idx] >= ref_val[k - 1] - tol)
+    if set(gpu_idx.tolist()) != set(ref_idx[:k].tolist()):
+        assert len(ref_val) > k and ref_val[k - 1] - ref_val[k] <= tol, (gpu_idx, ref_idx[:k], ref_val[:k + 1])
+        assert np.all(ref_scores_row[gpu_idx] >= ref_val[k - 1] - tol)
+    s = ref_scores_row[gpu_idx]
+    for i in range(k - 1):
+        assert s[i] >= s[i + 1:].max() - 2 * tol, (i, s)
 
 
 def _row_rel_err(got, ref):
@@ -99,11 +103,224 @@ def test_tiny_end_to_end(m):
     ds = m.msa_route_scores(index, lay.chunk_doc, lay.n_docs, dv["qr"])
     ref_ds, _ = O.route(krb, w.doc_chunk_off, w.qr(0))
     assert np.abs(_np(ds) - ref_ds).max() <= 1e-5
-    # selection and attention output of the round
-    idx, val, o = O.route_and_attend(krb, w.doc_chunk_off, np.stack([kb, vb], 1), w.qr(0)[0], w.q(0)[0],
-                                     w.k_new(0)[0], w.v_new(0)[0], 0, w.k, w.rope_base)
+    # selection, then the oracle's attention over the documents the GPU selected
     got_idx = idx_host[0][0].numpy()[0]
     assert_topk_matches(got_idx, ref_ds[0], w.k)
     assert set(got_idx[:2].tolist()) == {17, 42}
-    if np.array_equal(got_idx, idx):
-        assert _row_rel_err(_np(outs[0][0])[0], o) <= 1e-5
+    mem = O.gather_memory(np.stack([kb, vb], 1), w.doc_chunk_off, got_idx)
+    kl = O.apply_rope(w.k_new(0)[0], O.global_positions(w.k, 0, w.T0), w.rope_base)
+    qq = O.apply_rope(w.q(0)[0], O.global_positions(w.k, 0, w.T0), w.rope_base)
+    o = O.sparse_attention(qq, mem[:, 0], mem[:, 1], kl, w.v_new(0)[0], 0, 1 / np.sqrt(w.d))
+    assert _row_rel_err(_np(outs[0][0])[0], o) <= 1e-5
+
+
+# ------------------------------------------------------------------------------------------ helpers
+def oracle_encode_docs(w, layer, docs, names=("k", "v", "kr")):
+    """Oracle-pooled chunks of the given documents: {name: {doc: [n_chunks, heads, d]}} (K rotated
+    with document-wise positions)."""
+    out = {n: {} for n in names}
+    for doc in docs:
+        a, b = int(w.doc_tok_off[doc]), int(w.doc_tok_off[doc + 1])
+        rows = np.arange(a, b)
+        off = np.array([0, b - a])
+        t = {n: w.host_rows(layer, n, rows).reshape(b - a, -1, w.d) for n in names}
+        kb, vb, krb = O.encode_memory(t.get("k"), t.get("v"), t.get("kr"), off, w.chunk, w.rope_base)
+        for n, val in (("k", kb), ("v", vb), ("kr", krb)):
+            if n in names:
+                out[n][int(doc)] = val
+    return out
+
+
+def oracle_router_index(w, layer, group=64):
+    """Oracle K-bar^R of every chunk of a token-level workload, pooled group by group."""
+    parts = []
+    for d0 in range(0, w.n_docs, group):
+        d1 = min(w.n_docs, d0 + group)
+        a, b = int(w.doc_tok_off[d0]), int(w.doc_tok_off[d1])
+        x = w.host_rows(layer, "kr", np.arange(a, b)).reshape(b - a, w.H, w.d)
+        _, _, krb = O.encode_memory(None, None, x, w.doc_tok_off[d0:d1 + 1] - a, w.chunk, w.rope_base)
+        parts.append(krb)
+    return np.concatenate(parts)
+
+
+def oracle_route_prepooled(w, layer, qr, slice_docs=8192):
+    """Oracle doc scores of a pre-pooled workload over every chunk, generated slice by slice."""
+    out = []
+    for d0 in range(0, w.n_docs, slice_docs):
+        d1 = min(w.n_docs, d0 + slice_docs)
+        a, b = int(w.doc_chunk_off[d0]), int(w.doc_chunk_off[d1])
+        rows = w.host_rows(layer, "krbar", np.arange(a, b)).reshape(b - a, w.H, w.d)
+        ds, _ = O.route(rows, w.doc_chunk_off[d0:d1 + 1] - a, qr)
+        out.append(ds)
+    return np.concatenate(out, axis=1)
+
+
+def _free():
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+# ------------------------------------------------------------------------------------------ 1M
+def test_1m_end_to_end(m):
+    from routed_long_context_b200.bank import BankLayout, encode_tokens, to_host_bank
+
+    w = workloads.mem_1m()
+    lay = BankLayout.from_doc_lengths(w.doc_len, w.chunk)
+    cs = m.rope_table(4096, w.d, w.rope_base)
+    k, v, kr = (memory_tensor(w, 0, n) for n in ("k", "v", "kr"))
+    kvbar, index = encode_tokens(lay, k, v, kr, w.chunk, cs)
+    del k, v, kr
+    bank = to_host_bank(kvbar)
+    dv = small_tensors(w, 0)
+    local, outs, idx_host = alloc_round_buffers(w, 1)
+    run_round(m, w, lay, [dv], 0, cs, [index], [bank], local, outs, idx_host)
+    ds_gpu = _np(m.msa_route_scores(index, lay.chunk_doc, lay.n_docs, dv["qr"]))
+    assert m.device_status() == 0
+
+    krb = oracle_router_index(w, 0)
+    ref_ds, _ = O.route(krb, w.doc_chunk_off, w.qr(0))
+    assert np.abs(ds_gpu - ref_ds).max() <= 2e-3
+    np.testing.assert_allclose(_np(index), O.unit(krb).reshape(_np(index).shape), atol=2.0 ** -8)
+    gi = idx_host[0][0].numpy()[0]
+    assert_topk_matches(gi, ref_ds[0], w.k)
+    assert set(w.expected(0, 0, 0)) <= set(gi.tolist())
+    # pooled K-bar / V-bar of the selected documents, then attention over them
+    enc = oracle_encode_docs(w, 0, gi, ("k", "v"))
+    kb = np.concatenate([enc["k"][int(d)] for d in gi])
+    vb = np.concatenate([enc["v"][int(d)] for d in gi])
+    for d in gi:
+        a, b = int(w.doc_chunk_off[d]), int(w.doc_chunk_off[d + 1])
+        np.testing.assert_allclose(_np(kvbar[a:b, 0]), enc["k"][int(d)], atol=1e-5, rtol=2.0 ** -8)
+        np.testing.assert_allclose(_np(kvbar[a:b, 1]), enc["v"][int(d)], atol=1e-5, rtol=2.0 ** -8)
+    kl = O.apply_rope(w.k_new(0)[0], O.global_positions(w.k, 0, w.T0), w.rope_base)
+    qq = O.apply_rope(w.q(0)[0], O.global_positions(w.k, 0, w.T0), w.rope_base)
+    o = O.sparse_attention(qq, kb, vb, kl, w.v_new(0)[0], 0, 1 / np.sqrt(w.d))
+    assert _row_rel_err(_np(outs[0][0])[0], o) <= 2e-2
+    _free()
+
+
+# ------------------------------------------------------------------------------------------ 10M
+def test_10m_encode_and_decode_routing(m):
+    from routed_long_context_b200.bank import BankLayout, encode_tokens, to_host_bank
+
+    w = workloads.mem_10m()
+    lay = BankLayout.from_doc_lengths(w.doc_len, w.chunk)
+    cs = m.rope_table(4096, w.d, w.rope_base)
+    k, v, kr = (memory_tensor(w, 0, n) for n in ("k", "v", "kr"))
+    kvbar, index = encode_tokens(lay, k, v, kr, w.chunk, cs)
+    del k, v, kr
+    _free()
+    bank = to_host_bank(kvbar)
+    dv = small_tensors(w, 0)
+    local, outs, idx_host = alloc_round_buffers(w, 1)
+    run_round(m, w, lay, [dv], 0, cs, [index], [bank], local, outs, idx_host)
+    ds_gpu = _np(m.msa_route_scores(index, lay.chunk_doc, lay.n_docs, dv["qr"]))
+    assert m.device_status() == 0
+    gi = idx_host[0][0].numpy()                                    # [32, 16]
+
+    # documents checked one by one by the oracle: planted, selected, and a seeded random sample
+    rs = np.random.default_rng(10)
+    sample = rs.choice(w.n_docs, 400, replace=False)
+    planted = sorted({d for q in range(w.n_q) for d in w.expected(0, 0, q)})
+    docs = sorted(set(sample.tolist()) | set(gi.ravel().tolist()) | set(planted))
+    enc = oracle_encode_docs(w, 0, docs)
+    for d in docs[::7]:                                           # pooled bank and index rows
+        a, b = int(w.doc_chunk_off[d]), int(w.doc_chunk_off[d + 1])
+        np.testing.assert_allclose(_np(kvbar[a:b, 0]), enc["k"][d], atol=1e-5, rtol=2.0 ** -8)
+        np.testing.assert_allclose(_np(kvbar[a:b, 1]), enc["v"][d], atol=1e-5, rtol=2.0 ** -8)
+        np.testing.assert_allclose(_np(index[a:b]), O.unit(enc["kr"][d]), atol=1e-5, rtol=2.0 ** -8)
+    qr = w.qr(0)
+    for q in range(w.n_q):
+        ref = {d: O.chunk_scores_one_query(enc["kr"][d], qr[q]).max() for d in docs}
+        for d in docs:
+            assert abs(ds_gpu[q, d] - ref[d]) <= 2e-3, (q, d, ds_gpu[q, d], ref[d])
+        sel = set(gi[q].tolist())
+        assert set(w.expected(0, 0, q)) <= sel
+        kth = min(ref[d] for d in sel)
+        assert all(ref[d] <= kth + 2e-3 for d in docs if d not in sel)      # nothing better was left out
+        # attention of the decode token over its selected memory and itself
+        kb = np.concatenate([enc["k"][int(d)] for d in gi[q]])
+        vb = np.concatenate([enc["v"][int(d)] for d in gi[q]])
+        kl = O.apply_rope(w.k_new(0)[q], O.global_positions(w.k, 0, 1), w.rope_base)
+        qq = O.apply_rope(w.q(0)[q], O.global_positions(w.k, 0, 1), w.rope_base)
+        o = O.sparse_attention(qq, kb, vb, kl, w.v_new(0)[q], 0, 1 / np.sqrt(w.d))
+        assert _row_rel_err(_np(outs[0][0])[q], o) <= 2e-2
+    del kvbar, index
+    _free()
+
+
+# ------------------------------------------------------------------------------------------ pre-pooled
+def build_prepooled(m, w, n_layers):
+    from routed_long_context_b200.bank import BankLayout, index_from_prepooled
+
+    lay = BankLayout(w.doc_chunks)
+    index = [index_from_prepooled(lay, memory_tensor(w, l, "krbar")) for l in range(n_layers)]
+    banks = []
+    for s in range(min(w.n_host_banks, n_layers)):
+        dev = memory_tensor(w, s, "bank")
+        host = torch.empty(dev.shape, dtype=dev.dtype, pin_memory=True)
+        host.copy_(dev)
+        banks.append(host)
+        del dev
+    torch.cuda.synchronize()
+    return lay, index, banks
+
+
+def oracle_bank_rows(w, layer, docs):
+    rows = np.concatenate([np.arange(w.doc_chunk_off[d], w.doc_chunk_off[d + 1]) for d in docs])
+    return w.host_rows(layer, "bank", rows).reshape(len(rows), 2, w.hkv, w.d)
+
+
+def test_100m_two_layers_full_routing(m):
+    w = workloads.mem_100m(layers=2, n_host_banks=2)
+    lay, index, banks = build_prepooled(m, w, 2)
+    cs = m.rope_table(4096, w.d, w.rope_base)
+    dvs = [small_tensors(w, l) for l in range(2)]
+    local, outs, idx_host = alloc_round_buffers(w, 2)
+    run_round(m, w, lay, dvs, 0, cs, index, banks, local, outs, idx_host)
+    assert m.device_status() == 0
+    for l in range(2):
+        ds_gpu = _np(m.msa_route_scores(index[l], lay.chunk_doc, lay.n_docs, dvs[l]["qr"]))
+        ref = oracle_route_prepooled(w, l, w.qr(l))
+        assert np.abs(ds_gpu - ref).max() <= 2e-3
+        gi = idx_host[l][0].numpy()[0]
+        assert_topk_matches(gi, ref[0], w.k)
+        assert set(w.expected(l, 0, 0)) <= set(gi.tolist())
+        mem = oracle_bank_rows(w, l, gi)
+        kl = O.apply_rope(w.k_new(l)[0], O.global_positions(w.k, 0, w.T0), w.rope_base)
+        qq = O.apply_rope(w.q(l)[0], O.global_positions(w.k, 0, w.T0), w.rope_base)
+        o = O.sparse_attention(qq, mem[:, 0], mem[:, 1], kl, w.v_new(l)[0], 0, 1 / np.sqrt(w.d))
+        assert _row_rel_err(_np(outs[l][0])[0], o) <= 2e-2
+    del index
+    _free()
+
+
+def test_interleave_three_rounds(m):
+    """Two routed layers through three rounds, checked in full; the chain documents are selected
+    in the round they are planted for."""
+    w = workloads.interleave(layers=2, n_host_banks=2)
+    lay, index, banks = build_prepooled(m, w, 2)
+    cs = m.rope_table(4096, w.d, w.rope_base)
+    dvs = [small_tensors(w, l) for l in range(2)]
+    local, outs, idx_host = alloc_round_buffers(w, 2)
+    for r in range(w.rounds):
+        run_round(m, w, lay, dvs, r, cs, index, banks, local, outs, idx_host)
+    assert m.device_status() == 0
+    for l in range(2):
+        krbar = w.host_tensor(l, "krbar")
+        for r in range(w.rounds):
+            L_prev, tn = w.round_tokens(r)
+            ref_ds, _ = O.route(krbar, w.doc_chunk_off, w.qr(l)[:, :L_prev + tn])
+            gi_all = idx_host[l][r].numpy()
+            for q in range(w.n_q):
+                gi = gi_all[q]
+                assert_topk_matches(gi, ref_ds[q], w.k)
+                assert set(w.expected(l, r, q)) <= set(gi.tolist()), (l, r, q)
+                mem = oracle_bank_rows(w, l, gi)
+                L = L_prev + tn
+                kl = O.apply_rope(w.k_new(l)[q, :L], O.global_positions(w.k, 0, L), w.rope_base)
+                qq = O.apply_rope(w.q(l)[q, L_prev:L], O.global_positions(w.k, L_prev, tn), w.rope_base)
+                o = O.sparse_attention(qq, mem[:, 0], mem[:, 1], kl, w.v_new(l)[q, :L], L_prev, 1 / np.sqrt(w.d))
+                assert _row_rel_err(_np(outs[l][r])[q], o) <= 2e-2, (l, r, q)
+    del index
+    _free()
