@@ -36,7 +36,11 @@ def parse():
     ap.add_argument("--layers", type=int, default=18)
     ap.add_argument("--host-banks", type=int, default=2)
     ap.add_argument("--n-docs", type=int, default=97657, help="shorter bank for small profiling cases only")
-    ap.add_argument("--reserved-sms", type=int, default=8,
+    ap.add_argument("--fetch-mode", type=int, default=1, choices=[0, 1],
+                    help="0: host-issued cudaMemcpyAsync per selected document; 1: device-side fetch kernel")
+    ap.add_argument("--router-stages", type=int, default=0,
+                    help="cap on the router's pipeline stages (0 = default shared-memory budget)")
+    ap.add_argument("--reserved-sms", type=int, default=0,
                     help="SMs the routers leave free for the overlapped selection and attention")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -230,6 +234,7 @@ def main():
     from routed_long_context_b200.bank import BankLayout, index_from_prepooled
 
     torch.cuda.set_device(local_rank)
+    m.api.route_set_max_stages(args.router_stages)
     if world > 1:
         from datetime import timedelta
 
@@ -272,7 +277,8 @@ def main():
     rnd = m.InterleaveRound(layer_args, n_chunks=lay.n_chunks, n_docs=lay.n_docs, doc_chunk_off=lay.doc_chunk_off,
                             doc_chunk_off_host=lay.doc_chunk_off_host, chunk_doc=lay.chunk_doc, n_q=1, H=w.H, d=w.d,
                             hq=w.hq, hkv=w.hkv, k=w.k, L_prev=0, T_new=w.T0, new_q_stride=w.T0, L_max=w.T0,
-                            max_mem=w.max_mem, cos_sin=cs, dtype=dt, reserved_sms=args.reserved_sms)
+                            max_mem=w.max_mem, cos_sin=cs, dtype=dt, reserved_sms=args.reserved_sms,
+                            fetch_mode=args.fetch_mode)
 
     # ---- warm-up, then K timed steps (inputs are 1.6 GB per layer: larger than L2, no flush needed)
     for _ in range(args.warmup):
@@ -366,6 +372,8 @@ def main():
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
             "route_ms_per_layer": route_ms,
             "reserved_sms": args.reserved_sms,
+            "router_stages": args.router_stages or "default",
+            "fetch_mode": ["host cudaMemcpyAsync per document", "device fetch kernel"][args.fetch_mode],
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": None,
                          "kernel": "route_tc_kernel (+ its query-normalisation prepass)",
@@ -373,7 +381,9 @@ def main():
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms},
-            "gpu_launches": 7 * w.layers * args.steps,
+            # per layer: prepass, router, top-k, fetch kernel (mode 1) or memory lengths (mode 0),
+            # attention; per step: one fused append for every layer
+            "gpu_launches": (5 * w.layers + (w.layers + 23) // 24) * args.steps,
             "clocks": clk.summary(),
             "checks": {"planted_docs_selected": planted_ok, "device_status": status},
         }))

@@ -142,8 +142,14 @@ msa_status msa_route_scores(const void* kr_index, msa_dtype dt, int64_t n_chunks
 msa_status msa_route_workspace_size(int n_q, int T, int H, int d, msa_dtype dt, size_t* bytes);
 
 /* Selects the router kernel for testing: 0 = automatic, 1 = CUDA-core kernel, 2 = tensor-core
- * kernel (bf16 only). Process-wide. */
+ * kernel (bf16 only; the normalised queries stream from L2 with every index tile), 3 = tensor-core
+ * kernel with the normalised queries held in shared memory when they fit. Process-wide. */
 msa_status msa_route_set_impl(int impl);
+
+/* Tuning knob of the tensor-core router: at most n pipeline stages of index tiles (1 <= n <= 12;
+ * 0 = default, as many as fit in a shared-memory budget that leaves each SM room for one
+ * attention block and one top-k block running concurrently). Process-wide. */
+msa_status msa_route_set_max_stages(int n);
 
 /* Top-k document selection ([P1] §组件 1; [P2] Top-k 选择机制): for every query the k documents
  * with the largest doc_scores, in descending score order, ties broken by the lower document
@@ -187,6 +193,18 @@ msa_status msa_gather_kv(const void* host_bank, msa_dtype dt, int64_t n_chunks, 
                          int64_t n_docs, const int32_t* idx_host, int n_q, int k, int hkv, int d, int max_mem,
                          void* dev_mem_kv, int32_t* mem_len_host, void* copy_stream);
 
+/* Device-side variant of msa_gather_kv: a kernel on `stream` reads the selected documents' rows
+ * straight from the pinned host bank (mapped into the device address space; the pointer must come
+ * from cudaHostAlloc / torch pin_memory) with device-resident indices, so no host round trip sits
+ * between selection and fetch. Same layout and rank order as msa_gather_kv.
+ *   doc_chunk_off: device int64 [n_docs+1]; idx: device int32 [n_q][k]; mem_len: device int32 [n_q].
+ * Indices out of range or more rows than max_mem record MSA_DEV_BAD_INDEX and skip that query's
+ * copy (no out-of-range access). Returns MSA_ERR_INVALID_ARG if host_bank is not pinned, mapped
+ * host memory. */
+msa_status msa_gather_kv_device(const void* host_bank, msa_dtype dt, int64_t n_chunks, const int64_t* doc_chunk_off,
+                                int64_t n_docs, const int32_t* idx, int n_q, int k, int hkv, int d, int max_mem,
+                                void* dev_mem_kv, int32_t* mem_len, void* stream);
+
 /* Sparse attention ([P1] §组件 1 稀疏注意力机制; [P2] concatenation of the selected compressed
  * K/V with the query's local K/V): for query q, token t, head h (kv head g = h / (hq/hkv)):
  *   out = softmax(scale * q . [mem K-bar ; local K_j, j <= q_start + t, j < L]) [mem V-bar ; local V]
@@ -195,10 +213,15 @@ msa_status msa_gather_kv(const void* host_bank, msa_dtype dt, int64_t n_chunks, 
  *   local_k, local_v: device [n_q][L_max][hkv][d], rotated keys of the active context;
  *   out: device [n_q][T][hq][d]. All of dtype dt; arithmetic and softmax in fp32.
  * Memory rows are all visible; local keys are causal. A row with no visible key is 0.
+ * bf16 runs on tensor cores (mma.sync, fp32 accumulation), fp32 on CUDA cores.
  * Requires d == 128 and hq/hkv in {1, 2, 4, 8}. */
 msa_status msa_sparse_attn(const void* q, const void* mem_kv, const int32_t* mem_len, int max_mem,
                            const void* local_k, const void* local_v, int L_max, int L, int q_start, int n_q, int T,
                            int hq, int hkv, int d, float scale, void* out, msa_dtype dt, void* stream);
+
+/* Selects the bf16 attention kernel for testing: 0 = tensor cores (mma.sync m16n8k16, default),
+ * 1 = CUDA cores. fp32 always runs on CUDA cores. Process-wide. */
+msa_status msa_attn_set_impl(int impl);
 
 /* One routed layer of one Memory Interleave round (see msa_interleave_step). */
 typedef struct msa_layer_args {
@@ -234,6 +257,10 @@ typedef struct msa_interleave_args {
     float scale;                    /* attention scale, normally 1/sqrt(d) */
     int reserved_sms;               /* SMs the router kernels leave free for the overlapped selection
                                        and attention of earlier layers (0 = routers use every SM) */
+    int fetch_mode;                 /* 0: the host waits for each layer's selection and issues one
+                                       cudaMemcpyAsync per document on `copy` (msa_gather_kv);
+                                       1: a device kernel fetches from the mapped pinned bank right
+                                       after selection (msa_gather_kv_device), no host waits */
     void* ws;                       /* device workspace of msa_interleave_workspace_size bytes */
     size_t ws_bytes;
 } msa_interleave_args;
@@ -247,8 +274,9 @@ typedef struct msa_interleave_args {
  * `copy` and attend. The router kernels run back to back on `compute`; selection and attention
  * run on two library-owned streams (created once per device) that fork from and join back into
  * `compute`, so a layer's selection, fetch and attention overlap the routing of later layers.
- * The host waits for each layer's selection (polling with a deadline of host_wait_timeout_us,
- * giving MSA_ERR_TIMEOUT) before enqueueing its fetch. When the call returns, everything is
+ * With fetch_mode 0 the host waits for each layer's selection (polling with a deadline of
+ * host_wait_timeout_us, giving MSA_ERR_TIMEOUT) before enqueueing its copies; with fetch_mode 1
+ * the fetch is a device kernel and the call never waits. When the call returns, everything is
  * enqueued and `compute` is ordered after all of it. */
 msa_status msa_interleave_step(const msa_interleave_args* a, void* compute, void* copy, int64_t host_wait_timeout_us);
 msa_status msa_interleave_workspace_size(const msa_interleave_args* a, size_t* bytes);

@@ -29,7 +29,7 @@ class InterleaveArgs(ctypes.Structure):
                 ("hq", ctypes.c_int), ("hkv", ctypes.c_int), ("k", ctypes.c_int), ("L_prev", ctypes.c_int),
                 ("T_new", ctypes.c_int), ("new_q_stride", ctypes.c_int), ("L_max", ctypes.c_int),
                 ("max_mem", ctypes.c_int), ("rope_cos_sin", vp), ("rope_max_pos", i64), ("scale", f32),
-                ("reserved_sms", ctypes.c_int), ("ws", vp), ("ws_bytes", sz)]
+                ("reserved_sms", ctypes.c_int), ("fetch_mode", ctypes.c_int), ("ws", vp), ("ws_bytes", sz)]
 
 
 # name -> (restype, argtypes)
@@ -47,14 +47,18 @@ SIGNATURES = {
     "msa_route_workspace_size": (i32, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, i32,
                                        ctypes.POINTER(sz)]),
     "msa_route_set_impl": (i32, [ctypes.c_int]),
+    "msa_route_set_max_stages": (i32, [ctypes.c_int]),
     "msa_topk_docs": (i32, [vp, ctypes.c_int, i64, ctypes.c_int, vp, vp, vp, sz, vp]),
     "msa_topk_workspace_size": (i32, [ctypes.c_int, i64, ctypes.c_int, ctypes.POINTER(sz)]),
     "msa_topk_docs_noalloc": (i32, [vp, ctypes.c_int, i64, ctypes.c_int, vp, vp, vp]),
     "msa_topk_noalloc_max_scratch": (sz, []),
     "msa_gather_kv": (i32, [vp, i32, i64, vp, i64, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                             ctypes.c_int, vp, vp, vp]),
+    "msa_gather_kv_device": (i32, [vp, i32, i64, vp, i64, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                   ctypes.c_int, vp, vp, vp]),
     "msa_sparse_attn": (i32, [vp, vp, vp, ctypes.c_int, vp, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                               ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, f32, vp, i32, vp]),
+    "msa_attn_set_impl": (i32, [ctypes.c_int]),
     "msa_interleave_step": (i32, [ctypes.POINTER(InterleaveArgs), vp, vp, i64]),
     "msa_interleave_workspace_size": (i32, [ctypes.POINTER(InterleaveArgs), ctypes.POINTER(sz)]),
 }
@@ -62,7 +66,7 @@ SIGNATURES = {
 
 def load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"libmsa.so not found at {LIB_PATH}; build it with `python -m routed_long_context_b200.build`")
+        raise ImportError(f"libmsa.so not found at {LIB_PATH}; build it with `python routed_long_context_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     for name, (res, args) in SIGNATURES.items():
         fn = getattr(lib, name)

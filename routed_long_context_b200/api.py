@@ -101,8 +101,18 @@ def route_workspace_size(n_q: int, T: int, H: int, d: int, dtype) -> int:
     return n.value
 
 
+def attn_set_impl(impl: int) -> None:
+    """bf16 attention: 0 = tensor cores (default), 1 = CUDA cores."""
+    check(lib.msa_attn_set_impl(impl), "msa_attn_set_impl")
+
+
+def route_set_max_stages(n: int) -> None:
+    """Tuning knob: cap on the router's pipeline stages (0 = default budget)."""
+    check(lib.msa_route_set_max_stages(n), "msa_route_set_max_stages")
+
+
 def route_set_impl(impl: int) -> None:
-    """0 = automatic, 1 = CUDA-core kernel, 2 = tensor-core kernel."""
+    """0 = automatic, 1 = CUDA-core kernel, 2 = tensor-core kernel, 3 = tensor cores with qhat held in shared memory."""
     check(lib.msa_route_set_impl(impl), "msa_route_set_impl")
 
 
@@ -172,6 +182,22 @@ def msa_gather_kv(host_bank, doc_chunk_off_host, idx_host, max_mem: int, dev_mem
     return dev_mem_kv, mem_len
 
 
+def msa_gather_kv_device(host_bank, doc_chunk_off, idx, max_mem: int, dev_mem_kv=None, mem_len=None, stream=None):
+    """Device-side fetch: idx [n_q, k] int32 and doc_chunk_off on the device; the pinned host bank is
+    read by a kernel. Returns (dev_mem_kv [n_q, max_mem, 2, hkv, d], mem_len int32 [n_q] on the device)."""
+    C, _, hkv, d = host_bank.shape
+    n_q, k = idx.shape
+    dev = idx.device
+    if dev_mem_kv is None:
+        dev_mem_kv = torch.zeros((n_q, max_mem, 2, hkv, d), dtype=host_bank.dtype, device=dev)
+    if mem_len is None:
+        mem_len = torch.zeros(n_q, dtype=torch.int32, device=dev)
+    check(lib.msa_gather_kv_device(_ptr(host_bank), _dt(host_bank), C, _ptr(doc_chunk_off), doc_chunk_off.numel() - 1,
+                                   _ptr(idx), n_q, k, hkv, d, max_mem, _ptr(dev_mem_kv), _ptr(mem_len),
+                                   _stream(stream)), "msa_gather_kv_device")
+    return dev_mem_kv, mem_len
+
+
 def msa_sparse_attn(q, mem_kv, mem_len, local_k, local_v, L: int, q_start: int, scale: float | None = None,
                     out=None, stream=None):
     """q [n_q, T, hq, d] (rotated), mem_kv [n_q, max_mem, 2, hkv, d], mem_len int32 [n_q] (device),
@@ -193,7 +219,7 @@ class InterleaveRound:
 
     def __init__(self, layers, *, n_chunks, n_docs, doc_chunk_off, doc_chunk_off_host, chunk_doc, n_q, H, d, hq, hkv,
                  k, L_prev, T_new, new_q_stride, L_max, max_mem, cos_sin, scale=None, dtype=torch.bfloat16, ws=None,
-                 reserved_sms: int = 0):
+                 reserved_sms: int = 0, fetch_mode: int = 1):
         self.layer_structs = (_lib.LayerArgs * len(layers))()
         for i, y in enumerate(layers):
             s = self.layer_structs[i]
@@ -215,6 +241,7 @@ class InterleaveRound:
         a.rope_max_pos = cos_sin.shape[0]
         a.scale = 1.0 / math.sqrt(d) if scale is None else scale
         a.reserved_sms = reserved_sms
+        a.fetch_mode = fetch_mode
         self.args = a
         need = ctypes.c_size_t(0)
         a.ws, a.ws_bytes = None, 0

@@ -1,6 +1,8 @@
 """Builds libmsa.so (the C-ABI library) in-tree with nvcc for sm_100a.
 
-    python -m routed_long_context_b200.build [--ptxas-verbose]
+    python routed_long_context_b200/build.py [--ptxas-verbose]
+
+Run it by path (or load it with importlib by path): importing the package itself loads the library.
 """
 from __future__ import annotations
 

@@ -6,12 +6,15 @@
 // heads (q and K from shared memory, K rows padded to 129 floats so the 32 lanes hit 32 banks),
 // then an online softmax (running max and sum per head, exp2 with log2(e) folded into q) and
 // the P.V update, where lane r owns output dims 4r..4r+3. Arithmetic and softmax in fp32.
+#include <atomic>
+
 #include "common.cuh"
 
 namespace msa {
 namespace {
 
 constexpr int kD = 128;
+std::atomic<int> g_attn_impl{0};   // bf16: 0 = tensor cores (mma.sync), 1 = CUDA cores
 constexpr int kTokPerBlock = 8;
 constexpr int kKeyTile = 32;
 
@@ -199,12 +202,214 @@ msa_status launch(const AttnArgs& a, int n_q, cudaStream_t s) {
     }
 }
 
+
+// ------------------------------------------------------------------------------------------------
+// bf16 tensor-core variant (mma.sync m16n8k16, fp32 accumulation): one block of 4 warps per
+// (64 query rows, kv head g, query q); rows are (token, head) pairs r = t * G + h of the G heads
+// sharing kv head g; warp w owns rows 16w..16w+15. Per tile of 64 keys: S = Q K^T from K rows in
+// shared memory (row stride 136 elements: the 32-bit fragment loads of 8 keys x 4 lanes hit 32
+// distinct banks), online softmax on the accumulator fragments (row max/sum across the 4 lanes of
+// a row), then O += P V with V fragments from ldmatrix.trans. Q stays in registers.
+// ------------------------------------------------------------------------------------------------
+constexpr int kMmaRows = 64;
+constexpr int kMmaKeys = 64;
+constexpr int kKvStride = kD + 8;   // bf16 elements per shared-memory row
+
+__device__ __forceinline__ void mma_bf16_16816(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+template <int G>
+__global__ void __launch_bounds__(128) attn_mma_kernel(const AttnArgs a) {
+    __shared__ __align__(16) __nv_bfloat16 Ks[kMmaKeys][kKvStride];
+    __shared__ __align__(16) __nv_bfloat16 Vs[kMmaKeys][kKvStride];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int gid = lane >> 2, tig = lane & 3;
+    const int qi = blockIdx.z, g = blockIdx.y;
+    const int n_rows = a.T * G;
+    const int r0 = blockIdx.x * kMmaRows;
+    const int r_last = min(r0 + kMmaRows, n_rows) - 1;
+    const int t_last = r_last / G;
+    const int mem_len = max(min(a.mem_len[qi], a.max_mem), 0);
+    const int n_local = max(min(a.L, a.q_start + t_last + 1), 0);
+    const int n_keys = mem_len + n_local;
+
+    const __nv_bfloat16* Q = static_cast<const __nv_bfloat16*>(a.q);
+    const __nv_bfloat16* MKV = static_cast<const __nv_bfloat16*>(a.mem_kv);
+    const __nv_bfloat16* LK = static_cast<const __nv_bfloat16*>(a.local_k);
+    const __nv_bfloat16* LV = static_cast<const __nv_bfloat16*>(a.local_v);
+
+    // this thread's two rows (gid, gid + 8 of the warp's 16) and their tokens
+    const int ra = r0 + warp * 16 + gid, rb = ra + 8;
+    const bool va = ra < n_rows, vb = rb < n_rows;
+    const int ta = ra / G, tb = rb / G;
+    // Q fragments for the 8 k-steps of d = 128 (zeros for rows past the end)
+    uint32_t qf[kD / 16][4];
+    {
+        const uint32_t* qa = reinterpret_cast<const uint32_t*>(Q + (((int64_t)qi * a.T + ta) * a.hq + g * G + ra % G) * kD);
+        const uint32_t* qb = reinterpret_cast<const uint32_t*>(Q + (((int64_t)qi * a.T + tb) * a.hq + g * G + rb % G) * kD);
+#pragma unroll
+        for (int s = 0; s < kD / 16; ++s) {
+            qf[s][0] = va ? qa[s * 8 + tig] : 0u;
+            qf[s][1] = vb ? qb[s * 8 + tig] : 0u;
+            qf[s][2] = va ? qa[s * 8 + 4 + tig] : 0u;
+            qf[s][3] = vb ? qb[s * 8 + 4 + tig] : 0u;
+        }
+    }
+    const float ninf = -__int_as_float(0x7f800000);
+    float o[kD / 8][4];
+#pragma unroll
+    for (int nd = 0; nd < kD / 8; ++nd) o[nd][0] = o[nd][1] = o[nd][2] = o[nd][3] = 0.f;
+    float m_a = ninf, m_b = ninf, l_a = 0.f, l_b = 0.f;
+
+    for (int kb = 0; kb < n_keys; kb += kMmaKeys) {
+        __syncthreads();
+        // stage 64 keys and values: 16-byte vectors, zeros past the visible range
+        for (int v = threadIdx.x; v < kMmaKeys * (kD / 8) * 2; v += blockDim.x) {
+            const int which = v / (kMmaKeys * (kD / 8));
+            const int rem = v % (kMmaKeys * (kD / 8));
+            const int r = rem / (kD / 8), c = (rem % (kD / 8)) * 8;
+            const int kk = kb + r;
+            uint4 x = make_uint4(0, 0, 0, 0);
+            if (kk < mem_len)
+                x = *reinterpret_cast<const uint4*>(MKV + (((int64_t)qi * a.max_mem + kk) * 2 + which) * a.hkv * kD +
+                                                    g * kD + c);
+            else if (kk < n_keys)
+                x = *reinterpret_cast<const uint4*>((which ? LV : LK) +
+                                                    (((int64_t)qi * a.L_max + (kk - mem_len)) * a.hkv + g) * kD + c);
+            *reinterpret_cast<uint4*>(which ? &Vs[r][c] : &Ks[r][c]) = x;
+        }
+        __syncthreads();
+
+        // S = Q K^T for 8 blocks of 8 keys
+        float sc[kMmaKeys / 8][4];
+#pragma unroll
+        for (int nb = 0; nb < kMmaKeys / 8; ++nb) {
+            sc[nb][0] = sc[nb][1] = sc[nb][2] = sc[nb][3] = 0.f;
+            const uint32_t* krow = reinterpret_cast<const uint32_t*>(&Ks[nb * 8 + gid][0]);
+#pragma unroll
+            for (int s = 0; s < kD / 16; ++s) mma_bf16_16816(sc[nb], qf[s], krow[s * 8 + tig], krow[s * 8 + 4 + tig]);
+        }
+        // mask, scale (log2 domain) and tile row maxima
+        float tm_a = ninf, tm_b = ninf;
+#pragma unroll
+        for (int nb = 0; nb < kMmaKeys / 8; ++nb) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int kk = kb + nb * 8 + tig * 2 + e;
+                const bool vis_a = va && (kk < mem_len || (kk < n_keys && kk - mem_len <= a.q_start + ta));
+                const bool vis_b = vb && (kk < mem_len || (kk < n_keys && kk - mem_len <= a.q_start + tb));
+                sc[nb][e] = vis_a ? sc[nb][e] * a.scale_log2e : ninf;
+                sc[nb][2 + e] = vis_b ? sc[nb][2 + e] * a.scale_log2e : ninf;
+                tm_a = fmaxf(tm_a, sc[nb][e]);
+                tm_b = fmaxf(tm_b, sc[nb][2 + e]);
+            }
+        }
+        tm_a = fmaxf(tm_a, __shfl_xor_sync(0xffffffffu, tm_a, 1));
+        tm_a = fmaxf(tm_a, __shfl_xor_sync(0xffffffffu, tm_a, 2));
+        tm_b = fmaxf(tm_b, __shfl_xor_sync(0xffffffffu, tm_b, 1));
+        tm_b = fmaxf(tm_b, __shfl_xor_sync(0xffffffffu, tm_b, 2));
+        const float mn_a = fmaxf(m_a, tm_a), mn_b = fmaxf(m_b, tm_b);
+        const float f_a = mn_a == ninf ? 1.f : exp2f(m_a - mn_a);
+        const float f_b = mn_b == ninf ? 1.f : exp2f(m_b - mn_b);
+        m_a = mn_a;
+        m_b = mn_b;
+        float ps_a = 0.f, ps_b = 0.f;
+#pragma unroll
+        for (int nb = 0; nb < kMmaKeys / 8; ++nb) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                sc[nb][e] = mn_a == ninf ? 0.f : exp2f(sc[nb][e] - mn_a);
+                sc[nb][2 + e] = mn_b == ninf ? 0.f : exp2f(sc[nb][2 + e] - mn_b);
+                ps_a += sc[nb][e];
+                ps_b += sc[nb][2 + e];
+            }
+        }
+        l_a = l_a * f_a + ps_a;
+        l_b = l_b * f_b + ps_b;
+#pragma unroll
+        for (int nd = 0; nd < kD / 8; ++nd) {
+            o[nd][0] *= f_a; o[nd][1] *= f_a;
+            o[nd][2] *= f_b; o[nd][3] *= f_b;
+        }
+        // O += P V: P from the score fragments (bf16), V fragments by ldmatrix.trans
+#pragma unroll
+        for (int s2 = 0; s2 < kMmaKeys / 16; ++s2) {
+            uint32_t pa[4];
+            pa[0] = pack_bf16(sc[2 * s2][0], sc[2 * s2][1]);
+            pa[1] = pack_bf16(sc[2 * s2][2], sc[2 * s2][3]);
+            pa[2] = pack_bf16(sc[2 * s2 + 1][0], sc[2 * s2 + 1][1]);
+            pa[3] = pack_bf16(sc[2 * s2 + 1][2], sc[2 * s2 + 1][3]);
+#pragma unroll
+            for (int nd = 0; nd < kD / 8; nd += 2) {
+                // matrices: keys 16s2+0..7 / +8..15, dims 8nd..+7 / 8(nd+1)..+7
+                const int key = s2 * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+                const int dim = nd * 8 + (lane >> 4) * 8;
+                const uint32_t addr = static_cast<uint32_t>(__cvta_generic_to_shared(&Vs[key][dim]));
+                uint32_t b0, b1, b2, b3;
+                asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                             : "=r"(b0), "=r"(b1), "=r"(b2), "=r"(b3)
+                             : "r"(addr));
+                mma_bf16_16816(o[nd], pa, b0, b1);
+                mma_bf16_16816(o[nd + 1], pa, b2, b3);
+            }
+        }
+    }
+
+    l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
+    l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
+    l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
+    l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
+    const float ia = l_a > 0.f ? 1.f / l_a : 0.f, ib = l_b > 0.f ? 1.f / l_b : 0.f;
+    __nv_bfloat16* O = static_cast<__nv_bfloat16*>(a.out);
+    uint32_t* oa = reinterpret_cast<uint32_t*>(O + (((int64_t)qi * a.T + ta) * a.hq + g * G + ra % G) * kD);
+    uint32_t* ob = reinterpret_cast<uint32_t*>(O + (((int64_t)qi * a.T + tb) * a.hq + g * G + rb % G) * kD);
+#pragma unroll
+    for (int nd = 0; nd < kD / 8; ++nd) {
+        if (va) oa[nd * 4 + tig] = pack_bf16(o[nd][0] * ia, o[nd][1] * ia);
+        if (vb) ob[nd * 4 + tig] = pack_bf16(o[nd][2] * ib, o[nd][3] * ib);
+    }
+}
+
+template <int G>
+msa_status launch_mma_g(const AttnArgs& a, int n_q, cudaStream_t s) {
+    dim3 grid((a.T * G + kMmaRows - 1) / kMmaRows, a.hkv, n_q);
+    attn_mma_kernel<G><<<grid, 128, 0, s>>>(a);
+    MSA_LAUNCH_CHECK();
+    return MSA_OK;
+}
+
+msa_status launch_mma(const AttnArgs& a, int n_q, cudaStream_t s) {
+    switch (a.hq / a.hkv) {
+        case 1: return launch_mma_g<1>(a, n_q, s);
+        case 2: return launch_mma_g<2>(a, n_q, s);
+        case 4: return launch_mma_g<4>(a, n_q, s);
+        case 8: return launch_mma_g<8>(a, n_q, s);
+        default: return set_error(MSA_ERR_UNSUPPORTED, "msa_sparse_attn: hq/hkv unsupported");
+    }
+}
+
 }  // namespace
 }  // namespace msa
 
 using namespace msa;
 
 extern "C" {
+
+msa_status msa_attn_set_impl(int impl) {
+    MSA_REQUIRE(impl == 0 || impl == 1, "msa_attn_set_impl: impl must be 0 or 1");
+    g_attn_impl.store(impl);
+    return MSA_OK;
+}
 
 msa_status msa_sparse_attn(const void* q, const void* mem_kv, const int32_t* mem_len, int max_mem,
                            const void* local_k, const void* local_v, int L_max, int L, int q_start, int n_q, int T,
@@ -229,6 +434,7 @@ msa_status msa_sparse_attn(const void* q, const void* mem_kv, const int32_t* mem
     a.local_k = local_k; a.local_v = local_v; a.L_max = L_max; a.L = L; a.q_start = q_start;
     a.T = T; a.hq = hq; a.hkv = hkv; a.scale_log2e = scale * 1.4426950408889634f; a.out = out;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dt == MSA_BF16 && g_attn_impl.load() == 0) return launch_mma(a, n_q, s);
     return dt == MSA_BF16 ? launch<__nv_bfloat16>(a, n_q, s) : launch<float>(a, n_q, s);
 }
 

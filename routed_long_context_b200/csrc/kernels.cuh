@@ -26,6 +26,28 @@ struct RopeRowsArgs {
     int* err;
 };
 msa_status launch_rope_rows(const RopeRowsArgs& a, msa_dtype dt, cudaStream_t s);
+
+// One interleave round's appends for up to kMaxAppendLayers layers in one launch: new keys rotated
+// to positions pos_offset + t into local_k rows L_prev + t, values copied to local_v, queries
+// rotated into q_rot [n_q][T_new][hq][d]. New-token buffers: row (q * new_q_stride + t).
+struct AppendLayer {
+    const void* k_new;
+    const void* v_new;
+    const void* q_new;
+    void* local_k;
+    void* local_v;
+    void* q_rot;
+};
+constexpr int kMaxAppendLayers = 24;
+struct AppendArgs {
+    AppendLayer layer[kMaxAppendLayers];
+    int n_layers, n_q, T_new, new_q_stride, L_max, L_prev, hkv, hq, d;
+    int64_t pos_offset;
+    const float2* cs;
+    int64_t max_pos;
+    int* err;
+};
+msa_status launch_append(const AppendArgs& a, msa_dtype dt, cudaStream_t s);
 bool rope_layout_ok(msa_dtype dt, int d);
 
 // Tensor-core router (tcgen05 + TMA + TMEM) over a bf16 index in unit-vector form.
@@ -44,11 +66,14 @@ struct RouteTcArgs {
     int* err;
     int grid_cap;          // > 0: at most this many CTAs (SMs left free for concurrent work)
     int* tile_counter;     // zero at launch (route_prepare zeroes it)
+    bool resident;         // keep qhat in shared memory when it fits (default: stream it with the index)
 };
 // Returns MSA_ERR_UNSUPPORTED (without launching) when the shape does not fit the kernel.
 msa_status launch_route_tc(const RouteTcArgs& a, cudaStream_t s);
 // Rows the tensor-core path needs in qhat for N columns (0 if unsupported).
-int route_tc_pad_rows(int N, int K);
+int route_tc_pad_rows(int N, int K, bool resident = false);
+// Testing knob: cap on the router's pipeline stages (0 = as many as the shared-memory budget allows).
+void route_tc_set_max_stages(int n);
 
 // Router scoring split in two launches so a caller can hoist the (tiny) query prepass off the
 // router's stream: route_prepare normalises the queries into qhat and fills the score outputs with
@@ -58,6 +83,7 @@ struct RoutePlan {
     msa_dtype dt;
     int n_q, T, H, d, K, N, n_pad;
     bool use_tc;
+    bool resident;
 };
 msa_status route_plan(msa_dtype dt, int64_t n_chunks, int n_q, int T, int H, int d, RoutePlan* plan);
 msa_status route_prepare(const RoutePlan& p, const void* qr, void* ws, float* doc_scores, int64_t n_docs,
@@ -65,5 +91,10 @@ msa_status route_prepare(const RoutePlan& p, const void* qr, void* ws, float* do
 msa_status route_launch(const RoutePlan& p, const void* kr_index, int64_t n_chunks, const int32_t* chunk_doc,
                         int64_t n_docs, void* ws, float* doc_scores, float* chunk_scores, int grid_cap,
                         cudaStream_t s);
+
+// Device-side fetch of the selected documents' rows from a pinned (mapped) host bank.
+msa_status gather_device(const void* host_bank, msa_dtype dt, int64_t n_chunks, const int64_t* doc_chunk_off,
+                         int64_t n_docs, const int32_t* idx, int n_q, int k, int hkv, int d, int max_mem,
+                         void* dev_mem_kv, int32_t* mem_len, cudaStream_t s);
 
 }  // namespace msa

@@ -85,7 +85,11 @@ struct PoolArgs {
 template <typename TIn, typename TOut>
 __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const PoolArgs a) {
     constexpr int VEC = 16 / sizeof(TIn);
-    const int part = a.parts[blockIdx.y];
+    // block b handles tensor part b % n_parts of chunks b / n_parts, b / n_parts + stride, ...: the
+    // rotated-K blocks (heavier on the load units) interleave with the plain streaming ones
+    const int part = a.parts[blockIdx.x % a.n_parts];
+    const int64_t c_first = blockIdx.x / a.n_parts;
+    const int64_t c_stride = gridDim.x / a.n_parts;
     const TIn* __restrict__ src = static_cast<const TIn*>(a.src[part]);
     const int H = a.heads[part];
     const int d = a.d;
@@ -95,7 +99,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const PoolArgs a) {
     const bool rope = (part == 0) && a.fuse_rope;
     const int passes = (E + kPoolThreads * VEC - 1) / (kPoolThreads * VEC);
 
-    for (int64_t c = blockIdx.x; c < a.n_chunks; c += gridDim.x) {
+    for (int64_t c = c_first; c < a.n_chunks; c += c_stride) {
         const int64_t doc = a.chunk_doc[c];
         if (doc < 0 || doc >= a.n_docs) {
             if (threadIdx.x == 0) record_device_error(a.err, MSA_DEV_BAD_INDEX);
@@ -223,6 +227,58 @@ __global__ void __launch_bounds__(128) rope_rows_kernel(const RopeRowsArgs a) {
     }
 }
 
+
+// ---------------------------------------------------------------------------------------------
+// Fused append of one interleave round, every layer in one launch: block (layer, query, token)
+// rotates the new token's key to its global position into the local cache, copies its value, and
+// rotates its query into the attention workspace.
+template <typename T>
+__device__ __forceinline__ void rotate_copy_row(const T* __restrict__ src, T* __restrict__ dst, int E, int d,
+                                                const float2* __restrict__ cs_row, bool do_rotate) {
+    constexpr int VEC = 16 / sizeof(T);
+    const int half_lanes = (d / 2) / VEC;
+    const int passes = (E + 128 * VEC - 1) / (128 * VEC);
+    for (int pass = 0; pass < passes; ++pass) {
+        const int e0 = (pass * 128 + threadIdx.x) * VEC;
+        const bool active = e0 < E;
+        const uint4 raw = active ? *reinterpret_cast<const uint4*>(src + e0) : make_uint4(0, 0, 0, 0);
+        if (!do_rotate) {
+            if (active) *reinterpret_cast<uint4*>(dst + e0) = raw;
+            continue;
+        }
+        const uint4 praw = shfl_xor_u4(raw, half_lanes);
+        float x[VEC], px[VEC];
+        widen<T>(raw, x);
+        widen<T>(praw, px);
+        const int ih = e0 % d;
+        const bool first_half = ih < d / 2;
+        if (cs_row) msa::rotate<VEC>(x, px, cs_row, first_half ? ih : ih - d / 2, first_half);
+        if (active) store_f32<T, VEC>(dst + e0, x);
+    }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(128) append_kernel(const AppendArgs a) {
+    const int per_layer = a.n_q * a.T_new;
+    const int layer = blockIdx.x / per_layer;
+    const int rem = blockIdx.x % per_layer;
+    const int q = rem / a.T_new, t = rem % a.T_new;
+    const AppendLayer& y = a.layer[layer];
+    const int64_t p = a.pos_offset + t;
+    const bool pos_ok = p >= 0 && p < a.max_pos;
+    if (!pos_ok && threadIdx.x == 0) record_device_error(a.err, MSA_DEV_ROPE_POSITION);
+    const float2* cs_row = pos_ok ? a.cs + p * (a.d / 2) : nullptr;
+    const int Ek = a.hkv * a.d, Eq = a.hq * a.d;
+    const int64_t in_row = (int64_t)q * a.new_q_stride + t;
+    const int64_t cache_row = (int64_t)q * a.L_max + a.L_prev + t;
+    rotate_copy_row<T>(static_cast<const T*>(y.k_new) + in_row * Ek, static_cast<T*>(y.local_k) + cache_row * Ek, Ek,
+                       a.d, cs_row, true);
+    rotate_copy_row<T>(static_cast<const T*>(y.v_new) + in_row * Ek, static_cast<T*>(y.local_v) + cache_row * Ek, Ek,
+                       a.d, nullptr, false);
+    rotate_copy_row<T>(static_cast<const T*>(y.q_new) + in_row * Eq,
+                       static_cast<T*>(y.q_rot) + ((int64_t)q * a.T_new + t) * Eq, Eq, a.d, cs_row, true);
+}
+
 template <typename T>
 bool vec_layout_ok(int d) {
     constexpr int VEC = 16 / sizeof(T);
@@ -241,6 +297,17 @@ msa_status launch_rope_rows(const RopeRowsArgs& a, msa_dtype dt, cudaStream_t s)
         rope_rows_kernel<__nv_bfloat16><<<blocks, 128, 0, s>>>(a);
     else
         rope_rows_kernel<float><<<blocks, 128, 0, s>>>(a);
+    MSA_LAUNCH_CHECK();
+    return MSA_OK;
+}
+
+msa_status launch_append(const AppendArgs& a, msa_dtype dt, cudaStream_t s) {
+    const int64_t blocks = (int64_t)a.n_layers * a.n_q * a.T_new;
+    if (blocks == 0) return MSA_OK;
+    if (dt == MSA_BF16)
+        append_kernel<__nv_bfloat16><<<(unsigned)blocks, 128, 0, s>>>(a);
+    else
+        append_kernel<float><<<(unsigned)blocks, 128, 0, s>>>(a);
     MSA_LAUNCH_CHECK();
     return MSA_OK;
 }
@@ -315,7 +382,8 @@ msa_status msa_pool_chunks(const void* k, const void* v, const void* kr, msa_dty
     a.kvbar = kvbar; a.kr_index = kr_index; a.normalize = normalize_router;
     a.err = device_error_word();
     const int64_t cap = 1 << 20;
-    dim3 grid((unsigned)(n_chunks < cap ? n_chunks : cap), (unsigned)a.n_parts);
+    const int64_t per_part = n_chunks < cap ? n_chunks : cap;
+    dim3 grid((unsigned)(per_part * a.n_parts));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (in_dt == MSA_BF16 && out_dt == MSA_BF16)
         pool_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, kPoolThreads, 0, s>>>(a);

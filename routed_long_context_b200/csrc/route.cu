@@ -13,7 +13,7 @@
 namespace msa {
 namespace {
 
-std::atomic<int> g_route_impl{0};   // 0 auto, 1 CUDA cores, 2 tensor cores
+std::atomic<int> g_route_impl{0};   // 0 auto, 1 CUDA cores, 2 tensor cores, 3 tensor cores + resident qhat
 
 // q_hat rows [n_pad][K] of TQ; rows >= N are zero. Also fills doc_scores/chunk_scores with -inf.
 template <typename T, typename TQ>
@@ -177,9 +177,10 @@ msa_status route_plan(msa_dtype dt, int64_t n_chunks, int n_q, int T, int H, int
     RoutePlan p{};
     p.dt = dt; p.n_q = n_q; p.T = T; p.H = H; p.d = d; p.K = H * d; p.N = n_q * T;
     const int impl = g_route_impl.load();
-    const int tc_rows = dt == MSA_BF16 ? route_tc_pad_rows(p.N, p.K) : 0;
+    p.resident = impl == 3;
+    const int tc_rows = dt == MSA_BF16 ? route_tc_pad_rows(p.N, p.K, p.resident) : 0;
     p.use_tc = dt == MSA_BF16 && impl != 1 && tc_rows > 0 && n_chunks > 0;
-    if (impl == 2 && !p.use_tc)
+    if (impl >= 2 && !p.use_tc)
         return set_error(MSA_ERR_UNSUPPORTED, "msa_route_scores: tensor-core path unavailable for this shape");
     if (!p.use_tc && !simt_supported(dt, p.K))
         return set_error(MSA_ERR_UNSUPPORTED, "msa_route_scores: H*d = %d unsupported", p.K);
@@ -228,6 +229,7 @@ msa_status route_launch(const RoutePlan& p, const void* kr_index, int64_t n_chun
         a.index = kr_index; a.qhat = qhat; a.n_chunks = n_chunks; a.K = p.K; a.N = p.N; a.n_pad = p.n_pad;
         a.T = p.T; a.chunk_doc = chunk_doc; a.n_docs = n_docs; a.doc_scores = doc_scores;
         a.chunk_scores = chunk_scores; a.err = err; a.grid_cap = grid_cap; a.tile_counter = static_cast<int*>(ws);
+        a.resident = p.resident;
         return launch_route_tc(a, s);
     }
     if (p.dt == MSA_BF16)
@@ -244,8 +246,14 @@ using namespace msa;
 extern "C" {
 
 msa_status msa_route_set_impl(int impl) {
-    MSA_REQUIRE(impl >= 0 && impl <= 2, "msa_route_set_impl: impl must be 0, 1 or 2");
+    MSA_REQUIRE(impl >= 0 && impl <= 3, "msa_route_set_impl: impl must be 0, 1, 2 or 3");
     g_route_impl.store(impl);
+    return MSA_OK;
+}
+
+msa_status msa_route_set_max_stages(int n) {
+    MSA_REQUIRE(n >= 0 && n <= 12, "msa_route_set_max_stages: n must be in [0, 12]");
+    route_tc_set_max_stages(n);
     return MSA_OK;
 }
 

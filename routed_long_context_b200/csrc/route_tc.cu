@@ -14,12 +14,15 @@
 // atomic counter and publishes it to the MMA and epilogue warps through a 2-entry shared-memory
 // queue, so CTAs that start late (SMs still busy with concurrent kernels) simply take fewer tiles.
 // Modes: RESIDENT keeps all of qhat (<= 64 columns) in shared memory, loaded once per CTA,
-// so only the index streams from HBM; otherwise qhat tiles of BN <= 256 columns stream with A.
+// so only the index streams; by default qhat tiles of BN <= 256 columns stream (from L2) with A.
 // Every mbarrier wait is bounded (about 2 s of %globaltimer); on expiry the CTA records
 // MSA_DEV_WAIT_TIMEOUT, all roles leave their loops, in-flight copies and MMAs are waited for
 // (again bounded) and TMEM is freed before the kernel returns.
 #include <cuda.h>
 
+#include <algorithm>
+
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -31,8 +34,12 @@ namespace {
 constexpr int BM = 128;               // chunks per tile = MMA M = TMEM lanes
 constexpr int BK = 64;                // bf16 elements per 128-byte swizzled row
 constexpr int kThreads = 192;
-constexpr int kMaxStages = 8;
+constexpr int kMaxStages = 12;
 constexpr int kSmemLimit = 232448;    // max dynamic shared memory per block on sm_100
+// Default budget: leaves room on each SM (228 KB of shared memory) for one attention block
+// (35 KB) and one top-k block (5 KB) of the overlapped selection/attention of earlier layers.
+constexpr int kSmemBudget = 188 * 1024;
+std::atomic<int> g_max_stages{0};     // testing knob: 0 = as many stages as the budget allows
 constexpr int kStageA = BM * BK * 2;  // 16 KB
 constexpr uint64_t kWaitNs = 2000000000ull;
 
@@ -470,13 +477,15 @@ struct Plan {
     size_t smem;
 };
 
-bool make_plan(int N, int K, Plan* pl) {
+// Streamed qhat is the default: the query block is re-read from L2 with every index tile, which
+// leaves shared memory for more index stages in flight (measured faster than keeping qhat
+// resident at 64 columns). `resident` asks for qhat held in shared memory when it fits.
+bool make_plan(int N, int K, Plan* pl, bool resident = false) {
     if (N <= 0 || K <= 0 || K % BK != 0 || K > 8192) return false;
     const int kblocks = K / BK;
     const int n16 = (N + 15) / 16 * 16;
-    const size_t fixed = 1024 + 256;
-    // resident: all of qhat stays in shared memory, only the index streams
-    if (n16 <= 64) {
+    const size_t fixed = 1024 + 512;
+    if (resident && n16 <= 64) {
         const size_t b = (size_t)kblocks * n16 * BK * 2;
         if (fixed + b + 4 * kStageA <= (size_t)kSmemLimit) {
             int st = (int)((kSmemLimit - fixed - b) / kStageA);
@@ -488,23 +497,42 @@ bool make_plan(int N, int K, Plan* pl) {
     const int BN = n16 <= 256 ? n16 : 256;
     const int n_tiles_n = (N + BN - 1) / BN;
     const size_t stage = (size_t)kStageA + (size_t)BN * BK * 2;
-    int st = (int)((kSmemLimit - fixed) / stage);
+    const int forced = g_max_stages.load();
+    int st = (int)((kSmemBudget - fixed) / stage);
+    if (st < 4) st = (int)((kSmemLimit - fixed) / stage);      // wide query blocks: use it all
+    if (forced > 0) st = std::min(forced, (int)((kSmemLimit - fixed) / stage));
     if (st > kMaxStages) st = kMaxStages;
     if (st < 2) return false;
     *pl = Plan{false, BN, n_tiles_n * BN, n_tiles_n, st, fixed + (size_t)st * stage};
     return true;
 }
 
+// Opts both kernel variants into the largest dynamic shared memory once per device.
+msa_status allow_max_smem() {
+    static std::mutex mu;
+    static bool done[64] = {false};
+    int dev = 0;
+    MSA_CUDA_TRY(cudaGetDevice(&dev));
+    std::lock_guard<std::mutex> lk(mu);
+    if (dev >= 0 && dev < 64 && done[dev]) return MSA_OK;
+    MSA_CUDA_TRY(cudaFuncSetAttribute(route_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit));
+    MSA_CUDA_TRY(cudaFuncSetAttribute(route_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit));
+    if (dev >= 0 && dev < 64) done[dev] = true;
+    return MSA_OK;
+}
+
 }  // namespace
 
-int route_tc_pad_rows(int N, int K) {
+void route_tc_set_max_stages(int n) { g_max_stages.store(n); }
+
+int route_tc_pad_rows(int N, int K, bool resident) {
     Plan pl;
-    return make_plan(N, K, &pl) ? pl.n_pad : 0;
+    return make_plan(N, K, &pl, resident) ? pl.n_pad : 0;
 }
 
 msa_status launch_route_tc(const RouteTcArgs& a, cudaStream_t s) {
     Plan pl;
-    if (!make_plan(a.N, a.K, &pl) || pl.n_pad != a.n_pad)
+    if (!make_plan(a.N, a.K, &pl, a.resident) || pl.n_pad != a.n_pad)
         return set_error(MSA_ERR_UNSUPPORTED, "route (tensor cores): unsupported shape N=%d K=%d", a.N, a.K);
     CUtensorMap tmA, tmB;
     MSA_RETURN_IF(make_map(&tmA, a.index, (uint64_t)a.K, (uint64_t)a.n_chunks, BM, true));
@@ -531,15 +559,11 @@ msa_status launch_route_tc(const RouteTcArgs& a, cudaStream_t s) {
     if (!p.tile_counter) return set_error(MSA_ERR_INVALID_ARG, "route (tensor cores): no tile counter");
     int64_t grid = p.n_tiles < (int64_t)sm_count() ? p.n_tiles : (int64_t)sm_count();
     if (a.grid_cap > 0 && grid > a.grid_cap) grid = a.grid_cap;
-    if (pl.resident) {
-        auto kern = route_tc_kernel<true>;
-        MSA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem));
-        kern<<<(unsigned)grid, kThreads, pl.smem, s>>>(tmA, tmB, p);
-    } else {
-        auto kern = route_tc_kernel<false>;
-        MSA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem));
-        kern<<<(unsigned)grid, kThreads, pl.smem, s>>>(tmA, tmB, p);
-    }
+    MSA_RETURN_IF(allow_max_smem());
+    if (pl.resident)
+        route_tc_kernel<true><<<(unsigned)grid, kThreads, pl.smem, s>>>(tmA, tmB, p);
+    else
+        route_tc_kernel<false><<<(unsigned)grid, kThreads, pl.smem, s>>>(tmA, tmB, p);
     MSA_LAUNCH_CHECK();
     return MSA_OK;
 }

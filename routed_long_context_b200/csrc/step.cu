@@ -1,13 +1,15 @@
 // One Memory Interleave round over all routed layers: append -> route -> top-k -> fetch -> attend.
 //
-// Streams: R = the caller's compute stream (routers only), C = the caller's copy stream (fetches),
+// Streams: R = the caller's compute stream (routers only), C = the caller's copy stream (host-issued fetches),
 // S = select (library-owned: top-k, index copy to the host, memory lengths),
 // A = attend (library-owned: query prepasses, appends, attention).
-//   A: every layer's router prepass (record P_l), then every layer's append + query rotation.
+//   A: every layer's router prepass (record P_l), then one fused append + query rotation launch.
 //   R: for every layer: wait P_l, router kernel (optionally on fewer SMs than the GPU has), record R_l.
 //   S: for every layer: wait R_l, top-k, indices -> pinned host, memory lengths, record E_l.
-//   host: for every layer: wait E_l (bounded poll), enqueue the document fetches on C, record G_l;
-//         A waits G_l and runs the layer's attention.
+//   fetch_mode 0 (host-issued copies): for every layer the host waits E_l (bounded poll), enqueues one
+//         cudaMemcpyAsync per document on C, records G_l; A waits G_l and runs the layer's attention.
+//   fetch_mode 1 (device fetch): S runs the fetch kernel right after top-k (reading the mapped pinned
+//         bank), A waits E_l and attends; the host never waits.
 //   join: R waits for the last work of S and A.
 // The routers run back to back; selection, fetch and attention of layer l overlap the routing of
 // layers l+1.. (on SMs the routers leave free and in the copy engines).
@@ -78,7 +80,8 @@ msa_status validate(const msa_interleave_args* a, bool need_ws) {
     MSA_REQUIRE(dtype_ok(a->dt), "msa_interleave_step: bad dtype");
     MSA_REQUIRE(a->n_layers > 0 && a->layers, "msa_interleave_step: no layers");
     MSA_REQUIRE(a->n_q > 0 && a->H > 0 && a->d > 0 && a->hq > 0 && a->hkv > 0 && a->k > 0 && a->T_new > 0 &&
-                    a->L_prev >= 0 && a->n_docs > 0 && a->n_chunks > 0 && a->max_mem > 0 && a->reserved_sms >= 0,
+                    a->L_prev >= 0 && a->n_docs > 0 && a->n_chunks > 0 && a->max_mem > 0 && a->reserved_sms >= 0 &&
+                    (a->fetch_mode == 0 || a->fetch_mode == 1),
                 "msa_interleave_step: bad sizes");
     MSA_REQUIRE(a->L_prev + a->T_new <= a->L_max, "msa_interleave_step: local cache overflow (%d + %d > %d)", a->L_prev,
                 a->T_new, a->L_max);
@@ -111,12 +114,24 @@ msa_status wait_event(cudaEvent_t ev, std::chrono::steady_clock::time_point dead
     }
 }
 
-struct Events {
-    std::vector<cudaEvent_t> ev;
-    ~Events() {
-        for (cudaEvent_t e : ev) cudaEventDestroy(e);
+// Events reused across calls: a per-thread, per-device pool (an event belongs to one device;
+// re-recording an event does not disturb waits already enqueued on its earlier record).
+constexpr int kMaxEvDev = 64;
+thread_local std::vector<cudaEvent_t> t_events[kMaxEvDev];
+
+msa_status event_pool(size_t n, cudaEvent_t** out) {
+    int dev = 0;
+    MSA_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxEvDev) return set_error(MSA_ERR_UNSUPPORTED, "msa_interleave_step: device %d", dev);
+    std::vector<cudaEvent_t>& v = t_events[dev];
+    while (v.size() < n) {
+        cudaEvent_t e = nullptr;
+        MSA_CUDA_TRY(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+        v.push_back(e);
     }
-};
+    *out = v.data();
+    return MSA_OK;
+}
 
 // Library-owned auxiliary streams (select, attend), created once per device.
 constexpr int kMaxDev = 64;
@@ -175,47 +190,27 @@ msa_status msa_interleave_step(const msa_interleave_args* a, void* compute, void
     MSA_RETURN_IF(route_plan(a->dt, a->n_chunks, a->n_q, T_act, a->H, a->d, &plan));
     const int grid_cap = a->reserved_sms > 0 ? std::max(1, sm_count() - a->reserved_sms) : 0;
 
-    // events: fork, P_l, R_l, E_l, G_l, join x2
-    Events evs;
-    evs.ev.resize(4 * (size_t)L + 3, nullptr);
-    for (auto& e : evs.ev) MSA_CUDA_TRY(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
-    cudaEvent_t ev_fork = evs.ev[4 * L], ev_join_s = evs.ev[4 * L + 1], ev_join_a = evs.ev[4 * L + 2];
-    auto P = [&](int l) { return evs.ev[l]; };
-    auto R = [&](int l) { return evs.ev[L + l]; };
-    auto E = [&](int l) { return evs.ev[2 * L + l]; };
-    auto G = [&](int l) { return evs.ev[3 * L + l]; };
+    // events: P_l, R_l, E_l, G_l, fork, join x2
+    cudaEvent_t* ev = nullptr;
+    MSA_RETURN_IF(event_pool(4 * (size_t)L + 3, &ev));
+    cudaEvent_t ev_fork = ev[4 * L], ev_join_s = ev[4 * L + 1], ev_join_a = ev[4 * L + 2];
+    auto P = [&](int l) { return ev[l]; };
+    auto R = [&](int l) { return ev[L + l]; };
+    auto E = [&](int l) { return ev[2 * L + l]; };
+    auto G = [&](int l) { return ev[3 * L + l]; };
     auto slot = [&](int l, size_t off) { return ws + Lo.off_layers + Lo.per_layer * (size_t)l + off; };
 
     MSA_CUDA_TRY(cudaEventRecord(ev_fork, sR));
     MSA_CUDA_TRY(cudaStreamWaitEvent(sS, ev_fork, 0));
     MSA_CUDA_TRY(cudaStreamWaitEvent(sA, ev_fork, 0));
 
-    // ---- A: router prepasses of every layer, then appends and query rotations
-    for (int l = 0; l < L; ++l) {
-        MSA_RETURN_IF(route_prepare(plan, a->layers[l].qr, slot(l, Lo.o_route),
-                                    reinterpret_cast<float*>(slot(l, Lo.o_scores)), a->n_docs, nullptr, a->n_chunks, sA));
-        MSA_CUDA_TRY(cudaEventRecord(P(l), sA));
-    }
-    for (int l = 0; l < L; ++l) {
-        const msa_layer_args& y = a->layers[l];
-        RopeRowsArgs r{};
-        r.heads = a->hkv; r.d = a->d; r.n_rows = (int64_t)a->n_q * a->T_new; r.uniform_len = a->T_new;
-        r.in = y.k_new; r.out = y.local_k; r.in_stride = a->new_q_stride; r.out_stride = a->L_max; r.out_off = a->L_prev;
-        r.pos_offset = (int64_t)a->k + a->L_prev; r.cs = cs; r.max_pos = a->rope_max_pos; r.err = err;
-        MSA_RETURN_IF(launch_rope_rows(r, a->dt, sA));
-        const size_t vrow = (size_t)a->hkv * a->d * es;
-        MSA_CUDA_TRY(cudaMemcpy2DAsync(static_cast<char*>(y.local_v) + (size_t)a->L_prev * vrow, (size_t)a->L_max * vrow,
-                                       y.v_new, (size_t)a->new_q_stride * vrow, (size_t)a->T_new * vrow, a->n_q,
-                                       cudaMemcpyDeviceToDevice, sA));
-        RopeRowsArgs rq = r;
-        rq.heads = a->hq; rq.in = y.q_new; rq.out = slot(l, Lo.o_qrot); rq.out_stride = a->T_new; rq.out_off = 0;
-        MSA_RETURN_IF(launch_rope_rows(rq, a->dt, sA));
-    }
-
-    // ---- R: routers back to back; S: selection as each router finishes
+    // ---- per layer, in enqueue order: prepass on A, router on R, selection on S (the first router
+    // is on the GPU after two launches of host time; the rest enqueue while it runs)
     for (int l = 0; l < L; ++l) {
         const msa_layer_args& y = a->layers[l];
         float* scores = reinterpret_cast<float*>(slot(l, Lo.o_scores));
+        MSA_RETURN_IF(route_prepare(plan, y.qr, slot(l, Lo.o_route), scores, a->n_docs, nullptr, a->n_chunks, sA));
+        MSA_CUDA_TRY(cudaEventRecord(P(l), sA));
         MSA_CUDA_TRY(cudaStreamWaitEvent(sR, P(l), 0));
         MSA_RETURN_IF(route_launch(plan, y.kr_index, a->n_chunks, a->chunk_doc, a->n_docs, slot(l, Lo.o_route), scores,
                                    nullptr, grid_cap, sR));
@@ -224,12 +219,37 @@ msa_status msa_interleave_step(const msa_interleave_args* a, void* compute, void
         MSA_CUDA_TRY(cudaStreamWaitEvent(sS, R(l), 0));
         int32_t* idx = reinterpret_cast<int32_t*>(slot(l, Lo.o_idx));
         MSA_RETURN_IF(msa_topk_docs(scores, a->n_q, a->n_docs, a->k, idx, nullptr, ws + Lo.off_topk, Lo.topk_ws, sS));
-        MSA_CUDA_TRY(cudaMemcpyAsync(y.topk_idx_host, idx, (size_t)a->n_q * a->k * sizeof(int32_t),
-                                     cudaMemcpyDeviceToHost, sS));
-        mem_len_kernel<<<(a->n_q + 127) / 128, 128, 0, sS>>>(idx, a->n_q, a->k, a->doc_chunk_off, a->n_docs, a->max_mem,
-                                                            reinterpret_cast<int32_t*>(slot(l, Lo.o_len)), err);
-        MSA_LAUNCH_CHECK();
-        MSA_CUDA_TRY(cudaEventRecord(E(l), sS));
+        if (a->fetch_mode == 1) {
+            // fetch right behind the selection on the device; the index copy to the host is output only
+            MSA_RETURN_IF(gather_device(y.host_bank, a->dt, a->n_chunks, a->doc_chunk_off, a->n_docs, idx, a->n_q, a->k,
+                                        a->hkv, a->d, a->max_mem, slot(l, Lo.o_mem),
+                                        reinterpret_cast<int32_t*>(slot(l, Lo.o_len)), sS));
+            MSA_CUDA_TRY(cudaEventRecord(E(l), sS));
+            MSA_CUDA_TRY(cudaMemcpyAsync(y.topk_idx_host, idx, (size_t)a->n_q * a->k * sizeof(int32_t),
+                                         cudaMemcpyDeviceToHost, sS));
+        } else {
+            MSA_CUDA_TRY(cudaMemcpyAsync(y.topk_idx_host, idx, (size_t)a->n_q * a->k * sizeof(int32_t),
+                                         cudaMemcpyDeviceToHost, sS));
+            mem_len_kernel<<<(a->n_q + 127) / 128, 128, 0, sS>>>(idx, a->n_q, a->k, a->doc_chunk_off, a->n_docs,
+                                                                a->max_mem, reinterpret_cast<int32_t*>(slot(l, Lo.o_len)),
+                                                                err);
+            MSA_LAUNCH_CHECK();
+            MSA_CUDA_TRY(cudaEventRecord(E(l), sS));
+        }
+    }
+
+    // ---- A: appends and query rotations of every layer, one launch per kMaxAppendLayers layers
+    for (int l0 = 0; l0 < L; l0 += kMaxAppendLayers) {
+        AppendArgs ap{};
+        ap.n_layers = std::min(kMaxAppendLayers, L - l0);
+        for (int i = 0; i < ap.n_layers; ++i) {
+            const msa_layer_args& y = a->layers[l0 + i];
+            ap.layer[i] = AppendLayer{y.k_new, y.v_new, y.q_new, y.local_k, y.local_v, slot(l0 + i, Lo.o_qrot)};
+        }
+        ap.n_q = a->n_q; ap.T_new = a->T_new; ap.new_q_stride = a->new_q_stride; ap.L_max = a->L_max;
+        ap.L_prev = a->L_prev; ap.hkv = a->hkv; ap.hq = a->hq; ap.d = a->d;
+        ap.pos_offset = (int64_t)a->k + a->L_prev; ap.cs = cs; ap.max_pos = a->rope_max_pos; ap.err = err;
+        MSA_RETURN_IF(launch_append(ap, a->dt, sA));
     }
 
     // ---- host: per layer, wait for its selection, fetch on C, attend on A
@@ -237,11 +257,16 @@ msa_status msa_interleave_step(const msa_interleave_args* a, void* compute, void
     std::vector<int32_t> mem_len_host((size_t)a->n_q);
     for (int l = 0; l < L; ++l) {
         const msa_layer_args& y = a->layers[l];
-        MSA_RETURN_IF(wait_event(E(l), deadline));
-        MSA_RETURN_IF(msa_gather_kv(y.host_bank, a->dt, a->n_chunks, a->doc_chunk_off_host, a->n_docs, y.topk_idx_host,
-                                    a->n_q, a->k, a->hkv, a->d, a->max_mem, slot(l, Lo.o_mem), mem_len_host.data(), sC));
-        MSA_CUDA_TRY(cudaEventRecord(G(l), sC));
-        MSA_CUDA_TRY(cudaStreamWaitEvent(sA, G(l), 0));
+        if (a->fetch_mode == 1) {
+            MSA_CUDA_TRY(cudaStreamWaitEvent(sA, E(l), 0));
+        } else {
+            MSA_RETURN_IF(wait_event(E(l), deadline));
+            MSA_RETURN_IF(msa_gather_kv(y.host_bank, a->dt, a->n_chunks, a->doc_chunk_off_host, a->n_docs,
+                                        y.topk_idx_host, a->n_q, a->k, a->hkv, a->d, a->max_mem, slot(l, Lo.o_mem),
+                                        mem_len_host.data(), sC));
+            MSA_CUDA_TRY(cudaEventRecord(G(l), sC));
+            MSA_CUDA_TRY(cudaStreamWaitEvent(sA, G(l), 0));
+        }
         MSA_RETURN_IF(msa_sparse_attn(slot(l, Lo.o_qrot), slot(l, Lo.o_mem),
                                       reinterpret_cast<const int32_t*>(slot(l, Lo.o_len)), a->max_mem, y.local_k,
                                       y.local_v, a->L_max, T_act, a->L_prev, a->n_q, a->T_new, a->hq, a->hkv, a->d,

@@ -98,8 +98,21 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restr
 
     List<KT> L;
     L.clear();
-    for (int64_t i = (int64_t)blockIdx.x * kTopkThreads + threadIdx.x; i < n_docs; i += (int64_t)P * kTopkThreads)
-        L.insert(row[i], (int)i);
+    // batches of independent loads first, then the inserts (no load waits behind an insert)
+    const int64_t stride = (int64_t)P * kTopkThreads;
+    for (int64_t i0 = (int64_t)blockIdx.x * kTopkThreads + threadIdx.x; i0 < n_docs; i0 += 8 * stride) {
+        float v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int64_t i = i0 + u * stride;
+            v[u] = i < n_docs ? __ldg(row + i) : -__int_as_float(0x7f800000);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int64_t i = i0 + u * stride;
+            if (i < n_docs) L.insert(v[u], (int)i);
+        }
+    }
     block_merge<KT>(L, ws, wi, res_s, res_i);
 
     float* my_s = part_s + ((int64_t)q * P + blockIdx.x) * KT;
@@ -114,10 +127,22 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restr
 
     L.clear();
     for (int l = threadIdx.x; l < P; l += kTopkThreads) {
-        const float* ps = part_s + ((int64_t)q * P + l) * KT;
-        const int* pi = part_i + ((int64_t)q * P + l) * KT;
+        // the whole list in 16-byte loads first, then inserts (lists are sorted best-first)
+        const float4* ps = reinterpret_cast<const float4*>(part_s + ((int64_t)q * P + l) * KT);
+        const int4* pi = reinterpret_cast<const int4*>(part_i + ((int64_t)q * P + l) * KT);
+        float cs[KT];
+        int ci[KT];
+#pragma unroll
+        for (int j = 0; j < KT / 4; ++j) {
+            const float4 a = __ldcg(ps + j);
+            const int4 b = __ldcg(pi + j);
+            cs[4 * j] = a.x; cs[4 * j + 1] = a.y; cs[4 * j + 2] = a.z; cs[4 * j + 3] = a.w;
+            ci[4 * j] = b.x; ci[4 * j + 1] = b.y; ci[4 * j + 2] = b.z; ci[4 * j + 3] = b.w;
+        }
+        bool more = true;
+#pragma unroll
         for (int j = 0; j < KT; ++j)
-            if (!L.insert(__ldcg(ps + j), __ldcg(pi + j))) break;   // lists are sorted best-first
+            if (more) more = L.insert(cs[j], ci[j]);
     }
     block_merge<KT>(L, ws, wi, res_s, res_i);
     if (threadIdx.x < k) {

@@ -12,9 +12,12 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def lib():
-    from routed_long_context_b200 import build
+    import importlib.util
 
-    build.build()
+    spec = importlib.util.spec_from_file_location("msa_build", os.path.join(ROOT, "routed_long_context_b200", "build.py"))
+    builder = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(builder)
+    builder.build()                      # rebuilds only when a source is newer than the library
     from routed_long_context_b200 import _lib
 
     return _lib.lib
@@ -103,7 +106,7 @@ def test_route_and_attention_reject_bad_shapes(lib):
                              ctypes.c_void_p(256), ctypes.c_void_p(256), 8, 9, 0, 1, 4, 8, 2, 128, 0.125,
                              ctypes.c_void_p(256), 0, None)
     assert st == 1
-    assert lib.msa_route_set_impl(3) == 1 and lib.msa_route_set_impl(0) == 0
+    assert lib.msa_route_set_impl(4) == 1 and lib.msa_route_set_impl(0) == 0
 
 
 def test_interleave_rejects_local_cache_overflow(lib):

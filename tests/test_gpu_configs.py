@@ -46,7 +46,7 @@ def _row_rel_err(got, ref):
     return float((num / den).max())
 
 
-def run_round(m, w, lay, layers_dev, rnd, cs, index, banks, local, outs, idx_host):
+def run_round(m, w, lay, layers_dev, rnd, cs, index, banks, local, outs, idx_host, fetch_mode=1):
     """Marshal one interleave round of workload w over its layers and run it."""
     L_prev, tn = w.round_tokens(rnd)
     T_act = L_prev + tn
@@ -61,7 +61,8 @@ def run_round(m, w, lay, layers_dev, rnd, cs, index, banks, local, outs, idx_hos
     r = m.InterleaveRound(layer_args, n_chunks=lay.n_chunks, n_docs=lay.n_docs, doc_chunk_off=lay.doc_chunk_off,
                           doc_chunk_off_host=lay.doc_chunk_off_host, chunk_doc=lay.chunk_doc, n_q=w.n_q, H=w.H, d=w.d,
                           hq=w.hq, hkv=w.hkv, k=w.k, L_prev=L_prev, T_new=tn, new_q_stride=w.T_total,
-                          L_max=w.T_total, max_mem=w.max_mem, cos_sin=cs, dtype=TORCH_DT[w.dtype])
+                          L_max=w.T_total, max_mem=w.max_mem, cos_sin=cs, dtype=TORCH_DT[w.dtype],
+                          fetch_mode=fetch_mode)
     r.run()
     torch.cuda.synchronize()
     del keep
@@ -80,7 +81,8 @@ def alloc_round_buffers(w, n_layers):
 
 
 # ------------------------------------------------------------------------------------------ tiny
-def test_tiny_end_to_end(m):
+@pytest.mark.parametrize("fetch_mode", [0, 1])
+def test_tiny_end_to_end(m, fetch_mode):
     from routed_long_context_b200.bank import BankLayout, encode_tokens, to_host_bank
 
     w = workloads.tiny()
@@ -91,7 +93,7 @@ def test_tiny_end_to_end(m):
     bank = to_host_bank(kvbar)
     dv = small_tensors(w, 0)
     local, outs, idx_host = alloc_round_buffers(w, 1)
-    run_round(m, w, lay, [dv], 0, cs, [index], [bank], local, outs, idx_host)
+    run_round(m, w, lay, [dv], 0, cs, [index], [bank], local, outs, idx_host, fetch_mode)
     assert m.device_status() == 0
 
     kb, vb, krb = O.encode_memory(k, v, kr, w.doc_tok_off, w.chunk, w.rope_base)
@@ -271,13 +273,14 @@ def oracle_bank_rows(w, layer, docs):
     return w.host_rows(layer, "bank", rows).reshape(len(rows), 2, w.hkv, w.d)
 
 
-def test_100m_two_layers_full_routing(m):
+@pytest.mark.parametrize("fetch_mode", [0, 1])
+def test_100m_two_layers_full_routing(m, fetch_mode):
     w = workloads.mem_100m(layers=2, n_host_banks=2)
     lay, index, banks = build_prepooled(m, w, 2)
     cs = m.rope_table(4096, w.d, w.rope_base)
     dvs = [small_tensors(w, l) for l in range(2)]
     local, outs, idx_host = alloc_round_buffers(w, 2)
-    run_round(m, w, lay, dvs, 0, cs, index, banks, local, outs, idx_host)
+    run_round(m, w, lay, dvs, 0, cs, index, banks, local, outs, idx_host, fetch_mode)
     assert m.device_status() == 0
     for l in range(2):
         ds_gpu = _np(m.msa_route_scores(index[l], lay.chunk_doc, lay.n_docs, dvs[l]["qr"]))

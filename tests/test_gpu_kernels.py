@@ -155,13 +155,13 @@ def test_route_fp32_cuda_cores(m, n_q, T):
 
 
 @pytest.mark.parametrize("n_q,T", [(1, 16), (1, 64), (2, 48), (3, 100), (32, 1), (8, 128), (1, 3)])
-@pytest.mark.parametrize("impl", [0, 1])
+@pytest.mark.parametrize("impl", [2, 1, 3])
 def test_route_bf16_tensor_cores_and_cuda_cores(m, n_q, T, impl):
     from routed_long_context_b200.bank import BankLayout
 
     counts, off, index, qr = _route_case(n_q * 1000 + T, n_q, T, "bf16")
     lay = BankLayout(counts)
-    m.route_set_impl(2 if impl == 0 else 1)
+    m.route_set_impl(impl)          # 2 tensor cores, 1 CUDA cores, 3 tensor cores with resident qhat
     try:
         ds, cs_ = m.msa_route_scores(upload(index, "bf16"), lay.chunk_doc, lay.n_docs, upload(qr, "bf16"),
                                      want_chunk_scores=True)
@@ -235,17 +235,24 @@ def _row_rel_err(got, ref):
     return (num / den).max()
 
 
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dtype,impl", [("f32", 0), ("bf16", 0), ("bf16", 1)])
 @pytest.mark.parametrize("hq,hkv", [(32, 8), (8, 8), (16, 8), (32, 4)])
-def test_sparse_attention(m, dtype, hq, hkv):
-    n_q, T, d, max_mem, q_start = 3, 13, 128, 40, 7
+@pytest.mark.parametrize("T,max_mem,mem_lens,q_start", [(13, 40, (0, 5, 37), 7), (37, 140, (130, 64, 1), 50)])
+def test_sparse_attention(m, dtype, impl, hq, hkv, T, max_mem, mem_lens, q_start):
+    """Both bf16 kernels (tensor cores, CUDA cores) and fp32; one key tile and several key tiles
+    with ragged tails, rows past the end of a 64-row block, empty memory."""
+    n_q, d = 3, 128
     L = q_start + T
     q = _gen(90, (n_q, T, hq, d), dtype)
     mem = _gen(91, (n_q, max_mem, 2, hkv, d), dtype)
     lk, lv = _gen(92, (n_q, L + 3, hkv, d), dtype), _gen(93, (n_q, L + 3, hkv, d), dtype)
-    mem_len = np.array([0, 5, 37], dtype=np.int32)
-    out = m.msa_sparse_attn(upload(q, dtype), upload(mem, dtype), torch.from_numpy(mem_len).cuda(), upload(lk, dtype),
-                            upload(lv, dtype), L, q_start)
+    mem_len = np.array(mem_lens, dtype=np.int32)
+    m.attn_set_impl(impl)
+    try:
+        out = m.msa_sparse_attn(upload(q, dtype), upload(mem, dtype), torch.from_numpy(mem_len).cuda(),
+                                upload(lk, dtype), upload(lv, dtype), L, q_start)
+    finally:
+        m.attn_set_impl(0)
     got = _np(out)
     tol = 1e-5 if dtype == "f32" else 2e-2
     for qi in range(n_q):
@@ -253,6 +260,30 @@ def test_sparse_attention(m, dtype, hq, hkv):
         ref = O.sparse_attention(q[qi], mem[qi, :ml, 0], mem[qi, :ml, 1], lk[qi, :L], lv[qi, :L], q_start,
                                  1 / np.sqrt(d))
         assert _row_rel_err(got[qi], ref) <= tol
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_device_gather_matches_host_gather(m, dtype):
+    counts = np.array([3, 1, 4, 0, 2, 5, 8, 8], dtype=np.int64)
+    off = np.concatenate([[0], np.cumsum(counts)])
+    tdt = torch.float32 if dtype == "f32" else torch.bfloat16
+    bank = torch.from_numpy(_gen(81, (int(off[-1]), 2, 8, 128), dtype)).to(tdt).pin_memory()
+    idx = torch.tensor([[2, 0, 5], [3, 1, 4], [7, 6, 0]], dtype=torch.int32)
+    ref, ref_len = m.msa_gather_kv(bank, off, idx, max_mem=20)
+    dev, dev_len = m.msa_gather_kv_device(bank, torch.from_numpy(off).cuda(), idx.cuda(), max_mem=20)
+    torch.cuda.synchronize()
+    assert dev_len.cpu().tolist() == ref_len.tolist() == [12, 3, 19]
+    for q, n in enumerate(ref_len.tolist()):
+        assert torch.equal(dev[q, :n].cpu(), ref[q, :n].cpu())
+    _status(m)
+
+
+def test_device_gather_flags_bad_index_without_faulting(m):
+    bank = torch.zeros((10, 2, 8, 128), dtype=torch.bfloat16).pin_memory()
+    off = torch.tensor([0, 4, 10], dtype=torch.int64, device="cuda")
+    idx = torch.tensor([[1, 5]], dtype=torch.int32, device="cuda")     # doc 5 does not exist
+    m.msa_gather_kv_device(bank, off, idx, max_mem=16)
+    assert m.device_status() == 3                                      # MSA_DEV_BAD_INDEX
 
 
 def test_sparse_attention_no_keys_gives_zero(m):
