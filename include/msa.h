@@ -151,6 +151,12 @@ msa_status msa_route_set_impl(int impl);
  * attention block and one top-k block running concurrently). Process-wide. */
 msa_status msa_route_set_max_stages(int n);
 
+/* Failure-detection test hook of the tensor-core router: while on, each launch's producer
+ * publishes no tile and issues no copy, so the other warps' bounded waits expire (about 2 s); the
+ * kernel then records MSA_DEV_WAIT_TIMEOUT, frees its tensor memory and returns, leaving the
+ * context usable. Scores written by such launches are meaningless. Process-wide. */
+msa_status msa_route_inject_stall(int on);
+
 /* Top-k document selection ([P1] §组件 1; [P2] Top-k 选择机制): for every query the k documents
  * with the largest doc_scores, in descending score order, ties broken by the lower document
  * index. doc_scores: device float [n_q][n_docs]; idx: device int32 [n_q][k]; score: device
@@ -257,6 +263,9 @@ typedef struct msa_interleave_args {
     float scale;                    /* attention scale, normally 1/sqrt(d) */
     int reserved_sms;               /* SMs the router kernels leave free for the overlapped selection
                                        and attention of earlier layers (0 = routers use every SM) */
+    void* const* route_events;      /* optional (NULL = none): 2 * n_layers cudaEvent_t created by the
+                                       caller; [2l] and [2l+1] are recorded on `compute` just before and
+                                       after layer l's router kernel, to time it inside the round */
     int fetch_mode;                 /* 0: the host waits for each layer's selection and issues one
                                        cudaMemcpyAsync per document on `copy` (msa_gather_kv);
                                        1: a device kernel fetches from the mapped pinned bank right

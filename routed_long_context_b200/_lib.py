@@ -29,7 +29,8 @@ class InterleaveArgs(ctypes.Structure):
                 ("hq", ctypes.c_int), ("hkv", ctypes.c_int), ("k", ctypes.c_int), ("L_prev", ctypes.c_int),
                 ("T_new", ctypes.c_int), ("new_q_stride", ctypes.c_int), ("L_max", ctypes.c_int),
                 ("max_mem", ctypes.c_int), ("rope_cos_sin", vp), ("rope_max_pos", i64), ("scale", f32),
-                ("reserved_sms", ctypes.c_int), ("fetch_mode", ctypes.c_int), ("ws", vp), ("ws_bytes", sz)]
+                ("reserved_sms", ctypes.c_int), ("route_events", vp), ("fetch_mode", ctypes.c_int),
+                ("ws", vp), ("ws_bytes", sz)]
 
 
 # name -> (restype, argtypes)
@@ -48,6 +49,7 @@ SIGNATURES = {
                                        ctypes.POINTER(sz)]),
     "msa_route_set_impl": (i32, [ctypes.c_int]),
     "msa_route_set_max_stages": (i32, [ctypes.c_int]),
+    "msa_route_inject_stall": (i32, [ctypes.c_int]),
     "msa_topk_docs": (i32, [vp, ctypes.c_int, i64, ctypes.c_int, vp, vp, vp, sz, vp]),
     "msa_topk_workspace_size": (i32, [ctypes.c_int, i64, ctypes.c_int, ctypes.POINTER(sz)]),
     "msa_topk_docs_noalloc": (i32, [vp, ctypes.c_int, i64, ctypes.c_int, vp, vp, vp]),

@@ -249,9 +249,18 @@ class InterleaveRound:
         self.ws = _ws(need.value, doc_chunk_off.device) if ws is None else ws
         a.ws, a.ws_bytes = self.ws.data_ptr(), self.ws.numel()
 
-    def run(self, compute=None, copy=None, timeout_us: int = 30_000_000) -> None:
+    def run(self, compute=None, copy=None, timeout_us: int = 30_000_000, route_events=None) -> None:
+        """route_events: optional list of 2 * n_layers torch.cuda.Event(enable_timing=True), recorded around
+        each layer's router kernel on the compute stream."""
+        if route_events is not None:
+            arr = (ctypes.c_void_p * len(route_events))(*[e.cuda_event for e in route_events])
+            self.args.route_events = ctypes.cast(arr, ctypes.c_void_p)
+        else:
+            arr = None
+            self.args.route_events = None
         check(lib.msa_interleave_step(ctypes.byref(self.args), _stream(compute), _stream(copy), timeout_us),
               "msa_interleave_step")
+        del arr
 
 
 def msa_interleave_step(layers, compute=None, copy=None, timeout_us: int = 30_000_000, **kw) -> InterleaveRound:

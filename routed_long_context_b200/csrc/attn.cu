@@ -273,21 +273,26 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnArgs a) {
 
     for (int kb = 0; kb < n_keys; kb += kMmaKeys) {
         __syncthreads();
-        // stage 64 keys and values: 16-byte vectors, zeros past the visible range
+        // stage 64 keys and values with asynchronous 16-byte copies (all in flight at once);
+        // rows past the visible range are zero-filled without reading
         for (int v = threadIdx.x; v < kMmaKeys * (kD / 8) * 2; v += blockDim.x) {
             const int which = v / (kMmaKeys * (kD / 8));
             const int rem = v % (kMmaKeys * (kD / 8));
             const int r = rem / (kD / 8), c = (rem % (kD / 8)) * 8;
             const int kk = kb + r;
-            uint4 x = make_uint4(0, 0, 0, 0);
-            if (kk < mem_len)
-                x = *reinterpret_cast<const uint4*>(MKV + (((int64_t)qi * a.max_mem + kk) * 2 + which) * a.hkv * kD +
-                                                    g * kD + c);
-            else if (kk < n_keys)
-                x = *reinterpret_cast<const uint4*>((which ? LV : LK) +
-                                                    (((int64_t)qi * a.L_max + (kk - mem_len)) * a.hkv + g) * kD + c);
-            *reinterpret_cast<uint4*>(which ? &Vs[r][c] : &Ks[r][c]) = x;
+            const __nv_bfloat16* src = Q;     // any valid address: zero-filled copies read nothing
+            uint32_t bytes = 0;
+            if (kk < mem_len) {
+                src = MKV + (((int64_t)qi * a.max_mem + kk) * 2 + which) * a.hkv * kD + g * kD + c;
+                bytes = 16;
+            } else if (kk < n_keys) {
+                src = (which ? LV : LK) + (((int64_t)qi * a.L_max + (kk - mem_len)) * a.hkv + g) * kD + c;
+                bytes = 16;
+            }
+            const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(which ? &Vs[r][c] : &Ks[r][c]));
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(bytes) : "memory");
         }
+        asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
         __syncthreads();
 
         // S = Q K^T for 8 blocks of 8 keys

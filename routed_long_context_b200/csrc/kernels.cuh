@@ -74,6 +74,8 @@ msa_status launch_route_tc(const RouteTcArgs& a, cudaStream_t s);
 int route_tc_pad_rows(int N, int K, bool resident = false);
 // Testing knob: cap on the router's pipeline stages (0 = as many as the shared-memory budget allows).
 void route_tc_set_max_stages(int n);
+// Testing knob: launches withhold every tile so their bounded waits expire (MSA_DEV_WAIT_TIMEOUT).
+void route_tc_inject_stall(int on);
 
 // Router scoring split in two launches so a caller can hoist the (tiny) query prepass off the
 // router's stream: route_prepare normalises the queries into qhat and fills the score outputs with

@@ -251,6 +251,12 @@ msa_status msa_route_set_impl(int impl) {
     return MSA_OK;
 }
 
+msa_status msa_route_inject_stall(int on) {
+    MSA_REQUIRE(on == 0 || on == 1, "msa_route_inject_stall: on must be 0 or 1");
+    route_tc_inject_stall(on);
+    return MSA_OK;
+}
+
 msa_status msa_route_set_max_stages(int n) {
     MSA_REQUIRE(n >= 0 && n <= 12, "msa_route_set_max_stages: n must be in [0, 12]");
     route_tc_set_max_stages(n);

@@ -40,6 +40,7 @@ constexpr int kSmemLimit = 232448;    // max dynamic shared memory per block on 
 // (35 KB) and one top-k block (5 KB) of the overlapped selection/attention of earlier layers.
 constexpr int kSmemBudget = 188 * 1024;
 std::atomic<int> g_max_stages{0};     // testing knob: 0 = as many stages as the budget allows
+std::atomic<int> g_inject_stall{0};   // testing knob: make the next launches' waits time out
 constexpr int kStageA = BM * BK * 2;  // 16 KB
 constexpr uint64_t kWaitNs = 2000000000ull;
 
@@ -57,6 +58,7 @@ struct TcParams {
     float* chunk_scores;
     int* err;
     int* tile_counter;     // zero at launch; tiles are handed out in order by atomicAdd
+    int inject_stall;      // testing: the producer never publishes a tile, so every other wait times out
 };
 
 // ---------------------------------------------------------------------------------- PTX helpers
@@ -245,6 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = false;
                     break;
                 }
+                if (p.inject_stall) break;     // nothing issued: the consumers' bounded waits run out
                 const int t = atomicAdd(p.tile_counter, 1);
                 const int tile = (int64_t)t < p.n_tiles ? t : -1;
                 tile_q[tslot] = tile;
@@ -524,6 +527,7 @@ msa_status allow_max_smem() {
 }  // namespace
 
 void route_tc_set_max_stages(int n) { g_max_stages.store(n); }
+void route_tc_inject_stall(int on) { g_inject_stall.store(on); }
 
 int route_tc_pad_rows(int N, int K, bool resident) {
     Plan pl;
@@ -556,6 +560,7 @@ msa_status launch_route_tc(const RouteTcArgs& a, cudaStream_t s) {
     p.chunk_doc = a.chunk_doc; p.n_docs = a.n_docs; p.doc_scores = a.doc_scores; p.chunk_scores = a.chunk_scores;
     p.err = a.err;
     p.tile_counter = a.tile_counter;
+    p.inject_stall = g_inject_stall.load();
     if (!p.tile_counter) return set_error(MSA_ERR_INVALID_ARG, "route (tensor cores): no tile counter");
     int64_t grid = p.n_tiles < (int64_t)sm_count() ? p.n_tiles : (int64_t)sm_count();
     if (a.grid_cap > 0 && grid > a.grid_cap) grid = a.grid_cap;

@@ -212,8 +212,10 @@ msa_status msa_interleave_step(const msa_interleave_args* a, void* compute, void
         MSA_RETURN_IF(route_prepare(plan, y.qr, slot(l, Lo.o_route), scores, a->n_docs, nullptr, a->n_chunks, sA));
         MSA_CUDA_TRY(cudaEventRecord(P(l), sA));
         MSA_CUDA_TRY(cudaStreamWaitEvent(sR, P(l), 0));
+        if (a->route_events) MSA_CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(a->route_events[2 * l]), sR));
         MSA_RETURN_IF(route_launch(plan, y.kr_index, a->n_chunks, a->chunk_doc, a->n_docs, slot(l, Lo.o_route), scores,
                                    nullptr, grid_cap, sR));
+        if (a->route_events) MSA_CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(a->route_events[2 * l + 1]), sR));
         MSA_CUDA_TRY(cudaEventRecord(R(l), sR));
 
         MSA_CUDA_TRY(cudaStreamWaitEvent(sS, R(l), 0));

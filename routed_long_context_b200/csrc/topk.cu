@@ -1,4 +1,5 @@
-// Top-k document selection over doc_scores [n_q][n_docs].
+// Top-k document selection over doc_scores [n_q][n_docs]. k <= 32 uses warp-distributed lists
+// (topk_warp_kernel below); larger k uses per-thread lists merged by tournaments.
 //
 // Order: descending score, ties to the lower document index (a strict total order, so the
 // result is unique). One launch: P blocks per query each keep a per-thread sorted list of the
@@ -161,6 +162,176 @@ int pick_blocks(int64_t n_docs) {
     return (int)p;
 }
 
+
+// ------------------------------------------------------------------------------------------------
+// k <= 32: warp-distributed lists. Lane i of a warp holds rank i of the warp's sorted list
+// (lanes >= k hold sentinels). A batch of 32 candidates (one per lane) is filtered against the
+// list's k-th entry with one ballot; each survivor is inserted by a rank count (popc of a ballot)
+// and a one-lane shift. Per block: each warp scans a strided slice, then warp 0 folds the other
+// warps' lists in; the last block of a query (atomic ticket) folds the per-block lists.
+// ------------------------------------------------------------------------------------------------
+struct WList {
+    float s;
+    int i;
+};
+
+__device__ __forceinline__ void wl_clear(WList& w) {
+    w.s = -__int_as_float(0x7f800000);
+    w.i = INT_MAX;
+}
+
+// One compare-exchange step of a warp-wide bitonic network on (score, id) pairs: this lane keeps
+// the better of itself and lane ^ j when keep_better, else the worse.
+__device__ __forceinline__ void cmpx(float& s, int& i, int j, bool keep_better) {
+    const float ps = __shfl_xor_sync(0xffffffffu, s, j);
+    const int pi = __shfl_xor_sync(0xffffffffu, i, j);
+    const bool partner_better = better(ps, pi, s, i);
+    if (partner_better == keep_better) {
+        s = ps;
+        i = pi;
+    }
+}
+
+// Sorts the 32 lanes' pairs best-first (bitonic sort, 15 stages).
+__device__ __forceinline__ void warp_sort32(float& s, int& i) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int k = 2; k <= 32; k <<= 1)
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) cmpx(s, i, j, ((lane & j) == 0) == ((lane & k) == 0));
+}
+
+// w (sorted best-first) <- the 32 best of w and b (b sorted best-first): the half-cleaner on w and
+// reversed b leaves the 32 best as a bitonic sequence, which a 5-stage bitonic merge sorts.
+__device__ __forceinline__ void warp_merge32(WList& w, float bs, int bi) {
+    const int lane = threadIdx.x & 31;
+    const float rs = __shfl_sync(0xffffffffu, bs, 31 - lane);
+    const int ri = __shfl_sync(0xffffffffu, bi, 31 - lane);
+    if (better(rs, ri, w.s, w.i)) {
+        w.s = rs;
+        w.i = ri;
+    }
+#pragma unroll
+    for (int j = 16; j > 0; j >>= 1) cmpx(w.s, w.i, j, (lane & j) == 0);
+}
+
+// Inserts every lane's candidate (cv, ci) that beats the list's k-th entry; valid marks real ones.
+// One or two survivors go in by rank count and shift; more are sorted and merged in one go.
+__device__ __forceinline__ void wl_insert_batch(WList& w, int k, float cv, int ci, bool valid) {
+    const int lane = threadIdx.x & 31;
+    float ts = __shfl_sync(0xffffffffu, w.s, k - 1);
+    int ti = __shfl_sync(0xffffffffu, w.i, k - 1);
+    unsigned mask = __ballot_sync(0xffffffffu, valid && better(cv, ci, ts, ti));
+    if (__popc(mask) > 2) {
+        float s = (mask >> lane) & 1u ? cv : -__int_as_float(0x7f800000);
+        int i = (mask >> lane) & 1u ? ci : INT_MAX;
+        warp_sort32(s, i);
+        warp_merge32(w, s, i);
+        return;
+    }
+    while (mask) {
+        const int j = __ffs(mask) - 1;
+        const float s = __shfl_sync(0xffffffffu, cv, j);
+        const int id = __shfl_sync(0xffffffffu, ci, j);
+        const bool ahead = lane < k && better(w.s, w.i, s, id);
+        const int pos = __popc(__ballot_sync(0xffffffffu, ahead));
+        const float ps = __shfl_up_sync(0xffffffffu, w.s, 1);
+        const int pi = __shfl_up_sync(0xffffffffu, w.i, 1);
+        if (lane == pos) {
+            w.s = s;
+            w.i = id;
+        } else if (lane > pos && lane < k) {
+            w.s = ps;
+            w.i = pi;
+        }
+        ts = __shfl_sync(0xffffffffu, w.s, k - 1);
+        ti = __shfl_sync(0xffffffffu, w.i, k - 1);
+        mask &= ~(1u << j);
+        mask &= __ballot_sync(0xffffffffu, valid && better(cv, ci, ts, ti));
+    }
+}
+
+constexpr int kWarpTopkThreads = 256;
+
+__global__ void __launch_bounds__(kWarpTopkThreads) topk_warp_kernel(const float* __restrict__ scores, int64_t n_docs,
+                                                                      int k, int P, float* part_s, int* part_i,
+                                                                      int* counters, int32_t* out_idx, float* out_score) {
+    constexpr int W = kWarpTopkThreads / 32;
+    __shared__ float ls[W][32];
+    __shared__ int li[W][32];
+    __shared__ int is_last;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int q = blockIdx.y;
+    const float* row = scores + (int64_t)q * n_docs;
+    WList w;
+    wl_clear(w);
+    // this warp's slice: chunks of 32 consecutive docs, strided over all warps of all blocks
+    const int64_t gw = (int64_t)blockIdx.x * W + warp, nw = (int64_t)P * W;
+    for (int64_t base = gw * 32; base < n_docs; base += nw * 32 * 8) {
+        float v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int64_t i = base + u * nw * 32 + lane;
+            v[u] = i < n_docs ? __ldg(row + i) : -__int_as_float(0x7f800000);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int64_t i = base + u * nw * 32 + lane;
+            wl_insert_batch(w, k, v[u], (int)i, i < n_docs);
+        }
+    }
+    // fold the block's warp lists (sorted) into warp 0's
+    ls[warp][lane] = w.s;
+    li[warp][lane] = w.i;
+    __syncthreads();
+    if (warp == 0) {
+        for (int o = 1; o < W; ++o) warp_merge32(w, ls[o][lane], li[o][lane]);
+        part_s[((int64_t)q * P + blockIdx.x) * 32 + lane] = w.s;
+        part_i[((int64_t)q * P + blockIdx.x) * 32 + lane] = w.i;
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) is_last = (atomicAdd(counters + q, 1) == P - 1);
+    }
+    __syncthreads();
+    if (!is_last) return;
+    // last block: warp w folds partial lists w, w + W, ... (loads first), then warp 0 folds the warps
+    __threadfence();
+    wl_clear(w);
+    for (int b0 = warp; b0 < P; b0 += 4 * W) {
+        float cv[4];
+        int ci[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int b = b0 + u * W;
+            const int64_t off = ((int64_t)q * P + b) * 32 + lane;
+            cv[u] = b < P ? __ldcg(part_s + off) : -__int_as_float(0x7f800000);
+            ci[u] = b < P ? __ldcg(part_i + off) : INT_MAX;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (b0 + u * W < P) warp_merge32(w, cv[u], ci[u]);
+    }
+    __syncthreads();
+    ls[warp][lane] = w.s;
+    li[warp][lane] = w.i;
+    __syncthreads();
+    if (warp == 0) {
+        for (int o = 1; o < W; ++o) warp_merge32(w, ls[o][lane], li[o][lane]);
+        if (lane < k) {
+            out_idx[(int64_t)q * k + lane] = w.i;
+            if (out_score) out_score[(int64_t)q * k + lane] = w.s;
+        }
+    }
+}
+
+int pick_blocks_warp(int64_t n_docs) {
+    // about 16 batches of 32 docs per warp: few partial lists for the last block to fold
+    int64_t p = (n_docs + kWarpTopkThreads * 16 - 1) / (kWarpTopkThreads * 16);
+    const int64_t cap = (int64_t)sm_count() * 2;
+    if (p > cap) p = cap;
+    if (p < 1) p = 1;
+    return (int)p;
+}
 }  // namespace
 }  // namespace msa
 
@@ -171,7 +342,9 @@ extern "C" {
 msa_status msa_topk_workspace_size(int n_q, int64_t n_docs, int k, size_t* bytes) {
     MSA_REQUIRE(bytes, "msa_topk_workspace_size: bytes is NULL");
     MSA_REQUIRE(n_q > 0 && n_docs > 0 && k > 0 && k <= 64, "msa_topk_workspace_size: bad sizes");
-    const int P = pick_blocks(n_docs), KT = pick_kt(k);
+    const bool warp_lists = k <= 32;
+    const int P = warp_lists ? pick_blocks_warp(n_docs) : pick_blocks(n_docs);
+    const int KT = warp_lists ? 32 : pick_kt(k);
     const size_t lists = (size_t)n_q * P * KT;
     *bytes = align_up(lists * 4, 256) * 2 + align_up((size_t)n_q * 4, 256);
     return MSA_OK;
@@ -186,7 +359,9 @@ msa_status msa_topk_docs(const float* doc_scores, int n_q, int64_t n_docs, int k
     size_t need = 0;
     MSA_RETURN_IF(msa_topk_workspace_size(n_q, n_docs, k, &need));
     if (ws_bytes < need) return set_error(MSA_ERR_WORKSPACE, "msa_topk_docs: workspace %zu < %zu", ws_bytes, need);
-    const int P = pick_blocks(n_docs), KT = pick_kt(k);
+    const bool warp_lists = k <= 32;
+    const int P = warp_lists ? pick_blocks_warp(n_docs) : pick_blocks(n_docs);
+    const int KT = warp_lists ? 32 : pick_kt(k);
     const size_t lists = (size_t)n_q * P * KT;
     char* w = static_cast<char*>(ws);
     float* part_s = reinterpret_cast<float*>(w);
@@ -195,6 +370,11 @@ msa_status msa_topk_docs(const float* doc_scores, int n_q, int64_t n_docs, int k
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     MSA_CUDA_TRY(cudaMemsetAsync(counters, 0, (size_t)n_q * sizeof(int), s));
     dim3 grid(P, n_q);
+    if (warp_lists) {
+        topk_warp_kernel<<<grid, kWarpTopkThreads, 0, s>>>(doc_scores, n_docs, k, P, part_s, part_i, counters, idx, score);
+        MSA_LAUNCH_CHECK();
+        return MSA_OK;
+    }
     switch (KT) {
         case 8: topk_kernel<8><<<grid, kTopkThreads, 0, s>>>(doc_scores, n_docs, k, P, part_s, part_i, counters, idx, score); break;
         case 16: topk_kernel<16><<<grid, kTopkThreads, 0, s>>>(doc_scores, n_docs, k, P, part_s, part_i, counters, idx, score); break;
@@ -269,7 +449,9 @@ msa_status msa_topk_docs_noalloc(const float* doc_scores, int n_q, int64_t n_doc
                          n_q, (long long)n_docs, k, need, kNoAllocScratchBytes);
     void* ws = nullptr;
     MSA_RETURN_IF(scratch_address(&ws));
-    const int P = pick_blocks(n_docs), KT = pick_kt(k);
+    const bool warp_lists = k <= 32;
+    const int P = warp_lists ? pick_blocks_warp(n_docs) : pick_blocks(n_docs);
+    const int KT = warp_lists ? 32 : pick_kt(k);
     const size_t lists = (size_t)n_q * P * KT;
     char* w = static_cast<char*>(ws);
     float* part_s = reinterpret_cast<float*>(w);
@@ -279,6 +461,11 @@ msa_status msa_topk_docs_noalloc(const float* doc_scores, int n_q, int64_t n_doc
     // the array keeps the previous call's contents: the tickets must start at zero
     MSA_CUDA_TRY(cudaMemsetAsync(counters, 0, (size_t)n_q * sizeof(int), s));
     dim3 grid(P, n_q);
+    if (warp_lists) {
+        topk_warp_kernel<<<grid, kWarpTopkThreads, 0, s>>>(doc_scores, n_docs, k, P, part_s, part_i, counters, idx, score);
+        MSA_LAUNCH_CHECK();
+        return MSA_OK;
+    }
     switch (KT) {
         case 8: topk_kernel<8><<<grid, kTopkThreads, 0, s>>>(doc_scores, n_docs, k, P, part_s, part_i, counters, idx, score); break;
         case 16: topk_kernel<16><<<grid, kTopkThreads, 0, s>>>(doc_scores, n_docs, k, P, part_s, part_i, counters, idx, score); break;
