@@ -44,9 +44,11 @@ def parse():
                     help="SMs the routers leave free for the overlapped selection and attention")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="100m", choices=["100m", "encode10m"],
+    ap.add_argument("--workload", default="100m", choices=["100m", "encode10m", "interleave"],
                     help="100m: the routing step (the reported metric); encode10m: offline encoding of the "
-                         "10M-token bank (document-wise RoPE + chunk-mean pooling), reported separately")
+                         "10M-token bank (document-wise RoPE + chunk-mean pooling); interleave: three Memory "
+                         "Interleave rounds over a 10M-token bank (tensor-bound routing); the last two are "
+                         "reported separately")
     return ap.parse_args()
 
 
@@ -229,6 +231,99 @@ def encode_bench(args, rank, world, local_rank):
             "clocks": clk.summary(), "device_status": m.device_status()}))
 
 
+# ---------------------------------------------------------------------------------------------- interleave
+def interleave_bench(args, rank, world, local_rank):
+    """Three Memory Interleave rounds (64 + 32 + 32 tokens per query, 8 queries) over a 10M-token
+    pre-pooled bank (78,128 chunks of 128) and 18 routed layers; one step = the three rounds."""
+    import torch
+
+    import routed_long_context_b200 as m
+    from msa_inputs import workloads
+    from msa_inputs.device import memory_tensor, small_tensors
+    from routed_long_context_b200.bank import BankLayout, index_from_prepooled
+
+    torch.cuda.set_device(local_rank)
+    w = workloads.interleave(layers=args.layers, n_host_banks=args.host_banks)
+    lay = BankLayout(w.doc_chunks)
+    cs = m.rope_table(4096, w.d, w.rope_base)
+    dt = torch.bfloat16
+    index = [index_from_prepooled(lay, memory_tensor(w, l, "krbar")) for l in range(w.layers)]
+    banks = []
+    for s_ in range(w.n_host_banks):
+        dev = memory_tensor(w, s_, "bank")
+        h = torch.empty(dev.shape, dtype=dt, pin_memory=True)
+        h.copy_(dev)
+        banks.append(h)
+        del dev
+    small = [small_tensors(w, l) for l in range(w.layers)]
+    qr_round = [[small[l]["qr"][:, :w.round_tokens(r)[0] + w.round_tokens(r)[1]].contiguous() for r in range(w.rounds)]
+                for l in range(w.layers)]
+    local = [(torch.zeros((w.n_q, w.T_total, w.hkv, w.d), dtype=dt, device="cuda"),
+              torch.zeros((w.n_q, w.T_total, w.hkv, w.d), dtype=dt, device="cuda")) for _ in range(w.layers)]
+    outs = [[torch.empty((w.n_q, w.round_tokens(r)[1], w.hq, w.d), dtype=dt, device="cuda") for r in range(w.rounds)]
+            for _ in range(w.layers)]
+    idx_host = [[torch.empty((w.n_q, w.k), dtype=torch.int32, pin_memory=True) for _ in range(w.rounds)]
+                for _ in range(w.layers)]
+    compute, copy = torch.cuda.Stream(), torch.cuda.Stream()
+    rounds = []
+    for r in range(w.rounds):
+        L_prev, tn = w.round_tokens(r)
+        la = [dict(kr_index=index[l], host_bank=banks[w.host_bank_slot(l)], qr=qr_round[l][r],
+                   q_new=small[l]["q"][:, L_prev:], k_new=small[l]["k_new"][:, L_prev:],
+                   v_new=small[l]["v_new"][:, L_prev:], local_k=local[l][0], local_v=local[l][1], out=outs[l][r],
+                   topk_idx_host=idx_host[l][r]) for l in range(w.layers)]
+        rounds.append(m.InterleaveRound(la, n_chunks=lay.n_chunks, n_docs=lay.n_docs, doc_chunk_off=lay.doc_chunk_off,
+                                        doc_chunk_off_host=lay.doc_chunk_off_host, chunk_doc=lay.chunk_doc, n_q=w.n_q,
+                                        H=w.H, d=w.d, hq=w.hq, hkv=w.hkv, k=w.k, L_prev=L_prev, T_new=tn,
+                                        new_q_stride=w.T_total, L_max=w.T_total, max_mem=w.max_mem, cos_sin=cs,
+                                        dtype=dt, fetch_mode=args.fetch_mode))
+    for _ in range(args.warmup):
+        for rd in rounds:
+            rd.run(compute, copy)
+    torch.cuda.synchronize()
+    chain_ok = all(set(w.expected(l, r, q)) <= set(idx_host[l][r][q].tolist())
+                   for l in range(w.layers) for r in range(w.rounds) for q in range(w.n_q))
+    route_ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(2 * w.layers)] for _ in range(w.rounds)]
+                for _ in range(args.steps)]
+    for a in route_ev:
+        for b in a:
+            for e in b:
+                e.record(compute)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        e0.record(compute)
+        for i in range(args.steps):
+            for r, rd in enumerate(rounds):
+                rd.run(compute, copy, route_events=route_ev[i][r])
+        e1.record(compute)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    # router FLOPs per launch: 2 * (H*d) * chunks * (n_q * routing tokens of the round)
+    flops = [2.0 * w.H * w.d * lay.n_chunks * w.n_q * sum(w.round_tokens(r)) for r in range(w.rounds)]
+    rms = [sum(route_ev[i][r][2 * l].elapsed_time(route_ev[i][r][2 * l + 1]) for i in range(args.steps)
+               for l in range(w.layers)) / (args.steps * w.layers) for r in range(w.rounds)]
+    tflops = [f / (t / 1e3) / 1e12 for f, t in zip(flops, rms)]
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peak, kind = float(json.load(f)["bf16_tflops_sustained"]), "measured sustained bf16 (cuBLAS)"
+    except Exception:
+        peak, kind = 1400.0, "fallback sustained bf16"
+    if rank == 0:
+        tokens = lay.n_chunks * TOKENS_PER_CHUNK * w.layers * w.rounds
+        print(json.dumps({
+            "metric": "Memory Interleave: memory tokens routed/s (3 rounds x 18 layers over a 10M-token bank)",
+            "value": tokens / (ms / 1e3), "unit": "memory tokens/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "interleave: 78,128 chunks x 18 layers, 8 queries, 64/96/128 routing tokens, top-12"},
+            "route_ms_per_layer_by_round": rms, "route_tflops_by_round": tflops,
+            "roofline": {"bound": "tensor", "achieved": tflops[-1], "peak": peak, "unit": "TFLOP/s",
+                         "frac": tflops[-1] / peak, "traffic": None, "kernel": "route_tc_kernel, round 3 (1,024 columns)",
+                         "peak_kind": kind},
+            "checks": {"chain_docs_selected": chain_ok, "device_status": m.device_status()},
+            "clocks": clk.summary()}))
+
+
 # ---------------------------------------------------------------------------------------------- ours
 def main():
     args = parse()
@@ -239,6 +334,8 @@ def main():
         return reference_arm(args, rank)
     if args.workload == "encode10m":
         return encode_bench(args, rank, world, local_rank)
+    if args.workload == "interleave":
+        return interleave_bench(args, rank, world, local_rank)
 
     import numpy as np
     import torch

@@ -11,6 +11,7 @@ namespace msa {
 namespace {
 
 constexpr int kPoolThreads = 128;
+constexpr int kPoolUnroll = 8;   // 16-byte loads in flight per thread
 
 template <typename T>
 __device__ __forceinline__ uint4 load_stream(const T* p) {
@@ -145,12 +146,29 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const PoolArgs a) {
 
             const uint4 zero = make_uint4(0, 0, 0, 0);
             int64_t t = t0;
-            for (; t + 4 <= t1; t += 4) {
-                uint4 r[4];
+            if (rope) {
+                // rotated keys: 4 tokens in flight (the rotation's table reads and registers dominate)
+                for (; t + 4 <= t1; t += 4) {
+                    uint4 r[4];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) r[u] = active ? load_stream(src + (t + u) * E + e0) : zero;
+                    for (int u = 0; u < 4; ++u) r[u] = active ? load_stream(src + (t + u) * E + e0) : zero;
 #pragma unroll
-                for (int u = 0; u < 4; ++u) consume(r[u], t + u);
+                    for (int u = 0; u < 4; ++u) consume(r[u], t + u);
+                }
+            } else {
+                // plain streaming: kPoolUnroll tokens in flight
+                for (; t + kPoolUnroll <= t1; t += kPoolUnroll) {
+                    uint4 r[kPoolUnroll];
+#pragma unroll
+                    for (int u = 0; u < kPoolUnroll; ++u) r[u] = active ? load_stream(src + (t + u) * E + e0) : zero;
+#pragma unroll
+                    for (int u = 0; u < kPoolUnroll; ++u) {
+                        float x[VEC];
+                        widen<TIn>(r[u], x);
+#pragma unroll
+                        for (int j = 0; j < VEC; ++j) acc[j] += x[j];
+                    }
+                }
             }
             for (; t < t1; ++t) {
                 uint4 r = active ? load_stream(src + t * E + e0) : zero;
