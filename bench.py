@@ -196,7 +196,7 @@ def encode_bench(args, rank, world, local_rank):
     from routed_long_context_b200.bank import BankLayout, encode_tokens
 
     torch.cuda.set_device(local_rank)
-    w = workloads.mem_10m()
+    w = workloads.mem_10m(n_docs=9766 if args.n_docs == 97657 else args.n_docs)
     lay = BankLayout.from_doc_lengths(w.doc_len, w.chunk)
     cs = m.rope_table(4096, w.d, w.rope_base)
     k, v, kr = (memory_tensor(w, 0, n) for n in ("k", "v", "kr"))
@@ -225,7 +225,8 @@ def encode_bench(args, rank, world, local_rank):
             "metric": "10M-token offline encode (doc-wise RoPE + chunk-mean pooling) throughput", "value": w.n_tok / (ms / 1e3),
             "unit": "memory tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "encode10m: 9,766 docs x 1024 tokens, chunk 256, K/V/K^R bf16 [10,000,384 x 8 x 128]"},
+            "config": {"workload": f"encode10m: {w.n_docs:,} docs x 1024 tokens, chunk 256, K/V/K^R bf16 "
+                                   f"[{w.n_tok:,} x 8 x 128]"},
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
                          "traffic": None, "kernel": "pool_kernel", "peak_kind": kind},
             "clocks": clk.summary(), "device_status": m.device_status()}))

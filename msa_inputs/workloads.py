@@ -284,9 +284,10 @@ def mem_1m() -> Workload:
     return Workload("1m", seed, lens, 128, "bf16", n_q=1, T0=64, k=8, plant_kind="mix", plant_args={"n": 8})
 
 
-def mem_10m() -> Workload:
-    """9,766 docs x 1024 tokens, chunk 256, bf16; 32 queries of one decode token, 4 planted docs each."""
-    return Workload("10m", SEED_BASE + 2, np.full(9766, 1024), 256, "bf16", n_q=32, T0=1, k=16,
+def mem_10m(n_docs: int = 9766) -> Workload:
+    """9,766 docs x 1024 tokens, chunk 256, bf16; 32 queries of one decode token, 4 planted docs each.
+    A smaller n_docs keeps the shapes with a shorter bank (profiling of a small case)."""
+    return Workload("10m", SEED_BASE + 2, np.full(n_docs, 1024), 256, "bf16", n_q=32, T0=1, k=16,
                     plant_kind="per_query", plant_args={"per_query": 4})
 
 

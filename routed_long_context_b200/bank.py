@@ -55,3 +55,44 @@ def to_host_bank(kvbar: torch.Tensor) -> torch.Tensor:
     host = torch.empty(kvbar.shape, dtype=kvbar.dtype, pin_memory=True)
     host.copy_(kvbar)
     return host
+
+
+class GrowableBank:
+    """A layer's memory that grows by whole documents without re-encoding the earlier ones.
+
+    Holds the router index [capacity, hr, d] and the pooled K-bar/V-bar [capacity, 2, hkv, d] on the
+    device with spare capacity, plus the document metadata. append() encodes only the new documents
+    (document-wise RoPE + chunk-mean pooling, the same kernels as a full encode) straight into the
+    next free rows and extends the offsets; every earlier row is left untouched, so the result is
+    bit-identical to encoding all documents at once.
+    """
+
+    def __init__(self, capacity_chunks: int, hr: int, hkv: int, d: int, dtype=torch.bfloat16, device="cuda"):
+        self.capacity = int(capacity_chunks)
+        self.index = torch.empty((self.capacity, hr, d), dtype=dtype, device=device)
+        self.kvbar = torch.empty((self.capacity, 2, hkv, d), dtype=dtype, device=device)
+        self.device = device
+        self.doc_len = np.zeros(0, dtype=np.int64)
+        self.doc_chunk_off_host = np.zeros(1, dtype=np.int64)
+        self.layout = None
+
+    @property
+    def n_chunks(self) -> int:
+        return int(self.doc_chunk_off_host[-1])
+
+    def append(self, k, v, kr, doc_len, chunk: int, cos_sin, stream=None):
+        """Encode new documents (token-level k, v [n_tok, hkv, d], kr [n_tok, hr, d] of the new documents
+        only, doc_len their token counts) into the next free rows. Returns the slice of new chunk rows."""
+        doc_len = np.asarray(doc_len, dtype=np.int64)
+        new = BankLayout.from_doc_lengths(doc_len, chunk, self.device)
+        c0, c1 = self.n_chunks, self.n_chunks + new.n_chunks
+        if c1 > self.capacity:
+            raise ValueError(f"bank capacity {self.capacity} chunks exceeded ({c1} needed)")
+        if new.n_chunks:
+            api.msa_pool_chunks(k, v, kr, new.doc_tok_off, new.doc_chunk_off, new.chunk_doc, chunk, cos_sin=cos_sin,
+                                fuse_doc_rope=True, normalize_router=True, kvbar=self.kvbar[c0:c1],
+                                kr_index=self.index[c0:c1], stream=stream)
+        self.doc_len = np.concatenate([self.doc_len, doc_len])
+        self.doc_chunk_off_host = np.concatenate([self.doc_chunk_off_host, c0 + new.doc_chunk_off_host[1:]])
+        self.layout = BankLayout(np.diff(self.doc_chunk_off_host), self.device)
+        return slice(c0, c1)

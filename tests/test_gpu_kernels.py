@@ -292,3 +292,38 @@ def test_sparse_attention_no_keys_gives_zero(m):
     lk = torch.zeros((1, 4, 8, 128), device="cuda")
     out = m.msa_sparse_attn(q, mem, torch.zeros(1, dtype=torch.int32, device="cuda"), lk, lk, 0, 0)
     assert torch.count_nonzero(out) == 0
+
+
+# -------------------------------------------------------------------------------------- incremental append
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_growable_bank_append_equals_full_encode_bitwise(m, dtype):
+    """Appending documents encodes only them and reproduces a from-scratch encode bit for bit; routing
+    over the grown bank finds a planted document of the appended part."""
+    from routed_long_context_b200.bank import BankLayout, GrowableBank, encode_tokens
+
+    lens = np.array([300, 128, 1, 129, 257, 1024, 77, 640, 384, 200, 513, 90], dtype=np.int64)
+    n_old = 7
+    n_tok = int(lens.sum())
+    cut = int(lens[:n_old].sum())
+    k, v, kr = (_gen(300 + i, (n_tok, 8, 128), dtype) for i in range(3))
+    qr = _gen(310, (2, 9, 8, 128), dtype)
+    off = np.concatenate([[0], np.cumsum(lens)])
+    d_plant = n_old + 1                                              # the second appended document
+    kr[off[d_plant] + 128:off[d_plant] + 256] = rng.round_to(qr[1, 4], dtype)   # its whole chunk 1
+    cs = m.rope_table(2048, 128, 1e6)
+    tdt = torch.float32 if dtype == "f32" else torch.bfloat16
+    full = BankLayout.from_doc_lengths(lens, 128)
+    kv_ref, idx_ref = encode_tokens(full, upload(k, dtype), upload(v, dtype), upload(kr, dtype), 128, cs)
+
+    bank = GrowableBank(full.n_chunks + 5, 8, 8, 128, dtype=tdt)
+    s_old = bank.append(upload(k[:cut], dtype), upload(v[:cut], dtype), upload(kr[:cut], dtype), lens[:n_old], 128, cs)
+    s_new = bank.append(upload(k[cut:], dtype), upload(v[cut:], dtype), upload(kr[cut:], dtype), lens[n_old:], 128, cs)
+    torch.cuda.synchronize()
+    assert s_old.start == 0 and s_new.stop == full.n_chunks
+    np.testing.assert_array_equal(bank.doc_chunk_off_host, full.doc_chunk_off_host)
+    assert torch.equal(bank.index[:full.n_chunks], idx_ref)
+    assert torch.equal(bank.kvbar[:full.n_chunks], kv_ref)
+    assert torch.equal(bank.layout.chunk_doc, full.chunk_doc)
+    ds = m.msa_route_scores(bank.index[:bank.n_chunks], bank.layout.chunk_doc, bank.layout.n_docs, upload(qr, dtype))
+    assert int(torch.argmax(ds[1])) == d_plant
+    _status(m)
