@@ -25,6 +25,9 @@ sys.path.insert(0, ROOT)
 METRIC = "memory tokens routed/s per layer at 100M (frac of HBM peak); route+attn ms/step"
 UNIT = "memory tokens/s"
 TOKENS_PER_CHUNK = 128
+# DRAM bytes (read + write) of one full-size router launch: ncu --set full on a 99,994-chunk case of
+# the current kernel (205.48 MB read + 3.63 MB written), scaled by the chunk count to 781,250 chunks.
+ROUTER_TRAFFIC_BYTES = (205.48e6 + 3.63e6) * 781250 / 99994
 
 
 def parse():
@@ -494,7 +497,7 @@ def main():
             "router_stages": args.router_stages or "default",
             "fetch_mode": ["host cudaMemcpyAsync per document", "device fetch kernel"][args.fetch_mode],
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": None,
+                         "frac": achieved / peak, "traffic": ROUTER_TRAFFIC_BYTES if args.n_docs == 97657 else None,
                          "kernel": "route_tc_kernel, timed by events around each launch inside the timed steps",
                          "peak_kind": f"{peak_kind} (copy bandwidth)"},
             "cpu_baseline": cpu,
