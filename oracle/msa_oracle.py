@@ -129,6 +129,15 @@ def encode_memory(k, v, kr, doc_tok_off, chunk: int, base: float):
     return tuple(out)
 
 
+def token_bank(k, v, doc_tok_off, base: float) -> np.ndarray:
+    """Token-level memory of the fine stage: [n_tok, 2, hkv, d], row r = (K_r rotated to its position
+    inside its own document, V_r). Coarse-to-fine reading of [P5] 四個核心機制 §1 (routing on the
+    compressed chunks, then the selected documents' own tokens); the keys keep document-wise
+    positions as in [P1] §组件 2."""
+    pos = doc_positions(doc_tok_off)
+    return np.stack([apply_rope(k, pos, base), np.asarray(v, dtype=F64)], axis=1)
+
+
 # ---------------------------------------------------------------------------------------------
 # router scoring
 # ---------------------------------------------------------------------------------------------
@@ -273,6 +282,25 @@ def route_and_attend(krbar, doc_chunk_off, kvbar, qr_active, q_new, k_local_raw,
     ds, _ = route(krbar, doc_chunk_off, qr_active[None])
     idx, val = topk_docs(ds, k)
     mem = gather_memory(kvbar, doc_chunk_off, idx[0])
+    L = L_prev + T_new
+    k_local = apply_rope(k_local_raw[:L], global_positions(k, 0, L), base)
+    q_rot = apply_rope(q_new, global_positions(k, L_prev, T_new), base)
+    o = sparse_attention(q_rot, mem[:, 0], mem[:, 1], k_local, v_local[:L], L_prev, scale)
+    return idx[0], val[0], o
+
+
+def route_and_attend_fine(krbar, doc_chunk_off, tokbank, doc_tok_off, qr_active, q_new, k_local_raw, v_local,
+                          L_prev: int, k: int, base: float, scale: float | None = None):
+    """route_and_attend with the fine stage: routing and selection on the compressed chunks as
+    before, then attention over the selected documents' token-level K/V (token_bank rows, in rank
+    order) instead of their chunk means (coarse-to-fine reading of [P5] 四個核心機制 §1).
+    Returns (idx [k], doc scores of idx [k], output [T_new, hq, d])."""
+    T_new = q_new.shape[0]
+    d = q_new.shape[-1]
+    scale = 1.0 / np.sqrt(d) if scale is None else scale
+    ds, _ = route(krbar, doc_chunk_off, qr_active[None])
+    idx, val = topk_docs(ds, k)
+    mem = gather_memory(tokbank, doc_tok_off, idx[0])
     L = L_prev + T_new
     k_local = apply_rope(k_local_raw[:L], global_positions(k, 0, L), base)
     q_rot = apply_rope(q_new, global_positions(k, L_prev, T_new), base)

@@ -349,3 +349,81 @@ def test_tiny_workload_planted_docs_route_first(name):
     idx, val = O.topk_docs(ds, w.k)
     assert set(idx[0, :2]) == {17, 42}
     assert val[0, 1] > 0.9 and val[0, 2] < 0.5
+
+
+# ------------------------------------------------------------------------------- fine stage
+def test_token_bank_rows_rotate_keys_by_document_position():
+    """K of the first token of every document is unrotated (position 0), every V row is the raw
+    value, every key keeps its norm, and a key at position p equals the closed-form rotation."""
+    r = np.random.default_rng(21)
+    off = np.array([0, 5, 5, 12, 20])               # includes an empty document
+    k, v = r.standard_normal((20, 2, 8)), r.standard_normal((20, 2, 8))
+    tb = O.token_bank(k, v, off, 1e4)
+    assert tb.shape == (20, 2, 2, 8)
+    np.testing.assert_array_equal(tb[:, 1], v)
+    for s in (0, 5, 12):
+        np.testing.assert_array_equal(tb[s, 0], k[s])
+    np.testing.assert_allclose(np.linalg.norm(tb[:, 0], axis=-1), np.linalg.norm(k, axis=-1), rtol=1e-13)
+    # token 15 is position 3 of the document starting at 12: pair i rotates by 3 * 1e4^(-2i/8)
+    w = 1e4 ** (-2.0 * np.arange(4) / 8)
+    c, sn = np.cos(3 * w), np.sin(3 * w)
+    x = k[15]
+    want = np.concatenate([x[:, :4] * c - x[:, 4:] * sn, x[:, 4:] * c + x[:, :4] * sn], axis=-1)
+    np.testing.assert_allclose(tb[15, 0], want, atol=1e-14)
+
+
+def test_token_bank_translation_invariance():
+    """A document's token rows do not depend on where it sits in the bank (positions restart at 0)."""
+    r = np.random.default_rng(22)
+    doc = r.standard_normal((9, 1, 8)), r.standard_normal((9, 1, 8))
+    pre = r.standard_normal((7, 1, 8)), r.standard_normal((7, 1, 8))
+    a = O.token_bank(doc[0], doc[1], np.array([0, 9]), 1e6)
+    b = O.token_bank(np.concatenate([pre[0], doc[0]]), np.concatenate([pre[1], doc[1]]), np.array([0, 7, 16]), 1e6)
+    np.testing.assert_allclose(b[7:], a, atol=1e-15)
+
+
+def test_fine_stage_with_chunk_one_equals_coarse():
+    """With chunks of one token the chunk means are the tokens themselves, so the fine stage and the
+    coarse path attend over identical memories and give the same result."""
+    w = _small_chain(rounds=1)
+    r = np.random.default_rng(23)
+    n_docs = 12
+    off = np.arange(0, 4 * n_docs + 1, 4)
+    k, v = r.standard_normal((4 * n_docs, w.hkv, w.d)), r.standard_normal((4 * n_docs, w.hkv, w.d))
+    kr = r.standard_normal((4 * n_docs, w.H, w.d))
+    kbar, vbar, krbar = O.encode_memory(k, v, kr, off, 1, 1e6)
+    dco, _ = O.chunk_layout(off, 1)
+    qr, q, kn, vn = r.standard_normal((6, w.H, w.d)), r.standard_normal((6, w.hq, w.d)), \
+        r.standard_normal((6, w.hkv, w.d)), r.standard_normal((6, w.hkv, w.d))
+    coarse = O.route_and_attend(krbar, dco, np.stack([kbar, vbar], 1), qr, q, kn, vn, 0, 3, 1e6)
+    fine = O.route_and_attend_fine(krbar, dco, O.token_bank(k, v, off, 1e6), off, qr, q, kn, vn, 0, 3, 1e6)
+    np.testing.assert_array_equal(coarse[0], fine[0])
+    np.testing.assert_allclose(fine[2], coarse[2], atol=1e-13)
+
+
+def test_fine_stage_over_every_document_is_dense_attention():
+    """Selecting every document, the fine stage is dense softmax attention over all memory tokens
+    (doc-wise rotated keys, fully visible) followed by the causal local keys: compared with torch's
+    scaled_dot_product_attention on the concatenated keys with an explicit mask."""
+    r = np.random.default_rng(24)
+    off = np.array([0, 7, 19, 24])
+    hq, hkv, d, T = 4, 2, 16, 5
+    k, v = r.standard_normal((24, hkv, d)), r.standard_normal((24, hkv, d))
+    kr = r.standard_normal((24, 2, d))
+    _, _, krbar = O.encode_memory(None, None, kr, off, 8, 1e6)
+    dco, _ = O.chunk_layout(off, 8)
+    qr, q = r.standard_normal((T, 2, d)), r.standard_normal((T, hq, d))
+    kn, vn = r.standard_normal((T, hkv, d)), r.standard_normal((T, hkv, d))
+    idx, _, got = O.route_and_attend_fine(krbar, dco, O.token_bank(k, v, off, 1e6), off, qr, q, kn, vn, 0, 3, 1e6)
+    pos = np.concatenate([np.arange(7), np.arange(12), np.arange(5)])
+    mem_k = O.apply_rope(k, pos, 1e6)
+    order = np.concatenate([np.arange(off[i], off[i + 1]) for i in idx])
+    keys = np.concatenate([mem_k[order], O.apply_rope(kn, np.arange(3, 3 + T), 1e6)])
+    vals = np.concatenate([v[order], vn])
+    qt = torch.from_numpy(O.apply_rope(q, np.arange(3, 3 + T), 1e6)).permute(1, 0, 2)[None]
+    kt = torch.from_numpy(keys).permute(1, 0, 2).repeat_interleave(hq // hkv, 0)[None]
+    vt = torch.from_numpy(vals).permute(1, 0, 2).repeat_interleave(hq // hkv, 0)[None]
+    mask = torch.ones(T, 24 + T, dtype=torch.bool)
+    mask[:, 24:] = torch.tril(torch.ones(T, T, dtype=torch.bool))
+    want = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask)[0].permute(1, 0, 2).numpy()
+    np.testing.assert_allclose(got, want, atol=1e-12)
