@@ -47,11 +47,11 @@ def parse():
                     help="SMs the routers leave free for the overlapped selection and attention")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="100m", choices=["100m", "encode10m", "interleave"],
+    ap.add_argument("--workload", default="100m", choices=["100m", "encode10m", "interleave", "fine1m"],
                     help="100m: the routing step (the reported metric); encode10m: offline encoding of the "
                          "10M-token bank (document-wise RoPE + chunk-mean pooling); interleave: three Memory "
-                         "Interleave rounds over a 10M-token bank (tensor-bound routing); the last two are "
-                         "reported separately")
+                         "Interleave rounds over a 10M-token bank (tensor-bound routing); fine1m: the token-level "
+                         "fine stage on the 1M-token bank; the last three are reported separately")
     return ap.parse_args()
 
 
@@ -328,6 +328,122 @@ def interleave_bench(args, rank, world, local_rank):
             "clocks": clk.summary()}))
 
 
+# ---------------------------------------------------------------------------------------------- fine stage
+def host_link_gbs(nbytes: int = 1 << 30, reps: int = 5) -> float:
+    """Pinned host -> device copy bandwidth measured in this process (best of reps, CUDA events)."""
+    import torch
+
+    h = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
+    d = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    best = float("inf")
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        d.copy_(h, non_blocking=True)
+        b.record()
+        torch.cuda.synchronize()
+        best = min(best, a.elapsed_time(b))
+    del h, d
+    return nbytes / (best / 1e3) / 1e9
+
+
+def fine_bench(args, rank, world, local_rank):
+    """Token-level fine stage on the 1M-token bank: one step = route (pooled index) + top-8 + fetch of
+    the selected documents' token K/V from the pinned token bank + global RoPE of the local context +
+    split-key attention of 64 query tokens over those rows."""
+    import numpy as np
+    import torch
+
+    import routed_long_context_b200 as m
+    from msa_inputs import workloads
+    from msa_inputs.device import memory_tensor, small_tensors
+    from routed_long_context_b200.bank import BankLayout, to_host_bank
+
+    torch.cuda.set_device(local_rank)
+    w = workloads.mem_1m()
+    lay = BankLayout.from_doc_lengths(w.doc_len, w.chunk)
+    cs = m.rope_table(4096, w.d, w.rope_base)
+    k, v, kr = (memory_tensor(w, 0, n) for n in ("k", "v", "kr"))
+    _, index = m.msa_pool_chunks(None, None, kr, lay.doc_tok_off, lay.doc_chunk_off, lay.chunk_doc, w.chunk)
+    tok = m.msa_pack_tokens(k, v, lay.doc_tok_off, cs)
+    del k, v, kr
+    host_tok = to_host_bank(tok)
+    del tok
+    torch.cuda.empty_cache()
+    dv = small_tensors(w, 0)
+    T, max_mem = w.T0, w.k * int(w.doc_len.max())
+    seg = torch.tensor([0, T], dtype=torch.int64, device="cuda")
+    ds = torch.empty((w.n_q, lay.n_docs), dtype=torch.float32, device="cuda")
+    idx = torch.empty((w.n_q, w.k), dtype=torch.int32, device="cuda")
+    sc = torch.empty((w.n_q, w.k), dtype=torch.float32, device="cuda")
+    idx_h = torch.empty((w.n_q, w.k), dtype=torch.int32, pin_memory=True)
+    mem = torch.zeros((w.n_q, max_mem, 2, w.hkv, w.d), dtype=torch.bfloat16, device="cuda")
+    mem_len = torch.zeros(w.n_q, dtype=torch.int32, device="cuda")
+    lk, qq = torch.empty_like(dv["k_new"][0]), torch.empty_like(dv["q"][0])
+    out = torch.empty((w.n_q, T, w.hq, w.d), dtype=torch.bfloat16, device="cuda")
+    rws = m.api._ws(m.route_workspace_size(w.n_q, T, w.H, w.d, torch.bfloat16), "cuda")
+    tws = m.api._ws(m.topk_workspace_size(w.n_q, lay.n_docs, w.k), "cuda")
+    aws = m.api._ws(m.sparse_attn_split_workspace_size(w.n_q, T, w.hq, w.hkv, max_mem, T), "cuda")
+    s = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev: ev[0].record(s)
+        m.msa_route_scores(index, lay.chunk_doc, lay.n_docs, dv["qr"], doc_scores=ds, ws=rws)
+        m.msa_topk_docs(ds, w.k, idx=idx, score=sc, ws=tws)
+        if ev: ev[1].record(s)
+        if args.fetch_mode == 1:
+            m.msa_gather_kv_device(host_tok, lay.doc_tok_off, idx, max_mem, dev_mem_kv=mem, mem_len=mem_len)
+        else:
+            idx_h.copy_(idx, non_blocking=True)
+            s.synchronize()
+            _, ml = m.msa_gather_kv(host_tok, w.doc_tok_off, idx_h, max_mem, dev_mem_kv=mem, copy_stream=s)
+            mem_len.copy_(ml, non_blocking=True)
+        if ev: ev[2].record(s)
+        m.msa_rope_doc(dv["k_new"][0], seg, w.k, cs, out=lk)
+        m.msa_rope_doc(dv["q"][0], seg, w.k, cs, out=qq)
+        m.msa_sparse_attn_split(qq[None], mem, mem_len, lk[None], dv["v_new"], T, 0, out=out, ws=aws)
+        if ev: ev[3].record(s)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    rows = int(mem_len.cpu().sum())
+    gi = idx.cpu().numpy()[0]
+    planted_ok = set(w.expected(0, 0, 0)) <= set(gi.tolist())
+    steps = min(args.steps, 100)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        for i in range(steps):
+            step(evs[i])
+        torch.cuda.synchronize()
+    route_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / steps
+    fetch_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / steps
+    attn_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / steps
+    ms = sum(e[0].elapsed_time(e[3]) for e in evs) / steps
+    fetch_bytes = rows * 2 * w.hkv * w.d * 2
+    link = host_link_gbs()
+    fetch_gbs = fetch_bytes / (fetch_ms / 1e3) / 1e9
+    G = w.hq // w.hkv
+    attn_flops = 4.0 * w.n_q * T * w.hq * w.d * (rows + T / 2)
+    if rank == 0:
+        print(json.dumps({
+            "metric": "1M fine stage: token rows fetched and attended per second (route + top-8 + token fetch + "
+                      "split attention)",
+            "value": rows / (ms / 1e3), "unit": "memory token rows/s", "n_gpus": 1, "steps": steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"fine1m: {w.n_docs} docs ({w.n_tok:,} tokens), token bank "
+                                   f"{w.n_tok * 4096 / 1e9:.1f} GB pinned host, 64 query tokens, top-8 -> {rows} rows",
+                       "fetch_mode": args.fetch_mode},
+            "route_topk_ms": route_ms, "fetch_ms": fetch_ms, "attn_ms": attn_ms, "attn_tflops": attn_flops / attn_ms / 1e9,
+            "roofline": {"bound": "host-link", "achieved": fetch_gbs, "peak": link, "unit": "GB/s",
+                         "frac": fetch_gbs / link, "traffic": None,
+                         "kernel": "gather_device_kernel" if args.fetch_mode == 1 else "cudaMemcpyAsync per document",
+                         "peak_kind": "pinned host->device copy measured in this process", "bytes": fetch_bytes},
+            "checks": {"planted_docs_selected": planted_ok, "device_status": m.device_status(), "G": G},
+            "clocks": clk.summary()}))
+
+
 # ---------------------------------------------------------------------------------------------- ours
 def main():
     args = parse()
@@ -340,6 +456,8 @@ def main():
         return encode_bench(args, rank, world, local_rank)
     if args.workload == "interleave":
         return interleave_bench(args, rank, world, local_rank)
+    if args.workload == "fine1m":
+        return fine_bench(args, rank, world, local_rank)
 
     import numpy as np
     import torch

@@ -122,6 +122,21 @@ msa_status msa_pool_chunks(const void* k, const void* v, const void* kr, msa_dty
                            const float* cos_sin, int64_t max_pos, void* kvbar, void* kr_index, msa_dtype out_dt,
                            int normalize_router, void* stream);
 
+/* Token-level memory bank for the fine stage (coarse-to-fine reading of [P5] 四個核心機制 §1:
+ * after routing on the compressed chunks, attention may read the selected documents' own tokens;
+ * [P1] §组件 2: memory keys carry document-wise positions). For every token row r of document i
+ * (doc_tok_off[i] <= r < doc_tok_off[i+1]):
+ *   bank[r][0] = k[r] rotated to position r - doc_tok_off[i];  bank[r][1] = v[r].
+ *   k, v: device [n_tok][hkv][d] of dt; doc_tok_off: device int64 [n_docs+1] (doc_tok_off[0] = 0,
+ *   doc_tok_off[n_docs] = n_tok); cos_sin: device [max_pos][d/2][2] (msa_rope_table);
+ *   bank: device [n_tok][2][hkv][d] of dt — the layout msa_gather_kv and msa_gather_kv_device
+ *   read when given doc_tok_off in place of doc_chunk_off, so a document is one contiguous run.
+ * A position >= max_pos leaves that key unrotated and records MSA_DEV_ROPE_POSITION.
+ * Same head_dim rules as msa_rope_doc. */
+msa_status msa_pack_tokens(const void* k, const void* v, msa_dtype dt, int64_t n_tok, int hkv, int d,
+                           const int64_t* doc_tok_off, int64_t n_docs, const float* cos_sin, int64_t max_pos,
+                           void* bank, void* stream);
+
 /* Router scoring ([P1] §组件 1 key formula; [P2] §可学习记忆路由层的核心架构):
  *   S_{q,c} = max over tokens t of mean over heads h of cos(Q^R_{q,t,h}, K-bar^R_{c,h})
  *   doc_scores[q][i] = max over the chunks c of document i of S_{q,c}
@@ -183,6 +198,28 @@ msa_status msa_topk_docs_noalloc(const float* doc_scores, int n_q, int64_t n_doc
                                  void* stream);
 size_t msa_topk_noalloc_max_scratch(void);
 
+/* Memory Parallel merge ([P2] §工程实现的关键细节: the router keys are sharded over several GPUs,
+ * each scores its own keys and keeps its local best, and the local results are combined into the
+ * global top-k; [P3] §四大技术突破 3). Shard g holds the documents
+ * shard_doc_off[g] .. shard_doc_off[g+1]-1 and supplies its local top-k_cand list.
+ *   cand_score, cand_idx: device float / int32 lists [n_q][k_cand] of every shard, shard g's lists
+ *     starting shard_stride * g elements after cand_score / cand_idx (n_q * k_cand for two plain
+ *     [n_shards][n_q][k_cand] arrays; 2 * n_q * k_cand when every rank packed [scores ; indices]
+ *     into one buffer and an all_gather concatenated them). Indices are local to their shard, -1
+ *     for an empty slot;
+ *   shard_doc_off: HOST int64 [n_shards+1], non-decreasing;
+ *   idx: device int32 [n_q][k]: the k best candidates as GLOBAL document indices, by descending
+ *     score, equal scores to the lower global index (-0 equals +0, a NaN score ranks below -inf);
+ *     score: device float [n_q][k] (may be NULL). Slots past the number of candidates hold -1 and
+ *     -inf. With disjoint shards whose lists are their exact local top-k (k_cand >= k) the result is
+ *     exactly msa_topk_docs over all documents.
+ * Requires 1 <= n_shards <= 64, n_shards * k_cand <= 4096, 1 <= k <= 64, global indices < 2^31.
+ * A local index outside its shard (other than -1) records MSA_DEV_BAD_INDEX and counts as empty.
+ * Duplicate candidates are not removed. One block per query. */
+msa_status msa_topk_merge(const float* cand_score, const int32_t* cand_idx, int64_t shard_stride, int n_shards,
+                          int n_q, int k_cand, const int64_t* shard_doc_off, int k, int32_t* idx, float* score,
+                          void* stream);
+
 /* Fetch of the selected documents' compressed K-bar/V-bar from host memory
  * ([P2] §工程实现的关键细节: K-bar^R stays in GPU memory, K-bar/V-bar live in host DRAM and are
  * loaded asynchronously once routing has chosen the documents; [P5] §3 async prefetch).
@@ -193,7 +230,8 @@ size_t msa_topk_noalloc_max_scratch(void);
  *   concatenated in rank order from row 0; mem_len_host[q] (host int32, written before the
  *   call returns) is the number of rows filled.
  * One cudaMemcpyAsync per selected document on copy_stream (the copy engines over the host
- * link); the call returns once they are enqueued. Fails with MSA_ERR_INVALID_ARG, copying
+ * link); the call returns once they are enqueued. The fine stage passes the token bank of
+ * msa_pack_tokens with doc_tok_off in place of doc_chunk_off (rows are then tokens). Fails with MSA_ERR_INVALID_ARG, copying
  * nothing, if an index is out of range or a query's rows exceed max_mem. */
 msa_status msa_gather_kv(const void* host_bank, msa_dtype dt, int64_t n_chunks, const int64_t* doc_chunk_off_host,
                          int64_t n_docs, const int32_t* idx_host, int n_q, int k, int hkv, int d, int max_mem,
@@ -205,7 +243,8 @@ msa_status msa_gather_kv(const void* host_bank, msa_dtype dt, int64_t n_chunks, 
  * between selection and fetch. Same layout and rank order as msa_gather_kv.
  *   doc_chunk_off: device int64 [n_docs+1]; idx: device int32 [n_q][k]; mem_len: device int32 [n_q].
  * Indices out of range or more rows than max_mem record MSA_DEV_BAD_INDEX and skip that query's
- * copy (no out-of-range access). Returns MSA_ERR_INVALID_ARG if host_bank is not pinned, mapped
+ * copy (no out-of-range access). Long documents (token rows of the fine stage) are split over
+ * several blocks, chosen from max_mem / k. Returns MSA_ERR_INVALID_ARG if host_bank is not pinned, mapped
  * host memory. */
 msa_status msa_gather_kv_device(const void* host_bank, msa_dtype dt, int64_t n_chunks, const int64_t* doc_chunk_off,
                                 int64_t n_docs, const int32_t* idx, int n_q, int k, int hkv, int d, int max_mem,
@@ -228,6 +267,20 @@ msa_status msa_sparse_attn(const void* q, const void* mem_kv, const int32_t* mem
 /* Selects the bf16 attention kernel for testing: 0 = tensor cores (mma.sync m16n8k16, default),
  * 1 = CUDA cores. fp32 always runs on CUDA cores. Process-wide. */
 msa_status msa_attn_set_impl(int impl);
+
+/* Sparse attention over long memories (the token-level fine stage, thousands of memory rows per
+ * query): the same arguments, layout and result as msa_sparse_attn, computed with the keys of
+ * every (64-row block, kv head, query) split into n_split contiguous ranges of 64-key tiles that
+ * run as separate blocks. Each writes its unnormalised output and (running max, sum) in fp32 to
+ * the workspace; a second kernel merges the ranges' softmax statistics and writes out.
+ * n_split is chosen from the sizes so that the grid fits one wave of three blocks per SM (148
+ * SMs), at least four tiles per range. bf16 only (tensor cores); fp32 returns MSA_ERR_UNSUPPORTED.
+ * ws: device, msa_sparse_attn_split_workspace_size bytes, 16-byte aligned. */
+msa_status msa_sparse_attn_split(const void* q, const void* mem_kv, const int32_t* mem_len, int max_mem,
+                                 const void* local_k, const void* local_v, int L_max, int L, int q_start, int n_q,
+                                 int T, int hq, int hkv, int d, float scale, void* out, msa_dtype dt, void* ws,
+                                 size_t ws_bytes, void* stream);
+msa_status msa_sparse_attn_split_workspace_size(int n_q, int T, int hq, int hkv, int max_mem, int L, size_t* bytes);
 
 /* One routed layer of one Memory Interleave round (see msa_interleave_step). */
 typedef struct msa_layer_args {

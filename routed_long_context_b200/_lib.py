@@ -54,6 +54,7 @@ SIGNATURES = {
     "msa_topk_workspace_size": (i32, [ctypes.c_int, i64, ctypes.c_int, ctypes.POINTER(sz)]),
     "msa_topk_docs_noalloc": (i32, [vp, ctypes.c_int, i64, ctypes.c_int, vp, vp, vp]),
     "msa_topk_noalloc_max_scratch": (sz, []),
+    "msa_topk_merge": (i32, [vp, vp, i64, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, ctypes.c_int, vp, vp, vp]),
     "msa_gather_kv": (i32, [vp, i32, i64, vp, i64, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                             ctypes.c_int, vp, vp, vp]),
     "msa_gather_kv_device": (i32, [vp, i32, i64, vp, i64, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -61,6 +62,12 @@ SIGNATURES = {
     "msa_sparse_attn": (i32, [vp, vp, vp, ctypes.c_int, vp, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                               ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, f32, vp, i32, vp]),
     "msa_attn_set_impl": (i32, [ctypes.c_int]),
+    "msa_sparse_attn_split": (i32, [vp, vp, vp, ctypes.c_int, vp, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                    ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, f32, vp, i32,
+                                    vp, sz, vp]),
+    "msa_sparse_attn_split_workspace_size": (i32, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                   ctypes.c_int, ctypes.c_int, ctypes.POINTER(sz)]),
+    "msa_pack_tokens": (i32, [vp, vp, i32, i64, ctypes.c_int, ctypes.c_int, vp, i64, vp, i64, vp, vp]),
     "msa_interleave_step": (i32, [ctypes.POINTER(InterleaveArgs), vp, vp, i64]),
     "msa_interleave_workspace_size": (i32, [ctypes.POINTER(InterleaveArgs), ctypes.POINTER(sz)]),
 }

@@ -12,7 +12,7 @@ import numpy as np
 import torch
 
 from . import _lib
-from ._lib import MSA_BF16, MSA_F32, check, lib
+from ._lib import MSA_BF16, MSA_F32, MSAError, check, lib  # noqa: F401
 
 _DT = {torch.float32: MSA_F32, torch.bfloat16: MSA_BF16}
 
@@ -95,6 +95,17 @@ def msa_pool_chunks(k, v, kr, doc_tok_off, doc_chunk_off, chunk_doc, chunk: int,
     return (kvbar if k is not None else None), (kr_index if kr is not None else None)
 
 
+def msa_pack_tokens(k, v, doc_tok_off, cos_sin, bank=None, stream=None):
+    """Token-level memory bank of the fine stage: k, v [n_tok, hkv, d] -> bank [n_tok, 2, hkv, d] with each
+    key rotated to its position inside its document (doc_tok_off [n_docs+1], device int64)."""
+    n_tok, hkv, d = k.shape
+    if bank is None:
+        bank = torch.empty((n_tok, 2, hkv, d), dtype=k.dtype, device=k.device)
+    check(lib.msa_pack_tokens(_ptr(k), _ptr(v), _dt(k), n_tok, hkv, d, _ptr(doc_tok_off), doc_tok_off.numel() - 1,
+                              _ptr(cos_sin), cos_sin.shape[0], _ptr(bank), _stream(stream)), "msa_pack_tokens")
+    return bank
+
+
 def route_workspace_size(n_q: int, T: int, H: int, d: int, dtype) -> int:
     n = ctypes.c_size_t(0)
     check(lib.msa_route_workspace_size(n_q, T, H, d, _DT[dtype], ctypes.byref(n)), "msa_route_workspace_size")
@@ -166,6 +177,23 @@ def msa_topk_docs_noalloc(doc_scores, k: int, idx=None, score=None, stream=None)
     return idx, score
 
 
+def msa_topk_merge(cand_score, cand_idx, shard_doc_off, k: int, idx=None, score=None, shard_stride=None,
+                   stream=None):
+    """Memory Parallel merge: cand_score float32 / cand_idx int32 lists [n_q, k_cand] of every shard (device,
+    shard g's lists shard_stride elements after shard g-1's; default: plain [n_shards, n_q, k_cand] arrays),
+    shard_doc_off host int64 [n_shards + 1] -> (idx int32 [n_q, k] global, score float32 [n_q, k])."""
+    off = np.ascontiguousarray(shard_doc_off, dtype=np.int64)
+    n_shards = len(off) - 1
+    n_q, k_cand = cand_score.shape[-2:]
+    dev = cand_score.device
+    stride = n_q * k_cand if shard_stride is None else int(shard_stride)
+    idx = torch.empty((n_q, k), dtype=torch.int32, device=dev) if idx is None else idx
+    score = torch.empty((n_q, k), dtype=torch.float32, device=dev) if score is None else score
+    check(lib.msa_topk_merge(_ptr(cand_score), _ptr(cand_idx), stride, n_shards, n_q, k_cand, off.ctypes.data, k,
+                             _ptr(idx), _ptr(score), _stream(stream)), "msa_topk_merge")
+    return idx, score
+
+
 def msa_gather_kv(host_bank, doc_chunk_off_host, idx_host, max_mem: int, dev_mem_kv=None, device="cuda",
                   copy_stream=None):
     """Copy the selected docs' rows [*, 2, hkv, d] from the pinned host bank into
@@ -211,6 +239,31 @@ def msa_sparse_attn(q, mem_kv, mem_len, local_k, local_v, L: int, q_start: int, 
     check(lib.msa_sparse_attn(_ptr(q), _ptr(mem_kv), _ptr(mem_len), max_mem, _ptr(local_k), _ptr(local_v), L_max, L,
                               q_start, n_q, T, hq, hkv, d, scale, _ptr(out), _dt(q), _stream(stream)),
           "msa_sparse_attn")
+    return out
+
+
+def sparse_attn_split_workspace_size(n_q: int, T: int, hq: int, hkv: int, max_mem: int, L: int) -> int:
+    n = ctypes.c_size_t(0)
+    check(lib.msa_sparse_attn_split_workspace_size(n_q, T, hq, hkv, max_mem, L, ctypes.byref(n)),
+          "msa_sparse_attn_split_workspace_size")
+    return n.value
+
+
+def msa_sparse_attn_split(q, mem_kv, mem_len, local_k, local_v, L: int, q_start: int, scale: float | None = None,
+                          out=None, ws=None, stream=None):
+    """msa_sparse_attn for long memories (token-level fine stage): keys split into ranges that run as
+    separate blocks, then merged. Same arguments and result; bf16 only."""
+    n_q, T, hq, d = q.shape
+    max_mem = mem_kv.shape[1]
+    hkv = mem_kv.shape[3]
+    L_max = local_k.shape[1]
+    out = torch.empty_like(q) if out is None else out
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    if ws is None:
+        ws = _ws(sparse_attn_split_workspace_size(n_q, T, hq, hkv, max_mem, L), q.device)
+    check(lib.msa_sparse_attn_split(_ptr(q), _ptr(mem_kv), _ptr(mem_len), max_mem, _ptr(local_k), _ptr(local_v),
+                                    L_max, L, q_start, n_q, T, hq, hkv, d, scale, _ptr(out), _dt(q), _ptr(ws),
+                                    ws.numel(), _stream(stream)), "msa_sparse_attn_split")
     return out
 
 

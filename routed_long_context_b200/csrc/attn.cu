@@ -6,6 +6,7 @@
 // heads (q and K from shared memory, K rows padded to 129 floats so the 32 lanes hit 32 banks),
 // then an online softmax (running max and sum per head, exp2 with log2(e) folded into q) and
 // the P.V update, where lane r owns output dims 4r..4r+3. Arithmetic and softmax in fp32.
+#include <algorithm>
 #include <atomic>
 
 #include "common.cuh"
@@ -29,6 +30,9 @@ struct AttnArgs {
     int T, hq, hkv;
     float scale_log2e;
     void* out;
+    int n_split;       // split-KV variant: key ranges per (row block, kv head, query)
+    float* part_o;     // [n_split][n_q * T * hq][d] unnormalised outputs
+    float2* part_ml;   // [n_split][n_q * T * hq] (running max in log2 units, sum of weights)
 };
 
 template <typename T>
@@ -228,20 +232,38 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-template <int G>
-__global__ void __launch_bounds__(128) attn_mma_kernel(const AttnArgs a) {
-    __shared__ __align__(16) __nv_bfloat16 Ks[kMmaKeys][kKvStride];
-    __shared__ __align__(16) __nv_bfloat16 Vs[kMmaKeys][kKvStride];
+// Shared memory of one key/value stage: K and V tiles of 64 keys. The split variant double-buffers
+// (the next tile's copies are in flight while the current tile is computed); the plain variant keeps
+// one stage so that it fits beside the router's blocks on an SM.
+constexpr size_t kMmaStageBytes = (size_t)2 * kMmaKeys * kKvStride * sizeof(__nv_bfloat16);
+
+template <int G, bool SPLIT>
+__global__ void __launch_bounds__(128, SPLIT ? 3 : 1) attn_mma_kernel(const AttnArgs a) {
+    constexpr int STAGES = SPLIT ? 2 : 1;
+    extern __shared__ __align__(16) unsigned char attn_mma_smem[];
+    typedef __nv_bfloat16 Tile[kMmaKeys][kKvStride];
+    Tile* Kst = reinterpret_cast<Tile*>(attn_mma_smem);                                  // [STAGES]
+    Tile* Vst = reinterpret_cast<Tile*>(attn_mma_smem + STAGES * (kMmaStageBytes / 2));  // [STAGES]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gid = lane >> 2, tig = lane & 3;
     const int qi = blockIdx.z, g = blockIdx.y;
     const int n_rows = a.T * G;
-    const int r0 = blockIdx.x * kMmaRows;
+    const int split = SPLIT ? blockIdx.x % a.n_split : 0;
+    const int r0 = (SPLIT ? blockIdx.x / a.n_split : blockIdx.x) * kMmaRows;
     const int r_last = min(r0 + kMmaRows, n_rows) - 1;
     const int t_last = r_last / G;
     const int mem_len = max(min(a.mem_len[qi], a.max_mem), 0);
     const int n_local = max(min(a.L, a.q_start + t_last + 1), 0);
     const int n_keys = mem_len + n_local;
+    // keys of this block: all of them, or this split's contiguous range of 64-key tiles (ranges
+    // start on tile boundaries, so no tile straddles two splits)
+    int k_begin = 0, k_end = n_keys;
+    if constexpr (SPLIT) {
+        const int tiles = (n_keys + kMmaKeys - 1) / kMmaKeys;
+        const int per = (tiles + a.n_split - 1) / a.n_split;
+        k_begin = min(split * per, tiles) * kMmaKeys;
+        k_end = min(min(split * per + per, tiles) * kMmaKeys, n_keys);
+    }
 
     const __nv_bfloat16* Q = static_cast<const __nv_bfloat16*>(a.q);
     const __nv_bfloat16* MKV = static_cast<const __nv_bfloat16*>(a.mem_kv);
@@ -271,10 +293,9 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnArgs a) {
     for (int nd = 0; nd < kD / 8; ++nd) o[nd][0] = o[nd][1] = o[nd][2] = o[nd][3] = 0.f;
     float m_a = ninf, m_b = ninf, l_a = 0.f, l_b = 0.f;
 
-    for (int kb = 0; kb < n_keys; kb += kMmaKeys) {
-        __syncthreads();
-        // stage 64 keys and values with asynchronous 16-byte copies (all in flight at once);
-        // rows past the visible range are zero-filled without reading
+    // stage 64 keys and values of tile kb into buffer b with asynchronous 16-byte copies (all in
+    // flight at once); rows past the visible range are zero-filled without reading
+    auto stage = [&](int kb, int b) {
         for (int v = threadIdx.x; v < kMmaKeys * (kD / 8) * 2; v += blockDim.x) {
             const int which = v / (kMmaKeys * (kD / 8));
             const int rem = v % (kMmaKeys * (kD / 8));
@@ -289,11 +310,29 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnArgs a) {
                 src = (which ? LV : LK) + (((int64_t)qi * a.L_max + (kk - mem_len)) * a.hkv + g) * kD + c;
                 bytes = 16;
             }
-            const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(which ? &Vs[r][c] : &Ks[r][c]));
+            const uint32_t dst =
+                static_cast<uint32_t>(__cvta_generic_to_shared(which ? &Vst[b][r][c] : &Kst[b][r][c]));
             asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(bytes) : "memory");
         }
-        asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+
+    if (k_begin < k_end) stage(k_begin, 0);
+    int buf = 0;
+    for (int kb = k_begin; kb < k_end; kb += kMmaKeys) {
+        if constexpr (STAGES == 2) {
+            if (kb + kMmaKeys < k_end) {
+                stage(kb + kMmaKeys, buf ^ 1);   // that buffer's readers finished at the last barrier
+                asm volatile("cp.async.wait_group 1;" ::: "memory");
+            } else {
+                asm volatile("cp.async.wait_group 0;" ::: "memory");
+            }
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+        }
         __syncthreads();
+        const Tile& Ks = Kst[buf];
+        const Tile& Vs = Vst[buf];
 
         // S = Q K^T for 8 blocks of 8 keys
         float sc[kMmaKeys / 8][4];
@@ -368,12 +407,35 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnArgs a) {
                 mma_bf16_16816(o[nd + 1], pa, b2, b3);
             }
         }
+        __syncthreads();   // every warp is done with this buffer before it is refilled
+        if constexpr (STAGES == 2) {
+            buf ^= 1;
+        } else if (kb + kMmaKeys < k_end) {
+            stage(kb + kMmaKeys, 0);
+        }
     }
 
     l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
     l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
     l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
     l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
+    if constexpr (SPLIT) {
+        // partial result of this key range: unnormalised output and (max, sum) per row
+        const int64_t rows_total = (int64_t)gridDim.z * a.T * a.hq;
+        const int64_t row_a = ((int64_t)qi * a.T + ta) * a.hq + g * G + ra % G;
+        const int64_t row_b = ((int64_t)qi * a.T + tb) * a.hq + g * G + rb % G;
+        float* po = a.part_o + (int64_t)split * rows_total * kD;
+#pragma unroll
+        for (int nd = 0; nd < kD / 8; ++nd) {
+            if (va) *reinterpret_cast<float2*>(po + row_a * kD + nd * 8 + tig * 2) = make_float2(o[nd][0], o[nd][1]);
+            if (vb) *reinterpret_cast<float2*>(po + row_b * kD + nd * 8 + tig * 2) = make_float2(o[nd][2], o[nd][3]);
+        }
+        if (tig == 0) {
+            if (va) a.part_ml[(int64_t)split * rows_total + row_a] = make_float2(m_a, l_a);
+            if (vb) a.part_ml[(int64_t)split * rows_total + row_b] = make_float2(m_b, l_b);
+        }
+        return;
+    }
     const float ia = l_a > 0.f ? 1.f / l_a : 0.f, ib = l_b > 0.f ? 1.f / l_b : 0.f;
     __nv_bfloat16* O = static_cast<__nv_bfloat16*>(a.out);
     uint32_t* oa = reinterpret_cast<uint32_t*>(O + (((int64_t)qi * a.T + ta) * a.hq + g * G + ra % G) * kD);
@@ -385,22 +447,87 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnArgs a) {
     }
 }
 
-template <int G>
+// Merge of the split-KV partial results: one warp per (query, token, head) row, lane l owning dims
+// 4l..4l+3. out = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s with M = max_s m_s; a row whose
+// ranges saw no visible key (all m_s = -inf) is 0.
+__global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restrict__ part_o,
+                                                           const float2* __restrict__ part_ml, int n_split,
+                                                           int64_t rows, __nv_bfloat16* __restrict__ out) {
+    const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    const float ninf = -__int_as_float(0x7f800000);
+    float M = ninf;
+    for (int s = 0; s < n_split; ++s) M = fmaxf(M, part_ml[(int64_t)s * rows + row].x);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f}, L = 0.f;
+    if (M != ninf) {
+        for (int s = 0; s < n_split; ++s) {
+            const float2 ml = part_ml[(int64_t)s * rows + row];
+            if (ml.x == ninf) continue;
+            const float w = exp2f(ml.x - M);
+            L = fmaf(w, ml.y, L);
+            const float4 o = *reinterpret_cast<const float4*>(part_o + ((int64_t)s * rows + row) * kD + lane * 4);
+            acc[0] = fmaf(w, o.x, acc[0]);
+            acc[1] = fmaf(w, o.y, acc[1]);
+            acc[2] = fmaf(w, o.z, acc[2]);
+            acc[3] = fmaf(w, o.w, acc[3]);
+        }
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    uint2 u;
+    u.x = pack_bf16(acc[0] * inv, acc[1] * inv);
+    u.y = pack_bf16(acc[2] * inv, acc[3] * inv);
+    *reinterpret_cast<uint2*>(out + row * kD + lane * 4) = u;
+}
+
+template <int G, bool SPLIT>
 msa_status launch_mma_g(const AttnArgs& a, int n_q, cudaStream_t s) {
-    dim3 grid((a.T * G + kMmaRows - 1) / kMmaRows, a.hkv, n_q);
-    attn_mma_kernel<G><<<grid, 128, 0, s>>>(a);
+    const int row_blocks = (a.T * G + kMmaRows - 1) / kMmaRows;
+    dim3 grid(row_blocks * (SPLIT ? a.n_split : 1), a.hkv, n_q);
+    const size_t smem = (SPLIT ? 2 : 1) * kMmaStageBytes;
+    if constexpr (SPLIT)
+        MSA_CUDA_TRY(cudaFuncSetAttribute(attn_mma_kernel<G, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          (int)smem));
+    attn_mma_kernel<G, SPLIT><<<grid, 128, smem, s>>>(a);
     MSA_LAUNCH_CHECK();
+    if constexpr (SPLIT) {
+        const int64_t rows = (int64_t)n_q * a.T * a.hq;
+        attn_combine_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(a.part_o, a.part_ml, a.n_split, rows,
+                                                                       static_cast<__nv_bfloat16*>(a.out));
+        MSA_LAUNCH_CHECK();
+    }
     return MSA_OK;
 }
 
+template <bool SPLIT>
 msa_status launch_mma(const AttnArgs& a, int n_q, cudaStream_t s) {
     switch (a.hq / a.hkv) {
-        case 1: return launch_mma_g<1>(a, n_q, s);
-        case 2: return launch_mma_g<2>(a, n_q, s);
-        case 4: return launch_mma_g<4>(a, n_q, s);
-        case 8: return launch_mma_g<8>(a, n_q, s);
+        case 1: return launch_mma_g<1, SPLIT>(a, n_q, s);
+        case 2: return launch_mma_g<2, SPLIT>(a, n_q, s);
+        case 4: return launch_mma_g<4, SPLIT>(a, n_q, s);
+        case 8: return launch_mma_g<8, SPLIT>(a, n_q, s);
         default: return set_error(MSA_ERR_UNSUPPORTED, "msa_sparse_attn: hq/hkv unsupported");
     }
+}
+
+// Key ranges per (64-row block, kv head, query): as many as keep the grid within one wave of three
+// resident blocks per SM (148 SMs; the split kernel is register-bounded to 168 per thread for
+// that), at least four 64-key tiles per range.
+constexpr int kSplitTargetBlocks = 3 * 148;
+constexpr int kMinTilesPerSplit = 4;
+
+int pick_splits(int n_q, int T, int hq, int hkv, int max_mem, int L) {
+    const int G = hq / hkv;
+    const int64_t base = (int64_t)((T * G + kMmaRows - 1) / kMmaRows) * hkv * n_q;
+    const int tiles = (max_mem + L + kMmaKeys - 1) / kMmaKeys;
+    const int64_t want = kSplitTargetBlocks / base;
+    const int64_t cap = std::max(1, tiles / kMinTilesPerSplit);
+    return (int)std::max<int64_t>(1, std::min(want, cap));
+}
+
+size_t split_ws_bytes(int n_split, int n_q, int T, int hq) {
+    const size_t rows = (size_t)n_q * T * hq;
+    return align_up((size_t)n_split * rows * kD * 4, 256) + align_up((size_t)n_split * rows * 8, 256);
 }
 
 }  // namespace
@@ -439,8 +566,51 @@ msa_status msa_sparse_attn(const void* q, const void* mem_kv, const int32_t* mem
     a.local_k = local_k; a.local_v = local_v; a.L_max = L_max; a.L = L; a.q_start = q_start;
     a.T = T; a.hq = hq; a.hkv = hkv; a.scale_log2e = scale * 1.4426950408889634f; a.out = out;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (dt == MSA_BF16 && g_attn_impl.load() == 0) return launch_mma(a, n_q, s);
+    if (dt == MSA_BF16 && g_attn_impl.load() == 0) return launch_mma<false>(a, n_q, s);
     return dt == MSA_BF16 ? launch<__nv_bfloat16>(a, n_q, s) : launch<float>(a, n_q, s);
+}
+
+msa_status msa_sparse_attn_split_workspace_size(int n_q, int T, int hq, int hkv, int max_mem, int L, size_t* bytes) {
+    MSA_REQUIRE(bytes, "msa_sparse_attn_split_workspace_size: bytes is NULL");
+    MSA_REQUIRE(n_q > 0 && T >= 0 && hq > 0 && hkv > 0 && hq % hkv == 0 && max_mem >= 0 && L >= 0,
+                "msa_sparse_attn_split_workspace_size: bad sizes");
+    *bytes = split_ws_bytes(pick_splits(n_q, T, hq, hkv, max_mem, L), n_q, T, hq);
+    return MSA_OK;
+}
+
+msa_status msa_sparse_attn_split(const void* q, const void* mem_kv, const int32_t* mem_len, int max_mem,
+                                 const void* local_k, const void* local_v, int L_max, int L, int q_start, int n_q,
+                                 int T, int hq, int hkv, int d, float scale, void* out, msa_dtype dt, void* ws,
+                                 size_t ws_bytes, void* stream) {
+    MSA_REQUIRE(dtype_ok(dt), "msa_sparse_attn_split: bad dtype");
+    if (dt != MSA_BF16) return set_error(MSA_ERR_UNSUPPORTED, "msa_sparse_attn_split: bf16 only");
+    MSA_REQUIRE(n_q > 0 && T >= 0 && hq > 0 && hkv > 0 && hq % hkv == 0 && max_mem >= 0 && L >= 0 && L <= L_max &&
+                    q_start >= 0 && n_q <= 65535 && hkv <= 65535,
+                "msa_sparse_attn_split: bad sizes");
+    if (d != kD) return set_error(MSA_ERR_UNSUPPORTED, "msa_sparse_attn_split: head_dim must be 128, got %d", d);
+    const int G = hq / hkv;
+    if (G != 1 && G != 2 && G != 4 && G != 8)
+        return set_error(MSA_ERR_UNSUPPORTED, "msa_sparse_attn_split: hq/hkv = %d unsupported", G);
+    if (T == 0) return MSA_OK;
+    MSA_REQUIRE(q && out && mem_len && ws, "msa_sparse_attn_split: NULL pointer");
+    MSA_REQUIRE(max_mem == 0 || mem_kv, "msa_sparse_attn_split: NULL mem_kv");
+    MSA_REQUIRE(L == 0 || (local_k && local_v), "msa_sparse_attn_split: NULL local K/V");
+    MSA_REQUIRE(aligned16(q) && aligned16(out) && aligned16(ws) && (max_mem == 0 || aligned16(mem_kv)) &&
+                    (L == 0 || (aligned16(local_k) && aligned16(local_v))),
+                "msa_sparse_attn_split: pointers must be 16-byte aligned");
+    const int n_split = pick_splits(n_q, T, hq, hkv, max_mem, L);
+    const size_t need = split_ws_bytes(n_split, n_q, T, hq);
+    if (ws_bytes < need)
+        return set_error(MSA_ERR_WORKSPACE, "msa_sparse_attn_split: workspace %zu < %zu", ws_bytes, need);
+    AttnArgs a{};
+    a.q = q; a.mem_kv = mem_kv; a.mem_len = mem_len; a.max_mem = max_mem;
+    a.local_k = local_k; a.local_v = local_v; a.L_max = L_max; a.L = L; a.q_start = q_start;
+    a.T = T; a.hq = hq; a.hkv = hkv; a.scale_log2e = scale * 1.4426950408889634f; a.out = out;
+    a.n_split = n_split;
+    a.part_o = static_cast<float*>(ws);
+    a.part_ml = reinterpret_cast<float2*>(static_cast<char*>(ws) +
+                                          align_up((size_t)n_split * n_q * T * hq * kD * 4, 256));
+    return launch_mma<true>(a, n_q, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

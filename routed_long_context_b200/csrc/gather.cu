@@ -3,6 +3,8 @@
 // The bank is [n_chunks][2][hkv][d]: one document is one contiguous byte run, so each selected
 // document is one cudaMemcpyAsync host -> device on the copy stream (the copy engines over the
 // host link), written into the query's slot at the running row offset (rank order).
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -55,7 +57,9 @@ msa_status msa_gather_kv(const void* host_bank, msa_dtype dt, int64_t n_chunks, 
 // ------------------------------------------------------------------------------------------------
 // Device-side fetch: a kernel reads the selected documents' rows straight from the pinned host bank
 // (mapped into the device's address space) using device-resident indices, so selection and fetch
-// need no host round trip. One block per (rank, query); 16-byte loads over the host link.
+// need no host round trip. Blocks (rank, query, part): a document's 16-byte words are dealt out to
+// gridDim.z blocks (one for compressed chunk rows, up to 32 for the token rows of the fine stage)
+// so enough loads are in flight over the host link.
 // ------------------------------------------------------------------------------------------------
 namespace msa {
 namespace {
@@ -93,18 +97,19 @@ __global__ void __launch_bounds__(256) gather_device_kernel(const uint4* __restr
         if (threadIdx.x == 0) record_device_error(err, MSA_DEV_BAD_INDEX);
         return;
     }
-    if (r == k - 1 && threadIdx.x == 0) mem_len[q] = (int32_t)(at + rows);
+    if (r == k - 1 && blockIdx.z == 0 && threadIdx.x == 0) mem_len[q] = (int32_t)(at + rows);
     const uint4* src = bank + a * row_vec;
     uint4* dst = out + ((int64_t)q * max_mem + at) * row_vec;
     const int64_t n = rows * row_vec;
-    for (int64_t i = threadIdx.x; i < n; i += 4 * blockDim.x) {
+    const int64_t step = (int64_t)gridDim.z * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.z * blockDim.x + threadIdx.x; i < n; i += 4 * step) {
         uint4 v[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u)
-            if (i + u * blockDim.x < n) v[u] = src[i + u * blockDim.x];
+            if (i + u * step < n) v[u] = src[i + u * step];
 #pragma unroll
         for (int u = 0; u < 4; ++u)
-            if (i + u * blockDim.x < n) dst[i + u * blockDim.x] = v[u];
+            if (i + u * step < n) dst[i + u * step] = v[u];
     }
 }
 
@@ -121,7 +126,10 @@ msa_status gather_device(const void* host_bank, msa_dtype dt, int64_t n_chunks, 
     const size_t row = (size_t)2 * hkv * d * dtype_size(dt);
     if (row % 16 != 0 || !aligned16(dptr) || !aligned16(dev_mem_kv))
         return set_error(MSA_ERR_INVALID_ARG, "device fetch: rows and pointers must be 16-byte aligned");
-    dim3 grid(k, n_q);
+    // words per document if the rows were spread evenly; one block per 8K words, at most 32
+    const int64_t words = ((int64_t)max_mem * (int64_t)(row / 16)) / k;
+    const int parts = (int)std::min<int64_t>(32, std::max<int64_t>(1, (words + 8191) / 8192));
+    dim3 grid(k, n_q, parts);
     gather_device_kernel<<<grid, 256, 0, s>>>(static_cast<const uint4*>(dptr), n_chunks, doc_chunk_off, n_docs, idx, k,
                                               (int)(row / 16), max_mem, static_cast<uint4*>(dev_mem_kv), mem_len,
                                               device_error_word());

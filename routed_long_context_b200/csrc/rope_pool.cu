@@ -297,6 +297,42 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendArgs a) {
                        static_cast<T*>(y.q_rot) + ((int64_t)q * a.T_new + t) * Eq, Eq, a.d, cs_row, true);
 }
 
+// ---------------------------------------------------------------------------------------------
+// Token-level memory bank of the fine stage: block-stride over token rows; row r of document i
+// (found by binary search of the token offsets) gets its key rotated to its position inside the
+// document, r - doc_tok_off[i], into bank[r][0], and its value copied into bank[r][1].
+struct PackArgs {
+    const void* k;
+    const void* v;
+    int64_t n_tok;
+    int hkv, d;
+    const int64_t* doc_tok_off;
+    int64_t n_docs;
+    const float2* cs;
+    int64_t max_pos;
+    void* bank;
+    int* err;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(128) pack_tokens_kernel(const PackArgs a) {
+    const int E = a.hkv * a.d;
+    for (int64_t r = blockIdx.x; r < a.n_tok; r += gridDim.x) {
+        int64_t lo = 0, hi = a.n_docs - 1;   // largest i with doc_tok_off[i] <= r
+        while (lo < hi) {
+            const int64_t mid = (lo + hi + 1) >> 1;
+            if (a.doc_tok_off[mid] <= r) lo = mid; else hi = mid - 1;
+        }
+        const int64_t p = r - a.doc_tok_off[lo];
+        const bool pos_ok = p >= 0 && p < a.max_pos;
+        if (!pos_ok && threadIdx.x == 0) record_device_error(a.err, MSA_DEV_ROPE_POSITION);
+        T* dst = static_cast<T*>(a.bank) + r * 2 * (int64_t)E;
+        rotate_copy_row<T>(static_cast<const T*>(a.k) + r * E, dst, E, a.d, pos_ok ? a.cs + p * (a.d / 2) : nullptr,
+                           true);
+        rotate_copy_row<T>(static_cast<const T*>(a.v) + r * E, dst + E, E, a.d, nullptr, false);
+    }
+}
+
 template <typename T>
 bool vec_layout_ok(int d) {
     constexpr int VEC = 16 / sizeof(T);
@@ -330,6 +366,18 @@ msa_status launch_append(const AppendArgs& a, msa_dtype dt, cudaStream_t s) {
     return MSA_OK;
 }
 
+msa_status launch_pack_tokens(const PackArgs& a, msa_dtype dt, cudaStream_t s) {
+    if (a.n_tok == 0) return MSA_OK;
+    const int64_t cap = (int64_t)sm_count() * 16;
+    const unsigned blocks = (unsigned)(a.n_tok < cap ? a.n_tok : cap);
+    if (dt == MSA_BF16)
+        pack_tokens_kernel<__nv_bfloat16><<<blocks, 128, 0, s>>>(a);
+    else
+        pack_tokens_kernel<float><<<blocks, 128, 0, s>>>(a);
+    MSA_LAUNCH_CHECK();
+    return MSA_OK;
+}
+
 bool rope_layout_ok(msa_dtype dt, int d) {
     return dt == MSA_BF16 ? vec_layout_ok<__nv_bfloat16>(d) : vec_layout_ok<float>(d);
 }
@@ -357,6 +405,25 @@ msa_status msa_rope_doc(const void* x, void* out, msa_dtype dt, int64_t n_tok, i
     a.pos_offset = pos_offset; a.cs = reinterpret_cast<const float2*>(cos_sin); a.max_pos = max_pos;
     a.err = device_error_word();
     return launch_rope_rows(a, dt, static_cast<cudaStream_t>(stream));
+}
+
+msa_status msa_pack_tokens(const void* k, const void* v, msa_dtype dt, int64_t n_tok, int hkv, int d,
+                           const int64_t* doc_tok_off, int64_t n_docs, const float* cos_sin, int64_t max_pos,
+                           void* bank, void* stream) {
+    MSA_REQUIRE(dtype_ok(dt), "msa_pack_tokens: bad dtype %d", dt);
+    MSA_REQUIRE(n_tok >= 0 && hkv > 0 && d > 0 && n_docs > 0 && max_pos > 0, "msa_pack_tokens: bad sizes");
+    if (n_tok == 0) return MSA_OK;
+    MSA_REQUIRE(k && v && doc_tok_off && cos_sin && bank, "msa_pack_tokens: NULL pointer");
+    MSA_REQUIRE(aligned16(k) && aligned16(v) && aligned16(bank) && aligned16(cos_sin),
+                "msa_pack_tokens: pointers must be 16-byte aligned");
+    if (!rope_layout_ok(dt, d))
+        return set_error(MSA_ERR_UNSUPPORTED, "msa_pack_tokens: head layout hkv=%d d=%d unsupported", hkv, d);
+    PackArgs a{};
+    a.k = k; a.v = v; a.n_tok = n_tok; a.hkv = hkv; a.d = d;
+    a.doc_tok_off = doc_tok_off; a.n_docs = n_docs;
+    a.cs = reinterpret_cast<const float2*>(cos_sin); a.max_pos = max_pos;
+    a.bank = bank; a.err = device_error_word();
+    return launch_pack_tokens(a, dt, static_cast<cudaStream_t>(stream));
 }
 
 msa_status msa_pool_chunks(const void* k, const void* v, const void* kr, msa_dtype in_dt, int64_t n_tok, int hkv,

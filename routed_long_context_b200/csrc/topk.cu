@@ -477,3 +477,111 @@ msa_status msa_topk_docs_noalloc(const float* doc_scores, int n_q, int64_t n_doc
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------------------
+// Memory Parallel merge: the k best of every shard's local top-k candidates. Each candidate becomes
+// one 64-bit key, order-preserving float bits of its score above the complement of its global
+// document index, so that a larger key is a better candidate (higher score, then lower index);
+// no candidate (-1) gets key 0, a NaN score ranks below -inf. One block per query counts, for each
+// candidate, the candidates that beat it (ties of equal keys by position): that count is its rank.
+// ------------------------------------------------------------------------------------------------
+namespace msa {
+namespace {
+
+constexpr int kMergeMaxShards = 64;
+constexpr int kMergeMaxCand = 4096;
+constexpr int kMergeThreads = 256;
+
+struct MergeArgs {
+    const float* cand_score;
+    const int32_t* cand_idx;
+    int64_t shard_stride;
+    int n_shards, n_q, k_cand, k;
+    int64_t shard_off[kMergeMaxShards + 1];
+    int32_t* idx;
+    float* score;
+    int* err;
+};
+
+__device__ __forceinline__ uint32_t ordered_bits(float f) {
+    const uint32_t b = f == 0.f ? 0u : __float_as_uint(f);   // -0 and +0 compare equal
+    if (f != f) return 1u;                                  // NaN: just above "no candidate"
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+__device__ __forceinline__ float from_ordered_bits(uint32_t o) {
+    if (o == 1u) return __int_as_float(0x7fc00000);
+    return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
+}
+
+__global__ void __launch_bounds__(kMergeThreads) topk_merge_kernel(const MergeArgs a) {
+    __shared__ unsigned long long keys[kMergeMaxCand];
+    const int q = blockIdx.x;
+    const int n = a.n_shards * a.k_cand;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int g = i / a.k_cand, r = i % a.k_cand;
+        const int64_t at = (int64_t)g * a.shard_stride + (int64_t)q * a.k_cand + r;
+        const int32_t local = a.cand_idx[at];
+        const int64_t size = a.shard_off[g + 1] - a.shard_off[g];
+        unsigned long long key = 0ull;
+        if (local >= 0 && local < size) {
+            const uint32_t gi = (uint32_t)(a.shard_off[g] + local);
+            key = ((unsigned long long)ordered_bits(a.cand_score[at]) << 32) | (unsigned long long)(0xffffffffu - gi);
+        } else if (local != -1) {
+            record_device_error(a.err, MSA_DEV_BAD_INDEX);
+        }
+        keys[i] = key;
+    }
+    for (int r = n + threadIdx.x; r < a.k; r += blockDim.x) {   // fewer candidates than k
+        a.idx[(int64_t)q * a.k + r] = -1;
+        if (a.score) a.score[(int64_t)q * a.k + r] = -__int_as_float(0x7f800000);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const unsigned long long ki = keys[i];
+        int rank = 0;
+        for (int j = 0; j < n && rank < a.k; ++j) {
+            const unsigned long long kj = keys[j];
+            rank += (kj > ki) || (kj == ki && j < i);
+        }
+        if (rank < a.k) {
+            const bool valid = ki != 0ull;
+            a.idx[(int64_t)q * a.k + rank] = valid ? (int32_t)(0xffffffffu - (uint32_t)(ki & 0xffffffffull)) : -1;
+            if (a.score)
+                a.score[(int64_t)q * a.k + rank] =
+                    valid ? from_ordered_bits((uint32_t)(ki >> 32)) : -__int_as_float(0x7f800000);
+        }
+    }
+}
+
+}  // namespace
+}  // namespace msa
+
+extern "C" {
+
+msa_status msa_topk_merge(const float* cand_score, const int32_t* cand_idx, int64_t shard_stride, int n_shards,
+                          int n_q, int k_cand, const int64_t* shard_doc_off, int k, int32_t* idx, float* score,
+                          void* stream) {
+    MSA_REQUIRE(cand_score && cand_idx && shard_doc_off && idx, "msa_topk_merge: NULL pointer");
+    MSA_REQUIRE(n_shards >= 1 && n_shards <= kMergeMaxShards, "msa_topk_merge: 1 <= n_shards <= %d", kMergeMaxShards);
+    MSA_REQUIRE(n_q >= 1 && n_q <= INT_MAX / 2 && k_cand >= 1 && (int64_t)n_shards * k_cand <= kMergeMaxCand,
+                "msa_topk_merge: need n_q >= 1, k_cand >= 1, n_shards * k_cand <= %d", kMergeMaxCand);
+    MSA_REQUIRE(k >= 1 && k <= 64, "msa_topk_merge: need 1 <= k <= 64, got %d", k);
+    MSA_REQUIRE(shard_stride >= (int64_t)n_q * k_cand, "msa_topk_merge: shard_stride < n_q * k_cand");
+    MergeArgs a{};
+    a.shard_off[0] = shard_doc_off[0];
+    MSA_REQUIRE(shard_doc_off[0] >= 0, "msa_topk_merge: negative shard offset");
+    for (int g = 0; g < n_shards; ++g) {
+        MSA_REQUIRE(shard_doc_off[g + 1] >= shard_doc_off[g], "msa_topk_merge: shard offsets must not decrease");
+        a.shard_off[g + 1] = shard_doc_off[g + 1];
+    }
+    MSA_REQUIRE(shard_doc_off[n_shards] < (int64_t)INT_MAX, "msa_topk_merge: global document index exceeds int32");
+    a.cand_score = cand_score; a.cand_idx = cand_idx; a.shard_stride = shard_stride;
+    a.n_shards = n_shards; a.n_q = n_q; a.k_cand = k_cand; a.k = k;
+    a.idx = idx; a.score = score; a.err = device_error_word();
+    topk_merge_kernel<<<n_q, kMergeThreads, 0, static_cast<cudaStream_t>(stream)>>>(a);
+    MSA_LAUNCH_CHECK();
+    return MSA_OK;
+}
+
+}  // extern "C"

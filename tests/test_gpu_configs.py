@@ -201,6 +201,56 @@ def test_1m_end_to_end(m):
     _free()
 
 
+def test_1m_fine_stage(m):
+    """Token-level fine stage on the 1M configuration: route on the pooled index and select as
+    before, then fetch the selected documents' token rows from the pinned token bank (host-issued
+    copies and the device kernel, equal bit for bit) and attend over them with split key ranges;
+    against the oracle's token bank and attention over the same documents."""
+    from routed_long_context_b200.bank import BankLayout, to_host_bank
+
+    w = workloads.mem_1m()
+    lay = BankLayout.from_doc_lengths(w.doc_len, w.chunk)
+    cs = m.rope_table(4096, w.d, w.rope_base)
+    k, v, kr = (memory_tensor(w, 0, n) for n in ("k", "v", "kr"))
+    _, index = m.msa_pool_chunks(None, None, kr, lay.doc_tok_off, lay.doc_chunk_off, lay.chunk_doc, w.chunk)
+    tok = m.msa_pack_tokens(k, v, lay.doc_tok_off, cs)
+    del k, v, kr
+    host_tok = to_host_bank(tok)
+    del tok
+    _free()
+    dv = small_tensors(w, 0)
+    ds = m.msa_route_scores(index, lay.chunk_doc, lay.n_docs, dv["qr"])
+    idx, _ = m.msa_topk_docs(ds, w.k)
+    max_mem = w.k * int(w.doc_len.max())
+    mem_d, len_d = m.msa_gather_kv_device(host_tok, lay.doc_tok_off, idx, max_mem)
+    mem_h, len_h = m.msa_gather_kv(host_tok, w.doc_tok_off, idx.cpu(), max_mem)
+    T = w.T0
+    seg = torch.tensor([0, T], dtype=torch.int64, device="cuda")
+    lk = m.msa_rope_doc(dv["k_new"][0], seg, w.k, cs, out=torch.empty_like(dv["k_new"][0]))
+    qq = m.msa_rope_doc(dv["q"][0], seg, w.k, cs, out=torch.empty_like(dv["q"][0]))
+    out = m.msa_sparse_attn_split(qq[None], mem_d, len_d, lk[None], dv["v_new"], T, 0)
+    torch.cuda.synchronize()
+    assert m.device_status() == 0
+
+    gi = idx.cpu().numpy()[0]
+    assert set(w.expected(0, 0, 0)) <= set(gi.tolist())
+    n = int(len_h[0])
+    assert int(len_d.cpu()[0]) == n == int(sum(w.doc_len[gi]))
+    assert torch.equal(mem_d[0, :n].cpu(), mem_h[0, :n].cpu())
+    rows = np.concatenate([np.arange(w.doc_tok_off[d], w.doc_tok_off[d + 1]) for d in gi])
+    k_sel = w.host_rows(0, "k", rows).reshape(n, w.hkv, w.d)
+    v_sel = w.host_rows(0, "v", rows).reshape(n, w.hkv, w.d)
+    tb = O.token_bank(k_sel, v_sel, np.concatenate([[0], np.cumsum(w.doc_len[gi])]), w.rope_base)
+    got = _np(mem_d[0, :n])
+    np.testing.assert_allclose(got[:, 0], tb[:, 0], atol=1e-5, rtol=2.0 ** -8)
+    np.testing.assert_array_equal(got[:, 1], tb[:, 1])
+    kl = O.apply_rope(w.k_new(0)[0], O.global_positions(w.k, 0, T), w.rope_base)
+    qo = O.apply_rope(w.q(0)[0], O.global_positions(w.k, 0, T), w.rope_base)
+    o = O.sparse_attention(qo, tb[:, 0], tb[:, 1], kl, w.v_new(0)[0], 0, 1 / np.sqrt(w.d))
+    assert _row_rel_err(_np(out)[0], o) <= 2e-2
+    _free()
+
+
 # ------------------------------------------------------------------------------------------ 10M
 def test_10m_encode_and_decode_routing(m):
     from routed_long_context_b200.bank import BankLayout, encode_tokens, to_host_bank

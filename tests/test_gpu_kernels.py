@@ -294,6 +294,84 @@ def test_sparse_attention_no_keys_gives_zero(m):
     assert torch.count_nonzero(out) == 0
 
 
+# -------------------------------------------------------------------------------------- fine stage
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_pack_tokens_matches_oracle(m, dtype):
+    """Token bank of the fine stage: keys rotated to their position inside their document, values
+    copied bit for bit; empty and one-token documents included."""
+    off = np.array([0, 300, 300, 555, 1000, 1001], dtype=np.int64)
+    n, hkv, d = int(off[-1]), 8, 128
+    k, v = _gen(100, (n, hkv, d), dtype), _gen(101, (n, hkv, d), dtype)
+    cs = m.rope_table(1024, d, 1e6)
+    bank = m.msa_pack_tokens(upload(k, dtype), upload(v, dtype), torch.from_numpy(off).cuda(), cs)
+    _status(m)
+    ref = O.token_bank(k, v, off, 1e6)
+    _close(_np(bank[:, 0]), ref[:, 0], dtype, "token bank K")
+    np.testing.assert_array_equal(_np(bank[:, 1]), v)
+
+
+def test_pack_tokens_position_past_table_is_flagged_not_faulted(m):
+    off = np.array([0, 40], dtype=np.int64)
+    k = upload(_gen(106, (40, 8, 128)), "f32")
+    m.msa_pack_tokens(k, k, torch.from_numpy(off).cuda(), m.rope_table(32, 128, 1e6))
+    assert m.device_status() == 1                                      # MSA_DEV_ROPE_POSITION
+
+
+def test_device_gather_token_rows_over_many_blocks(m):
+    """Token-level documents (hundreds of rows each) are fetched by several blocks per document;
+    the result equals the host-issued copies and the rank-ordered row copy."""
+    lens = np.array([1000, 1792, 0, 256, 1500, 77], dtype=np.int64)
+    off = np.concatenate([[0], np.cumsum(lens)])
+    bank = torch.from_numpy(_gen(107, (int(off[-1]), 2, 8, 128), "bf16")).to(torch.bfloat16).pin_memory()
+    idx = torch.tensor([[1, 0, 4], [3, 5, 2]], dtype=torch.int32)
+    max_mem = 3 * 1792
+    ref, ref_len = m.msa_gather_kv(bank, off, idx, max_mem=max_mem)
+    dev, dev_len = m.msa_gather_kv_device(bank, torch.from_numpy(off).cuda(), idx.cuda(), max_mem=max_mem)
+    torch.cuda.synchronize()
+    assert dev_len.cpu().tolist() == ref_len.tolist() == [4292, 333]
+    host = bank.float().numpy()
+    for q, n in enumerate(ref_len.tolist()):
+        assert torch.equal(dev[q, :n].cpu(), ref[q, :n].cpu())
+        np.testing.assert_array_equal(dev[q, :n].float().cpu().numpy(), O.gather_memory(host, off, idx[q].tolist()))
+    _status(m)
+
+
+@pytest.mark.parametrize("hq,hkv", [(32, 8), (8, 8), (32, 4)])
+@pytest.mark.parametrize("T,mem_lens,q_start", [(64, (0, 700, 1537), 0), (24, (4099, 1, 64), 40)])
+def test_sparse_attention_split_long_memory(m, hq, hkv, T, mem_lens, q_start):
+    """Split-key attention over long memories: several key ranges per block (some empty), ragged
+    tails, empty memory, causal local keys; against the oracle within the bf16 bound."""
+    n_q, d, dtype = 3, 128, "bf16"
+    max_mem = max(mem_lens) + 5
+    L = q_start + T
+    q = _gen(102, (n_q, T, hq, d), dtype)
+    mem = _gen(103, (n_q, max_mem, 2, hkv, d), dtype)
+    lk, lv = _gen(104, (n_q, L + 3, hkv, d), dtype), _gen(105, (n_q, L + 3, hkv, d), dtype)
+    mem_len = np.array(mem_lens, dtype=np.int32)
+    rows = n_q * T * hq
+    assert m.sparse_attn_split_workspace_size(n_q, T, hq, hkv, max_mem, L) >= 2 * rows * (d * 4 + 8)   # >= 2 ranges
+    out = m.msa_sparse_attn_split(upload(q, dtype), upload(mem, dtype), torch.from_numpy(mem_len).cuda(),
+                                  upload(lk, dtype), upload(lv, dtype), L, q_start)
+    _status(m)
+    got = _np(out)
+    for qi in range(n_q):
+        ml = mem_len[qi]
+        ref = O.sparse_attention(q[qi], mem[qi, :ml, 0], mem[qi, :ml, 1], lk[qi, :L], lv[qi, :L], q_start,
+                                 1 / np.sqrt(d))
+        assert _row_rel_err(got[qi], ref) <= 2e-2
+
+
+def test_sparse_attention_split_no_keys_gives_zero_and_rejects_fp32(m):
+    q = upload(_gen(108, (2, 4, 32, 128), "bf16"), "bf16")
+    mem = torch.zeros((2, 300, 2, 8, 128), dtype=torch.bfloat16, device="cuda")
+    lk = torch.zeros((2, 4, 8, 128), dtype=torch.bfloat16, device="cuda")
+    out = m.msa_sparse_attn_split(q, mem, torch.zeros(2, dtype=torch.int32, device="cuda"), lk, lk, 0, 0)
+    assert torch.count_nonzero(out) == 0
+    with pytest.raises(m.MSAError):
+        m.msa_sparse_attn_split(q.float(), mem.float(), torch.zeros(2, dtype=torch.int32, device="cuda"), lk.float(),
+                                lk.float(), 0, 0)
+
+
 # -------------------------------------------------------------------------------------- incremental append
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_growable_bank_append_equals_full_encode_bitwise(m, dtype):
