@@ -4,3 +4,4 @@ Only the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline /
 reference arm may import this package; the product path never does.
 """
 from .msa_oracle import *  # noqa: F401,F403
+from .msa_backward import *  # noqa: F401,F403
