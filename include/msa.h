@@ -240,11 +240,12 @@ msa_status msa_gather_kv(const void* host_bank, msa_dtype dt, int64_t n_chunks, 
 /* Device-side variant of msa_gather_kv: a kernel on `stream` reads the selected documents' rows
  * straight from the pinned host bank (mapped into the device address space; the pointer must come
  * from cudaHostAlloc / torch pin_memory) with device-resident indices, so no host round trip sits
- * between selection and fetch. Same layout and rank order as msa_gather_kv.
+ * between selection and fetch. Same layout and rank order as msa_gather_kv. A bank in the current
+ * device's own memory (a training context) is accepted too and read directly.
  *   doc_chunk_off: device int64 [n_docs+1]; idx: device int32 [n_q][k]; mem_len: device int32 [n_q].
  * Indices out of range or more rows than max_mem record MSA_DEV_BAD_INDEX and skip that query's
  * copy (no out-of-range access). Long documents (token rows of the fine stage) are split over
- * several blocks, chosen from max_mem / k. Returns MSA_ERR_INVALID_ARG if host_bank is not pinned, mapped
+ * several blocks, chosen from max_mem / k. Returns MSA_ERR_INVALID_ARG if host_bank is neither device memory nor pinned, mapped
  * host memory. */
 msa_status msa_gather_kv_device(const void* host_bank, msa_dtype dt, int64_t n_chunks, const int64_t* doc_chunk_off,
                                 int64_t n_docs, const int32_t* idx, int n_q, int k, int hkv, int d, int max_mem,
@@ -275,12 +276,88 @@ msa_status msa_attn_set_impl(int impl);
  * the workspace; a second kernel merges the ranges' softmax statistics and writes out.
  * n_split is chosen from the sizes so that the grid fits one wave of three blocks per SM (148
  * SMs), at least four tiles per range. bf16 only (tensor cores); fp32 returns MSA_ERR_UNSUPPORTED.
+ * lse: optional device float [n_q][T][hq]: ln sum_j exp(scale * q . k_j) over the row's visible
+ * keys (-inf for a row without one), what msa_sparse_attn_backward needs from the forward pass.
  * ws: device, msa_sparse_attn_split_workspace_size bytes, 16-byte aligned. */
 msa_status msa_sparse_attn_split(const void* q, const void* mem_kv, const int32_t* mem_len, int max_mem,
                                  const void* local_k, const void* local_v, int L_max, int L, int q_start, int n_q,
-                                 int T, int hq, int hkv, int d, float scale, void* out, msa_dtype dt, void* ws,
-                                 size_t ws_bytes, void* stream);
+                                 int T, int hq, int hkv, int d, float scale, void* out, float* lse, msa_dtype dt,
+                                 void* ws, size_t ws_bytes, void* stream);
 msa_status msa_sparse_attn_split_workspace_size(int n_q, int T, int hq, int hkv, int max_mem, int L, size_t* bytes);
+
+/* ---------------------------------------------------------------------------------------------
+ * Backward pass (end-to-end training: [P1] 核心创新 端到端可训练性 — routing, compression and
+ * attention are optimised in one gradient flow; [P1] §训练策略 and [P2] §训练层面 — a weighted
+ * auxiliary loss supervises every layer's router). The top-k selection carries no gradient. All
+ * gradients are fp32; device pointers; calls are asynchronous on `stream`.
+ * --------------------------------------------------------------------------------------------- */
+
+/* Gradients of msa_sparse_attn / msa_sparse_attn_split with respect to q, the fetched memory and
+ * the local K/V, given dout = dL/dout. Same layouts and sizes as the forward; out (bf16) and
+ * lse (msa_sparse_attn_split's log-sum-exp) come from the forward pass.
+ *   dq: [n_q][T][hq][d]; dmem_kv: [n_q][max_mem][2][hkv][d] (rows < mem_len[q] written);
+ *   dlocal_k, dlocal_v: [n_q][L_max][hkv][d] (rows < L written). All overwritten, not added to.
+ * For each row, with P the softmax of the forward: dV = P^T dO, dS = P * (dO V^T - rowsum(dO*O)),
+ * dq = scale dS K, dK = scale dS^T q, summed over the query heads that share a kv head. Tensor
+ * cores (mma.sync, bf16 operands: P and dS are rounded to bf16, fp32 accumulation); each key's
+ * gradient is accumulated by one block over every row (no atomics). bf16 only, d == 128,
+ * hq/hkv in {1, 2, 4, 8}. ws: msa_sparse_attn_backward_workspace_size bytes. */
+msa_status msa_sparse_attn_backward(const void* q, const void* mem_kv, const int32_t* mem_len, int max_mem,
+                                    const void* local_k, const void* local_v, int L_max, int L, int q_start, int n_q,
+                                    int T, int hq, int hkv, int d, float scale, const void* out, const void* dout,
+                                    const float* lse, msa_dtype dt, float* dq, float* dmem_kv, float* dlocal_k,
+                                    float* dlocal_v, void* ws, size_t ws_bytes, void* stream);
+msa_status msa_sparse_attn_backward_workspace_size(int n_q, int T, int hq, size_t* bytes);
+
+/* Adjoint of the fetch (msa_gather_kv_device): query q's memory-row gradients dmem_kv
+ * [n_q][max_mem][2][hkv][d] (fp32) are ADDED to the chunk rows of dkvbar [n_chunks][2][hkv][d]
+ * (fp32, zeroed by the caller) they were copied from, following idx [n_q][k] and doc_chunk_off
+ * (device) in rank order; a document selected by several queries receives the sum (fp32 atomic
+ * adds, so the summation order varies). Bad indices record MSA_DEV_BAD_INDEX and are skipped. */
+msa_status msa_gather_kv_backward(const float* dmem_kv, int64_t n_chunks, const int64_t* doc_chunk_off,
+                                  int64_t n_docs, const int32_t* idx, int n_q, int k, int hkv, int d, int max_mem,
+                                  float* dkvbar, void* stream);
+
+/* Adjoint of msa_pool_chunks: token gradients from chunk gradients.
+ *   dkvbar: fp32 [n_chunks][2][hkv][d] (dK-bar, dV-bar) or NULL; then dk, dv: fp32 [n_tok][hkv][d]
+ *     with dk[t] = R(-p_t) dK-bar[c] / n_c (p_t the token's position in its document; without
+ *     fuse_doc_rope no rotation) and dv[t] = dV-bar[c] / n_c for every token t of chunk c (n_c tokens).
+ *   dkr_index: fp32 [n_chunks][hr][d] or NULL, the gradient with respect to the stored router index;
+ *     then dkr: fp32 [n_tok][hr][d]. With normalize_router the index was unit(K-bar^R) per head and
+ *     the gradient passes through the normalisation, (g - k_hat (k_hat . g)) / |K-bar^R|, the raw
+ *     chunk mean K-bar^R being recomputed from kr (token K^R [n_tok][hr][d] of kr_dt); without it
+ *     kr may be NULL. Needs hr * d <= 1024 and (normalised) d a multiple of 32 up to 256.
+ * Offsets, table and chunking as for msa_pool_chunks. */
+msa_status msa_pool_chunks_backward(const float* dkvbar, const float* dkr_index, const void* kr, msa_dtype kr_dt,
+                                    int64_t n_tok, int hkv, int hr, int d, const int64_t* doc_tok_off,
+                                    const int64_t* doc_chunk_off, const int32_t* chunk_doc, int64_t n_docs,
+                                    int64_t n_chunks, int chunk, int fuse_doc_rope, const float* cos_sin,
+                                    int64_t max_pos, int normalize_router, float* dk, float* dv, float* dkr,
+                                    void* stream);
+
+/* Auxiliary router loss and its gradient (reading of [P1] §训练策略 辅助损失, which states the
+ * supervision but no formula): for query q with evidence documents E_q (evidence [n_q][n_ev] int32,
+ * -1 = padding), s = doc_scores[q] / tau,
+ *   loss[q] = -(1/|E_q|) sum_{e in E_q} (s_e - log sum_i exp s_i)      (loss may be NULL)
+ *   d_doc_scores[q][i] = (softmax(s)_i - [i in E_q] / |E_q|) / tau / n_q
+ * i.e. the gradient of the mean of loss[] over the queries. One block per query. */
+msa_status msa_router_aux_loss(const float* doc_scores, int n_q, int64_t n_docs, const int32_t* evidence, int n_ev,
+                               float tau, float* loss, float* d_doc_scores, void* stream);
+
+/* Gradients of msa_route_scores' document scores given d_doc_scores [n_q][n_docs] (fp32):
+ * each document's score is attained at one (chunk, query token) pair — the first chunk, then the
+ * first token, on exact ties — and only that pair receives its gradient:
+ *   dqr [n_q][T][H][d] (fp32): with respect to the raw router queries, through their per-head
+ *     normalisation;
+ *   dkhat [n_chunks][H][d] (fp32, overwritten): with respect to the stored index vectors as used
+ *     in the dot product (msa_pool_chunks_backward carries it through the index normalisation).
+ * Scores are recomputed in fp32 on CUDA cores to find the attaining pairs (a training-context
+ * bank, not the 100M inference index). kr_index and qr of dtype dt; H * d <= 1024.
+ * ws: msa_route_backward_workspace_size bytes. */
+msa_status msa_route_backward(const void* kr_index, msa_dtype dt, int64_t n_chunks, const int64_t* doc_chunk_off,
+                              int64_t n_docs, const void* qr, int n_q, int T, int H, int d, const float* d_doc_scores,
+                              float* dqr, float* dkhat, void* ws, size_t ws_bytes, void* stream);
+msa_status msa_route_backward_workspace_size(int64_t n_chunks, int n_q, int T, int H, int d, size_t* bytes);
 
 /* One routed layer of one Memory Interleave round (see msa_interleave_step). */
 typedef struct msa_layer_args {

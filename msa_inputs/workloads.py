@@ -307,4 +307,12 @@ def interleave(layers: int = 18, n_host_banks: int = 2) -> Workload:
                     plant_kind="chain")
 
 
-CONFIGS = {"tiny": tiny, "1m": mem_1m, "10m": mem_10m, "100m": mem_100m, "interleave": interleave}
+def train64k() -> Workload:
+    """Training context: 16 docs x 4096 tokens (65,536), chunk 128, bf16; one query of 512 tokens that
+    routes and attends (causal over itself); top-4; 2 planted documents (the router's evidence)."""
+    return Workload("train64k", SEED_BASE + 5, np.full(16, 4096), 128, "bf16", n_q=1, T0=512, k=4,
+                    plant_kind="single", plant_args={"n": 2})
+
+
+CONFIGS = {"tiny": tiny, "1m": mem_1m, "10m": mem_10m, "100m": mem_100m, "interleave": interleave,
+           "train64k": train64k}

@@ -140,12 +140,13 @@ def router_aux_loss(doc_scores: np.ndarray, evidence, tau: float):
     return loss / n_q, grad
 
 
-def route_argmax(kr_index: np.ndarray, doc_chunk_off: np.ndarray, qr: np.ndarray):
+def route_argmax(kr_index: np.ndarray, doc_chunk_off: np.ndarray, qr: np.ndarray, index_is_unit: bool = False):
     """For every (query, document): the chunk c and query token t where the document's score
     max_c max_t mean_h cos is attained (the lowest chunk, then the lowest token, on exact ties;
-    -1 for a document without chunks)."""
+    -1 for a document without chunks). With index_is_unit the key vectors are taken as stored
+    (the index form, already normalised once) instead of being normalised again."""
     qh = unit(np.asarray(qr, dtype=F64))                  # [n_q, T, H, d]
-    kh = unit(np.asarray(kr_index, dtype=F64))            # [C, H, d]
+    kh = np.asarray(kr_index, dtype=F64) if index_is_unit else unit(np.asarray(kr_index, dtype=F64))
     H = kh.shape[1]
     D = len(doc_chunk_off) - 1
     n_q = qh.shape[0]
@@ -161,19 +162,23 @@ def route_argmax(kr_index: np.ndarray, doc_chunk_off: np.ndarray, qr: np.ndarray
     return arg_c, arg_t
 
 
-def route_backward(kr_index: np.ndarray, doc_chunk_off: np.ndarray, qr: np.ndarray, d_doc_scores: np.ndarray):
+def route_backward(kr_index: np.ndarray, doc_chunk_off: np.ndarray, qr: np.ndarray, d_doc_scores: np.ndarray,
+                   index_is_unit: bool = False):
     """Gradients of the router's document scores (msa_oracle.route) given dL/d doc score.
 
     The max over chunks and tokens passes the gradient to the attaining pair only; there
     score = (1/H) sum_h <q_hat_h, k_hat_h>, so dq_hat_h = ds k_hat_h / H and dk_hat_h = ds q_hat_h / H.
     Returns (dqr [n_q, T, H, d], the gradient with respect to the raw router queries, through their
     normalisation; dk_hat [C, H, d], the gradient with respect to the unit key vectors k_hat =
-    unit(kr_index); unit_backward(kr_index, dk_hat) carries it to kr_index itself)."""
+    unit(kr_index); unit_backward(kr_index, dk_hat) carries it to kr_index itself). With index_is_unit
+    the stored index vectors are the k_hat themselves (how the index form is scored: a dot product
+    with vectors normalised once and stored), which also decides the attaining chunks."""
     qr = np.asarray(qr, dtype=F64)
     ds = np.atleast_2d(np.asarray(d_doc_scores, dtype=F64))
-    qh, kh = unit(qr), unit(np.asarray(kr_index, dtype=F64))
+    qh = unit(qr)
+    kh = np.asarray(kr_index, dtype=F64) if index_is_unit else unit(np.asarray(kr_index, dtype=F64))
     H = kh.shape[1]
-    arg_c, arg_t = route_argmax(kr_index, doc_chunk_off, qr)
+    arg_c, arg_t = route_argmax(kr_index, doc_chunk_off, qr, index_is_unit)
     dqh = np.zeros_like(qh)
     dkh = np.zeros_like(kh)
     for q in range(ds.shape[0]):

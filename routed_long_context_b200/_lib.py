@@ -63,11 +63,24 @@ SIGNATURES = {
                               ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, f32, vp, i32, vp]),
     "msa_attn_set_impl": (i32, [ctypes.c_int]),
     "msa_sparse_attn_split": (i32, [vp, vp, vp, ctypes.c_int, vp, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                                    ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, f32, vp, i32,
-                                    vp, sz, vp]),
+                                    ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, f32, vp, vp,
+                                    i32, vp, sz, vp]),
     "msa_sparse_attn_split_workspace_size": (i32, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                    ctypes.c_int, ctypes.c_int, ctypes.POINTER(sz)]),
     "msa_pack_tokens": (i32, [vp, vp, i32, i64, ctypes.c_int, ctypes.c_int, vp, i64, vp, i64, vp, vp]),
+    "msa_sparse_attn_backward": (i32, [vp, vp, vp, ctypes.c_int, vp, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                       ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, f32, vp,
+                                       vp, vp, i32, vp, vp, vp, vp, vp, sz, vp]),
+    "msa_sparse_attn_backward_workspace_size": (i32, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.POINTER(sz)]),
+    "msa_gather_kv_backward": (i32, [vp, i64, vp, i64, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                     ctypes.c_int, vp, vp]),
+    "msa_pool_chunks_backward": (i32, [vp, vp, vp, i32, i64, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp, vp,
+                                       i64, i64, ctypes.c_int, ctypes.c_int, vp, i64, ctypes.c_int, vp, vp, vp, vp]),
+    "msa_router_aux_loss": (i32, [vp, ctypes.c_int, i64, vp, ctypes.c_int, f32, vp, vp, vp]),
+    "msa_route_backward": (i32, [vp, i32, i64, vp, i64, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                 vp, vp, vp, vp, sz, vp]),
+    "msa_route_backward_workspace_size": (i32, [i64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                ctypes.POINTER(sz)]),
     "msa_interleave_step": (i32, [ctypes.POINTER(InterleaveArgs), vp, vp, i64]),
     "msa_interleave_workspace_size": (i32, [ctypes.POINTER(InterleaveArgs), ctypes.POINTER(sz)]),
 }

@@ -250,9 +250,10 @@ def sparse_attn_split_workspace_size(n_q: int, T: int, hq: int, hkv: int, max_me
 
 
 def msa_sparse_attn_split(q, mem_kv, mem_len, local_k, local_v, L: int, q_start: int, scale: float | None = None,
-                          out=None, ws=None, stream=None):
+                          out=None, ws=None, lse=None, stream=None):
     """msa_sparse_attn for long memories (token-level fine stage): keys split into ranges that run as
-    separate blocks, then merged. Same arguments and result; bf16 only."""
+    separate blocks, then merged. Same arguments and result; bf16 only. lse: optional float32
+    [n_q, T, hq] output, the log-sum-exp of each row's logits (for the backward pass)."""
     n_q, T, hq, d = q.shape
     max_mem = mem_kv.shape[1]
     hkv = mem_kv.shape[3]
@@ -262,9 +263,102 @@ def msa_sparse_attn_split(q, mem_kv, mem_len, local_k, local_v, L: int, q_start:
     if ws is None:
         ws = _ws(sparse_attn_split_workspace_size(n_q, T, hq, hkv, max_mem, L), q.device)
     check(lib.msa_sparse_attn_split(_ptr(q), _ptr(mem_kv), _ptr(mem_len), max_mem, _ptr(local_k), _ptr(local_v),
-                                    L_max, L, q_start, n_q, T, hq, hkv, d, scale, _ptr(out), _dt(q), _ptr(ws),
-                                    ws.numel(), _stream(stream)), "msa_sparse_attn_split")
+                                    L_max, L, q_start, n_q, T, hq, hkv, d, scale, _ptr(out), _ptr(lse), _dt(q),
+                                    _ptr(ws), ws.numel(), _stream(stream)), "msa_sparse_attn_split")
     return out
+
+
+# ------------------------------------------------------------------------------------------------ backward
+def msa_sparse_attn_backward(q, mem_kv, mem_len, local_k, local_v, L: int, q_start: int, out, dout, lse,
+                             scale: float | None = None, grads=None, ws=None, stream=None):
+    """Gradients of the sparse attention (bf16 inputs): returns (dq [n_q, T, hq, d], dmem_kv [n_q, max_mem, 2,
+    hkv, d], dlocal_k, dlocal_v [n_q, L_max, hkv, d]), fp32; `grads` may supply those four buffers."""
+    n_q, T, hq, d = q.shape
+    max_mem, hkv = mem_kv.shape[1], mem_kv.shape[3]
+    L_max = local_k.shape[1]
+    dev = q.device
+    if grads is None:
+        grads = (torch.zeros((n_q, T, hq, d), dtype=torch.float32, device=dev),
+                 torch.zeros((n_q, max_mem, 2, hkv, d), dtype=torch.float32, device=dev),
+                 torch.zeros((n_q, L_max, hkv, d), dtype=torch.float32, device=dev),
+                 torch.zeros((n_q, L_max, hkv, d), dtype=torch.float32, device=dev))
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    if ws is None:
+        n = ctypes.c_size_t(0)
+        check(lib.msa_sparse_attn_backward_workspace_size(n_q, T, hq, ctypes.byref(n)),
+              "msa_sparse_attn_backward_workspace_size")
+        ws = _ws(n.value, dev)
+    dq, dmem, dlk, dlv = grads
+    check(lib.msa_sparse_attn_backward(_ptr(q), _ptr(mem_kv), _ptr(mem_len), max_mem, _ptr(local_k), _ptr(local_v),
+                                       L_max, L, q_start, n_q, T, hq, hkv, d, scale, _ptr(out), _ptr(dout), _ptr(lse),
+                                       _dt(q), _ptr(dq), _ptr(dmem), _ptr(dlk), _ptr(dlv), _ptr(ws), ws.numel(),
+                                       _stream(stream)), "msa_sparse_attn_backward")
+    return grads
+
+
+def msa_gather_kv_backward(dmem_kv, doc_chunk_off, idx, n_chunks: int, dkvbar=None, stream=None):
+    """Adds the memory-row gradients [n_q, max_mem, 2, hkv, d] (fp32) into dkvbar [n_chunks, 2, hkv, d]."""
+    n_q, max_mem, _, hkv, d = dmem_kv.shape
+    k = idx.shape[1]
+    if dkvbar is None:
+        dkvbar = torch.zeros((n_chunks, 2, hkv, d), dtype=torch.float32, device=dmem_kv.device)
+    check(lib.msa_gather_kv_backward(_ptr(dmem_kv), n_chunks, _ptr(doc_chunk_off), doc_chunk_off.numel() - 1,
+                                     _ptr(idx), n_q, k, hkv, d, max_mem, _ptr(dkvbar), _stream(stream)),
+          "msa_gather_kv_backward")
+    return dkvbar
+
+
+def msa_pool_chunks_backward(dkvbar, dkr_index, doc_tok_off, doc_chunk_off, chunk_doc, chunk: int, n_tok: int,
+                             kr=None, cos_sin=None, fuse_doc_rope: bool = True, normalize_router: bool = True,
+                             stream=None):
+    """Token gradients (dk, dv [n_tok, hkv, d], dkr [n_tok, hr, d], fp32; None where not asked) from the chunk
+    gradients dkvbar [C, 2, hkv, d] and dkr_index [C, hr, d] (either may be None)."""
+    ref = dkvbar if dkvbar is not None else dkr_index
+    dev = ref.device
+    C, d = chunk_doc.numel(), ref.shape[-1]
+    hkv = dkvbar.shape[2] if dkvbar is not None else 0
+    hr = dkr_index.shape[1] if dkr_index is not None else 0
+    dk = dv = dkr = None
+    if dkvbar is not None:
+        dk = torch.empty((n_tok, hkv, d), dtype=torch.float32, device=dev)
+        dv = torch.empty((n_tok, hkv, d), dtype=torch.float32, device=dev)
+    if dkr_index is not None:
+        dkr = torch.empty((n_tok, hr, d), dtype=torch.float32, device=dev)
+    fuse = bool(fuse_doc_rope and dkvbar is not None)
+    check(lib.msa_pool_chunks_backward(_ptr(dkvbar), _ptr(dkr_index), _ptr(kr), _dt(kr) if kr is not None else MSA_F32,
+                                       n_tok, hkv, hr, d, _ptr(doc_tok_off), _ptr(doc_chunk_off), _ptr(chunk_doc),
+                                       doc_tok_off.numel() - 1, C, chunk, int(fuse), _ptr(cos_sin) if fuse else None,
+                                       cos_sin.shape[0] if fuse else 0, int(normalize_router), _ptr(dk), _ptr(dv),
+                                       _ptr(dkr), _stream(stream)), "msa_pool_chunks_backward")
+    return dk, dv, dkr
+
+
+def msa_router_aux_loss(doc_scores, evidence, tau: float, stream=None):
+    """(loss per query [n_q], dL/d doc_scores [n_q, D]) of the auxiliary router loss; evidence int32 [n_q, n_ev]
+    (-1 padding). The gradient is that of the mean of the per-query losses."""
+    n_q, D = doc_scores.shape
+    loss = torch.empty(n_q, dtype=torch.float32, device=doc_scores.device)
+    grad = torch.empty_like(doc_scores)
+    ev = evidence.to(device=doc_scores.device, dtype=torch.int32).contiguous()
+    check(lib.msa_router_aux_loss(_ptr(doc_scores), n_q, D, _ptr(ev), ev.shape[1], tau, _ptr(loss), _ptr(grad),
+                                  _stream(stream)), "msa_router_aux_loss")
+    return loss, grad
+
+
+def msa_route_backward(kr_index, doc_chunk_off, qr, d_doc_scores, stream=None):
+    """(dqr [n_q, T, H, d], dkhat [C, H, d]) fp32: gradients of the router's document scores."""
+    C, H, d = kr_index.shape
+    n_q, T = qr.shape[:2]
+    dev = qr.device
+    n = ctypes.c_size_t(0)
+    check(lib.msa_route_backward_workspace_size(C, n_q, T, H, d, ctypes.byref(n)), "msa_route_backward_workspace_size")
+    ws = _ws(n.value, dev)
+    dqr = torch.empty((n_q, T, H, d), dtype=torch.float32, device=dev)
+    dkhat = torch.empty((C, H, d), dtype=torch.float32, device=dev)
+    check(lib.msa_route_backward(_ptr(kr_index), _dt(kr_index), C, _ptr(doc_chunk_off), doc_chunk_off.numel() - 1,
+                                 _ptr(qr), n_q, T, H, d, _ptr(d_doc_scores), _ptr(dqr), _ptr(dkhat), _ptr(ws),
+                                 ws.numel(), _stream(stream)), "msa_route_backward")
+    return dqr, dkhat
 
 
 class InterleaveRound:

@@ -10,6 +10,7 @@
 #include <atomic>
 
 #include "common.cuh"
+#include "mma.cuh"
 
 namespace msa {
 namespace {
@@ -33,6 +34,7 @@ struct AttnArgs {
     int n_split;       // split-KV variant: key ranges per (row block, kv head, query)
     float* part_o;     // [n_split][n_q * T * hq][d] unnormalised outputs
     float2* part_ml;   // [n_split][n_q * T * hq] (running max in log2 units, sum of weights)
+    float* lse;        // split variant, optional: [n_q * T * hq] natural-log log-sum-exp of the logits
 };
 
 template <typename T>
@@ -218,19 +220,6 @@ msa_status launch(const AttnArgs& a, int n_q, cudaStream_t s) {
 constexpr int kMmaRows = 64;
 constexpr int kMmaKeys = 64;
 constexpr int kKvStride = kD + 8;   // bf16 elements per shared-memory row
-
-__device__ __forceinline__ void mma_bf16_16816(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&v);
-}
 
 // Shared memory of one key/value stage: K and V tiles of 64 keys. The split variant double-buffers
 // (the next tile's copies are in flight while the current tile is computed); the plain variant keeps
@@ -452,7 +441,8 @@ __global__ void __launch_bounds__(128, SPLIT ? 3 : 1) attn_mma_kernel(const Attn
 // ranges saw no visible key (all m_s = -inf) is 0.
 __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restrict__ part_o,
                                                            const float2* __restrict__ part_ml, int n_split,
-                                                           int64_t rows, __nv_bfloat16* __restrict__ out) {
+                                                           int64_t rows, __nv_bfloat16* __restrict__ out,
+                                                           float* __restrict__ lse) {
     const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= rows) return;
@@ -474,6 +464,8 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
         }
     }
     const float inv = L > 0.f ? 1.f / L : 0.f;
+    // natural-log log-sum-exp of the scaled logits (M and the sums are in log2 units)
+    if (lse && lane == 0) lse[row] = L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : ninf;
     uint2 u;
     u.x = pack_bf16(acc[0] * inv, acc[1] * inv);
     u.y = pack_bf16(acc[2] * inv, acc[3] * inv);
@@ -493,7 +485,7 @@ msa_status launch_mma_g(const AttnArgs& a, int n_q, cudaStream_t s) {
     if constexpr (SPLIT) {
         const int64_t rows = (int64_t)n_q * a.T * a.hq;
         attn_combine_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(a.part_o, a.part_ml, a.n_split, rows,
-                                                                       static_cast<__nv_bfloat16*>(a.out));
+                                                                       static_cast<__nv_bfloat16*>(a.out), a.lse);
         MSA_LAUNCH_CHECK();
     }
     return MSA_OK;
@@ -580,8 +572,8 @@ msa_status msa_sparse_attn_split_workspace_size(int n_q, int T, int hq, int hkv,
 
 msa_status msa_sparse_attn_split(const void* q, const void* mem_kv, const int32_t* mem_len, int max_mem,
                                  const void* local_k, const void* local_v, int L_max, int L, int q_start, int n_q,
-                                 int T, int hq, int hkv, int d, float scale, void* out, msa_dtype dt, void* ws,
-                                 size_t ws_bytes, void* stream) {
+                                 int T, int hq, int hkv, int d, float scale, void* out, float* lse, msa_dtype dt,
+                                 void* ws, size_t ws_bytes, void* stream) {
     MSA_REQUIRE(dtype_ok(dt), "msa_sparse_attn_split: bad dtype");
     if (dt != MSA_BF16) return set_error(MSA_ERR_UNSUPPORTED, "msa_sparse_attn_split: bf16 only");
     MSA_REQUIRE(n_q > 0 && T >= 0 && hq > 0 && hkv > 0 && hq % hkv == 0 && max_mem >= 0 && L >= 0 && L <= L_max &&
@@ -607,6 +599,7 @@ msa_status msa_sparse_attn_split(const void* q, const void* mem_kv, const int32_
     a.local_k = local_k; a.local_v = local_v; a.L_max = L_max; a.L = L; a.q_start = q_start;
     a.T = T; a.hq = hq; a.hkv = hkv; a.scale_log2e = scale * 1.4426950408889634f; a.out = out;
     a.n_split = n_split;
+    a.lse = lse;
     a.part_o = static_cast<float*>(ws);
     a.part_ml = reinterpret_cast<float2*>(static_cast<char*>(ws) +
                                           align_up((size_t)n_split * n_q * T * hq * kD * 4, 256));

@@ -118,11 +118,23 @@ __global__ void __launch_bounds__(256) gather_device_kernel(const uint4* __restr
 msa_status gather_device(const void* host_bank, msa_dtype dt, int64_t n_chunks, const int64_t* doc_chunk_off,
                          int64_t n_docs, const int32_t* idx, int n_q, int k, int hkv, int d, int max_mem,
                          void* dev_mem_kv, int32_t* mem_len, cudaStream_t s) {
+    // a bank in this device's memory (training) is read directly; a host bank through its mapping
     void* dptr = nullptr;
-    const cudaError_t e = cudaHostGetDevicePointer(&dptr, const_cast<void*>(host_bank), 0);
-    if (e != cudaSuccess)
-        return set_error(MSA_ERR_INVALID_ARG, "device fetch: the host bank is not pinned, mapped host memory (%s)",
-                         cudaGetErrorString(e));
+    cudaPointerAttributes attr{};
+    int dev = -1;
+    if (cudaPointerGetAttributes(&attr, host_bank) == cudaSuccess && attr.type == cudaMemoryTypeDevice &&
+        cudaGetDevice(&dev) == cudaSuccess && attr.device == dev) {
+        dptr = const_cast<void*>(host_bank);
+    } else {
+        (void)cudaGetLastError();
+        const cudaError_t e = cudaHostGetDevicePointer(&dptr, const_cast<void*>(host_bank), 0);
+        if (e != cudaSuccess) {
+            (void)cudaGetLastError();
+            return set_error(MSA_ERR_INVALID_ARG,
+                             "device fetch: the bank is neither this device's memory nor pinned, mapped host memory (%s)",
+                             cudaGetErrorString(e));
+        }
+    }
     const size_t row = (size_t)2 * hkv * d * dtype_size(dt);
     if (row % 16 != 0 || !aligned16(dptr) || !aligned16(dev_mem_kv))
         return set_error(MSA_ERR_INVALID_ARG, "device fetch: rows and pointers must be 16-byte aligned");

@@ -1,0 +1,209 @@
+"""Backward pass of the CUDA path (through the C ABI) against the fp64 backward oracle: attention,
+fetch, pooling with document-wise RoPE and index normalisation, the auxiliary router loss, the
+router's gradient, and the chained training loss on a 64K-token training context."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from msa_inputs import rng, workloads
+from msa_inputs.device import memory_tensor, small_tensors, upload
+
+pytestmark = pytest.mark.gpu
+
+SEED = 0xBAC4
+
+
+@pytest.fixture(scope="module")
+def m():
+    import routed_long_context_b200 as m
+
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return m
+
+
+def _gen(tid, shape, dtype="f32", sigma=1.0):
+    return rng.normal(SEED, tid, 0, int(np.prod(shape)), sigma, dtype).reshape(shape)
+
+
+def _np(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def _rel(got, ref):
+    """Relative Frobenius error of a whole gradient tensor."""
+    return float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30))
+
+
+# The bf16 attention backward rounds P and dS to bf16 as tensor-core operands (2^-9 relative each)
+# and takes D = rowsum(dO * O) from the bf16 forward output; fp32 accumulation. Per gradient tensor
+# that stays within 1e-2 of the exact result in relative Frobenius norm.
+ATTN_BWD_TOL = 1e-2
+
+
+@pytest.mark.parametrize("hq,hkv", [(32, 8), (8, 8), (32, 4)])
+@pytest.mark.parametrize("T,max_mem,mem_lens,q_start", [(13, 40, (0, 5, 37), 7), (64, 140, (130, 64, 1), 0),
+                                                        (100, 300, (256, 300, 77), 20)])
+def test_attention_backward_matches_oracle(m, hq, hkv, T, max_mem, mem_lens, q_start):
+    n_q, d, dt = 3, 128, "bf16"
+    L = q_start + T
+    q = _gen(1, (n_q, T, hq, d), dt)
+    mem = _gen(2, (n_q, max_mem, 2, hkv, d), dt)
+    lk, lv = _gen(3, (n_q, L + 3, hkv, d), dt), _gen(4, (n_q, L + 3, hkv, d), dt)
+    dout = _gen(5, (n_q, T, hq, d), dt)
+    mem_len = torch.from_numpy(np.array(mem_lens, dtype=np.int32)).cuda()
+    qd, memd, lkd, lvd, dod = (upload(x, dt) for x in (q, mem, lk, lv, dout))
+    lse = torch.empty((n_q, T, hq), dtype=torch.float32, device="cuda")
+    out = m.msa_sparse_attn_split(qd, memd, mem_len, lkd, lvd, L, q_start, lse=lse)
+    dq, dmem, dlk, dlv = m.msa_sparse_attn_backward(qd, memd, mem_len, lkd, lvd, L, q_start, out, dod, lse)
+    assert m.device_status() == 0
+    scale = 1 / np.sqrt(d)
+    for qi in range(n_q):
+        ml = mem_lens[qi]
+        ref = O.sparse_attention_backward(q[qi], mem[qi, :ml, 0], mem[qi, :ml, 1], lk[qi, :L], lv[qi, :L], q_start,
+                                          scale, dout[qi])
+        got = (_np(dq[qi]), _np(dmem[qi, :ml, 0]), _np(dmem[qi, :ml, 1]), _np(dlk[qi, :L]), _np(dlv[qi, :L]))
+        for name, g, r in zip(("dq", "dmem_k", "dmem_v", "dlocal_k", "dlocal_v"), got, ref):
+            if r.size:
+                assert _rel(g, r) <= ATTN_BWD_TOL, (qi, name, _rel(g, r))
+        # log-sum-exp of the forward rows
+        o_lse = []
+        for h in range(hq):
+            g_ = h // (hq // hkv)
+            keys = np.concatenate([mem[qi, :ml, 0, g_], lk[qi, :L, g_]])
+            lg = (q[qi, :, h] @ keys.T) * scale
+            vis = np.ones_like(lg, dtype=bool)
+            vis[:, ml:] = np.arange(L)[None, :] <= q_start + np.arange(T)[:, None]
+            lg = np.where(vis, lg, -np.inf)
+            mx = lg.max(axis=1)
+            o_lse.append(mx + np.log(np.exp(lg - mx[:, None]).sum(axis=1)))
+        np.testing.assert_allclose(_np(lse[qi]), np.stack(o_lse, axis=1), atol=2e-3)
+
+
+def test_gather_backward_sums_rows_of_documents_fetched_twice(m):
+    counts = np.array([3, 1, 4, 0, 2, 5], dtype=np.int64)
+    off = np.concatenate([[0], np.cumsum(counts)])
+    C = int(off[-1])
+    idx = np.array([[2, 0, 5], [5, 1, 2]], dtype=np.int32)           # documents 2 and 5 twice
+    dmem = _gen(6, (2, 14, 2, 8, 128))
+    got = m.msa_gather_kv_backward(torch.from_numpy(dmem).float().cuda(), torch.from_numpy(off).cuda(),
+                                   torch.from_numpy(idx).cuda(), C)
+    assert m.device_status() == 0
+    ref = sum(O.gather_memory_backward(dmem[q], off, idx[q].tolist(), C) for q in range(2))
+    np.testing.assert_allclose(_np(got), ref, rtol=1e-6, atol=1e-6)
+
+
+@pytest.mark.parametrize("kr_dt", ["f32", "bf16"])
+def test_pool_backward_matches_oracle(m, kr_dt):
+    """Token gradients of pooling: keys through the transposed document-wise rotation, values, and
+    router keys through the index normalisation; ragged documents (one empty)."""
+    from routed_long_context_b200.bank import BankLayout
+
+    lens = np.array([300, 0, 255, 129, 1000, 1], dtype=np.int64)
+    chunk, hkv, hr, d, base = 128, 8, 8, 128, 1e6
+    lay = BankLayout.from_doc_lengths(lens, chunk)
+    n = int(lay.doc_tok_off_host[-1])
+    C = lay.n_chunks
+    kr = _gen(7, (n, hr, d), kr_dt)
+    dkv = _gen(8, (C, 2, hkv, d))
+    dki = _gen(9, (C, hr, d))
+    cs = m.rope_table(2048, d, base)
+    dk, dv, dkr = m.msa_pool_chunks_backward(torch.from_numpy(dkv).float().cuda(), torch.from_numpy(dki).float().cuda(),
+                                             lay.doc_tok_off, lay.doc_chunk_off, lay.chunk_doc, chunk, n,
+                                             kr=upload(kr, kr_dt), cos_sin=cs)
+    assert m.device_status() == 0
+    _, _, krb = O.encode_memory(None, None, kr, lay.doc_tok_off_host, chunk, base)
+    rk, rv, rkr = O.encode_memory_backward(dkv[:, 0], dkv[:, 1], O.unit_backward(krb, dki), lay.doc_tok_off_host,
+                                           chunk, base)
+    np.testing.assert_allclose(_np(dk), rk, rtol=1e-5, atol=1e-6)
+    np.testing.assert_allclose(_np(dv), rv, rtol=1e-6, atol=1e-7)
+    np.testing.assert_allclose(_np(dkr), rkr, rtol=1e-4, atol=1e-6)
+
+
+@pytest.mark.parametrize("n_q,D,tau", [(3, 1000, 0.1), (2, 97657, 0.05)])
+def test_aux_loss_matches_oracle(m, n_q, D, tau):
+    s = np.clip(_gen(10, (n_q, D)) * 0.3, -1, 1).astype(np.float32)
+    ev = np.full((n_q, 3), -1, dtype=np.int32)
+    ev[0, :2] = [5, D - 1]
+    ev[1, :1] = [17]
+    if n_q > 2:
+        ev[2] = [0, 1, 2]
+    loss, grad = m.msa_router_aux_loss(torch.from_numpy(s).cuda(), torch.from_numpy(ev), tau)
+    assert m.device_status() == 0
+    rl, rg = O.router_aux_loss(s, [[e for e in row if e >= 0] for row in ev], tau)
+    assert abs(float(loss.mean()) - rl) <= 1e-4 * max(1.0, abs(rl))
+    np.testing.assert_allclose(_np(grad), rg, rtol=1e-3, atol=1e-7 / n_q)
+
+
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+def test_route_backward_matches_oracle(m, dt):
+    """The index is built on the host (unit vectors rounded to dt) and both sides score those stored
+    values as they are, so they find the same attaining (chunk, token) pairs."""
+    r = np.random.default_rng(12)
+    counts = r.integers(0, 13, 40)
+    off = np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
+    C, H, d, n_q, T = int(off[-1]), 8, 128, 2, 17
+    index = rng.round_to(O.unit(_gen(11, (C, H, d))).astype(np.float32), dt).astype(np.float64)
+    qr = _gen(13, (n_q, T, H, d), dt)
+    ds = _gen(14, (n_q, 40))
+    dqr, dkh = m.msa_route_backward(upload(index, dt), torch.from_numpy(off).cuda(), upload(qr, dt),
+                                    torch.from_numpy(ds).float().cuda())
+    assert m.device_status() == 0
+    rq, rk = O.route_backward(index, off, qr, ds, index_is_unit=True)
+    assert _rel(_np(dqr), rq) <= 1e-4 and _rel(_np(dkh), rk) <= 1e-4
+
+
+def test_training_loss_gradients_on_a_64k_context(m):
+    """L = <W, attention output> + lam * aux(router scores) on the train64k context, selection held at
+    the GPU's top-k: the chained library calls (encode, route, top-k, fetch, split attention with
+    log-sum-exp; attention backward, fetch backward, aux loss, router backward, pooling backward) give
+    the token gradients of K, V and K^R of the chained backward oracle."""
+    from routed_long_context_b200.bank import BankLayout, encode_tokens
+
+    w = workloads.train64k()
+    lay = BankLayout.from_doc_lengths(w.doc_len, w.chunk)
+    cs = m.rope_table(8192, w.d, w.rope_base)
+    k, v, kr = (memory_tensor(w, 0, n) for n in ("k", "v", "kr"))
+    kvbar, index = encode_tokens(lay, k, v, kr, w.chunk, cs)
+    sm = small_tensors(w, 0)
+    T, lam, tau = w.T0, 0.5, 1.0
+    ds = m.msa_route_scores(index, lay.chunk_doc, lay.n_docs, sm["qr"])
+    idx, _ = m.msa_topk_docs(ds, w.k)
+    max_mem = w.k * int(w.doc_chunks.max())
+    mem, mem_len = m.msa_gather_kv_device(kvbar, lay.doc_chunk_off, idx, max_mem)
+    seg = torch.tensor([0, T], dtype=torch.int64, device="cuda")
+    lk = m.msa_rope_doc(sm["k_new"][0], seg, w.k, cs, out=torch.empty_like(sm["k_new"][0]))
+    qq = m.msa_rope_doc(sm["q"][0], seg, w.k, cs, out=torch.empty_like(sm["q"][0]))
+    lse = torch.empty((1, T, w.hq), dtype=torch.float32, device="cuda")
+    out = m.msa_sparse_attn_split(qq[None], mem, mem_len, lk[None], sm["v_new"], T, 0, lse=lse)
+    W = _gen(15, (1, T, w.hq, w.d), "bf16")
+    _, dmem, _, _ = m.msa_sparse_attn_backward(qq[None], mem, mem_len, lk[None], sm["v_new"], T, 0, out,
+                                               upload(W, "bf16"), lse)
+    dkvbar = m.msa_gather_kv_backward(dmem, lay.doc_chunk_off, idx, lay.n_chunks)
+    evidence = np.array([w.expected(0, 0, 0)], dtype=np.int32)
+    _, g_aux = m.msa_router_aux_loss(ds, torch.from_numpy(evidence), tau)
+    _, dkhat = m.msa_route_backward(index, lay.doc_chunk_off, sm["qr"], g_aux * lam)
+    dk, dv, dkr = m.msa_pool_chunks_backward(dkvbar, dkhat, lay.doc_tok_off, lay.doc_chunk_off, lay.chunk_doc, w.chunk,
+                                             w.n_tok, kr=kr, cos_sin=cs)
+    assert m.device_status() == 0
+    gi = idx.cpu().numpy()[0]
+    assert set(evidence[0].tolist()) <= set(gi.tolist())
+
+    # the chained oracle
+    kh, vh, krh = (w.host_tensor(0, n) for n in ("k", "v", "kr"))
+    kb, vb, krb = O.encode_memory(kh, vh, krh, w.doc_tok_off, w.chunk, w.rope_base)
+    qr = w.qr(0)
+    memo = O.gather_memory(np.stack([kb, vb], 1), w.doc_chunk_off, gi)
+    pos = O.global_positions(w.k, 0, T)
+    _, dmk, dmv, _, _ = O.sparse_attention_backward(O.apply_rope(w.q(0)[0], pos, w.rope_base), memo[:, 0], memo[:, 1],
+                                                    O.apply_rope(w.k_new(0)[0], pos, w.rope_base), w.v_new(0)[0], 0,
+                                                    1 / np.sqrt(w.d), W[0])
+    dbar = O.gather_memory_backward(np.stack([dmk, dmv], 1), w.doc_chunk_off, gi, w.n_chunks)
+    _, g = O.router_aux_loss(O.route(krb, w.doc_chunk_off, qr)[0], [evidence[0].tolist()], tau)
+    stored = rng.round_to(O.unit(krb).astype(np.float32), "bf16").astype(np.float64)   # the index's stored form
+    _, dkh = O.route_backward(stored, w.doc_chunk_off, qr, lam * g, index_is_unit=True)
+    rk, rv, rkr = O.encode_memory_backward(dbar[:, 0], dbar[:, 1], O.unit_backward(krb, dkh), w.doc_tok_off, w.chunk,
+                                           w.rope_base)
+    assert _rel(_np(dk), rk) <= ATTN_BWD_TOL
+    assert _rel(_np(dv), rv) <= ATTN_BWD_TOL
+    assert _rel(_np(dkr), rkr) <= ATTN_BWD_TOL

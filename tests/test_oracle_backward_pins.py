@@ -134,6 +134,19 @@ def test_route_backward_matches_finite_differences():
     np.testing.assert_allclose(dkr.flat[ik], _fd(f_k, kr, ik), atol=1e-7)
 
 
+def test_route_backward_on_exact_unit_index_equals_normalising_form():
+    """For exactly unit key vectors, scoring them as stored (index form) is the cosine itself."""
+    r = _rng(8)
+    off = np.array([0, 2, 5, 9])
+    kr = O.unit(r.standard_normal((9, 2, 6)))
+    qr = r.standard_normal((2, 3, 2, 6))
+    w = r.standard_normal((2, 3))
+    a = O.route_backward(kr, off, qr, w)
+    b = O.route_backward(kr, off, qr, w, index_is_unit=True)
+    np.testing.assert_allclose(a[0], b[0], atol=1e-14)
+    np.testing.assert_allclose(a[1], b[1], atol=1e-14)
+
+
 # ------------------------------------------------------------------------------------------ chained training loss
 def test_training_loss_gradient_through_encode_route_and_attention():
     """L = <W, attention output> + lam * aux(router scores) with the selection held fixed: the
