@@ -47,11 +47,12 @@ def parse():
                     help="SMs the routers leave free for the overlapped selection and attention")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="100m", choices=["100m", "encode10m", "interleave", "fine1m"],
+    ap.add_argument("--workload", default="100m", choices=["100m", "encode10m", "interleave", "fine1m", "train64k"],
                     help="100m: the routing step (the reported metric); encode10m: offline encoding of the "
                          "10M-token bank (document-wise RoPE + chunk-mean pooling); interleave: three Memory "
                          "Interleave rounds over a 10M-token bank (tensor-bound routing); fine1m: the token-level "
-                         "fine stage on the 1M-token bank; the last three are reported separately")
+                         "fine stage on the 1M-token bank; train64k: a training step (forward + backward) on a "
+                         "64K-token context; the last four are reported separately")
     return ap.parse_args()
 
 
@@ -444,6 +445,124 @@ def fine_bench(args, rank, world, local_rank):
             "clocks": clk.summary()}))
 
 
+# ---------------------------------------------------------------------------------------------- training step
+def train_bench(args, rank, world, local_rank):
+    """One training step of a routed layer on the 64K-token training context (16 docs x 4096 tokens,
+    chunk 128; one query of 512 tokens; top-4): forward (encode, route, top-k, fetch, split attention
+    with log-sum-exp) and backward (attention, fetch, auxiliary router loss, router, pooling), each
+    call timed with CUDA events."""
+    import numpy as np
+    import torch
+
+    import routed_long_context_b200 as m
+    from msa_inputs import rng, workloads
+    from msa_inputs.device import memory_tensor, small_tensors, upload
+    from routed_long_context_b200.bank import BankLayout
+
+    torch.cuda.set_device(local_rank)
+    w = workloads.train64k()
+    lay = BankLayout.from_doc_lengths(w.doc_len, w.chunk)
+    cs = m.rope_table(8192, w.d, w.rope_base)
+    k, v, kr = (memory_tensor(w, 0, n) for n in ("k", "v", "kr"))
+    sm = small_tensors(w, 0)
+    T, C, dt = w.T0, lay.n_chunks, torch.bfloat16
+    max_mem = w.k * int(w.doc_chunks.max())
+    kvbar = torch.empty((C, 2, w.hkv, w.d), dtype=dt, device="cuda")
+    index = torch.empty((C, w.H, w.d), dtype=dt, device="cuda")
+    ds = torch.empty((1, lay.n_docs), dtype=torch.float32, device="cuda")
+    idx = torch.empty((1, w.k), dtype=torch.int32, device="cuda")
+    sc = torch.empty((1, w.k), dtype=torch.float32, device="cuda")
+    mem = torch.zeros((1, max_mem, 2, w.hkv, w.d), dtype=dt, device="cuda")
+    mem_len = torch.zeros(1, dtype=torch.int32, device="cuda")
+    seg = torch.tensor([0, T], dtype=torch.int64, device="cuda")
+    lk, qq = torch.empty_like(sm["k_new"][0]), torch.empty_like(sm["q"][0])
+    out = torch.empty((1, T, w.hq, w.d), dtype=dt, device="cuda")
+    lse = torch.empty((1, T, w.hq), dtype=torch.float32, device="cuda")
+    dout = upload(rng.normal(w.seed, 1 << 50, 0, T * w.hq * w.d, 1.0, "bf16").reshape(1, T, w.hq, w.d), "bf16")
+    grads = (torch.zeros((1, T, w.hq, w.d), dtype=torch.float32, device="cuda"),
+             torch.zeros((1, max_mem, 2, w.hkv, w.d), dtype=torch.float32, device="cuda"),
+             torch.zeros((1, T, w.hkv, w.d), dtype=torch.float32, device="cuda"),
+             torch.zeros((1, T, w.hkv, w.d), dtype=torch.float32, device="cuda"))
+    dkvbar = torch.zeros((C, 2, w.hkv, w.d), dtype=torch.float32, device="cuda")
+    evidence = torch.tensor([w.expected(0, 0, 0)], dtype=torch.int32, device="cuda")
+    rws = m.api._ws(m.route_workspace_size(1, T, w.H, w.d, dt), "cuda")
+    tws = m.api._ws(m.topk_workspace_size(1, lay.n_docs, w.k), "cuda")
+    aws = m.api._ws(m.sparse_attn_split_workspace_size(1, T, w.hq, w.hkv, max_mem, T), "cuda")
+    s = torch.cuda.current_stream()
+    names = ["encode", "route+topk", "fetch", "attn_fwd", "attn_bwd", "fetch_bwd", "aux_loss", "route_bwd", "pool_bwd"]
+
+    def step(ev=None):
+        def mark(i):
+            if ev:
+                ev[i].record(s)
+        mark(0)
+        m.msa_pool_chunks(k, v, kr, lay.doc_tok_off, lay.doc_chunk_off, lay.chunk_doc, w.chunk, cos_sin=cs,
+                          kvbar=kvbar, kr_index=index)
+        mark(1)
+        m.msa_route_scores(index, lay.chunk_doc, lay.n_docs, sm["qr"], doc_scores=ds, ws=rws)
+        m.msa_topk_docs(ds, w.k, idx=idx, score=sc, ws=tws)
+        mark(2)
+        m.msa_gather_kv_device(kvbar, lay.doc_chunk_off, idx, max_mem, dev_mem_kv=mem, mem_len=mem_len)
+        mark(3)
+        m.msa_rope_doc(sm["k_new"][0], seg, w.k, cs, out=lk)
+        m.msa_rope_doc(sm["q"][0], seg, w.k, cs, out=qq)
+        m.msa_sparse_attn_split(qq[None], mem, mem_len, lk[None], sm["v_new"], T, 0, out=out, ws=aws, lse=lse)
+        mark(4)
+        m.msa_sparse_attn_backward(qq[None], mem, mem_len, lk[None], sm["v_new"], T, 0, out, dout, lse, grads=grads)
+        mark(5)
+        m.msa_gather_kv_backward(grads[1], lay.doc_chunk_off, idx, C, dkvbar=dkvbar)
+        mark(6)
+        _, g_aux = m.msa_router_aux_loss(ds, evidence, 1.0)
+        mark(7)
+        _, dkhat = m.msa_route_backward(index, lay.doc_chunk_off, sm["qr"], g_aux)
+        mark(8)
+        m.msa_pool_chunks_backward(dkvbar, dkhat, lay.doc_tok_off, lay.doc_chunk_off, lay.chunk_doc, w.chunk, w.n_tok,
+                                   kr=kr, cos_sin=cs)
+        mark(9)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    planted_ok = set(w.expected(0, 0, 0)) <= set(idx.cpu().numpy()[0].tolist())
+    steps = min(args.steps, 100)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(10)] for _ in range(steps)]
+    with ClockSampler(local_rank) as clk:
+        for i in range(steps):
+            step(evs[i])
+        torch.cuda.synchronize()
+    part = {n: sum(e[j].elapsed_time(e[j + 1]) for e in evs) / steps for j, n in enumerate(names)}
+    ms = sum(e[0].elapsed_time(e[9]) for e in evs) / steps
+    # attention backward FLOPs: rows x visible keys x d x 2, for S, dP, dV, dK (key tiles) and S, dP, dQ (row blocks)
+    rows = T * w.hq
+    keys = float(mem_len.item()) + (T + 1) / 2.0
+    bwd_flops = 7 * 2.0 * rows * keys * w.d
+    pool_bwd_bytes = 3 * w.n_tok * w.hkv * w.d * 4 + w.n_tok * w.H * w.d * 2 + C * 3 * w.H * w.d * 4
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            pk = json.load(f)
+        bf16_peak, hbm_peak, kind = float(pk["bf16_tflops"]), float(pk["hbm_gbs"]), "measured"
+    except Exception:
+        bf16_peak, hbm_peak, kind = 1590.0, 6650.0, "fallback"
+    if rank == 0:
+        pool_gbs = pool_bwd_bytes / (part["pool_bwd"] / 1e3) / 1e9
+        print(json.dumps({
+            "metric": "train64k: training step of one routed layer (forward + backward), memory tokens/s",
+            "value": w.n_tok / (ms / 1e3), "unit": "memory tokens/s", "n_gpus": 1, "steps": steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "train64k: 16 docs x 4096 tokens, chunk 128, 1 query x 512 tokens, top-4, "
+                                   "GQA 32/8, d 128, aux loss tau 1"},
+            "ms_by_call": part,
+            "attn_bwd_tflops": bwd_flops / (part["attn_bwd"] / 1e3) / 1e12,
+            "roofline": {"bound": "hbm", "achieved": pool_gbs, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": pool_gbs / hbm_peak, "traffic": None, "kernel": "pool_bwd_kernel",
+                         "bytes": pool_bwd_bytes, "peak_kind": kind},
+            "attn_bwd_roofline": {"bound": "tensor", "achieved": bwd_flops / (part["attn_bwd"] / 1e3) / 1e12,
+                                  "peak": bf16_peak, "unit": "TFLOP/s",
+                                  "frac": bwd_flops / (part["attn_bwd"] / 1e3) / 1e12 / bf16_peak},
+            "checks": {"planted_docs_selected": planted_ok, "device_status": m.device_status()},
+            "clocks": clk.summary()}))
+
+
 # ---------------------------------------------------------------------------------------------- ours
 def main():
     args = parse()
@@ -458,6 +577,8 @@ def main():
         return interleave_bench(args, rank, world, local_rank)
     if args.workload == "fine1m":
         return fine_bench(args, rank, world, local_rank)
+    if args.workload == "train64k":
+        return train_bench(args, rank, world, local_rank)
 
     import numpy as np
     import torch

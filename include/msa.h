@@ -300,23 +300,26 @@ msa_status msa_sparse_attn_split_workspace_size(int n_q, int T, int hq, int hkv,
  * For each row, with P the softmax of the forward: dV = P^T dO, dS = P * (dO V^T - rowsum(dO*O)),
  * dq = scale dS K, dK = scale dS^T q, summed over the query heads that share a kv head. Tensor
  * cores (mma.sync, bf16 operands: P and dS are rounded to bf16, fp32 accumulation); each key's
- * gradient is accumulated by one block over every row (no atomics). bf16 only, d == 128,
- * hq/hkv in {1, 2, 4, 8}. ws: msa_sparse_attn_backward_workspace_size bytes. */
+ * gradient is accumulated over contiguous ranges of rows by as many blocks as fill about one wave,
+ * the ranges' partial sums then added in a fixed order (deterministic, no atomics). bf16 only,
+ * d == 128, hq/hkv in {1, 2, 4, 8}. ws: msa_sparse_attn_backward_workspace_size bytes. */
 msa_status msa_sparse_attn_backward(const void* q, const void* mem_kv, const int32_t* mem_len, int max_mem,
                                     const void* local_k, const void* local_v, int L_max, int L, int q_start, int n_q,
                                     int T, int hq, int hkv, int d, float scale, const void* out, const void* dout,
                                     const float* lse, msa_dtype dt, float* dq, float* dmem_kv, float* dlocal_k,
                                     float* dlocal_v, void* ws, size_t ws_bytes, void* stream);
-msa_status msa_sparse_attn_backward_workspace_size(int n_q, int T, int hq, size_t* bytes);
+msa_status msa_sparse_attn_backward_workspace_size(int n_q, int T, int hq, int hkv, int max_mem, int L,
+                                                   size_t* bytes);
 
 /* Adjoint of the fetch (msa_gather_kv_device): query q's memory-row gradients dmem_kv
- * [n_q][max_mem][2][hkv][d] (fp32) are ADDED to the chunk rows of dkvbar [n_chunks][2][hkv][d]
- * (fp32, zeroed by the caller) they were copied from, following idx [n_q][k] and doc_chunk_off
- * (device) in rank order; a document selected by several queries receives the sum (fp32 atomic
- * adds, so the summation order varies). Bad indices record MSA_DEV_BAD_INDEX and are skipped. */
+ * [n_q][max_mem][2][hkv][d] (fp32) are added to the chunk rows of dkvbar [n_chunks][2][hkv][d]
+ * (fp32) they were copied from, following idx [n_q][k] and doc_chunk_off (device) in rank order;
+ * a document selected by several queries receives the sum (fp32 atomic adds, so the summation
+ * order varies). With accumulate == 0 dkvbar is zeroed first (on the stream), else added to.
+ * Bad indices record MSA_DEV_BAD_INDEX and are skipped. */
 msa_status msa_gather_kv_backward(const float* dmem_kv, int64_t n_chunks, const int64_t* doc_chunk_off,
                                   int64_t n_docs, const int32_t* idx, int n_q, int k, int hkv, int d, int max_mem,
-                                  float* dkvbar, void* stream);
+                                  float* dkvbar, int accumulate, void* stream);
 
 /* Adjoint of msa_pool_chunks: token gradients from chunk gradients.
  *   dkvbar: fp32 [n_chunks][2][hkv][d] (dK-bar, dV-bar) or NULL; then dk, dv: fp32 [n_tok][hkv][d]

@@ -71,9 +71,10 @@ SIGNATURES = {
     "msa_sparse_attn_backward": (i32, [vp, vp, vp, ctypes.c_int, vp, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                        ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, f32, vp,
                                        vp, vp, i32, vp, vp, vp, vp, vp, sz, vp]),
-    "msa_sparse_attn_backward_workspace_size": (i32, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.POINTER(sz)]),
+    "msa_sparse_attn_backward_workspace_size": (i32, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                      ctypes.c_int, ctypes.c_int, ctypes.POINTER(sz)]),
     "msa_gather_kv_backward": (i32, [vp, i64, vp, i64, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                                     ctypes.c_int, vp, vp]),
+                                     ctypes.c_int, vp, ctypes.c_int, vp]),
     "msa_pool_chunks_backward": (i32, [vp, vp, vp, i32, i64, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp, vp,
                                        i64, i64, ctypes.c_int, ctypes.c_int, vp, i64, ctypes.c_int, vp, vp, vp, vp]),
     "msa_router_aux_loss": (i32, [vp, ctypes.c_int, i64, vp, ctypes.c_int, f32, vp, vp, vp]),

@@ -285,7 +285,7 @@ def msa_sparse_attn_backward(q, mem_kv, mem_len, local_k, local_v, L: int, q_sta
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     if ws is None:
         n = ctypes.c_size_t(0)
-        check(lib.msa_sparse_attn_backward_workspace_size(n_q, T, hq, ctypes.byref(n)),
+        check(lib.msa_sparse_attn_backward_workspace_size(n_q, T, hq, hkv, max_mem, L, ctypes.byref(n)),
               "msa_sparse_attn_backward_workspace_size")
         ws = _ws(n.value, dev)
     dq, dmem, dlk, dlv = grads
@@ -296,15 +296,18 @@ def msa_sparse_attn_backward(q, mem_kv, mem_len, local_k, local_v, L: int, q_sta
     return grads
 
 
-def msa_gather_kv_backward(dmem_kv, doc_chunk_off, idx, n_chunks: int, dkvbar=None, stream=None):
-    """Adds the memory-row gradients [n_q, max_mem, 2, hkv, d] (fp32) into dkvbar [n_chunks, 2, hkv, d]."""
+def msa_gather_kv_backward(dmem_kv, doc_chunk_off, idx, n_chunks: int, dkvbar=None, accumulate: bool = False,
+                           stream=None):
+    """Memory-row gradients [n_q, max_mem, 2, hkv, d] (fp32) into chunk-row gradients dkvbar [n_chunks, 2, hkv, d]
+    (zeroed first unless accumulate)."""
     n_q, max_mem, _, hkv, d = dmem_kv.shape
     k = idx.shape[1]
     if dkvbar is None:
-        dkvbar = torch.zeros((n_chunks, 2, hkv, d), dtype=torch.float32, device=dmem_kv.device)
+        dkvbar = torch.empty((n_chunks, 2, hkv, d), dtype=torch.float32, device=dmem_kv.device)
+        accumulate = False
     check(lib.msa_gather_kv_backward(_ptr(dmem_kv), n_chunks, _ptr(doc_chunk_off), doc_chunk_off.numel() - 1,
-                                     _ptr(idx), n_q, k, hkv, d, max_mem, _ptr(dkvbar), _stream(stream)),
-          "msa_gather_kv_backward")
+                                     _ptr(idx), n_q, k, hkv, d, max_mem, _ptr(dkvbar), int(accumulate),
+                                     _stream(stream)), "msa_gather_kv_backward")
     return dkvbar
 
 

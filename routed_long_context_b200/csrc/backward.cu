@@ -44,6 +44,9 @@ struct BwdArgs {
     float* dmem;             // [n_q][max_mem][2][hkv][d]
     float* dlk;              // [n_q][L_max][hkv][d]
     float* dlv;
+    int n_rsplit;            // dK/dV: row ranges per key tile (1 = write the gradients directly)
+    int key_pad;             // key tiles x 64
+    float* part_dkv;         // [n_rsplit][n_q][key_pad][2][hkv][d] partial dK (x scale) / dV per row range
 };
 
 __device__ __forceinline__ bool key_visible(int kk, int mem_len, int n_keys, int q_start, int t) {
@@ -102,11 +105,17 @@ __global__ void __launch_bounds__(128) attn_bwd_dkdv_kernel(const BwdArgs a) {
     float* D_s = lse_s + kTile;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
-    const int qi = blockIdx.z, g = blockIdx.y, kb = blockIdx.x * kTile;
+    const int qi = blockIdx.z, g = blockIdx.y;
+    const int rsplit = blockIdx.x % a.n_rsplit, kb = (blockIdx.x / a.n_rsplit) * kTile;
     const int mem_len = max(min(a.mem_len[qi], a.max_mem), 0);
     const int n_keys = mem_len + a.L;
     if (kb >= n_keys) return;
     const int n_rows = a.T * G;
+    // this block's contiguous range of 64-row blocks
+    const int row_blocks = (n_rows + kTile - 1) / kTile;
+    const int rb_per = (row_blocks + a.n_rsplit - 1) / a.n_rsplit;
+    const int r_begin = min(rsplit * rb_per, row_blocks) * kTile;
+    const int r_end = min(min(rsplit * rb_per + rb_per, row_blocks) * kTile, n_rows);
     const float ninf = -__int_as_float(0x7f800000);
 
     stage_rows(Ks, [&](int r) { return kb + r < n_keys ? key_row(a, qi, g, kb + r, mem_len, 0) : nullptr; }, a.q);
@@ -124,7 +133,7 @@ __global__ void __launch_bounds__(128) attn_bwd_dkdv_kernel(const BwdArgs a) {
     const int key_a = kb + warp * 16 + gid, key_b = key_a + 8;
     const int kr_a = warp * 16 + gid, kr_b = kr_a + 8;   // rows of Ks / Vs
 
-    for (int r0 = (t_first * G / kTile) * kTile; r0 < n_rows; r0 += kTile) {
+    for (int r0 = max(r_begin, (t_first * G / kTile) * kTile); r0 < r_end; r0 += kTile) {
         __syncthreads();                                  // previous row block's readers are done
         auto row_src = [&](const __nv_bfloat16* base, int r) -> const __nv_bfloat16* {
             const int row = r0 + r;
@@ -214,8 +223,12 @@ __global__ void __launch_bounds__(128) attn_bwd_dkdv_kernel(const BwdArgs a) {
         }
     }
 
-    // write this thread's two keys' gradients (dims nd*8 + 2 tig, +1)
+    // write this thread's two keys' gradients (dims nd*8 + 2 tig, +1): directly, or as this row
+    // range's partial sums for the reduction
     auto dst = [&](int key, int which) -> float* {
+        if (a.n_rsplit > 1)
+            return a.part_dkv +
+                   ((((int64_t)rsplit * gridDim.z + qi) * a.key_pad + key) * 2 + which) * a.hkv * kD + g * kD;
         if (key < mem_len) return a.dmem + (((int64_t)qi * a.max_mem + key) * 2 + which) * a.hkv * kD + g * kD;
         return (which ? a.dlv : a.dlk) + (((int64_t)qi * a.L_max + (key - mem_len)) * a.hkv + g) * kD;
     };
@@ -342,7 +355,51 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_kernel(const BwdArgs a) {
     }
 }
 
+// Sum of the row ranges' partial dK/dV into the outputs: one warp per (query, key, K or V, kv head),
+// lane l owning dims 4l..4l+3, the ranges added in order (deterministic).
+__global__ void __launch_bounds__(256) attn_bwd_dkdv_reduce_kernel(const BwdArgs a, int n_q) {
+    const int64_t w = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    const int64_t per_q = (int64_t)a.key_pad * 2 * a.hkv;
+    if (w >= n_q * per_q) return;
+    const int qi = (int)(w / per_q);
+    const int64_t rem = w % per_q;
+    const int key = (int)(rem / (2 * a.hkv));
+    const int which = (int)((rem / a.hkv) % 2), g = (int)(rem % a.hkv);
+    const int mem_len = max(min(a.mem_len[qi], a.max_mem), 0);
+    if (key >= mem_len + a.L) return;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int r = 0; r < a.n_rsplit; ++r) {
+        const float4 v = *reinterpret_cast<const float4*>(
+            a.part_dkv + ((((int64_t)r * n_q + qi) * a.key_pad + key) * 2 + which) * a.hkv * kD + g * kD + lane * 4);
+        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    float* out = key < mem_len
+                     ? a.dmem + (((int64_t)qi * a.max_mem + key) * 2 + which) * a.hkv * kD + g * kD
+                     : (which ? a.dlv : a.dlk) + (((int64_t)qi * a.L_max + (key - mem_len)) * a.hkv + g) * kD;
+    *reinterpret_cast<float4*>(out + lane * 4) = acc;
+}
+
 constexpr size_t kDkdvSmem = 4 * sizeof(Tile) + 2 * kTile * sizeof(float);
+// dK/dV blocks resident per SM (255 registers x 128 threads) on 148 SMs: the row ranges per key
+// tile are chosen so that the grid fills about one such wave
+constexpr int kDkdvWave = 2 * 148;
+
+int pick_rsplit(int n_q, int T, int hq, int hkv, int max_mem, int L) {
+    const int key_tiles = (max_mem + L + kTile - 1) / kTile;
+    const int64_t base = (int64_t)key_tiles * hkv * n_q;
+    const int row_blocks = (T * (hq / hkv) + kTile - 1) / kTile;
+    if (base <= 0) return 1;
+    return (int)std::max<int64_t>(1, std::min<int64_t>(row_blocks, kDkdvWave / base));
+}
+
+size_t bwd_ws_bytes(int n_q, int T, int hq, int hkv, int max_mem, int L) {
+    const size_t dvec = align_up((size_t)n_q * T * hq * sizeof(float), 256);
+    const int r = pick_rsplit(n_q, T, hq, hkv, max_mem, L);
+    if (r <= 1) return dvec;
+    const size_t key_pad = (size_t)((max_mem + L + kTile - 1) / kTile) * kTile;
+    return dvec + align_up((size_t)r * n_q * key_pad * 2 * hkv * kD * sizeof(float), 256);
+}
 
 template <int G>
 msa_status launch_attn_bwd_g(const BwdArgs& a, int n_q, cudaStream_t s) {
@@ -350,8 +407,13 @@ msa_status launch_attn_bwd_g(const BwdArgs& a, int n_q, cudaStream_t s) {
     if (key_tiles > 0) {
         MSA_CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dkdv_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           (int)kDkdvSmem));
-        attn_bwd_dkdv_kernel<G><<<dim3(key_tiles, a.hkv, n_q), 128, kDkdvSmem, s>>>(a);
+        attn_bwd_dkdv_kernel<G><<<dim3(key_tiles * a.n_rsplit, a.hkv, n_q), 128, kDkdvSmem, s>>>(a);
         MSA_LAUNCH_CHECK();
+        if (a.n_rsplit > 1) {
+            const int64_t warps = (int64_t)n_q * a.key_pad * 2 * a.hkv;
+            attn_bwd_dkdv_reduce_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, s>>>(a, n_q);
+            MSA_LAUNCH_CHECK();
+        }
     }
     attn_bwd_dq_kernel<G><<<dim3((a.T * G + kTile - 1) / kTile, a.hkv, n_q), 128, 0, s>>>(a);
     MSA_LAUNCH_CHECK();
@@ -384,7 +446,9 @@ __global__ void __launch_bounds__(256) gather_bwd_kernel(const float* __restrict
     }
     const float* src = dmem + ((int64_t)q * max_mem + at) * row_len;
     float* dst = dkvbar + c0 * row_len;
-    for (int64_t i = threadIdx.x; i < rows * row_len; i += blockDim.x) atomicAdd(dst + i, src[i]);
+    const int64_t step = (int64_t)gridDim.z * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.z * blockDim.x + threadIdx.x; i < rows * row_len; i += step)
+        atomicAdd(dst + i, src[i]);
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -419,11 +483,34 @@ __device__ __forceinline__ float load_elem(const void* p, int64_t i, int bf16) {
     return static_cast<const float*>(p)[i];
 }
 
-__global__ void __launch_bounds__(128) pool_bwd_kernel(const PoolBwdArgs a) {
-    __shared__ float gsh[1024 + 32];
+// Four consecutive elements at index i (a multiple of 4) of a bf16 or fp32 array, as fp32.
+__device__ __forceinline__ float4 load4(const void* p, int64_t i, int bf16) {
+    if (bf16) {
+        const uint2 u = *reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(p) + i);
+        return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u), __uint_as_float(u.y << 16),
+                           __uint_as_float(u.y & 0xffff0000u));
+    }
+    return *reinterpret_cast<const float4*>(static_cast<const float*>(p) + i);
+}
+
+__device__ __forceinline__ float4 scale4(float4 v, float s) { return make_float4(v.x * s, v.y * s, v.z * s, v.w * s); }
+
+// Block per (chunk, tensor part); thread i owns elements 4i..4i+3 of a token row (rows of at most
+// 1024 elements, one head = d/4 consecutive lanes of a warp). The chunk's gradient is read once;
+// every token of the chunk then gets one 16-byte streaming store per thread.
+constexpr int kPoolBwdThreads = 256;
+
+__global__ void __launch_bounds__(kPoolBwdThreads) pool_bwd_kernel(const PoolBwdArgs a) {
     const int part = a.parts[blockIdx.x % a.n_parts];
     const int64_t c_stride = gridDim.x / a.n_parts;
     const int d = a.d;
+    const int E = (part == 2 ? a.hr : a.hkv) * d;
+    const int e0 = threadIdx.x * 4;
+    const bool active = e0 < E;
+    const int ih = e0 % d;
+    const bool first = ih < d / 2;
+    const int hi = first ? ih : ih - d / 2;
+    const int head_lanes = d / 4;
     for (int64_t c = blockIdx.x / a.n_parts; c < a.n_chunks; c += c_stride) {
         const int64_t doc = a.chunk_doc[c];
         if (doc < 0 || doc >= a.n_docs) {
@@ -438,67 +525,61 @@ __global__ void __launch_bounds__(128) pool_bwd_kernel(const PoolBwdArgs a) {
             continue;
         }
         const float inv_n = 1.0f / (float)(t1 - t0);
-        if (part == 0 || part == 1) {
-            const int E = a.hkv * d;
-            const float* g = a.dkvbar + (c * 2 + part) * (int64_t)E;
-            float* out = part == 0 ? a.dk : a.dv;
-            for (int64_t t = t0; t < t1; ++t) {
-                const int64_t p = t - doc_start;
-                const bool rot = part == 0 && a.fuse_rope;
-                if (rot && p >= a.max_pos && threadIdx.x == 0) record_device_error(a.err, MSA_DEV_ROPE_POSITION);
-                for (int e = threadIdx.x; e < E; e += blockDim.x) {
-                    float x = g[e] * inv_n;
-                    if (rot && p < a.max_pos) {
-                        const int i = e % d;
-                        const int hi = i < d / 2 ? i : i - d / 2;
-                        const float2 cs = a.cs[p * (d / 2) + hi];
-                        const int partner = i < d / 2 ? e + d / 2 : e - d / 2;
-                        const float y = g[partner] * inv_n;
-                        // transpose of the rotation: first half x cos + y sin, second half x cos - y sin
-                        x = i < d / 2 ? fmaf(x, cs.x, y * cs.y) : fmaf(x, cs.x, -y * cs.y);
-                    }
-                    out[t * E + e] = x;
-                }
-            }
-        } else {
-            const int E = a.hr * d;
-            const float* g = a.dkr_index + c * (int64_t)E;
-            // gradient with respect to the raw pooled router key of every head
-            for (int e = threadIdx.x; e < E; e += blockDim.x) gsh[e] = g[e];
-            __syncthreads();
+        const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (part == 2) {
+            float4 g = active ? *reinterpret_cast<const float4*>(a.dkr_index + c * (int64_t)E + e0) : zero;
             if (a.normalize) {
-                // raw chunk mean into shared memory (second half of the buffer is not enough for
-                // E = 1024, so the mean overwrites nothing: use registers per element)
-                for (int h = threadIdx.x >> 5; h < a.hr; h += blockDim.x >> 5) {
-                    const int lane = threadIdx.x & 31;
-                    float ss = 0.f, dot = 0.f;
-                    float mean[8];
-                    for (int j = 0; j < d / 32 && j < 8; ++j) {
-                        const int e = h * d + lane + 32 * j;
-                        float m = 0.f;
-                        for (int64_t t = t0; t < t1; ++t) m += load_elem(a.kr, t * E + e, a.kr_bf16);
-                        m *= inv_n;
-                        mean[j] = m;
-                        ss = fmaf(m, m, ss);
-                        dot = fmaf(m, gsh[e], dot);
+                // the chunk's raw mean router key (this thread's 4 elements), then per head
+                // (g - k_hat (k_hat . g)) / |k| with k_hat = mean / |mean|
+                float4 mu = zero;
+                if (active)
+                    for (int64_t t = t0; t < t1; ++t) {
+                        const float4 x = load4(a.kr, t * E + e0, a.kr_bf16);
+                        mu.x += x.x; mu.y += x.y; mu.z += x.z; mu.w += x.w;
                     }
-#pragma unroll
-                    for (int o = 16; o >= 1; o >>= 1) {
-                        ss += __shfl_xor_sync(0xffffffffu, ss, o);
-                        dot += __shfl_xor_sync(0xffffffffu, dot, o);
-                    }
-                    const float nrm = sqrtf(ss);
-                    for (int j = 0; j < d / 32 && j < 8; ++j) {
-                        const int e = h * d + lane + 32 * j;
-                        // (g - k_hat (k_hat . g)) / |k| with k_hat = mean / |mean|
-                        gsh[e] = nrm > 0.f ? (gsh[e] - mean[j] * dot / (nrm * nrm)) / nrm : 0.f;
-                    }
+                mu = scale4(mu, inv_n);
+                float ss = mu.x * mu.x + mu.y * mu.y + mu.z * mu.z + mu.w * mu.w;
+                float dg = mu.x * g.x + mu.y * g.y + mu.z * g.z + mu.w * g.w;
+                for (int o = head_lanes / 2; o >= 1; o >>= 1) {
+                    ss += __shfl_xor_sync(0xffffffffu, ss, o);
+                    dg += __shfl_xor_sync(0xffffffffu, dg, o);
                 }
-                __syncthreads();
+                const float inv = ss > 0.f ? rsqrtf(ss) : 0.f;
+                const float proj = ss > 0.f ? dg / ss : 0.f;
+                g = make_float4((g.x - mu.x * proj) * inv, (g.y - mu.y * proj) * inv, (g.z - mu.z * proj) * inv,
+                                (g.w - mu.w * proj) * inv);
             }
-            for (int64_t t = t0; t < t1; ++t)
-                for (int e = threadIdx.x; e < E; e += blockDim.x) a.dkr[t * E + e] = gsh[e] * inv_n;
-            __syncthreads();
+            g = scale4(g, inv_n);
+            if (active)
+                for (int64_t t = t0; t < t1; ++t) __stcs(reinterpret_cast<float4*>(a.dkr + t * E + e0), g);
+            continue;
+        }
+        const float* grow = a.dkvbar + (c * 2 + part) * (int64_t)E;
+        const float4 g = active ? scale4(*reinterpret_cast<const float4*>(grow + e0), inv_n) : zero;
+        float* out = part == 0 ? a.dk : a.dv;
+        if (part == 1 || !a.fuse_rope) {
+            if (active)
+                for (int64_t t = t0; t < t1; ++t) __stcs(reinterpret_cast<float4*>(out + t * E + e0), g);
+            continue;
+        }
+        // keys: the transposed rotation of each token's position, R(-p):
+        // first half x cos + y sin, second half x cos - y sin (y the rotate-half partner)
+        const float4 y = active ? scale4(*reinterpret_cast<const float4*>(grow + (first ? e0 + d / 2 : e0 - d / 2)),
+                                         inv_n)
+                                : zero;
+        const float sg = first ? 1.f : -1.f;
+        for (int64_t t = t0; t < t1; ++t) {
+            const int64_t p = t - doc_start;
+            float4 o = g;
+            if (p < a.max_pos) {
+                const float4 c01 = *reinterpret_cast<const float4*>(a.cs + p * (d / 2) + hi);
+                const float4 c23 = *reinterpret_cast<const float4*>(a.cs + p * (d / 2) + hi + 2);
+                o = make_float4(fmaf(g.x, c01.x, sg * y.x * c01.y), fmaf(g.y, c01.z, sg * y.y * c01.w),
+                                fmaf(g.z, c23.x, sg * y.z * c23.y), fmaf(g.w, c23.z, sg * y.w * c23.w));
+            } else if (threadIdx.x == 0) {
+                record_device_error(a.err, MSA_DEV_ROPE_POSITION);
+            }
+            if (active) __stcs(reinterpret_cast<float4*>(out + t * E + e0), o);
         }
     }
 }
@@ -588,40 +669,74 @@ __global__ void __launch_bounds__(128) route_bwd_qhat_kernel(const void* __restr
     for (int i = lane; i < d; i += 32) qhat[w * d + i] = load_elem(qr, w * d + i, qr_bf16) * inv;
 }
 
-// (2) per (query, chunk): best folded score over the query tokens and the first token attaining it.
-//     Block per chunk (grid-stride), the chunk's index row in shared memory, warp per token.
+// (2) per (query, chunk): best folded score over the query tokens and the first token attaining it,
+//     as one 64-bit key (order-preserving bits of the score, then the complement of the token) so
+//     that an atomic max keeps the best score and, among equal scores, the first token.
+//     Block per (group of 8 chunks, slice of 64 tokens), grid-stride: the chunks' index rows in
+//     shared memory, each warp scores one token against all 8 chunks per read of its qhat.
+constexpr int kBestChunks = 8;
+constexpr int kBestTokens = 64;
+
+__device__ __forceinline__ unsigned long long best_key(float score, int t) {
+    const uint32_t b = __float_as_uint(score);
+    const uint32_t o = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+    return ((unsigned long long)o << 32) | (unsigned long long)(0xffffffffu - (uint32_t)t);
+}
+
+__device__ __forceinline__ float best_score(unsigned long long key) {
+    const uint32_t o = (uint32_t)(key >> 32);
+    return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
+}
+
 __global__ void __launch_bounds__(256) route_bwd_best_kernel(const void* __restrict__ index, int idx_bf16,
                                                              int64_t n_chunks, const float* __restrict__ qhat, int n_q,
-                                                             int T, int K, float* __restrict__ best,
-                                                             int* __restrict__ best_t) {
-    __shared__ float krow[1024];
-    __shared__ float wbest[8];
-    __shared__ int wt[8];
+                                                             int T, int K, unsigned long long* __restrict__ best) {
+    __shared__ float krow[kBestChunks][1024];
+    __shared__ unsigned long long wbest[8][kBestChunks];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int64_t c = blockIdx.x; c < n_chunks; c += gridDim.x) {
+    const int64_t groups = (n_chunks + kBestChunks - 1) / kBestChunks;
+    const int slices = (T + kBestTokens - 1) / kBestTokens;
+    for (int64_t w = blockIdx.x; w < groups * slices; w += gridDim.x) {
+        const int64_t c0 = (w / slices) * kBestChunks;
+        const int tb = (int)(w % slices) * kBestTokens, te = min(tb + kBestTokens, T);
+        const int nc = (int)min((int64_t)kBestChunks, n_chunks - c0);
         __syncthreads();
-        for (int i = threadIdx.x; i < K; i += blockDim.x) krow[i] = load_elem(index, c * K + i, idx_bf16);
+        for (int i = threadIdx.x; i < kBestChunks * K; i += blockDim.x) {
+            const int j = i / K, e = i % K;
+            krow[j][e] = j < nc ? load_elem(index, (c0 + j) * K + e, idx_bf16) : 0.f;
+        }
         __syncthreads();
         for (int q = 0; q < n_q; ++q) {
-            float bs = -__int_as_float(0x7f800000);
-            int bt = 0x7fffffff;
-            for (int t = warp; t < T; t += 8) {
-                const float* qv = qhat + ((int64_t)q * T + t) * K;
-                float acc = 0.f;
-                for (int i = lane; i < K; i += 32) acc = fmaf(qv[i], krow[i], acc);
+            unsigned long long bk[kBestChunks];
 #pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-                if (acc > bs) { bs = acc; bt = t; }             // t increases: first maximum kept
+            for (int j = 0; j < kBestChunks; ++j) bk[j] = 0ull;
+            for (int t = tb + warp; t < te; t += 8) {
+                const float* qv = qhat + ((int64_t)q * T + t) * K;
+                float acc[kBestChunks];
+#pragma unroll
+                for (int j = 0; j < kBestChunks; ++j) acc[j] = 0.f;
+                for (int i = lane; i < K; i += 32) {
+                    const float x = qv[i];
+#pragma unroll
+                    for (int j = 0; j < kBestChunks; ++j) acc[j] = fmaf(x, krow[j][i], acc[j]);
+                }
+#pragma unroll
+                for (int j = 0; j < kBestChunks; ++j) {
+#pragma unroll
+                    for (int o = 16; o >= 1; o >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
+                    const unsigned long long key = best_key(acc[j], t);
+                    bk[j] = key > bk[j] ? key : bk[j];
+                }
             }
-            if (lane == 0) { wbest[warp] = bs; wt[warp] = bt; }
+            if (lane == 0)
+#pragma unroll
+                for (int j = 0; j < kBestChunks; ++j) wbest[warp][j] = bk[j];
             __syncthreads();
-            if (threadIdx.x == 0) {
-                float b = wbest[0];
-                int tt = wt[0];
-                for (int w = 1; w < 8; ++w)
-                    if (wbest[w] > b || (wbest[w] == b && wt[w] < tt)) { b = wbest[w]; tt = wt[w]; }
-                best[(int64_t)q * n_chunks + c] = b;
-                best_t[(int64_t)q * n_chunks + c] = tt < T ? tt : -1;
+            if (threadIdx.x < nc) {
+                const int j = threadIdx.x;
+                unsigned long long b = wbest[0][j];
+                for (int x = 1; x < 8; ++x) b = wbest[x][j] > b ? wbest[x][j] : b;
+                if (b) atomicMax(best + (int64_t)q * n_chunks + c0 + j, b);
             }
             __syncthreads();
         }
@@ -634,8 +749,7 @@ __global__ void __launch_bounds__(256) route_bwd_best_kernel(const void* __restr
 __global__ void __launch_bounds__(256) route_bwd_scatter_kernel(const void* __restrict__ index, int idx_bf16,
                                                                 const int64_t* __restrict__ doc_chunk_off,
                                                                 int64_t n_docs, int64_t n_chunks,
-                                                                const float* __restrict__ best,
-                                                                const int* __restrict__ best_t,
+                                                                const unsigned long long* __restrict__ best,
                                                                 const float* __restrict__ qhat,
                                                                 const float* __restrict__ dscore, int n_q, int T,
                                                                 int H, int K, float* __restrict__ dqhat,
@@ -650,9 +764,11 @@ __global__ void __launch_bounds__(256) route_bwd_scatter_kernel(const void* __re
     if (ds == 0.f || b <= a || a < 0 || b > n_chunks) return;
     int64_t cbest = a;
     for (int64_t c = a + 1; c < b; ++c)
-        if (best[(int64_t)q * n_chunks + c] > best[(int64_t)q * n_chunks + cbest]) cbest = c;
-    const int t = best_t[(int64_t)q * n_chunks + cbest];
-    if (t < 0) return;
+        if (best_score(best[(int64_t)q * n_chunks + c]) > best_score(best[(int64_t)q * n_chunks + cbest])) cbest = c;
+    const unsigned long long key = best[(int64_t)q * n_chunks + cbest];
+    if (key == 0ull) return;
+    const int t = (int)(0xffffffffu - (uint32_t)(key & 0xffffffffull));
+    if (t < 0 || t >= T) return;
     const float* qv = qhat + ((int64_t)q * T + t) * K;
     const float invH = 1.0f / H;
     for (int i = lane; i < K; i += 32) {
@@ -694,9 +810,11 @@ using namespace msa;
 
 extern "C" {
 
-msa_status msa_sparse_attn_backward_workspace_size(int n_q, int T, int hq, size_t* bytes) {
-    MSA_REQUIRE(bytes && n_q > 0 && T >= 0 && hq > 0, "msa_sparse_attn_backward_workspace_size: bad arguments");
-    *bytes = align_up((size_t)n_q * T * hq * sizeof(float), 256);
+msa_status msa_sparse_attn_backward_workspace_size(int n_q, int T, int hq, int hkv, int max_mem, int L,
+                                                   size_t* bytes) {
+    MSA_REQUIRE(bytes && n_q > 0 && T >= 0 && hq > 0 && hkv > 0 && hq % hkv == 0 && max_mem >= 0 && L >= 0,
+                "msa_sparse_attn_backward_workspace_size: bad arguments");
+    *bytes = bwd_ws_bytes(n_q, T, hq, hkv, max_mem, L);
     return MSA_OK;
 }
 
@@ -724,7 +842,7 @@ msa_status msa_sparse_attn_backward(const void* q, const void* mem_kv, const int
                                 aligned16(dlocal_v))),
                 "msa_sparse_attn_backward: pointers must be 16-byte aligned");
     size_t need = 0;
-    MSA_RETURN_IF(msa_sparse_attn_backward_workspace_size(n_q, T, hq, &need));
+    MSA_RETURN_IF(msa_sparse_attn_backward_workspace_size(n_q, T, hq, hkv, max_mem, L, &need));
     if (ws_bytes < need)
         return set_error(MSA_ERR_WORKSPACE, "msa_sparse_attn_backward: workspace %zu < %zu", ws_bytes, need);
     BwdArgs a{};
@@ -739,6 +857,9 @@ msa_status msa_sparse_attn_backward(const void* q, const void* mem_kv, const int
     a.dout = static_cast<const __nv_bfloat16*>(dout);
     a.lse = lse; a.Dvec = static_cast<float*>(ws);
     a.dq = dq; a.dmem = dmem_kv; a.dlk = dlocal_k; a.dlv = dlocal_v;
+    a.n_rsplit = pick_rsplit(n_q, T, hq, hkv, max_mem, L);
+    a.key_pad = ((max_mem + L + kTile - 1) / kTile) * kTile;
+    a.part_dkv = reinterpret_cast<float*>(static_cast<char*>(ws) + align_up((size_t)n_q * T * hq * sizeof(float), 256));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int64_t rows = (int64_t)n_q * T * hq;
     attn_bwd_prep_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(a.out, a.dout, rows, a.Dvec);
@@ -753,11 +874,17 @@ msa_status msa_sparse_attn_backward(const void* q, const void* mem_kv, const int
 
 msa_status msa_gather_kv_backward(const float* dmem_kv, int64_t n_chunks, const int64_t* doc_chunk_off,
                                   int64_t n_docs, const int32_t* idx, int n_q, int k, int hkv, int d, int max_mem,
-                                  float* dkvbar, void* stream) {
+                                  float* dkvbar, int accumulate, void* stream) {
     MSA_REQUIRE(dmem_kv && doc_chunk_off && idx && dkvbar, "msa_gather_kv_backward: NULL pointer");
     MSA_REQUIRE(n_q > 0 && n_q <= 65535 && k > 0 && hkv > 0 && d > 0 && max_mem >= 0 && n_docs > 0 && n_chunks >= 0,
                 "msa_gather_kv_backward: bad sizes");
-    gather_bwd_kernel<<<dim3(k, n_q), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+    if (!accumulate)
+        MSA_CUDA_TRY(cudaMemsetAsync(dkvbar, 0, (size_t)n_chunks * 2 * hkv * d * sizeof(float),
+                                     static_cast<cudaStream_t>(stream)));
+    // a document's rows dealt out to several blocks (about 4K elements each, at most 64)
+    const int64_t per_doc = ((int64_t)max_mem * 2 * hkv * d) / k;
+    const int parts = (int)std::min<int64_t>(64, std::max<int64_t>(1, (per_doc + 4095) / 4096));
+    gather_bwd_kernel<<<dim3(k, n_q, parts), 256, 0, static_cast<cudaStream_t>(stream)>>>(
         dmem_kv, n_chunks, doc_chunk_off, n_docs, idx, k, 2 * hkv * d, max_mem, dkvbar, device_error_word());
     MSA_LAUNCH_CHECK();
     return MSA_OK;
@@ -776,16 +903,24 @@ msa_status msa_pool_chunks_backward(const float* dkvbar, const float* dkr_index,
     MSA_REQUIRE(doc_tok_off && doc_chunk_off && chunk_doc, "msa_pool_chunks_backward: NULL offsets");
     PoolBwdArgs a{};
     a.n_parts = 0;
+    // one thread per 4 elements of a row, a head on d/4 lanes of one warp
+    if (d % 8 != 0 || d / 4 > 32 || ((d / 4) & (d / 4 - 1)) != 0)
+        return set_error(MSA_ERR_UNSUPPORTED, "msa_pool_chunks_backward: head_dim %d unsupported (8..128, d/4 a power of two)", d);
     if (dkvbar) {
-        MSA_REQUIRE(hkv > 0 && dk && dv, "msa_pool_chunks_backward: K/V gradients need hkv > 0, dk and dv");
-        MSA_REQUIRE(!fuse_doc_rope || (cos_sin && max_pos > 0), "msa_pool_chunks_backward: RoPE needs a table");
+        MSA_REQUIRE(hkv > 0 && (size_t)hkv * d <= 4 * kPoolBwdThreads && dk && dv,
+                    "msa_pool_chunks_backward: K/V gradients need 0 < hkv * d <= 1024, dk and dv");
+        MSA_REQUIRE(aligned16(dkvbar) && aligned16(dk) && aligned16(dv), "msa_pool_chunks_backward: unaligned K/V pointer");
+        MSA_REQUIRE(!fuse_doc_rope || (cos_sin && max_pos > 0 && aligned16(cos_sin)),
+                    "msa_pool_chunks_backward: RoPE needs a table");
         a.parts[a.n_parts++] = 0;
         a.parts[a.n_parts++] = 1;
     }
     if (dkr_index) {
-        MSA_REQUIRE(hr > 0 && dkr && (size_t)hr * d <= 1024, "msa_pool_chunks_backward: K^R needs hr * d <= 1024, dkr");
-        MSA_REQUIRE(!normalize_router || (kr && dtype_ok(kr_dt) && d % 32 == 0 && d <= 256),
-                    "msa_pool_chunks_backward: the normalised index needs the token K^R and d a multiple of 32 <= 256");
+        MSA_REQUIRE(hr > 0 && dkr && (size_t)hr * d <= 4 * kPoolBwdThreads,
+                    "msa_pool_chunks_backward: K^R needs 0 < hr * d <= 1024 and dkr");
+        MSA_REQUIRE(aligned16(dkr_index) && aligned16(dkr), "msa_pool_chunks_backward: unaligned K^R pointer");
+        MSA_REQUIRE(!normalize_router || (kr && dtype_ok(kr_dt) && aligned16(kr)),
+                    "msa_pool_chunks_backward: the normalised index needs the token K^R");
         a.parts[a.n_parts++] = 2;
     }
     a.dkvbar = dkvbar; a.dkr_index = dkr_index; a.kr = kr; a.kr_bf16 = kr_dt == MSA_BF16;
@@ -795,8 +930,8 @@ msa_status msa_pool_chunks_backward(const float* dkvbar, const float* dkr_index,
     a.fuse_rope = fuse_doc_rope; a.normalize = normalize_router;
     a.cs = reinterpret_cast<const float2*>(cos_sin); a.max_pos = max_pos;
     a.dk = dk; a.dv = dv; a.dkr = dkr; a.err = device_error_word();
-    const int64_t per_part = std::min<int64_t>(n_chunks, (int64_t)sm_count() * 16);
-    pool_bwd_kernel<<<(unsigned)(per_part * a.n_parts), 128, 0, static_cast<cudaStream_t>(stream)>>>(a);
+    const int64_t per_part = std::min<int64_t>(n_chunks, (int64_t)1 << 20);
+    pool_bwd_kernel<<<(unsigned)(per_part * a.n_parts), kPoolBwdThreads, 0, static_cast<cudaStream_t>(stream)>>>(a);
     MSA_LAUNCH_CHECK();
     return MSA_OK;
 }
@@ -814,7 +949,7 @@ msa_status msa_router_aux_loss(const float* doc_scores, int n_q, int64_t n_docs,
 msa_status msa_route_backward_workspace_size(int64_t n_chunks, int n_q, int T, int H, int d, size_t* bytes) {
     MSA_REQUIRE(bytes && n_chunks >= 0 && n_q > 0 && T > 0 && H > 0 && d > 0, "msa_route_backward_workspace_size: bad sizes");
     const size_t qk = (size_t)n_q * T * H * d * sizeof(float);
-    *bytes = 2 * align_up(qk, 256) + 2 * align_up((size_t)n_q * n_chunks * 4, 256);
+    *bytes = 2 * align_up(qk, 256) + align_up((size_t)n_q * n_chunks * 8, 256);
     return MSA_OK;
 }
 
@@ -833,20 +968,21 @@ msa_status msa_route_backward(const void* kr_index, msa_dtype dt, int64_t n_chun
     char* w = static_cast<char*>(ws);
     float* qhat = reinterpret_cast<float*>(w);
     float* dqhat = reinterpret_cast<float*>(w + qk);
-    float* best = reinterpret_cast<float*>(w + 2 * qk);
-    int* best_t = reinterpret_cast<int*>(w + 2 * qk + align_up((size_t)n_q * n_chunks * 4, 256));
+    unsigned long long* best = reinterpret_cast<unsigned long long*>(w + 2 * qk);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int bf = dt == MSA_BF16;
     const int64_t rows = (int64_t)n_q * T;
     MSA_CUDA_TRY(cudaMemsetAsync(dqhat, 0, (size_t)n_q * T * K * sizeof(float), s));
     MSA_CUDA_TRY(cudaMemsetAsync(dkhat, 0, (size_t)n_chunks * K * sizeof(float), s));
+    MSA_CUDA_TRY(cudaMemsetAsync(best, 0, (size_t)n_q * n_chunks * sizeof(unsigned long long), s));
     route_bwd_qhat_kernel<<<(unsigned)((rows * H + 3) / 4), 128, 0, s>>>(qr, bf, rows, H, d, qhat);
     MSA_LAUNCH_CHECK();
-    const unsigned best_blocks = (unsigned)std::min<int64_t>(n_chunks, (int64_t)sm_count() * 8);
-    route_bwd_best_kernel<<<best_blocks, 256, 0, s>>>(kr_index, bf, n_chunks, qhat, n_q, T, K, best, best_t);
+    const int64_t work = ((n_chunks + kBestChunks - 1) / kBestChunks) * ((T + kBestTokens - 1) / kBestTokens);
+    const unsigned best_blocks = (unsigned)std::min<int64_t>(work, (int64_t)sm_count() * 8);
+    route_bwd_best_kernel<<<best_blocks, 256, 0, s>>>(kr_index, bf, n_chunks, qhat, n_q, T, K, best);
     MSA_LAUNCH_CHECK();
     route_bwd_scatter_kernel<<<(unsigned)(((int64_t)n_q * n_docs + 7) / 8), 256, 0, s>>>(
-        kr_index, bf, doc_chunk_off, n_docs, n_chunks, best, best_t, qhat, d_doc_scores, n_q, T, H, K, dqhat, dkhat);
+        kr_index, bf, doc_chunk_off, n_docs, n_chunks, best, qhat, d_doc_scores, n_q, T, H, K, dqhat, dkhat);
     MSA_LAUNCH_CHECK();
     route_bwd_qr_kernel<<<(unsigned)((rows * H + 3) / 4), 128, 0, s>>>(qr, bf, rows, H, d, dqhat, dqr);
     MSA_LAUNCH_CHECK();
