@@ -265,15 +265,18 @@ msa_status msa_sparse_attn(const void* q, const void* mem_kv, const int32_t* mem
                            const void* local_k, const void* local_v, int L_max, int L, int q_start, int n_q, int T,
                            int hq, int hkv, int d, float scale, void* out, msa_dtype dt, void* stream);
 
-/* Selects the bf16 attention kernel for testing: 0 = tensor cores (mma.sync m16n8k16, default),
- * 1 = CUDA cores. fp32 always runs on CUDA cores. Process-wide. */
+/* Selects the bf16 attention kernels for testing: 0 = default (msa_sparse_attn_split on tcgen05
+ * tensor cores with TMEM accumulators, msa_sparse_attn on mma.sync m16n8k16 so that it can run
+ * beside the router's blocks), 1 = CUDA cores for msa_sparse_attn, 2 = mma.sync for both.
+ * fp32 always runs on CUDA cores. Process-wide. */
 msa_status msa_attn_set_impl(int impl);
 
 /* Sparse attention over long memories (the token-level fine stage, thousands of memory rows per
  * query): the same arguments, layout and result as msa_sparse_attn, computed with the keys of
  * every (64-row block, kv head, query) split into n_split contiguous ranges of 64-key tiles that
- * run as separate blocks. Each writes its unnormalised output and (running max, sum) in fp32 to
- * the workspace; a second kernel merges the ranges' softmax statistics and writes out.
+ * run as separate blocks (tcgen05: one CTA per 128 (token, head) rows, S and O accumulated in
+ * TMEM; see msa_attn_set_impl). Each writes its unnormalised output and (running max, sum) in
+ * fp32 to the workspace; a second kernel merges the ranges' softmax statistics and writes out.
  * n_split is chosen from the sizes so that the grid fits one wave of three blocks per SM (148
  * SMs), at least four tiles per range. bf16 only (tensor cores); fp32 returns MSA_ERR_UNSUPPORTED.
  * lse: optional device float [n_q][T][hq]: ln sum_j exp(scale * q . k_j) over the row's visible

@@ -113,7 +113,8 @@ def route_workspace_size(n_q: int, T: int, H: int, d: int, dtype) -> int:
 
 
 def attn_set_impl(impl: int) -> None:
-    """bf16 attention: 0 = tensor cores (default), 1 = CUDA cores."""
+    """bf16 attention: 0 = default (split variant on tcgen05, plain on mma.sync), 1 = CUDA cores for the
+    plain variant, 2 = mma.sync for both."""
     check(lib.msa_attn_set_impl(impl), "msa_attn_set_impl")
 
 

@@ -13,10 +13,18 @@
 #include "mma.cuh"
 
 namespace msa {
+
+msa_status launch_attn_tc(const void* q, const void* mem_kv, const int32_t* mem_len, int max_mem, const void* local_k,
+                          const void* local_v, int L_max, int L, int q_start, int n_q, int T, int hq, int hkv,
+                          float scale_log2e, int n_split, float* part_o, float2* part_ml, cudaStream_t s);
+int attn_tc_splits(int n_q, int T, int hq, int hkv, int max_mem, int L);
+
 namespace {
 
 constexpr int kD = 128;
-std::atomic<int> g_attn_impl{0};   // bf16: 0 = tensor cores (mma.sync), 1 = CUDA cores
+// bf16: 0 = default (split variant on tcgen05, plain on mma.sync), 1 = CUDA cores for the plain
+// variant, 2 = mma.sync for both
+std::atomic<int> g_attn_impl{0};
 constexpr int kTokPerBlock = 8;
 constexpr int kKeyTile = 32;
 
@@ -125,7 +133,7 @@ __global__ void __launch_bounds__(kTokPerBlock * 32) attn_kernel(const AttnArgs 
         if (!tok_ok) continue;
 
         const int kk = tb + lane;
-        const bool visible = kk < mem_len || (kk < n_keys && kk - mem_len <= a.q_start + t);
+        const bool visible = (kk < mem_len) | ((kk < n_keys) & (kk - mem_len <= a.q_start + t));
         float s[G];
 #pragma unroll
         for (int h = 0; h < G; ++h) s[h] = 0.f;
@@ -339,8 +347,9 @@ __global__ void __launch_bounds__(128, SPLIT ? 3 : 1) attn_mma_kernel(const Attn
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 const int kk = kb + nb * 8 + tig * 2 + e;
-                const bool vis_a = va && (kk < mem_len || (kk < n_keys && kk - mem_len <= a.q_start + ta));
-                const bool vis_b = vb && (kk < mem_len || (kk < n_keys && kk - mem_len <= a.q_start + tb));
+                // branch-free (bitwise) masks: a memory row, or a causal local key inside the range
+                const bool vis_a = va & ((kk < mem_len) | ((kk < n_keys) & (kk - mem_len <= a.q_start + ta)));
+                const bool vis_b = vb & ((kk < mem_len) | ((kk < n_keys) & (kk - mem_len <= a.q_start + tb)));
                 sc[nb][e] = vis_a ? sc[nb][e] * a.scale_log2e : ninf;
                 sc[nb][2 + e] = vis_b ? sc[nb][2 + e] * a.scale_log2e : ninf;
                 tm_a = fmaxf(tm_a, sc[nb][e]);
@@ -352,8 +361,9 @@ __global__ void __launch_bounds__(128, SPLIT ? 3 : 1) attn_mma_kernel(const Attn
         tm_b = fmaxf(tm_b, __shfl_xor_sync(0xffffffffu, tm_b, 1));
         tm_b = fmaxf(tm_b, __shfl_xor_sync(0xffffffffu, tm_b, 2));
         const float mn_a = fmaxf(m_a, tm_a), mn_b = fmaxf(m_b, tm_b);
-        const float f_a = mn_a == ninf ? 1.f : exp2f(m_a - mn_a);
-        const float f_b = mn_b == ninf ? 1.f : exp2f(m_b - mn_b);
+        const float f_a = mn_a == ninf ? 1.f : ex2(m_a - mn_a);
+        const float f_b = mn_b == ninf ? 1.f : ex2(m_b - mn_b);
+        const float ref_a = mn_a == ninf ? 0.f : mn_a, ref_b = mn_b == ninf ? 0.f : mn_b;   // masked: 2^-inf = 0
         m_a = mn_a;
         m_b = mn_b;
         float ps_a = 0.f, ps_b = 0.f;
@@ -361,8 +371,8 @@ __global__ void __launch_bounds__(128, SPLIT ? 3 : 1) attn_mma_kernel(const Attn
         for (int nb = 0; nb < kMmaKeys / 8; ++nb) {
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-                sc[nb][e] = mn_a == ninf ? 0.f : exp2f(sc[nb][e] - mn_a);
-                sc[nb][2 + e] = mn_b == ninf ? 0.f : exp2f(sc[nb][2 + e] - mn_b);
+                sc[nb][e] = ex2(sc[nb][e] - ref_a);
+                sc[nb][2 + e] = ex2(sc[nb][2 + e] - ref_b);
                 ps_a += sc[nb][e];
                 ps_b += sc[nb][2 + e];
             }
@@ -472,6 +482,14 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
     *reinterpret_cast<uint2*>(out + row * kD + lane * 4) = u;
 }
 
+msa_status launch_combine(const AttnArgs& a, int n_q, cudaStream_t s) {
+    const int64_t rows = (int64_t)n_q * a.T * a.hq;
+    attn_combine_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(a.part_o, a.part_ml, a.n_split, rows,
+                                                                   static_cast<__nv_bfloat16*>(a.out), a.lse);
+    MSA_LAUNCH_CHECK();
+    return MSA_OK;
+}
+
 template <int G, bool SPLIT>
 msa_status launch_mma_g(const AttnArgs& a, int n_q, cudaStream_t s) {
     const int row_blocks = (a.T * G + kMmaRows - 1) / kMmaRows;
@@ -482,12 +500,7 @@ msa_status launch_mma_g(const AttnArgs& a, int n_q, cudaStream_t s) {
                                           (int)smem));
     attn_mma_kernel<G, SPLIT><<<grid, 128, smem, s>>>(a);
     MSA_LAUNCH_CHECK();
-    if constexpr (SPLIT) {
-        const int64_t rows = (int64_t)n_q * a.T * a.hq;
-        attn_combine_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(a.part_o, a.part_ml, a.n_split, rows,
-                                                                       static_cast<__nv_bfloat16*>(a.out), a.lse);
-        MSA_LAUNCH_CHECK();
-    }
+    if constexpr (SPLIT) return launch_combine(a, n_q, s);
     return MSA_OK;
 }
 
@@ -517,6 +530,10 @@ int pick_splits(int n_q, int T, int hq, int hkv, int max_mem, int L) {
     return (int)std::max<int64_t>(1, std::min(want, cap));
 }
 
+int split_ws_splits(int n_q, int T, int hq, int hkv, int max_mem, int L) {
+    return std::max(pick_splits(n_q, T, hq, hkv, max_mem, L), attn_tc_splits(n_q, T, hq, hkv, max_mem, L));
+}
+
 size_t split_ws_bytes(int n_split, int n_q, int T, int hq) {
     const size_t rows = (size_t)n_q * T * hq;
     return align_up((size_t)n_split * rows * kD * 4, 256) + align_up((size_t)n_split * rows * 8, 256);
@@ -530,7 +547,7 @@ using namespace msa;
 extern "C" {
 
 msa_status msa_attn_set_impl(int impl) {
-    MSA_REQUIRE(impl == 0 || impl == 1, "msa_attn_set_impl: impl must be 0 or 1");
+    MSA_REQUIRE(impl >= 0 && impl <= 2, "msa_attn_set_impl: impl must be 0, 1 or 2");
     g_attn_impl.store(impl);
     return MSA_OK;
 }
@@ -566,7 +583,7 @@ msa_status msa_sparse_attn_split_workspace_size(int n_q, int T, int hq, int hkv,
     MSA_REQUIRE(bytes, "msa_sparse_attn_split_workspace_size: bytes is NULL");
     MSA_REQUIRE(n_q > 0 && T >= 0 && hq > 0 && hkv > 0 && hq % hkv == 0 && max_mem >= 0 && L >= 0,
                 "msa_sparse_attn_split_workspace_size: bad sizes");
-    *bytes = split_ws_bytes(pick_splits(n_q, T, hq, hkv, max_mem, L), n_q, T, hq);
+    *bytes = split_ws_bytes(split_ws_splits(n_q, T, hq, hkv, max_mem, L), n_q, T, hq);
     return MSA_OK;
 }
 
@@ -590,8 +607,9 @@ msa_status msa_sparse_attn_split(const void* q, const void* mem_kv, const int32_
     MSA_REQUIRE(aligned16(q) && aligned16(out) && aligned16(ws) && (max_mem == 0 || aligned16(mem_kv)) &&
                     (L == 0 || (aligned16(local_k) && aligned16(local_v))),
                 "msa_sparse_attn_split: pointers must be 16-byte aligned");
-    const int n_split = pick_splits(n_q, T, hq, hkv, max_mem, L);
-    const size_t need = split_ws_bytes(n_split, n_q, T, hq);
+    const bool tc = g_attn_impl.load() == 0;
+    const int n_split = tc ? attn_tc_splits(n_q, T, hq, hkv, max_mem, L) : pick_splits(n_q, T, hq, hkv, max_mem, L);
+    const size_t need = split_ws_bytes(split_ws_splits(n_q, T, hq, hkv, max_mem, L), n_q, T, hq);
     if (ws_bytes < need)
         return set_error(MSA_ERR_WORKSPACE, "msa_sparse_attn_split: workspace %zu < %zu", ws_bytes, need);
     AttnArgs a{};
@@ -603,7 +621,13 @@ msa_status msa_sparse_attn_split(const void* q, const void* mem_kv, const int32_
     a.part_o = static_cast<float*>(ws);
     a.part_ml = reinterpret_cast<float2*>(static_cast<char*>(ws) +
                                           align_up((size_t)n_split * n_q * T * hq * kD * 4, 256));
-    return launch_mma<true>(a, n_q, static_cast<cudaStream_t>(stream));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (tc) {
+        MSA_RETURN_IF(launch_attn_tc(q, mem_kv, mem_len, max_mem, local_k, local_v, L_max, L, q_start, n_q, T, hq, hkv,
+                                     a.scale_log2e, n_split, a.part_o, a.part_ml, st));
+        return launch_combine(a, n_q, st);
+    }
+    return launch_mma<true>(a, n_q, st);
 }
 
 }  // extern "C"

@@ -49,8 +49,9 @@ struct BwdArgs {
     float* part_dkv;         // [n_rsplit][n_q][key_pad][2][hkv][d] partial dK (x scale) / dV per row range
 };
 
+// branch-free (bitwise) visibility: a memory row, or a causal local key inside the key range
 __device__ __forceinline__ bool key_visible(int kk, int mem_len, int n_keys, int q_start, int t) {
-    return kk < mem_len || (kk < n_keys && kk - mem_len <= q_start + t);
+    return (kk < mem_len) | ((kk < n_keys) & (kk - mem_len <= q_start + t));
 }
 
 // D_r = sum_d dO . O: one warp per row, lane l owns dims 4l..4l+3.
@@ -190,8 +191,8 @@ __global__ void __launch_bounds__(128) attn_bwd_dkdv_kernel(const BwdArgs a) {
                 const int row = r0 + rl;
                 const int key = e < 2 ? key_a : key_b;
                 const float l2 = lse_s[rl];
-                const bool vis = row < n_rows && l2 != ninf && key_visible(key, mem_len, n_keys, a.q_start, row / G);
-                const float p = vis ? exp2f(st[nb][e] * a.scale_log2e - l2) : 0.f;
+                const bool vis = (row < n_rows) & (l2 != ninf) & key_visible(key, mem_len, n_keys, a.q_start, row / G);
+                const float p = ex2(vis ? st[nb][e] * a.scale_log2e - l2 : ninf);
                 st[nb][e] = p;
                 dpt[nb][e] = p * (dpt[nb][e] - D_s[rl]);
             }
@@ -322,9 +323,9 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_kernel(const BwdArgs a) {
             for (int e = 0; e < 4; ++e) {
                 const int kk = kb + nb * 8 + tig * 2 + (e & 1);
                 const bool first = e < 2;
-                const bool vis = (first ? va : vb) && (first ? l2a : l2b) != ninf &&
+                const bool vis = (first ? va : vb) & ((first ? l2a : l2b) != ninf) &
                                  key_visible(kk, mem_len, n_keys_all, a.q_start, first ? ta : tb);
-                const float p = vis ? exp2f(sc[nb][e] * a.scale_log2e - (first ? l2a : l2b)) : 0.f;
+                const float p = ex2(vis ? sc[nb][e] * a.scale_log2e - (first ? l2a : l2b) : ninf);
                 dp[nb][e] = p * (dp[nb][e] - (first ? Da : Db));
             }
         }

@@ -1,9 +1,16 @@
 // Internal launchers shared between translation units of the library.
 #pragma once
 
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace msa {
+
+// Tensor map of a bf16 array for TMA loads with the 128-byte swizzle (defined with the router):
+// dims[0] innermost in elements, strides[i] in bytes for dims i + 1, box in elements.
+msa_status make_tensor_map_bf16(CUtensorMap* map, const void* ptr, int rank, const uint64_t* dims,
+                                const uint64_t* strides, const uint32_t* box);
 
 // Rotates rows of [*, heads, d] vectors. Row r of the launch belongs to segment s at offset u:
 //   uniform_len > 0: s = r / uniform_len, u = r % uniform_len,

@@ -16,6 +16,14 @@ __device__ __forceinline__ void mma_bf16_16816(float* c, const uint32_t* a, uint
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// 2^x by the hardware base-2 exponential (PTX ex2.approx.ftz.f32, relative error about 2^-22;
+// 2^-inf = 0). Used where the result is rounded to a bf16 operand right after.
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);

@@ -336,11 +336,14 @@ def test_device_gather_token_rows_over_many_blocks(m):
     _status(m)
 
 
+@pytest.mark.parametrize("impl", [0, 2])
 @pytest.mark.parametrize("hq,hkv", [(32, 8), (8, 8), (32, 4)])
-@pytest.mark.parametrize("T,mem_lens,q_start", [(64, (0, 700, 1537), 0), (24, (4099, 1, 64), 40)])
-def test_sparse_attention_split_long_memory(m, hq, hkv, T, mem_lens, q_start):
-    """Split-key attention over long memories: several key ranges per block (some empty), ragged
-    tails, empty memory, causal local keys; against the oracle within the bf16 bound."""
+@pytest.mark.parametrize("T,mem_lens,q_start", [(64, (0, 700, 1537), 0), (24, (4099, 1, 64), 40),
+                                                (300, (130, 2200, 64), 5)])
+def test_sparse_attention_split_long_memory(m, impl, hq, hkv, T, mem_lens, q_start):
+    """Split-key attention over long memories, on tcgen05 (impl 0) and on mma.sync (impl 2): several
+    key ranges per block (some empty), ragged tails, empty memory, causal local keys, several
+    128-row blocks; against the oracle within the bf16 bound."""
     n_q, d, dtype = 3, 128, "bf16"
     max_mem = max(mem_lens) + 5
     L = q_start + T
@@ -349,9 +352,14 @@ def test_sparse_attention_split_long_memory(m, hq, hkv, T, mem_lens, q_start):
     lk, lv = _gen(104, (n_q, L + 3, hkv, d), dtype), _gen(105, (n_q, L + 3, hkv, d), dtype)
     mem_len = np.array(mem_lens, dtype=np.int32)
     rows = n_q * T * hq
-    assert m.sparse_attn_split_workspace_size(n_q, T, hq, hkv, max_mem, L) >= 2 * rows * (d * 4 + 8)   # >= 2 ranges
-    out = m.msa_sparse_attn_split(upload(q, dtype), upload(mem, dtype), torch.from_numpy(mem_len).cuda(),
-                                  upload(lk, dtype), upload(lv, dtype), L, q_start)
+    if T < 300:   # short query blocks: the memory is split into several key ranges
+        assert m.sparse_attn_split_workspace_size(n_q, T, hq, hkv, max_mem, L) >= 2 * rows * (d * 4 + 8)
+    m.attn_set_impl(impl)
+    try:
+        out = m.msa_sparse_attn_split(upload(q, dtype), upload(mem, dtype), torch.from_numpy(mem_len).cuda(),
+                                      upload(lk, dtype), upload(lv, dtype), L, q_start)
+    finally:
+        m.attn_set_impl(0)
     _status(m)
     got = _np(out)
     for qi in range(n_q):
