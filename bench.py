@@ -678,30 +678,81 @@ def main():
     torch.cuda.synchronize()
     route_ms = r0.elapsed_time(r1) / (reps * w.layers)
 
-    # ---- end to end through the public API with host buffers: H2D of every layer's query-side
-    # inputs from pinned memory, the round, D2H of every layer's attention output (idx already host)
-    host_in = [{k: v.cpu().pin_memory() for k, v in small[l].items()} for l in range(w.layers)]
-    host_out = [torch.empty(outs[l].shape, dtype=dt, pin_memory=True) for l in range(w.layers)]
-    h2d = sum(t.numel() * t.element_size() for d_ in host_in for t in d_.values())
-    d2h = sum(t.numel() * t.element_size() for t in host_out) + sum(t.numel() * 4 for t in idx_host)
-    e_steps = max(3, args.steps // 4)
+    # ---- end to end through the public API with host buffers, pipelined as a serving loop runs it:
+    # two sets of device input and output buffers; every step copies its query-side inputs (all
+    # layers, one contiguous pinned buffer) host -> device on an input stream while the previous
+    # step computes, and reads its attention outputs (and, inside the round, the selected indices)
+    # back device -> host on an output stream while the next step computes. The timed region ends
+    # after the last read-back, so every step's copies are inside it.
+    names = ("qr", "q", "k_new", "v_new")
+    in_bytes = [[small[l][k_].numel() * small[l][k_].element_size() for k_ in names] for l in range(w.layers)]
+    total_in = sum(sum(b_) for b_ in in_bytes)
+    host_in = torch.empty(total_in, dtype=torch.uint8, pin_memory=True)
+    at = 0
+    for l in range(w.layers):
+        for k_, nb in zip(names, in_bytes[l]):
+            host_in[at:at + nb].copy_(small[l][k_].contiguous().view(-1).view(torch.uint8).cpu())
+            at += nb
+    out_shape = (w.layers,) + tuple(outs[0].shape)
+    sets = []
+    for b_ in range(2):
+        dev_in = torch.empty(total_in, dtype=torch.uint8, device="cuda")
+        dev_in.copy_(host_in)
+        dev_out = torch.empty(out_shape, dtype=dt, device="cuda")
+        views, at = [], 0
+        for l in range(w.layers):
+            v_ = {}
+            for k_, nb in zip(names, in_bytes[l]):
+                v_[k_] = dev_in[at:at + nb].view(dt).view(small[l][k_].shape)
+                at += nb
+            views.append(v_)
+        la = [dict(layer_args[l], qr=views[l]["qr"], q_new=views[l]["q"], k_new=views[l]["k_new"],
+                   v_new=views[l]["v_new"], out=dev_out[l]) for l in range(w.layers)]
+        rd = m.InterleaveRound(la, n_chunks=lay.n_chunks, n_docs=lay.n_docs, doc_chunk_off=lay.doc_chunk_off,
+                               doc_chunk_off_host=lay.doc_chunk_off_host, chunk_doc=lay.chunk_doc, n_q=1, H=w.H,
+                               d=w.d, hq=w.hq, hkv=w.hkv, k=w.k, L_prev=0, T_new=w.T0, new_q_stride=w.T0,
+                               L_max=w.T0, max_mem=w.max_mem, cos_sin=cs, dtype=dt, reserved_sms=args.reserved_sms,
+                               fetch_mode=args.fetch_mode)
+        host_out = torch.empty(out_shape, dtype=dt, pin_memory=True)
+        sets.append((dev_in, dev_out, rd, host_out))
+    h2d = total_in
+    d2h = sets[0][1].numel() * sets[0][1].element_size() + sum(t.numel() * 4 for t in idx_host)
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    done = [torch.cuda.Event() for _ in range(2)]
+    ready = [torch.cuda.Event() for _ in range(2)]
+    read = [torch.cuda.Event() for _ in range(2)]
+    for b_ in range(2):
+        done[b_].record(compute)
+        read[b_].record(s_out)
+    for b_ in range(2):                                        # warm the second set's round
+        sets[b_][2].run(compute, copy)
+    e_steps = max(4, args.steps // 4)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     e0.record(compute)
-    for _ in range(e_steps):
-        with torch.cuda.stream(compute):
-            for l in range(w.layers):
-                for k_, v_ in host_in[l].items():
-                    small[l][k_].copy_(v_, non_blocking=True)
-        rnd.run(compute, copy)
-        with torch.cuda.stream(compute):
-            for l in range(w.layers):
-                host_out[l].copy_(outs[l], non_blocking=True)
+    s_in.wait_stream(compute)
+    for i in range(e_steps):
+        b_ = i % 2
+        dev_in, dev_out, rd, host_out = sets[b_]
+        s_in.wait_event(done[b_])                               # this set's inputs are free again
+        with torch.cuda.stream(s_in):
+            dev_in.copy_(host_in, non_blocking=True)
+        ready[b_].record(s_in)
+        compute.wait_event(ready[b_])
+        compute.wait_event(read[b_])                            # its previous outputs were read back
+        rd.run(compute, copy)
+        done[b_].record(compute)
+        s_out.wait_event(done[b_])
+        with torch.cuda.stream(s_out):
+            host_out.copy_(dev_out, non_blocking=True)
+        read[b_].record(s_out)
+    compute.wait_stream(s_out)
     e1.record(compute)
     torch.cuda.synchronize()
     barrier()
     e2e_ms = e0.elapsed_time(e1) / e_steps
+    assert torch.equal(sets[(e_steps - 1) % 2][3][0].cuda(), sets[(e_steps - 1) % 2][1][0])
 
     # ---- max over ranks
     ms_step, e2e_ms, route_ms, route_ms_live = max_over_ranks([ms_step, e2e_ms, route_ms, route_ms_live], "cuda")
@@ -741,7 +792,9 @@ def main():
                          "peak_kind": f"{peak_kind} (copy bandwidth)"},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "ms_per_step": e2e_ms},
+                    "ms_per_step": e2e_ms,
+                    "how": "public API with pinned host buffers; double-buffered: each step's H2D and D2H on their "
+                           "own streams overlap the neighbouring steps' compute, all inside the timed region"},
             # per layer: prepass, router, top-k, fetch kernel (mode 1) or memory lengths (mode 0),
             # attention; per step: one fused append for every layer
             "gpu_launches": (5 * w.layers + (w.layers + 23) // 24) * args.steps,

@@ -533,11 +533,22 @@ __global__ void __launch_bounds__(kPoolBwdThreads) pool_bwd_kernel(const PoolBwd
                 // the chunk's raw mean router key (this thread's 4 elements), then per head
                 // (g - k_hat (k_hat . g)) / |k| with k_hat = mean / |mean|
                 float4 mu = zero;
-                if (active)
-                    for (int64_t t = t0; t < t1; ++t) {
+                if (active) {
+                    int64_t t = t0;
+                    for (; t + 4 <= t1; t += 4) {                // four loads in flight, added in token order
+                        float4 x[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) x[u] = load4(a.kr, (t + u) * E + e0, a.kr_bf16);
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            mu.x += x[u].x; mu.y += x[u].y; mu.z += x[u].z; mu.w += x[u].w;
+                        }
+                    }
+                    for (; t < t1; ++t) {
                         const float4 x = load4(a.kr, t * E + e0, a.kr_bf16);
                         mu.x += x.x; mu.y += x.y; mu.z += x.z; mu.w += x.w;
                     }
+                }
                 mu = scale4(mu, inv_n);
                 float ss = mu.x * mu.x + mu.y * mu.y + mu.z * mu.z + mu.w * mu.w;
                 float dg = mu.x * g.x + mu.y * g.y + mu.z * g.z + mu.w * g.w;
