@@ -542,6 +542,10 @@ size_t split_ws_bytes(int n_split, int n_q, int T, int hq) {
 }  // namespace
 }  // namespace msa
 
+namespace msa {
+int attn_impl_setting() { return g_attn_impl.load(); }
+}  // namespace msa
+
 using namespace msa;
 
 extern "C" {

@@ -67,34 +67,12 @@ struct AttnTcArgs {
     float2* part_ml;
     int* err;
     int use_tma;           // memory tiles by TMA from tm_mem (otherwise every tile by cp.async)
+    int use_tma_loc;       // local-key tiles by TMA from tm_lk / tm_lv
 };
 
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
-            dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
-        : "memory");
-}
-
-__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, bool valid) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0) : "memory");
-}
-
-// Offset of 16-byte chunk c (0..15 over d = 128) of row r in a tile stored as two 64-element halves
-// of [rows][128 B] with the 128-byte swizzle (chunk index XOR row % 8).
-__device__ __forceinline__ uint32_t swz(int r, int c, int half_bytes) {
-    return (uint32_t)((c >> 3) * half_bytes + r * 128 + (((c & 7) ^ (r & 7)) << 4));
-}
-
-// MN-major operand in the 128-byte swizzle: 8 rows along K at 128 B, 8-row groups 1024 B apart
-// (stride byte offset), 64-element MN atoms `lbo` bytes apart (leading byte offset).
-__device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t saddr, uint32_t lbo) {
-    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(lbo >> 4) << 16) | ((uint64_t)(1024 >> 4) << 32) |
-           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ CUtensorMap tm_mem,
+                                                              const __grid_constant__ CUtensorMap tm_lk,
+                                                              const __grid_constant__ CUtensorMap tm_lv,
                                                               const AttnTcArgs a) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = a.G;
@@ -215,6 +193,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             const uint32_t stage = smem_u32(sKV + st * kStageBytes);
             const uint32_t full = smem_u32(&kv_full[st]);
             const int kb = k_begin + j * kKeys;
+            const bool loc_tile = a.use_tma_loc && kb >= mem_len && kb + kKeys <= k_end;
+            if (loc_tile) {                       // 64 local keys: K and V halves from the local caches
+                if (lane == 0) {
+                    mbar_expect_tx(full, (uint32_t)kStageBytes);
+                    const int z = qi * a.L_max + (kb - mem_len);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        tma_load_3d(stage + h * kHalfKV, &tm_lk, h * 64, g, z, full);
+                        tma_load_3d(stage + 2 * kHalfKV + h * kHalfKV, &tm_lv, h * 64, g, z, full);
+                    }
+                }
+                tma_phase[st] = (j / kStages) & 1;
+                continue;
+            }
             if (a.use_tma && kb + kKeys <= mem_len) {
                 if (lane == 0) {
                     mbar_expect_tx(full, (uint32_t)kStageBytes);
@@ -482,8 +474,19 @@ msa_status launch_attn_tc(const void* q, const void* mem_kv, const int32_t* mem_
         MSA_RETURN_IF(make_tensor_map_bf16(&tm, mem_kv, 3, dims, strides, box));
         a.use_tma = 1;
     }
+    // local caches [n_q * L_max][hkv][d]: dims (d, head, row), box (64, 1, 64)
+    CUtensorMap tlk{}, tlv{};
+    a.use_tma_loc = 0;
+    if (L_max >= kKeys && L > 0 && local_k && local_v) {
+        const uint64_t dims[3] = {(uint64_t)kD, (uint64_t)hkv, (uint64_t)n_q * L_max};
+        const uint64_t strides[2] = {(uint64_t)kD * 2, (uint64_t)hkv * kD * 2};
+        const uint32_t box[3] = {64, 1, (uint32_t)kKeys};
+        MSA_RETURN_IF(make_tensor_map_bf16(&tlk, local_k, 3, dims, strides, box));
+        MSA_RETURN_IF(make_tensor_map_bf16(&tlv, local_v, 3, dims, strides, box));
+        a.use_tma_loc = 1;
+    }
     const int row_blocks = (T * a.G + kRows - 1) / kRows;
-    attn_tc_kernel<<<dim3(row_blocks * n_split, hkv, n_q), kThreads, kSmemBytes, s>>>(tm, a);
+    attn_tc_kernel<<<dim3(row_blocks * n_split, hkv, n_q), kThreads, kSmemBytes, s>>>(tm, tlk, tlv, a);
     MSA_LAUNCH_CHECK();
     return MSA_OK;
 }

@@ -402,6 +402,7 @@ size_t bwd_ws_bytes(int n_q, int T, int hq, int hkv, int max_mem, int L) {
     return dvec + align_up((size_t)r * n_q * key_pad * 2 * hkv * kD * sizeof(float), 256);
 }
 
+
 template <int G>
 msa_status launch_attn_bwd_g(const BwdArgs& a, int n_q, cudaStream_t s) {
     const int key_tiles = (a.max_mem + a.L + kTile - 1) / kTile;
@@ -415,6 +416,14 @@ msa_status launch_attn_bwd_g(const BwdArgs& a, int n_q, cudaStream_t s) {
             attn_bwd_dkdv_reduce_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, s>>>(a, n_q);
             MSA_LAUNCH_CHECK();
         }
+    }
+    if (attn_impl_setting() == 0) {   // dQ on tcgen05
+        DqTcArgs d{};
+        d.q = a.q; d.mem_kv = a.mem_kv; d.mem_len = a.mem_len; d.max_mem = a.max_mem;
+        d.local_k = a.local_k; d.local_v = a.local_v; d.L_max = a.L_max; d.L = a.L; d.q_start = a.q_start;
+        d.T = a.T; d.hq = a.hq; d.hkv = a.hkv; d.G = G; d.scale = a.scale; d.scale_log2e = a.scale_log2e;
+        d.dout = a.dout; d.lse = a.lse; d.Dvec = a.Dvec; d.dq = a.dq; d.err = device_error_word();
+        return launch_attn_bwd_dq_tc(d, n_q, s);
     }
     attn_bwd_dq_kernel<G><<<dim3((a.T * G + kTile - 1) / kTile, a.hkv, n_q), 128, 0, s>>>(a);
     MSA_LAUNCH_CHECK();

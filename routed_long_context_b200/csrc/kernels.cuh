@@ -12,6 +12,30 @@ namespace msa {
 msa_status make_tensor_map_bf16(CUtensorMap* map, const void* ptr, int rank, const uint64_t* dims,
                                 const uint64_t* strides, const uint32_t* box);
 
+// The bf16 attention kernel choice of msa_attn_set_impl (0 = default: tcgen05 where it applies).
+int attn_impl_setting();
+
+// dQ of the attention backward on tcgen05 (bf16, d = 128): the forward's operands, dout, its
+// log-sum-exp (natural log) and D = rowsum(dO * O); dq fp32 [n_q][T][hq][d] is overwritten.
+struct DqTcArgs {
+    const __nv_bfloat16* q;
+    const __nv_bfloat16* mem_kv;
+    const int32_t* mem_len;
+    int max_mem;
+    const __nv_bfloat16* local_k;
+    const __nv_bfloat16* local_v;
+    int L_max, L, q_start, T, hq, hkv, G;
+    float scale, scale_log2e;
+    const __nv_bfloat16* dout;
+    const float* lse;
+    const float* Dvec;
+    float* dq;
+    int* err;
+    int use_tma;
+    int use_tma_loc;
+};
+msa_status launch_attn_bwd_dq_tc(DqTcArgs a, int n_q, cudaStream_t s);
+
 // Rotates rows of [*, heads, d] vectors. Row r of the launch belongs to segment s at offset u:
 //   uniform_len > 0: s = r / uniform_len, u = r % uniform_len,
 //                    input row s*in_stride + u, output row s*out_stride + out_off + u;

@@ -41,10 +41,12 @@ def _rel(got, ref):
 ATTN_BWD_TOL = 1e-2
 
 
+@pytest.mark.parametrize("impl", [0, 2])
 @pytest.mark.parametrize("hq,hkv", [(32, 8), (8, 8), (32, 4)])
 @pytest.mark.parametrize("T,max_mem,mem_lens,q_start", [(13, 40, (0, 5, 37), 7), (64, 140, (130, 64, 1), 0),
                                                         (100, 300, (256, 300, 77), 20)])
-def test_attention_backward_matches_oracle(m, hq, hkv, T, max_mem, mem_lens, q_start):
+def test_attention_backward_matches_oracle(m, impl, hq, hkv, T, max_mem, mem_lens, q_start):
+    """impl 0: tcgen05 (forward split and dQ), impl 2: mma.sync throughout."""
     n_q, d, dt = 3, 128, "bf16"
     L = q_start + T
     q = _gen(1, (n_q, T, hq, d), dt)
@@ -54,8 +56,12 @@ def test_attention_backward_matches_oracle(m, hq, hkv, T, max_mem, mem_lens, q_s
     mem_len = torch.from_numpy(np.array(mem_lens, dtype=np.int32)).cuda()
     qd, memd, lkd, lvd, dod = (upload(x, dt) for x in (q, mem, lk, lv, dout))
     lse = torch.empty((n_q, T, hq), dtype=torch.float32, device="cuda")
-    out = m.msa_sparse_attn_split(qd, memd, mem_len, lkd, lvd, L, q_start, lse=lse)
-    dq, dmem, dlk, dlv = m.msa_sparse_attn_backward(qd, memd, mem_len, lkd, lvd, L, q_start, out, dod, lse)
+    m.attn_set_impl(impl)
+    try:
+        out = m.msa_sparse_attn_split(qd, memd, mem_len, lkd, lvd, L, q_start, lse=lse)
+        dq, dmem, dlk, dlv = m.msa_sparse_attn_backward(qd, memd, mem_len, lkd, lvd, L, q_start, out, dod, lse)
+    finally:
+        m.attn_set_impl(0)
     assert m.device_status() == 0
     scale = 1 / np.sqrt(d)
     for qi in range(n_q):
