@@ -273,12 +273,14 @@ msa_status msa_attn_set_impl(int impl);
 
 /* Sparse attention over long memories (the token-level fine stage, thousands of memory rows per
  * query): the same arguments, layout and result as msa_sparse_attn, computed with the keys of
- * every (64-row block, kv head, query) split into n_split contiguous ranges of 64-key tiles that
- * run as separate blocks (tcgen05: one CTA per 128 (token, head) rows, S and O accumulated in
- * TMEM; see msa_attn_set_impl). Each writes its unnormalised output and (running max, sum) in
- * fp32 to the workspace; a second kernel merges the ranges' softmax statistics and writes out.
- * n_split is chosen from the sizes so that the grid fits one wave of three blocks per SM (148
- * SMs), at least four tiles per range. bf16 only (tensor cores); fp32 returns MSA_ERR_UNSUPPORTED.
+ * every row block (of kv head g and query q) split into n_split contiguous ranges of 64-key tiles
+ * that run as separate blocks. Default (msa_attn_set_impl(0)): tcgen05 tensor cores, one CTA of
+ * 192 threads per 128 (token, head) rows and key range, S and O accumulated in TMEM, K/V tiles of
+ * memory rows and of local keys loaded by TMA; n_split sized for one wave of one CTA per SM (148
+ * SMs). impl 2: mma.sync, 64-row blocks, one wave of three blocks per SM. Ranges hold at least
+ * four tiles. Each range writes its unnormalised output and (running max, sum) in fp32 to the
+ * workspace; a second kernel merges the ranges' softmax statistics and writes out.
+ * bf16 only (tensor cores); fp32 returns MSA_ERR_UNSUPPORTED.
  * lse: optional device float [n_q][T][hq]: ln sum_j exp(scale * q . k_j) over the row's visible
  * keys (-inf for a row without one), what msa_sparse_attn_backward needs from the forward pass.
  * ws: device, msa_sparse_attn_split_workspace_size bytes, 16-byte aligned. */

@@ -127,3 +127,31 @@ def test_interleave_rejects_local_cache_overflow(lib):
     assert b"overflow" in lib.msa_last_error()
     a.L_prev = 56
     assert lib.msa_interleave_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0 and n.value > 0
+
+
+def test_new_entry_points_validate_on_the_host(lib):
+    """Fine stage, Memory Parallel merge and backward calls reject bad arguments before any launch."""
+    P = ctypes.c_void_p(256)
+    # token bank: odd head_dim
+    assert lib.msa_pack_tokens(P, P, 1, 10, 8, 127, P, 2, P, 64, P, None) != 0
+    # merge: too many shards, k out of range, shard offsets decreasing
+    off = np.array([0, 5, 3], dtype=np.int64)
+    assert lib.msa_topk_merge(P, P, 16, 65, 1, 4, off.ctypes.data, 4, P, P, None) == 1
+    good = np.array([0, 5, 9], dtype=np.int64)
+    assert lib.msa_topk_merge(P, P, 16, 2, 1, 4, good.ctypes.data, 65, P, P, None) == 1
+    assert lib.msa_topk_merge(P, P, 16, 2, 1, 4, off.ctypes.data, 4, P, P, None) == 1
+    assert b"decrease" in lib.msa_last_error()
+    # split attention and the backward are bf16 only
+    assert lib.msa_sparse_attn_split(P, P, P, 8, P, P, 8, 8, 0, 1, 4, 32, 8, 128, 0.1, P, None, 0, P, 1 << 20,
+                                     None) == 2
+    assert lib.msa_sparse_attn_backward(P, P, P, 8, P, P, 8, 8, 0, 1, 4, 32, 8, 128, 0.1, P, P, P, 0, P, P, P, P,
+                                        P, 1 << 20, None) == 2
+    # aux loss: tau must be positive; pooling backward: nothing to do
+    assert lib.msa_router_aux_loss(P, 1, 10, P, 2, 0.0, None, P, None) == 1
+    assert lib.msa_pool_chunks_backward(None, None, None, 0, 10, 8, 8, 128, P, P, P, 2, 4, 4, 1, P, 64, 1, P, P, P,
+                                        None) == 1
+    # workspace sizes are queries only
+    n = ctypes.c_size_t(0)
+    assert lib.msa_sparse_attn_split_workspace_size(1, 64, 32, 8, 8064, 64, ctypes.byref(n)) == 0 and n.value > 0
+    assert lib.msa_sparse_attn_backward_workspace_size(1, 512, 32, 8, 128, 512, ctypes.byref(n)) == 0
+    assert lib.msa_route_backward_workspace_size(512, 1, 512, 8, 128, ctypes.byref(n)) == 0 and n.value > 0
