@@ -41,3 +41,48 @@ def test_router_wait_timeout_is_reported_and_context_survives():
     ref, _ = O.route(index, lay.doc_chunk_off_host, qr)
     assert np.abs(ds.float().cpu().numpy() - ref).max() <= 2e-3
     assert m.device_status() == 0
+
+
+def test_host_wait_deadline_reports_timeout_and_the_next_round_is_correct():
+    """A round whose host-side wait (fetch mode 0) cannot be met returns MSA_ERR_TIMEOUT instead of
+    blocking: the router is made to withhold its tiles (bounded, about 2 s), the round is given a
+    deadline of 0. After the stalled launch has given up, the next round selects the planted
+    documents and reports no device error."""
+    import routed_long_context_b200 as m
+    from msa_inputs import workloads
+    from msa_inputs.device import memory_tensor, small_tensors
+    from routed_long_context_b200 import _lib
+    from routed_long_context_b200.bank import BankLayout, index_from_prepooled
+
+    w = workloads.mem_100m(layers=1, n_host_banks=1, n_docs=2000)
+    lay = BankLayout(w.doc_chunks)
+    index = index_from_prepooled(lay, memory_tensor(w, 0, "krbar"))
+    dev = memory_tensor(w, 0, "bank")
+    bank = torch.empty(dev.shape, dtype=dev.dtype, pin_memory=True)
+    bank.copy_(dev)
+    sm = small_tensors(w, 0)
+    cs = m.rope_table(4096, w.d, w.rope_base)
+    local = [torch.zeros((1, w.T0, w.hkv, w.d), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    out = torch.empty((1, w.T0, w.hq, w.d), dtype=torch.bfloat16, device="cuda")
+    idx_host = torch.empty((1, w.k), dtype=torch.int32, pin_memory=True)
+    layer = dict(kr_index=index, host_bank=bank, qr=sm["qr"], q_new=sm["q"], k_new=sm["k_new"], v_new=sm["v_new"],
+                 local_k=local[0], local_v=local[1], out=out, topk_idx_host=idx_host)
+    rnd = m.InterleaveRound([layer], n_chunks=lay.n_chunks, n_docs=lay.n_docs, doc_chunk_off=lay.doc_chunk_off,
+                            doc_chunk_off_host=lay.doc_chunk_off_host, chunk_doc=lay.chunk_doc, n_q=1, H=w.H, d=w.d,
+                            hq=w.hq, hkv=w.hkv, k=w.k, L_prev=0, T_new=w.T0, new_q_stride=w.T0, L_max=w.T0,
+                            max_mem=w.max_mem, cos_sin=cs, fetch_mode=0)
+    compute, copy = torch.cuda.Stream(), torch.cuda.Stream()
+    assert m.device_status() == 0
+    _lib.check(_lib.lib.msa_route_inject_stall(1), "inject")
+    try:
+        with pytest.raises(m.MSAError) as err:
+            rnd.run(compute, copy, timeout_us=0)
+        assert err.value.status == _lib.MSA_ERR_TIMEOUT
+    finally:
+        _lib.check(_lib.lib.msa_route_inject_stall(0), "inject")
+    torch.cuda.synchronize()                   # the stalled router returns after its bounded waits
+    assert m.device_status() == 2              # MSA_DEV_WAIT_TIMEOUT, now cleared
+    rnd.run(compute, copy)
+    torch.cuda.synchronize()
+    assert m.device_status() == 0
+    assert set(w.expected(0, 0, 0)) <= set(idx_host[0].tolist())

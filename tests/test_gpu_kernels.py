@@ -413,3 +413,54 @@ def test_growable_bank_append_equals_full_encode_bitwise(m, dtype):
     ds = m.msa_route_scores(bank.index[:bank.n_chunks], bank.layout.chunk_doc, bank.layout.n_docs, upload(qr, dtype))
     assert int(torch.argmax(ds[1])) == d_plant
     _status(m)
+
+
+# -------------------------------------------------------------------------------------- output bounds
+def _canaried(shape, dtype, pattern):
+    """A tensor of `shape` that is the head of a larger buffer whose 4 KB tail holds `pattern` bits."""
+    n = int(np.prod(shape))
+    el = torch.empty((), dtype=dtype).element_size()
+    extra = 4096 // el
+    int_dt = {2: torch.int16, 4: torch.int32}[el]
+    buf = torch.full((n + extra,), pattern, dtype=int_dt, device="cuda").view(dtype)
+    return buf[:n].view(shape), buf, n
+
+
+def _tail_intact(buf, n, pattern):
+    int_dt = {2: torch.int16, 4: torch.int32}[buf.element_size()]
+    return bool((buf[n:].view(int_dt) == pattern).all())
+
+
+def test_new_kernels_write_nothing_past_their_outputs(m):
+    """Canary words after the outputs of the token bank, the split attention (and its log-sum-exp),
+    the attention backward, the Memory Parallel merge and the pooling backward stay untouched."""
+    bf, f32 = torch.bfloat16, torch.float32
+    n_q, T, hq, hkv, d, L = 2, 24, 32, 8, 128, 30
+    mem_lens = np.array([700, 0], dtype=np.int32)
+    max_mem = 704
+    q = upload(_gen(120, (n_q, T, hq, d), "bf16"), "bf16")
+    mem = upload(_gen(121, (n_q, max_mem, 2, hkv, d), "bf16"), "bf16")
+    lk, lv = upload(_gen(122, (n_q, L, hkv, d), "bf16"), "bf16"), upload(_gen(123, (n_q, L, hkv, d), "bf16"), "bf16")
+    ml = torch.from_numpy(mem_lens).cuda()
+    out, ob, on = _canaried((n_q, T, hq, d), bf, 0x3C5A)
+    lse, lb, ln_ = _canaried((n_q, T, hq), f32, 0x7FC0DEAD)
+    m.msa_sparse_attn_split(q, mem, ml, lk, lv, L, 6, out=out, lse=lse)
+    grads = [_canaried(s_, f32, 0x7FC0BEEF) for s_ in ((n_q, T, hq, d), (n_q, max_mem, 2, hkv, d), (n_q, L, hkv, d),
+                                                        (n_q, L, hkv, d))]
+    m.msa_sparse_attn_backward(q, mem, ml, lk, lv, L, 6, out, q, lse, grads=tuple(g_[0] for g_ in grads))
+    off = np.array([0, 300, 300, 555, 1000], dtype=np.int64)
+    kt = upload(_gen(124, (1000, hkv, d), "bf16"), "bf16")
+    bank, bb, bn = _canaried((1000, 2, hkv, d), bf, 0x3C5A)
+    m.msa_pack_tokens(kt, kt, torch.from_numpy(off).cuda(), m.rope_table(1024, d, 1e6), bank=bank)
+    cand = torch.rand((3, 2, 16), device="cuda")
+    cidx = torch.randint(0, 50, (3, 2, 16), dtype=torch.int32, device="cuda")
+    midx, mb, mn = _canaried((2, 16), torch.int32, 0x5A5A5A5A)
+    msc, sb, sn = _canaried((2, 16), f32, 0x7FC0DEAD)
+    m.msa_topk_merge(cand, cidx, np.array([0, 50, 100, 150]), 16, idx=midx, score=msc)
+    torch.cuda.synchronize()
+    _status(m)
+    assert _tail_intact(ob, on, 0x3C5A) and _tail_intact(lb, ln_, 0x7FC0DEAD)
+    for g_, b_, n_ in grads:
+        assert _tail_intact(b_, n_, 0x7FC0BEEF)
+    assert _tail_intact(bb, bn, 0x3C5A)
+    assert _tail_intact(mb, mn, 0x5A5A5A5A) and _tail_intact(sb, sn, 0x7FC0DEAD)
