@@ -115,12 +115,29 @@ msa_status msa_rope_doc(const void* x, void* out, msa_dtype dt, int64_t n_tok, i
  *     head vector is divided by its L2 norm (a zero vector stays zero): the "index form" that
  *     msa_route_scores reads. Pre-pooled router keys are put into index form by calling this
  *     with chunk = 1, one document per chunk run, k = v = NULL.
- * Arithmetic is fp32; outputs are rounded once to out_dt. */
+ * Arithmetic is fp32 (each element summed in token order); outputs are rounded once to out_dt.
+ * Two kernels give the same bits: register streaming (one block per chunk and tensor part) and
+ * bulk copy (token rows, and for rotated keys their RoPE table rows, staged in shared memory by
+ * cp.async.bulk into a ring of pipeline stages fed by one producer lane; every wait bounded,
+ * MSA_DEV_WAIT_TIMEOUT on expiry). By default the bulk-copy kernel runs when chunks x parts is at
+ * most two waves of the register kernel's resident blocks, the register kernel otherwise; layouts
+ * whose token row exceeds a stage always use the register kernel. */
 msa_status msa_pool_chunks(const void* k, const void* v, const void* kr, msa_dtype in_dt, int64_t n_tok, int hkv,
                            int hr, int d, const int64_t* doc_tok_off, const int64_t* doc_chunk_off,
                            const int32_t* chunk_doc, int64_t n_docs, int64_t n_chunks, int chunk, int fuse_doc_rope,
                            const float* cos_sin, int64_t max_pos, void* kvbar, void* kr_index, msa_dtype out_dt,
                            int normalize_router, void* stream);
+
+/* Selects the pooling kernel: 0 = by size (default), 1 = register streaming, 2 = bulk copy where
+ * the layout allows. Process-wide. */
+msa_status msa_pool_set_impl(int impl);
+
+/* Tuning knob of the bulk-copy pooling kernel: n_stages pipeline stages (2..16) of stage_bytes
+ * bytes (a multiple of 1024 in [2048, 65536]), each filled by bulk copies of copy_bytes (a multiple
+ * of 16, rounded down to whole token rows, at least one row); 0 keeps the default (3 stages of
+ * 32 KiB, one copy per stage). The ring (n_stages * stage_bytes) must stay within 200 KiB.
+ * Process-wide. */
+msa_status msa_pool_set_pipeline(int n_stages, int stage_bytes, int copy_bytes);
 
 /* Token-level memory bank for the fine stage (coarse-to-fine reading of [P5] 四個核心機制 §1:
  * after routing on the compressed chunks, attention may read the selected documents' own tokens;

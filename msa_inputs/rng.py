@@ -144,6 +144,9 @@ def uniform_int(seed: int, tid: int, n: int, hi: int) -> np.ndarray:
 def distinct_ints(seed: int, tid: int, n: int, hi: int, exclude=()) -> np.ndarray:
     """n distinct integers in [0, hi), not in ``exclude``, taken in draw order."""
     got, seen, start = [], set(int(e) for e in exclude), 0
+    free = hi - len({e for e in seen if 0 <= e < hi})
+    if n > free:
+        raise ValueError(f"distinct_ints: {n} distinct values asked from {free} available in [0, {hi})")
     while len(got) < n:
         d = draw_u64(seed, tid, start, 4 * n + 16)
         start += len(d)

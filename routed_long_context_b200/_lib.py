@@ -43,6 +43,8 @@ SIGNATURES = {
     "msa_rope_doc": (i32, [vp, vp, i32, i64, ctypes.c_int, ctypes.c_int, vp, i64, i64, vp, i64, vp]),
     "msa_pool_chunks": (i32, [vp, vp, vp, i32, i64, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp, vp, i64, i64,
                               ctypes.c_int, ctypes.c_int, vp, i64, vp, vp, i32, ctypes.c_int, vp]),
+    "msa_pool_set_impl": (i32, [ctypes.c_int]),
+    "msa_pool_set_pipeline": (i32, [ctypes.c_int, ctypes.c_int, ctypes.c_int]),
     "msa_route_scores": (i32, [vp, i32, i64, vp, i64, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp,
                                vp, vp, sz, vp]),
     "msa_route_workspace_size": (i32, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, i32,

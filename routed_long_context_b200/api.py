@@ -118,6 +118,16 @@ def attn_set_impl(impl: int) -> None:
     check(lib.msa_attn_set_impl(impl), "msa_attn_set_impl")
 
 
+def pool_set_impl(impl: int) -> None:
+    """Chunk-mean pooling: 0 = by size (default), 1 = register streaming, 2 = bulk copy where the layout allows."""
+    check(lib.msa_pool_set_impl(impl), "msa_pool_set_impl")
+
+
+def pool_set_pipeline(n_stages: int = 0, stage_bytes: int = 0, copy_bytes: int = 0) -> None:
+    """Tuning knob of the bulk-copy pooling kernel (zeros = default: 3 stages of 32 KiB, one copy per stage)."""
+    check(lib.msa_pool_set_pipeline(n_stages, stage_bytes, copy_bytes), "msa_pool_set_pipeline")
+
+
 def route_set_max_stages(n: int) -> None:
     """Tuning knob: cap on the router's pipeline stages (0 = default budget)."""
     check(lib.msa_route_set_max_stages(n), "msa_route_set_max_stages")

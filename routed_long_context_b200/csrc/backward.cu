@@ -483,8 +483,9 @@ struct PoolBwdArgs {
     float* dk;
     float* dv;
     float* dkr;
-    int n_parts;
-    int parts[3];
+    int64_t n_kr_items;      // router-key chunks (0 without dkr_index)
+    int64_t n_kv_items;      // (chunk, K or V, token slice) items (0 without dkvbar)
+    int kv_slices, slice_tok;
     int* err;
 };
 
@@ -505,23 +506,39 @@ __device__ __forceinline__ float4 load4(const void* p, int64_t i, int bf16) {
 
 __device__ __forceinline__ float4 scale4(float4 v, float s) { return make_float4(v.x * s, v.y * s, v.z * s, v.w * s); }
 
-// Block per (chunk, tensor part); thread i owns elements 4i..4i+3 of a token row (rows of at most
-// 1024 elements, one head = d/4 consecutive lanes of a warp). The chunk's gradient is read once;
-// every token of the chunk then gets one 16-byte streaming store per thread.
+// Work items: first one per chunk of the router-key gradient (it reads the chunk's tokens again
+// for the normalisation's backward, so it keeps the whole chunk), then one per (chunk, K or V,
+// slice of kPoolBwdSliceTok tokens) — small, even items that the block scheduler spreads over
+// the SMs with a short tail. Thread i owns elements 4i..4i+3 of a token row (rows of at most 1024
+// elements, one head = d/4 consecutive lanes of a warp); every token gets one 16-byte streaming
+// store per thread.
 constexpr int kPoolBwdThreads = 256;
+constexpr int kPoolBwdSliceTok = 32;
 
 __global__ void __launch_bounds__(kPoolBwdThreads) pool_bwd_kernel(const PoolBwdArgs a) {
-    const int part = a.parts[blockIdx.x % a.n_parts];
-    const int64_t c_stride = gridDim.x / a.n_parts;
     const int d = a.d;
-    const int E = (part == 2 ? a.hr : a.hkv) * d;
     const int e0 = threadIdx.x * 4;
-    const bool active = e0 < E;
     const int ih = e0 % d;
     const bool first = ih < d / 2;
     const int hi = first ? ih : ih - d / 2;
     const int head_lanes = d / 4;
-    for (int64_t c = blockIdx.x / a.n_parts; c < a.n_chunks; c += c_stride) {
+    const int64_t total = a.n_kr_items + a.n_kv_items;
+    for (int64_t item = blockIdx.x; item < total; item += gridDim.x) {
+        int part, slice = 0;
+        int64_t c;
+        if (item < a.n_kr_items) {
+            part = 2;
+            c = item;
+        } else {
+            const int64_t j = item - a.n_kr_items;
+            const int64_t per_chunk = 2 * (int64_t)a.kv_slices;
+            c = j / per_chunk;
+            const int r = (int)(j - c * per_chunk);
+            part = r / a.kv_slices;
+            slice = r - part * a.kv_slices;
+        }
+        const int E = (part == 2 ? a.hr : a.hkv) * d;
+        const bool active = e0 < E;
         const int64_t doc = a.chunk_doc[c];
         if (doc < 0 || doc >= a.n_docs) {
             if (threadIdx.x == 0) record_device_error(a.err, MSA_DEV_BAD_INDEX);
@@ -530,7 +547,7 @@ __global__ void __launch_bounds__(kPoolBwdThreads) pool_bwd_kernel(const PoolBwd
         const int64_t doc_start = a.doc_tok_off[doc];
         const int64_t t0 = doc_start + (c - a.doc_chunk_off[doc]) * (int64_t)a.chunk;
         const int64_t t1 = min(t0 + (int64_t)a.chunk, a.doc_tok_off[doc + 1]);
-        if (t0 < doc_start || t0 >= t1 || t1 > a.n_tok) {
+        if (doc_start < 0 || t0 < doc_start || t0 >= t1 || t1 > a.n_tok) {
             if (threadIdx.x == 0) record_device_error(a.err, MSA_DEV_BAD_INDEX);
             continue;
         }
@@ -575,12 +592,15 @@ __global__ void __launch_bounds__(kPoolBwdThreads) pool_bwd_kernel(const PoolBwd
                 for (int64_t t = t0; t < t1; ++t) __stcs(reinterpret_cast<float4*>(a.dkr + t * E + e0), g);
             continue;
         }
+        const int64_t ta = t0 + (int64_t)slice * a.slice_tok;
+        if (ta >= t1) continue;
+        const int64_t tb = min(ta + (int64_t)a.slice_tok, t1);
         const float* grow = a.dkvbar + (c * 2 + part) * (int64_t)E;
         const float4 g = active ? scale4(*reinterpret_cast<const float4*>(grow + e0), inv_n) : zero;
         float* out = part == 0 ? a.dk : a.dv;
         if (part == 1 || !a.fuse_rope) {
             if (active)
-                for (int64_t t = t0; t < t1; ++t) __stcs(reinterpret_cast<float4*>(out + t * E + e0), g);
+                for (int64_t t = ta; t < tb; ++t) __stcs(reinterpret_cast<float4*>(out + t * E + e0), g);
             continue;
         }
         // keys: the transposed rotation of each token's position, R(-p):
@@ -589,7 +609,7 @@ __global__ void __launch_bounds__(kPoolBwdThreads) pool_bwd_kernel(const PoolBwd
                                          inv_n)
                                 : zero;
         const float sg = first ? 1.f : -1.f;
-        for (int64_t t = t0; t < t1; ++t) {
+        for (int64_t t = ta; t < tb; ++t) {
             const int64_t p = t - doc_start;
             float4 o = g;
             if (p < a.max_pos) {
@@ -923,7 +943,6 @@ msa_status msa_pool_chunks_backward(const float* dkvbar, const float* dkr_index,
     if (n_chunks == 0) return MSA_OK;
     MSA_REQUIRE(doc_tok_off && doc_chunk_off && chunk_doc, "msa_pool_chunks_backward: NULL offsets");
     PoolBwdArgs a{};
-    a.n_parts = 0;
     // one thread per 4 elements of a row, a head on d/4 lanes of one warp
     if (d % 8 != 0 || d / 4 > 32 || ((d / 4) & (d / 4 - 1)) != 0)
         return set_error(MSA_ERR_UNSUPPORTED, "msa_pool_chunks_backward: head_dim %d unsupported (8..128, d/4 a power of two)", d);
@@ -933,8 +952,6 @@ msa_status msa_pool_chunks_backward(const float* dkvbar, const float* dkr_index,
         MSA_REQUIRE(aligned16(dkvbar) && aligned16(dk) && aligned16(dv), "msa_pool_chunks_backward: unaligned K/V pointer");
         MSA_REQUIRE(!fuse_doc_rope || (cos_sin && max_pos > 0 && aligned16(cos_sin)),
                     "msa_pool_chunks_backward: RoPE needs a table");
-        a.parts[a.n_parts++] = 0;
-        a.parts[a.n_parts++] = 1;
     }
     if (dkr_index) {
         MSA_REQUIRE(hr > 0 && dkr && (size_t)hr * d <= 4 * kPoolBwdThreads,
@@ -942,7 +959,6 @@ msa_status msa_pool_chunks_backward(const float* dkvbar, const float* dkr_index,
         MSA_REQUIRE(aligned16(dkr_index) && aligned16(dkr), "msa_pool_chunks_backward: unaligned K^R pointer");
         MSA_REQUIRE(!normalize_router || (kr && dtype_ok(kr_dt) && aligned16(kr)),
                     "msa_pool_chunks_backward: the normalised index needs the token K^R");
-        a.parts[a.n_parts++] = 2;
     }
     a.dkvbar = dkvbar; a.dkr_index = dkr_index; a.kr = kr; a.kr_bf16 = kr_dt == MSA_BF16;
     a.hkv = hkv; a.hr = hr; a.d = d;
@@ -951,8 +967,13 @@ msa_status msa_pool_chunks_backward(const float* dkvbar, const float* dkr_index,
     a.fuse_rope = fuse_doc_rope; a.normalize = normalize_router;
     a.cs = reinterpret_cast<const float2*>(cos_sin); a.max_pos = max_pos;
     a.dk = dk; a.dv = dv; a.dkr = dkr; a.err = device_error_word();
-    const int64_t per_part = std::min<int64_t>(n_chunks, (int64_t)1 << 20);
-    pool_bwd_kernel<<<(unsigned)(per_part * a.n_parts), kPoolBwdThreads, 0, static_cast<cudaStream_t>(stream)>>>(a);
+    a.slice_tok = kPoolBwdSliceTok;
+    a.kv_slices = (chunk + kPoolBwdSliceTok - 1) / kPoolBwdSliceTok;
+    a.n_kr_items = dkr_index ? n_chunks : 0;
+    a.n_kv_items = dkvbar ? n_chunks * 2 * a.kv_slices : 0;
+    const int64_t items = a.n_kr_items + a.n_kv_items;
+    const unsigned grid = (unsigned)std::min<int64_t>(items, (int64_t)1 << 24);
+    pool_bwd_kernel<<<grid, kPoolBwdThreads, 0, static_cast<cudaStream_t>(stream)>>>(a);
     MSA_LAUNCH_CHECK();
     return MSA_OK;
 }

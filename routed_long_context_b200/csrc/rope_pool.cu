@@ -4,8 +4,12 @@
 // by d/VEC consecutive lanes of one warp, so the rotate-half partner of element i (i + d/2) sits
 // in lane ^ (d/2)/VEC and is fetched with one shuffle per 32-bit word. RoPE angles come from a
 // host-built fp64 -> fp32 table [max_pos][d/2] of (cos, sin).
+#include <atomic>
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.cuh"
+#include "tc.cuh"
 
 namespace msa {
 namespace {
@@ -81,6 +85,12 @@ struct PoolArgs {
     int hkv;
     int normalize;
     int* err;
+    // bulk-copy variant only
+    int rows_per_stage[3];   // token rows of each tensor part per pipeline stage
+    int rows_per_copy[3];    // token rows of each tensor part per bulk copy (a stage takes one or more)
+    int tab_bytes;           // bytes of one RoPE table row (d/2 cos/sin pairs), staged after rotated rows
+    int n_stages;
+    int stage_bytes;
 };
 
 template <typename TIn, typename TOut>
@@ -110,7 +120,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const PoolArgs a) {
         const int64_t t0 = doc_start + (c - a.doc_chunk_off[doc]) * (int64_t)a.chunk;
         const int64_t doc_end = a.doc_tok_off[doc + 1];
         const int64_t t1 = min(t0 + (int64_t)a.chunk, doc_end);
-        if (t0 < doc_start || t0 >= t1 || t1 > a.n_tok) {   // inconsistent metadata: skip, never read out of range
+        if (doc_start < 0 || t0 < doc_start || t0 >= t1 || t1 > a.n_tok) {   // inconsistent metadata: skip
             if (threadIdx.x == 0) record_device_error(a.err, MSA_DEV_BAD_INDEX);
             continue;
         }
@@ -197,6 +207,224 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const PoolArgs a) {
             }
         }
         (void)lane;
+    }
+}
+
+
+// ---------------------------------------------------------------------------------------------
+// Chunk-mean pooling with the token rows staged in shared memory by bulk copies.
+//
+// A chunk's rows of one tensor part are one contiguous run of HBM ([t0, t1) x H*d). The CTA walks
+// its (chunk, part) work items; one producer lane streams each item's run into a ring of
+// n_stages stages (stage_bytes each, whole rows) with cp.async.bulk, completing on the stage's
+// mbarrier; for rotated keys the RoPE table rows of the stage's positions (contiguous, since the
+// positions are) are copied into the stage behind the data rows. The consumer warps (one thread
+// per VEC elements of a row) read every row of the stage from shared memory, rotate K (partner
+// element and cos/sin from the same stage), accumulate in fp32 and release the stage. The copy queue never drains between a thread's load batches, so the
+// SM keeps its share of the HBM bandwidth in flight. Every wait is bounded: on expiry the CTA
+// records MSA_DEV_WAIT_TIMEOUT, leaves its loops and lets the copies it issued land before exiting.
+struct PoolItem {
+    int64_t c, doc_start, t0, t1;
+    int part;
+};
+
+__device__ __forceinline__ bool pool_item(const PoolArgs& a, int64_t item, PoolItem& it) {
+    it.c = item / a.n_parts;
+    it.part = a.parts[item % a.n_parts];
+    const int64_t doc = a.chunk_doc[it.c];
+    if (doc < 0 || doc >= a.n_docs) return false;
+    it.doc_start = a.doc_tok_off[doc];
+    it.t0 = it.doc_start + (it.c - a.doc_chunk_off[doc]) * (int64_t)a.chunk;
+    const int64_t doc_end = a.doc_tok_off[doc + 1];
+    it.t1 = min(it.t0 + (int64_t)a.chunk, doc_end);
+    return !(it.doc_start < 0 || it.t0 < it.doc_start || it.t0 >= it.t1 || it.t1 > a.n_tok);
+}
+
+constexpr int kBulkMaxConsumers = 256;
+
+template <typename TIn, typename TOut>
+__global__ void __launch_bounds__(kBulkMaxConsumers + 32) pool_bulk_kernel(const PoolArgs a) {
+    constexpr int VEC = 16 / sizeof(TIn);
+    extern __shared__ __align__(128) unsigned char pool_smem[];
+    const int S = a.n_stages;
+    unsigned char* ring = pool_smem;
+    uint64_t* full = reinterpret_cast<uint64_t*>(ring + (size_t)S * a.stage_bytes);
+    uint64_t* empty = full + S;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + S);
+    const int nc = (int)blockDim.x - 32;   // consumer threads; the last warp produces
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    if (tid == 0) {
+        for (int i = 0; i < S; ++i) {
+            mbar_init(smem_u32(full + i), 1);
+            mbar_init(smem_u32(empty + i), nc / 32);
+        }
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    __syncthreads();
+    const int64_t n_items = a.n_chunks * a.n_parts;
+    const int d = a.d;
+
+    // producer state, read again by the drain after the final barrier
+    int p_st = 0;
+    uint32_t p_ph = 0;
+    int64_t p_issued = 0;
+
+    if (tid >= nc) {
+        if (lane == 0) {
+            const uint64_t pol = policy_evict_first();
+            bool stop = false;
+            for (int64_t item = blockIdx.x; item < n_items && !stop; item += gridDim.x) {
+                PoolItem it;
+                if (!pool_item(a, item, it)) continue;
+                const int64_t E = (int64_t)a.heads[it.part] * d;
+                const TIn* src = static_cast<const TIn*>(a.src[it.part]);
+                const int R = a.rows_per_stage[it.part];
+                for (int64_t r0 = it.t0; r0 < it.t1; r0 += R) {
+                    const int64_t n = min((int64_t)R, it.t1 - r0);
+                    if (!mbar_wait(smem_u32(empty + p_st), p_ph ^ 1u, abort_flag)) {
+                        stop = true;
+                        break;
+                    }
+                    const int64_t row_bytes = E * (int64_t)sizeof(TIn);
+                    // rotated keys: the table rows of the stage's positions follow its R data rows
+                    int64_t n_tab = 0;
+                    if (it.part == 0 && a.fuse_rope) {
+                        n_tab = min(n, a.max_pos - (r0 - it.doc_start));
+                        if (n_tab < 0) n_tab = 0;
+                    }
+                    const uint32_t stage_addr = smem_u32(ring + (size_t)p_st * a.stage_bytes);
+                    mbar_expect_tx(smem_u32(full + p_st), (uint32_t)(n * row_bytes + n_tab * a.tab_bytes));
+                    const int64_t CR = a.rows_per_copy[it.part];
+                    for (int64_t cr = 0; cr < n; cr += CR) {
+                        const int64_t m = min(CR, n - cr);
+                        bulk_load_evict_first(stage_addr + (uint32_t)(cr * row_bytes), src + (r0 + cr) * E,
+                                              (uint32_t)(m * row_bytes), smem_u32(full + p_st), pol);
+                    }
+                    if (n_tab > 0)
+                        bulk_load_evict_first(stage_addr + (uint32_t)(R * row_bytes),
+                                              a.cs + (r0 - it.doc_start) * (int64_t)(d / 2),
+                                              (uint32_t)(n_tab * a.tab_bytes), smem_u32(full + p_st), pol);
+                    ++p_issued;
+                    if (++p_st == S) {
+                        p_st = 0;
+                        p_ph ^= 1u;
+                    }
+                }
+            }
+        }
+    } else {
+        int st = 0;
+        uint32_t ph = 0;
+        bool stop = false;
+        const int half_lanes = (d / 2) / VEC;
+        for (int64_t item = blockIdx.x; item < n_items && !stop; item += gridDim.x) {
+            PoolItem it;
+            if (!pool_item(a, item, it)) {
+                if (tid == 0) record_device_error(a.err, MSA_DEV_BAD_INDEX);
+                continue;
+            }
+            const int part = it.part;
+            const int E = a.heads[part] * d;
+            const int e0 = tid * VEC;
+            const bool active = e0 < E;
+            const int ih = e0 % d;
+            const bool first_half = ih < d / 2;
+            const int ci = first_half ? ih : ih - d / 2;
+            const int pe0 = first_half ? e0 + d / 2 : e0 - d / 2;   // rotate-half partner
+            const bool rope = (part == 0) && a.fuse_rope;
+            const int R = a.rows_per_stage[part];
+            const int row_bytes = E * (int)sizeof(TIn);
+            float acc[VEC];
+#pragma unroll
+            for (int j = 0; j < VEC; ++j) acc[j] = 0.f;
+
+            for (int64_t r0 = it.t0; r0 < it.t1; r0 += R) {
+                const int n = (int)min((int64_t)R, it.t1 - r0);
+                // every lane of the warp takes the same way out, so the shuffles below stay converged
+                if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(full + st), ph, abort_flag))) {
+                    stop = true;
+                    break;
+                }
+                const unsigned char* stage = ring + (size_t)st * a.stage_bytes;
+                if (active) {
+                    if (rope) {
+                        const unsigned char* tab = stage + R * row_bytes;
+#pragma unroll 2
+                        for (int r = 0; r < n; ++r) {
+                            const unsigned char* row = stage + r * row_bytes;
+                            float x[VEC], px[VEC];
+                            widen<TIn>(*reinterpret_cast<const uint4*>(row + e0 * (int)sizeof(TIn)), x);
+                            widen<TIn>(*reinterpret_cast<const uint4*>(row + pe0 * (int)sizeof(TIn)), px);
+                            const int64_t p = r0 + r - it.doc_start;
+                            if (p < a.max_pos)
+                                rotate<VEC>(x, px, reinterpret_cast<const float2*>(tab + r * a.tab_bytes), ci,
+                                            first_half);
+                            else
+                                record_device_error(a.err, MSA_DEV_ROPE_POSITION);
+#pragma unroll
+                            for (int j = 0; j < VEC; ++j) acc[j] += x[j];
+                        }
+                    } else {
+#pragma unroll 4
+                        for (int r = 0; r < n; ++r) {
+                            float x[VEC];
+                            widen<TIn>(*reinterpret_cast<const uint4*>(stage + r * row_bytes + e0 * (int)sizeof(TIn)),
+                                       x);
+#pragma unroll
+                            for (int j = 0; j < VEC; ++j) acc[j] += x[j];
+                        }
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(empty + st));
+                if (++st == S) {
+                    st = 0;
+                    ph ^= 1u;
+                }
+            }
+            if (stop) break;
+
+            const float inv_n = 1.0f / (float)(it.t1 - it.t0);
+            float mean[VEC];
+#pragma unroll
+            for (int j = 0; j < VEC; ++j) mean[j] = acc[j] * inv_n;
+            if (part == 2) {
+                if (a.normalize) {
+                    float ss = 0.f;
+#pragma unroll
+                    for (int j = 0; j < VEC; ++j) ss = fmaf(mean[j], mean[j], ss);
+                    for (int m = half_lanes; m >= 1; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+                    const float inv = ss > 0.f ? 1.0f / sqrtf(ss) : 0.f;
+#pragma unroll
+                    for (int j = 0; j < VEC; ++j) mean[j] *= inv;
+                }
+                if (active) store_f32<TOut, VEC>(static_cast<TOut*>(a.kr_index) + it.c * (int64_t)E + e0, mean);
+            } else if (active) {
+                TOut* dst = static_cast<TOut*>(a.kvbar) + (it.c * 2 + part) * (int64_t)a.hkv * d + e0;
+                store_f32<TOut, VEC>(dst, mean);
+            }
+        }
+    }
+    __syncwarp();
+    __syncthreads();
+    if (*abort_flag) {
+        if (tid == 0) record_device_error(a.err, MSA_DEV_WAIT_TIMEOUT);
+        if (tid == nc) {
+            // the last min(issued, S) stages hold the only copies that can still be in flight
+            const int64_t back = p_issued < S ? p_issued : S;
+            for (int64_t j = 1; j <= back; ++j) {
+                int s2 = p_st - (int)j;
+                uint32_t ph2 = p_ph;
+                if (s2 < 0) {
+                    s2 += S;
+                    ph2 ^= 1u;
+                }
+                mbar_wait_drain(smem_u32(full + s2), ph2);
+            }
+        }
     }
 }
 
@@ -378,6 +606,71 @@ msa_status launch_pack_tokens(const PackArgs& a, msa_dtype dt, cudaStream_t s) {
     return MSA_OK;
 }
 
+namespace {
+
+std::atomic<int> g_pool_impl{0};          // 0: by size, 1: register streaming, 2: bulk copy where the layout allows
+std::atomic<int> g_pool_stages{0};        // 0: default
+std::atomic<int> g_pool_stage_bytes{0};   // 0: default
+std::atomic<int> g_pool_copy_bytes{0};    // 0: one bulk copy per stage
+constexpr int kBulkStagesDefault = 3;
+constexpr int kBulkStageBytesDefault = 32768;
+
+// Launches the bulk-copy pooling kernel when every part's row fits a stage and a row needs at most
+// kBulkMaxConsumers threads; *launched tells whether it did.
+template <typename TIn, typename TOut>
+msa_status launch_pool_bulk(PoolArgs a, cudaStream_t s, bool* launched) {
+    constexpr int VEC = 16 / sizeof(TIn);
+    *launched = false;
+    a.tab_bytes = (a.d / 2) * (int)sizeof(float2);
+    const int S = g_pool_stages.load() > 0 ? g_pool_stages.load() : kBulkStagesDefault;
+    const int SB = g_pool_stage_bytes.load() > 0 ? g_pool_stage_bytes.load() : kBulkStageBytesDefault;
+    int max_e = 0;
+    for (int i = 0; i < a.n_parts; ++i) {
+        const int part = a.parts[i];
+        const int E = a.heads[part] * a.d;
+        const int row_bytes = E * (int)sizeof(TIn);
+        // rotated keys carry their table rows in the stage
+        const int per_row = row_bytes + ((part == 0 && a.fuse_rope) ? a.tab_bytes : 0);
+        if (per_row > SB || row_bytes % 16 != 0 || a.tab_bytes % 16 != 0) return MSA_OK;
+        a.rows_per_stage[part] = SB / per_row;
+        const int CB = g_pool_copy_bytes.load();
+        a.rows_per_copy[part] = CB > 0 ? (CB / row_bytes > 0 ? CB / row_bytes : 1) : a.rows_per_stage[part];
+        max_e = E > max_e ? E : max_e;
+    }
+    const int nc = (max_e / VEC + 31) / 32 * 32;
+    if (nc > kBulkMaxConsumers) return MSA_OK;
+    a.n_stages = S;
+    a.stage_bytes = SB;
+    const size_t smem = (size_t)S * SB + 2 * (size_t)S * sizeof(uint64_t) + 16;
+    static std::mutex mu;
+    static size_t opted[64] = {0};
+    int dev = 0;
+    MSA_CUDA_TRY(cudaGetDevice(&dev));
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        if (dev < 0 || dev >= 64 || opted[dev] < smem) {
+            MSA_CUDA_TRY(cudaFuncSetAttribute(pool_bulk_kernel<TIn, TOut>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              (int)smem));
+            // ask for the whole unified L1 as shared memory, so the occupancy computed below is reached
+            MSA_CUDA_TRY(cudaFuncSetAttribute(pool_bulk_kernel<TIn, TOut>,
+                                              cudaFuncAttributePreferredSharedMemoryCarveout, 100));
+            if (dev >= 0 && dev < 64) opted[dev] = smem;
+        }
+    }
+    int occ = 0;
+    MSA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, pool_bulk_kernel<TIn, TOut>, nc + 32, smem));
+    if (occ < 1) return MSA_OK;
+    const int64_t n_items = a.n_chunks * a.n_parts;
+    const int64_t cap = (int64_t)sm_count() * occ;
+    const unsigned grid = (unsigned)(n_items < cap ? n_items : cap);
+    pool_bulk_kernel<TIn, TOut><<<grid, nc + 32, smem, s>>>(a);
+    MSA_LAUNCH_CHECK();
+    *launched = true;
+    return MSA_OK;
+}
+
+}  // namespace
+
 bool rope_layout_ok(msa_dtype dt, int d) {
     return dt == MSA_BF16 ? vec_layout_ok<__nv_bfloat16>(d) : vec_layout_ok<float>(d);
 }
@@ -466,10 +759,37 @@ msa_status msa_pool_chunks(const void* k, const void* v, const void* kr, msa_dty
     a.cs = reinterpret_cast<const float2*>(cos_sin); a.max_pos = max_pos;
     a.kvbar = kvbar; a.kr_index = kr_index; a.normalize = normalize_router;
     a.err = device_error_word();
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // By size: the register-streaming kernel (one block per chunk and part) keeps more loads in flight
+    // per SM once its grid runs for several waves; on grids of under two waves its rotated-key blocks,
+    // which wait on their RoPE table reads, make a tail, and the bulk-copy kernel (table rows staged
+    // with the keys, items spread over a persistent grid) is faster.
+    int impl = g_pool_impl.load();
+    if (impl == 0) {
+        int occ = 0;
+        MSA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+            &occ, in_dt == MSA_BF16 ? (out_dt == MSA_BF16 ? (const void*)pool_kernel<__nv_bfloat16, __nv_bfloat16>
+                                                         : (const void*)pool_kernel<__nv_bfloat16, float>)
+                                   : (out_dt == MSA_BF16 ? (const void*)pool_kernel<float, __nv_bfloat16>
+                                                         : (const void*)pool_kernel<float, float>),
+            kPoolThreads, 0));
+        impl = n_chunks * a.n_parts <= 2 * (int64_t)sm_count() * (occ > 0 ? occ : 1) ? 2 : 1;
+    }
+    if (impl == 2) {
+        bool launched = false;
+        if (in_dt == MSA_BF16 && out_dt == MSA_BF16)
+            MSA_RETURN_IF((launch_pool_bulk<__nv_bfloat16, __nv_bfloat16>(a, s, &launched)));
+        else if (in_dt == MSA_BF16)
+            MSA_RETURN_IF((launch_pool_bulk<__nv_bfloat16, float>(a, s, &launched)));
+        else if (out_dt == MSA_BF16)
+            MSA_RETURN_IF((launch_pool_bulk<float, __nv_bfloat16>(a, s, &launched)));
+        else
+            MSA_RETURN_IF((launch_pool_bulk<float, float>(a, s, &launched)));
+        if (launched) return MSA_OK;
+    }
     const int64_t cap = 1 << 20;
     const int64_t per_part = n_chunks < cap ? n_chunks : cap;
     dim3 grid((unsigned)(per_part * a.n_parts));
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (in_dt == MSA_BF16 && out_dt == MSA_BF16)
         pool_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, kPoolThreads, 0, s>>>(a);
     else if (in_dt == MSA_BF16)
@@ -479,6 +799,26 @@ msa_status msa_pool_chunks(const void* k, const void* v, const void* kr, msa_dty
     else
         pool_kernel<float, float><<<grid, kPoolThreads, 0, s>>>(a);
     MSA_LAUNCH_CHECK();
+    return MSA_OK;
+}
+
+msa_status msa_pool_set_impl(int impl) {
+    MSA_REQUIRE(impl >= 0 && impl <= 2, "msa_pool_set_impl: impl must be 0, 1 or 2");
+    g_pool_impl.store(impl);
+    return MSA_OK;
+}
+
+msa_status msa_pool_set_pipeline(int n_stages, int stage_bytes, int copy_bytes) {
+    MSA_REQUIRE(n_stages == 0 || (n_stages >= 2 && n_stages <= 16), "msa_pool_set_pipeline: n_stages must be 0 or in [2, 16]");
+    MSA_REQUIRE(stage_bytes == 0 || (stage_bytes >= 2048 && stage_bytes <= 65536 && stage_bytes % 1024 == 0),
+                "msa_pool_set_pipeline: stage_bytes must be 0 or a multiple of 1024 in [2048, 65536]");
+    const int S = n_stages ? n_stages : kBulkStagesDefault;
+    const int SB = stage_bytes ? stage_bytes : kBulkStageBytesDefault;
+    MSA_REQUIRE((int64_t)S * SB <= 200 * 1024, "msa_pool_set_pipeline: %d stages of %d bytes exceed 200 KiB", S, SB);
+    MSA_REQUIRE(copy_bytes >= 0 && copy_bytes % 16 == 0, "msa_pool_set_pipeline: copy_bytes must be a multiple of 16");
+    g_pool_stages.store(n_stages);
+    g_pool_stage_bytes.store(stage_bytes);
+    g_pool_copy_bytes.store(copy_bytes);
     return MSA_OK;
 }
 

@@ -99,14 +99,16 @@ def test_gather_backward_sums_rows_of_documents_fetched_twice(m):
     np.testing.assert_allclose(_np(got), ref, rtol=1e-6, atol=1e-6)
 
 
-@pytest.mark.parametrize("kr_dt", ["f32", "bf16"])
-def test_pool_backward_matches_oracle(m, kr_dt):
+@pytest.mark.parametrize("kr_dt,chunk,parts", [("f32", 128, "both"), ("bf16", 128, "both"), ("bf16", 96, "kv"),
+                                               ("bf16", 96, "kr"), ("f32", 1, "both"), ("bf16", 200, "both")])
+def test_pool_backward_matches_oracle(m, kr_dt, chunk, parts):
     """Token gradients of pooling: keys through the transposed document-wise rotation, values, and
-    router keys through the index normalisation; ragged documents (one empty)."""
+    router keys through the index normalisation; ragged documents (one empty), chunks that end
+    inside a token slice, and either group of gradients alone."""
     from routed_long_context_b200.bank import BankLayout
 
     lens = np.array([300, 0, 255, 129, 1000, 1], dtype=np.int64)
-    chunk, hkv, hr, d, base = 128, 8, 8, 128, 1e6
+    hkv, hr, d, base = 8, 8, 128, 1e6
     lay = BankLayout.from_doc_lengths(lens, chunk)
     n = int(lay.doc_tok_off_host[-1])
     C = lay.n_chunks
@@ -114,16 +116,23 @@ def test_pool_backward_matches_oracle(m, kr_dt):
     dkv = _gen(8, (C, 2, hkv, d))
     dki = _gen(9, (C, hr, d))
     cs = m.rope_table(2048, d, base)
-    dk, dv, dkr = m.msa_pool_chunks_backward(torch.from_numpy(dkv).float().cuda(), torch.from_numpy(dki).float().cuda(),
-                                             lay.doc_tok_off, lay.doc_chunk_off, lay.chunk_doc, chunk, n,
+    g_kv = torch.from_numpy(dkv).float().cuda() if parts in ("both", "kv") else None
+    g_kr = torch.from_numpy(dki).float().cuda() if parts in ("both", "kr") else None
+    dk, dv, dkr = m.msa_pool_chunks_backward(g_kv, g_kr, lay.doc_tok_off, lay.doc_chunk_off, lay.chunk_doc, chunk, n,
                                              kr=upload(kr, kr_dt), cos_sin=cs)
     assert m.device_status() == 0
     _, _, krb = O.encode_memory(None, None, kr, lay.doc_tok_off_host, chunk, base)
     rk, rv, rkr = O.encode_memory_backward(dkv[:, 0], dkv[:, 1], O.unit_backward(krb, dki), lay.doc_tok_off_host,
                                            chunk, base)
-    np.testing.assert_allclose(_np(dk), rk, rtol=1e-5, atol=1e-6)
-    np.testing.assert_allclose(_np(dv), rv, rtol=1e-6, atol=1e-7)
-    np.testing.assert_allclose(_np(dkr), rkr, rtol=1e-4, atol=1e-6)
+    if g_kv is not None:
+        np.testing.assert_allclose(_np(dk), rk, rtol=1e-5, atol=1e-6)
+        np.testing.assert_allclose(_np(dv), rv, rtol=1e-6, atol=1e-7)
+    else:
+        assert dk is None and dv is None
+    if g_kr is not None:
+        np.testing.assert_allclose(_np(dkr), rkr, rtol=1e-4, atol=1e-6)
+    else:
+        assert dkr is None
 
 
 @pytest.mark.parametrize("n_q,D,tau", [(3, 1000, 0.1), (2, 97657, 0.05)])

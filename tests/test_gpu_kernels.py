@@ -107,6 +107,41 @@ def test_pool_chunks_ragged_documents(m, in_dt, out_dt):
     _status(m)
 
 
+@pytest.mark.parametrize("in_dt,out_dt", [("bf16", "bf16"), ("f32", "f32"), ("bf16", "f32"), ("f32", "bf16")])
+@pytest.mark.parametrize("pipeline", [(0, 0, 0), (2, 4096, 0), (3, 5120, 0), (16, 12288, 0), (6, 16384, 2048),
+                                      (4, 16384, 1040)])
+def test_pool_bulk_copy_kernel_matches_register_kernel_bitwise(m, in_dt, out_dt, pipeline):
+    """The bulk-copy pipeline and the register-streaming kernel sum every element in token order with
+    the same rotation: identical bits, for ragged documents, router heads != K/V heads and pipeline
+    shapes whose stages hold one row, a row and a half (the rest unused) or several rows, filled by
+    one copy or by several (of whole rows; a copy size below one row still copies a row)."""
+    from routed_long_context_b200.bank import BankLayout
+
+    chunk = 96
+    lay = BankLayout.from_doc_lengths(RAGGED, chunk)
+    n_tok = sum(RAGGED)
+    k, v = (upload(_gen(60 + i, (n_tok, 8, 128), in_dt), in_dt) for i in range(2))
+    kr = upload(_gen(62, (n_tok, 4, 128), in_dt), in_dt)
+    cs = m.rope_table(2048, 128, 1e6)
+    odt = torch.float32 if out_dt == "f32" else torch.bfloat16
+    got = []
+    try:
+        for impl in (1, 2):
+            m.pool_set_impl(impl)
+            m.pool_set_pipeline(*pipeline)
+            got.append(m.msa_pool_chunks(k, v, kr, lay.doc_tok_off, lay.doc_chunk_off, lay.chunk_doc, chunk,
+                                         cos_sin=cs, out_dtype=odt))
+    finally:
+        m.pool_set_impl(0)
+        m.pool_set_pipeline(0, 0, 0)
+    torch.cuda.synchronize()
+    _status(m)
+    assert torch.equal(got[0][0], got[1][0]) and torch.equal(got[0][1], got[1][1])
+    kb, vb, krb = O.encode_memory(_np(k), _np(v), _np(kr), lay.doc_tok_off_host, chunk, 1e6)
+    _close(_np(got[1][0][:, 0]), kb, out_dt, "K-bar")
+    _close(_np(got[1][1]), O.unit(krb), out_dt, "router index")
+
+
 def test_pool_document_translation_invariance_bitwise(m):
     """Document-wise positions: a document's pooled, rotated K-bar is bit-identical wherever it sits."""
     from routed_long_context_b200.bank import BankLayout
@@ -433,7 +468,7 @@ def _tail_intact(buf, n, pattern):
 
 def test_new_kernels_write_nothing_past_their_outputs(m):
     """Canary words after the outputs of the token bank, the split attention (and its log-sum-exp),
-    the attention backward, the Memory Parallel merge and the pooling backward stay untouched."""
+    the attention backward, the Memory Parallel merge and the bulk-copy pooling stay untouched."""
     bf, f32 = torch.bfloat16, torch.float32
     n_q, T, hq, hkv, d, L = 2, 24, 32, 8, 128, 30
     mem_lens = np.array([700, 0], dtype=np.int32)
@@ -457,8 +492,15 @@ def test_new_kernels_write_nothing_past_their_outputs(m):
     midx, mb, mn = _canaried((2, 16), torch.int32, 0x5A5A5A5A)
     msc, sb, sn = _canaried((2, 16), f32, 0x7FC0DEAD)
     m.msa_topk_merge(cand, cidx, np.array([0, 50, 100, 150]), 16, idx=midx, score=msc)
+    from routed_long_context_b200.bank import BankLayout
+    play = BankLayout.from_doc_lengths([300, 0, 255, 445], 96)
+    pkv, pkb, pkn = _canaried((play.n_chunks, 2, hkv, d), bf, 0x3C5A)
+    pki, pib, pin_ = _canaried((play.n_chunks, hkv, d), bf, 0x3C5A)
+    m.msa_pool_chunks(kt, kt, kt, play.doc_tok_off, play.doc_chunk_off, play.chunk_doc, 96,
+                      cos_sin=m.rope_table(1024, d, 1e6), kvbar=pkv, kr_index=pki)
     torch.cuda.synchronize()
     _status(m)
+    assert _tail_intact(pkb, pkn, 0x3C5A) and _tail_intact(pib, pin_, 0x3C5A)
     assert _tail_intact(ob, on, 0x3C5A) and _tail_intact(lb, ln_, 0x7FC0DEAD)
     for g_, b_, n_ in grads:
         assert _tail_intact(b_, n_, 0x7FC0BEEF)

@@ -33,6 +33,14 @@ def test_generator_moments_and_support():
     np.testing.assert_array_equal(rng.normal(123, 7, 1000, 50), x[1000:1050].astype(np.float32))
 
 
+def test_distinct_ints_are_distinct_and_refuse_impossible_requests():
+    got = rng.distinct_ints(5, 9, 40, 50, exclude=(3, 7, 60))
+    assert len(set(got.tolist())) == 40 and not ({3, 7} & set(got.tolist())) and got.min() >= 0 and got.max() < 50
+    assert sorted(rng.distinct_ints(5, 9, 48, 50, exclude=(3, 7)).tolist()) == [i for i in range(50) if i not in (3, 7)]
+    with pytest.raises(ValueError):
+        rng.distinct_ints(5, 9, 49, 50, exclude=(3, 7))   # 48 values exist: no endless draw
+
+
 def test_bf16_round_to_nearest_even():
     one = np.float32(1.0)
     cases = np.array([one + 2.0 ** -8, one + 3 * 2.0 ** -8, one + 2.0 ** -9, -(one + 2.0 ** -8)], dtype=np.float32)
