@@ -376,9 +376,12 @@ msa_status msa_router_aux_loss(const float* doc_scores, int n_q, int64_t n_docs,
  *     normalisation;
  *   dkhat [n_chunks][H][d] (fp32, overwritten): with respect to the stored index vectors as used
  *     in the dot product (msa_pool_chunks_backward carries it through the index normalisation).
- * Scores are recomputed in fp32 on CUDA cores to find the attaining pairs (a training-context
- * bank, not the 100M inference index). kr_index and qr of dtype dt; H * d <= 1024.
- * ws: msa_route_backward_workspace_size bytes. */
+ * Scores are recomputed to find the attaining pairs (a training-context bank, not the 100M
+ * inference index): for a bf16 index with H * d a multiple of 64, on the tcgen05 tensor cores with
+ * the fp32 normalised queries split exactly into three bf16 terms (fp32 accumulation in TMEM;
+ * msa_route_set_impl(1) selects the CUDA-core search instead); otherwise in fp32 on CUDA cores.
+ * kr_index and qr of dtype dt; H * d <= 1024.
+ * ws: msa_route_backward_workspace_size bytes (device, 256-byte aligned). */
 msa_status msa_route_backward(const void* kr_index, msa_dtype dt, int64_t n_chunks, const int64_t* doc_chunk_off,
                               int64_t n_docs, const void* qr, int n_q, int T, int H, int d, const float* d_doc_scores,
                               float* dqr, float* dkhat, void* ws, size_t ws_bytes, void* stream);

@@ -17,7 +17,7 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libmsa.so")
 SOURCES = ["api.cu", "rope_pool.cu", "route.cu", "route_tc.cu", "topk.cu", "gather.cu", "attn.cu", "step.cu",
-           "backward.cu", "attn_tc.cu", "attn_bwd_tc.cu"]
+           "backward.cu", "attn_tc.cu", "attn_bwd_tc.cu", "route_bwd_tc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-I", os.path.join(ROOT, "include"),
          "--expt-relaxed-constexpr"]

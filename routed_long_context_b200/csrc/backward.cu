@@ -692,9 +692,13 @@ __global__ void __launch_bounds__(1024) aux_loss_kernel(const float* __restrict_
 
 // ---------------------------------------------------------------------------------------------
 // Router backward.
-// (1) qhat: unit router queries per head, divided by H (the folded form) [n_q][T][H*d] fp32.
+// (1) qhat: unit router queries per head, divided by H (the folded form) [n_q][T][H*d] fp32;
+//     with qsplit, also its exact three-term bf16 split for the tensor-core search, rows
+//     [3][n_q][T_pad][H*d] (term, query, token).
 __global__ void __launch_bounds__(128) route_bwd_qhat_kernel(const void* __restrict__ qr, int qr_bf16, int64_t rows,
-                                                             int H, int d, float* __restrict__ qhat) {
+                                                             int H, int d, float* __restrict__ qhat,
+                                                             __nv_bfloat16* __restrict__ qsplit, int T, int T_pad,
+                                                             int n_q) {
     // one warp per (row, head)
     const int64_t w = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
@@ -707,7 +711,27 @@ __global__ void __launch_bounds__(128) route_bwd_qhat_kernel(const void* __restr
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     const float inv = ss > 0.f ? 1.0f / (sqrtf(ss) * H) : 0.f;
-    for (int i = lane; i < d; i += 32) qhat[w * d + i] = load_elem(qr, w * d + i, qr_bf16) * inv;
+    const int64_t row = w / H;
+    const int h = (int)(w - row * H);
+    const int64_t qi = row / T, t = row - qi * T;
+    const int64_t K = (int64_t)H * d;
+    for (int i = lane; i < d; i += 32) {
+        const float x = load_elem(qr, w * d + i, qr_bf16) * inv;
+        qhat[w * d + i] = x;
+        if (qsplit) {
+            // x = hi + mid + lo: each term the bf16 rounding of what the previous ones leave (the
+            // differences are exact in fp32)
+            const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+            const float r1 = x - __bfloat162float(hi);
+            const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+            const int64_t o = (qi * T_pad + t) * K + (int64_t)h * d + i;
+            const int64_t term = (int64_t)n_q * T_pad * K;
+            qsplit[o] = hi;
+            qsplit[o + term] = mid;
+            qsplit[o + 2 * term] = lo;
+        }
+    }
 }
 
 // (2) per (query, chunk): best folded score over the query tokens and the first token attaining it,
@@ -991,7 +1015,10 @@ msa_status msa_router_aux_loss(const float* doc_scores, int n_q, int64_t n_docs,
 msa_status msa_route_backward_workspace_size(int64_t n_chunks, int n_q, int T, int H, int d, size_t* bytes) {
     MSA_REQUIRE(bytes && n_chunks >= 0 && n_q > 0 && T > 0 && H > 0 && d > 0, "msa_route_backward_workspace_size: bad sizes");
     const size_t qk = (size_t)n_q * T * H * d * sizeof(float);
-    *bytes = 2 * align_up(qk, 256) + align_up((size_t)n_q * n_chunks * 8, 256);
+    const int tile = route_bwd_tc_token_tile();
+    const size_t t_pad = (size_t)(T + tile - 1) / tile * tile;
+    const size_t split = 3 * (size_t)n_q * t_pad * H * d * sizeof(__nv_bfloat16);
+    *bytes = 2 * align_up(qk, 256) + align_up((size_t)n_q * n_chunks * 8, 256) + align_up(split, 256);
     return MSA_OK;
 }
 
@@ -1011,18 +1038,32 @@ msa_status msa_route_backward(const void* kr_index, msa_dtype dt, int64_t n_chun
     float* qhat = reinterpret_cast<float*>(w);
     float* dqhat = reinterpret_cast<float*>(w + qk);
     unsigned long long* best = reinterpret_cast<unsigned long long*>(w + 2 * qk);
+    const int tile = route_bwd_tc_token_tile();
+    const int T_pad = (T + tile - 1) / tile * tile;
+    __nv_bfloat16* qsplit =
+        reinterpret_cast<__nv_bfloat16*>(w + 2 * qk + align_up((size_t)n_q * n_chunks * 8, 256));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int bf = dt == MSA_BF16;
     const int64_t rows = (int64_t)n_q * T;
+    // best-token search: tcgen05 for a bf16 index (K a multiple of 64), CUDA cores otherwise or when
+    // the router is set to its CUDA-core kernel
+    const bool tc = bf && K % 64 == 0 && route_impl_setting() != 1 && T_pad / tile <= 65535 && n_q <= 65535;
     MSA_CUDA_TRY(cudaMemsetAsync(dqhat, 0, (size_t)n_q * T * K * sizeof(float), s));
     MSA_CUDA_TRY(cudaMemsetAsync(dkhat, 0, (size_t)n_chunks * K * sizeof(float), s));
     MSA_CUDA_TRY(cudaMemsetAsync(best, 0, (size_t)n_q * n_chunks * sizeof(unsigned long long), s));
-    route_bwd_qhat_kernel<<<(unsigned)((rows * H + 3) / 4), 128, 0, s>>>(qr, bf, rows, H, d, qhat);
+    if (tc && T_pad != T)   // padding token rows of the split: zero (their columns are never read)
+        MSA_CUDA_TRY(cudaMemsetAsync(qsplit, 0, 3 * (size_t)n_q * T_pad * K * sizeof(__nv_bfloat16), s));
+    route_bwd_qhat_kernel<<<(unsigned)((rows * H + 3) / 4), 128, 0, s>>>(qr, bf, rows, H, d, qhat, tc ? qsplit : nullptr,
+                                                                         T, T_pad, n_q);
     MSA_LAUNCH_CHECK();
-    const int64_t work = ((n_chunks + kBestChunks - 1) / kBestChunks) * ((T + kBestTokens - 1) / kBestTokens);
-    const unsigned best_blocks = (unsigned)std::min<int64_t>(work, (int64_t)sm_count() * 8);
-    route_bwd_best_kernel<<<best_blocks, 256, 0, s>>>(kr_index, bf, n_chunks, qhat, n_q, T, K, best);
-    MSA_LAUNCH_CHECK();
+    if (tc) {
+        MSA_RETURN_IF(launch_route_bwd_best_tc(kr_index, n_chunks, qsplit, n_q, T, T_pad, K, best, s));
+    } else {
+        const int64_t work = ((n_chunks + kBestChunks - 1) / kBestChunks) * ((T + kBestTokens - 1) / kBestTokens);
+        const unsigned best_blocks = (unsigned)std::min<int64_t>(work, (int64_t)sm_count() * 8);
+        route_bwd_best_kernel<<<best_blocks, 256, 0, s>>>(kr_index, bf, n_chunks, qhat, n_q, T, K, best);
+        MSA_LAUNCH_CHECK();
+    }
     route_bwd_scatter_kernel<<<(unsigned)(((int64_t)n_q * n_docs + 7) / 8), 256, 0, s>>>(
         kr_index, bf, doc_chunk_off, n_docs, n_chunks, best, qhat, d_doc_scores, n_q, T, H, K, dqhat, dkhat);
     MSA_LAUNCH_CHECK();

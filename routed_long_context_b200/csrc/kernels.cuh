@@ -14,6 +14,14 @@ msa_status make_tensor_map_bf16(CUtensorMap* map, const void* ptr, int rank, con
 
 // The bf16 attention kernel choice of msa_attn_set_impl (0 = default: tcgen05 where it applies).
 int attn_impl_setting();
+int route_impl_setting();   // msa_route_set_impl's value (1 = CUDA-core kernels)
+
+// Router backward best-token search on tcgen05 (route_bwd_tc.cu): index [n_chunks][K] bf16,
+// qsplit [3][n_q][T_pad][K] bf16 (the exact three-term split of qhat), best [n_q][n_chunks]
+// 64-bit keys (zeroed by the caller), T_pad a multiple of route_bwd_tc_token_tile().
+int route_bwd_tc_token_tile();
+msa_status launch_route_bwd_best_tc(const void* index, int64_t n_chunks, const void* qsplit, int n_q, int T,
+                                    int T_pad, int K, unsigned long long* best, cudaStream_t s);
 
 // dQ of the attention backward on tcgen05 (bf16, d = 128): the forward's operands, dout, its
 // log-sum-exp (natural log) and D = rowsum(dO * O); dq fp32 [n_q][T][hq][d] is overwritten.

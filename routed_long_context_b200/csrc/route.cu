@@ -168,6 +168,8 @@ size_t qhat_bytes(int N, int K) {
 
 }  // namespace
 
+int route_impl_setting() { return g_route_impl.load(); }
+
 msa_status route_plan(msa_dtype dt, int64_t n_chunks, int n_q, int T, int H, int d, RoutePlan* plan) {
     MSA_REQUIRE(dtype_ok(dt), "msa_route_scores: bad dtype %d", dt);
     MSA_REQUIRE(n_q > 0 && T > 0 && H > 0 && d > 0, "msa_route_scores: bad sizes");

@@ -150,22 +150,37 @@ def test_aux_loss_matches_oracle(m, n_q, D, tau):
     np.testing.assert_allclose(_np(grad), rg, rtol=1e-3, atol=1e-7 / n_q)
 
 
-@pytest.mark.parametrize("dt", ["f32", "bf16"])
-def test_route_backward_matches_oracle(m, dt):
+@pytest.mark.parametrize("dt,impl,n_docs,T", [("f32", 0, 40, 17), ("bf16", 0, 40, 17), ("bf16", 1, 40, 17),
+                                              ("bf16", 0, 300, 70), ("bf16", 1, 300, 70), ("bf16", 0, 3, 64)])
+def test_route_backward_matches_oracle(m, dt, impl, n_docs, T):
     """The index is built on the host (unit vectors rounded to dt) and both sides score those stored
-    values as they are, so they find the same attaining (chunk, token) pairs."""
+    values as they are, so they find the same attaining (chunk, token) pairs. bf16 runs the best-token
+    search on the tensor cores (impl 0: chunk tiles of 128, token tiles of 32, padded token rows) or on
+    CUDA cores (impl 1). Query 0 repeats token 3 at token 9 and at token T-2, so its scores tie exactly
+    within a token tile and across tiles: the first token must take the gradient."""
     r = np.random.default_rng(12)
-    counts = r.integers(0, 13, 40)
+    counts = r.integers(0, 13, n_docs)
+    counts[0] = max(counts[0], 1)
     off = np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
-    C, H, d, n_q, T = int(off[-1]), 8, 128, 2, 17
+    C, H, d, n_q = int(off[-1]), 8, 128, 2
     index = rng.round_to(O.unit(_gen(11, (C, H, d))).astype(np.float32), dt).astype(np.float64)
     qr = _gen(13, (n_q, T, H, d), dt)
-    ds = _gen(14, (n_q, 40))
-    dqr, dkh = m.msa_route_backward(upload(index, dt), torch.from_numpy(off).cuda(), upload(qr, dt),
-                                    torch.from_numpy(ds).float().cuda())
-    assert m.device_status() == 0
+    qr[0, 9] = qr[0, 3]
+    qr[0, T - 2] = qr[0, 3]
+    # chunk 0 is attained by the repeated token
+    index[0] = rng.round_to(O.unit(qr[0, 3]).astype(np.float32), dt)
+    ds = _gen(14, (n_q, n_docs))
+    m.route_set_impl(impl)
+    try:
+        dqr, dkh = m.msa_route_backward(upload(index, dt), torch.from_numpy(off).cuda(), upload(qr, dt),
+                                        torch.from_numpy(ds).float().cuda())
+        assert m.device_status() == 0
+    finally:
+        m.route_set_impl(0)
     rq, rk = O.route_backward(index, off, qr, ds, index_is_unit=True)
     assert _rel(_np(dqr), rq) <= 1e-4 and _rel(_np(dkh), rk) <= 1e-4
+    g = _np(dqr)
+    assert np.abs(g[0, 3]).max() > 0 and np.abs(g[0, 9]).max() == 0 and np.abs(g[0, T - 2]).max() == 0
 
 
 def test_training_loss_gradients_on_a_64k_context(m):
