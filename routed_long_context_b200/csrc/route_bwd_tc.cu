@@ -17,6 +17,8 @@
 // 64-bit key with one atomic max per chunk. Every mbarrier wait is bounded; on expiry the CTA
 // records MSA_DEV_WAIT_TIMEOUT, writes nothing, waits (bounded) for its copies and MMAs and frees
 // TMEM.
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.cuh"
 #include "tc.cuh"
@@ -216,13 +218,18 @@ msa_status launch_route_bwd_best_tc(const void* index, int64_t n_chunks, const v
               | ((uint32_t)(BM >> 4) << 24);       // M / 16 ; A and B K-major
     p.best = best;
     p.err = device_error_word();
-    static bool opted[64] = {false};
-    int dev = 0;
-    MSA_CUDA_TRY(cudaGetDevice(&dev));
-    if (dev < 0 || dev >= 64 || !opted[dev]) {
-        MSA_CUDA_TRY(cudaFuncSetAttribute(route_bwd_best_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          kSmemBytes));
-        if (dev >= 0 && dev < 64) opted[dev] = true;
+    {
+        // once per device: opt the kernel into its dynamic shared memory
+        static std::mutex mu;
+        static bool opted[64] = {false};
+        int dev = 0;
+        MSA_CUDA_TRY(cudaGetDevice(&dev));
+        std::lock_guard<std::mutex> lk(mu);
+        if (dev < 0 || dev >= 64 || !opted[dev]) {
+            MSA_CUDA_TRY(cudaFuncSetAttribute(route_bwd_best_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              kSmemBytes));
+            if (dev >= 0 && dev < 64) opted[dev] = true;
+        }
     }
     const dim3 grid((unsigned)((n_chunks + BM - 1) / BM), (unsigned)(T_pad / BN), (unsigned)n_q);
     route_bwd_best_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(tmA, tmB, p);
