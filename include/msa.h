@@ -284,7 +284,9 @@ msa_status msa_sparse_attn(const void* q, const void* mem_kv, const int32_t* mem
 
 /* Selects the bf16 attention kernels for testing: 0 = default (msa_sparse_attn_split on tcgen05
  * tensor cores with TMEM accumulators, msa_sparse_attn on mma.sync m16n8k16 so that it can run
- * beside the router's blocks), 1 = CUDA cores for msa_sparse_attn, 2 = mma.sync for both.
+ * beside the router's blocks), 1 = CUDA cores for msa_sparse_attn, 2 = mma.sync for both,
+ * 3 = as 0, and the attention backward's dK / dV on tcgen05 as well (by default they run on
+ * mma.sync, dQ on tcgen05). impl 3 has not yet been validated on a GPU: opt-in only.
  * fp32 always runs on CUDA cores. Process-wide. */
 msa_status msa_attn_set_impl(int impl);
 

@@ -114,7 +114,8 @@ def route_workspace_size(n_q: int, T: int, H: int, d: int, dtype) -> int:
 
 def attn_set_impl(impl: int) -> None:
     """bf16 attention: 0 = default (split variant on tcgen05, plain on mma.sync), 1 = CUDA cores for the
-    plain variant, 2 = mma.sync for both."""
+    plain variant, 2 = mma.sync for both, 3 = as 0 plus the backward's dK/dV on tcgen05 (opt-in; not yet
+    validated on a GPU)."""
     check(lib.msa_attn_set_impl(impl), "msa_attn_set_impl")
 
 

@@ -551,7 +551,7 @@ using namespace msa;
 extern "C" {
 
 msa_status msa_attn_set_impl(int impl) {
-    MSA_REQUIRE(impl >= 0 && impl <= 2, "msa_attn_set_impl: impl must be 0, 1 or 2");
+    MSA_REQUIRE(impl >= 0 && impl <= 3, "msa_attn_set_impl: impl must be 0, 1, 2 or 3");
     g_attn_impl.store(impl);
     return MSA_OK;
 }
@@ -579,7 +579,7 @@ msa_status msa_sparse_attn(const void* q, const void* mem_kv, const int32_t* mem
     a.local_k = local_k; a.local_v = local_v; a.L_max = L_max; a.L = L; a.q_start = q_start;
     a.T = T; a.hq = hq; a.hkv = hkv; a.scale_log2e = scale * 1.4426950408889634f; a.out = out;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (dt == MSA_BF16 && g_attn_impl.load() == 0) return launch_mma<false>(a, n_q, s);
+    if (dt == MSA_BF16 && (g_attn_impl.load() == 0 || g_attn_impl.load() == 3)) return launch_mma<false>(a, n_q, s);
     return dt == MSA_BF16 ? launch<__nv_bfloat16>(a, n_q, s) : launch<float>(a, n_q, s);
 }
 
@@ -611,7 +611,7 @@ msa_status msa_sparse_attn_split(const void* q, const void* mem_kv, const int32_
     MSA_REQUIRE(aligned16(q) && aligned16(out) && aligned16(ws) && (max_mem == 0 || aligned16(mem_kv)) &&
                     (L == 0 || (aligned16(local_k) && aligned16(local_v))),
                 "msa_sparse_attn_split: pointers must be 16-byte aligned");
-    const bool tc = g_attn_impl.load() == 0;
+    const bool tc = g_attn_impl.load() == 0 || g_attn_impl.load() == 3;
     const int n_split = tc ? attn_tc_splits(n_q, T, hq, hkv, max_mem, L) : pick_splits(n_q, T, hq, hkv, max_mem, L);
     const size_t need = split_ws_bytes(split_ws_splits(n_q, T, hq, hkv, max_mem, L), n_q, T, hq);
     if (ws_bytes < need)

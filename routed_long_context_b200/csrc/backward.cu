@@ -407,17 +407,27 @@ template <int G>
 msa_status launch_attn_bwd_g(const BwdArgs& a, int n_q, cudaStream_t s) {
     const int key_tiles = (a.max_mem + a.L + kTile - 1) / kTile;
     if (key_tiles > 0) {
-        MSA_CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dkdv_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          (int)kDkdvSmem));
-        attn_bwd_dkdv_kernel<G><<<dim3(key_tiles * a.n_rsplit, a.hkv, n_q), 128, kDkdvSmem, s>>>(a);
-        MSA_LAUNCH_CHECK();
+        if (attn_impl_setting() == 3) {   // dK / dV on tcgen05 (opt-in)
+            DkdvTcArgs k{};
+            k.q = a.q; k.mem_kv = a.mem_kv; k.mem_len = a.mem_len; k.max_mem = a.max_mem;
+            k.local_k = a.local_k; k.local_v = a.local_v; k.L_max = a.L_max; k.L = a.L; k.q_start = a.q_start;
+            k.T = a.T; k.hq = a.hq; k.hkv = a.hkv; k.G = G; k.scale = a.scale; k.scale_log2e = a.scale_log2e;
+            k.dout = a.dout; k.lse = a.lse; k.Dvec = a.Dvec; k.dmem = a.dmem; k.dlk = a.dlk; k.dlv = a.dlv;
+            k.n_rsplit = a.n_rsplit; k.key_pad = a.key_pad; k.part_dkv = a.part_dkv; k.err = device_error_word();
+            MSA_RETURN_IF(launch_attn_bwd_dkdv_tc(k, n_q, s));
+        } else {
+            MSA_CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dkdv_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              (int)kDkdvSmem));
+            attn_bwd_dkdv_kernel<G><<<dim3(key_tiles * a.n_rsplit, a.hkv, n_q), 128, kDkdvSmem, s>>>(a);
+            MSA_LAUNCH_CHECK();
+        }
         if (a.n_rsplit > 1) {
             const int64_t warps = (int64_t)n_q * a.key_pad * 2 * a.hkv;
             attn_bwd_dkdv_reduce_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, s>>>(a, n_q);
             MSA_LAUNCH_CHECK();
         }
     }
-    if (attn_impl_setting() == 0) {   // dQ on tcgen05
+    if (attn_impl_setting() == 0 || attn_impl_setting() == 3) {   // dQ on tcgen05
         DqTcArgs d{};
         d.q = a.q; d.mem_kv = a.mem_kv; d.mem_len = a.mem_len; d.max_mem = a.max_mem;
         d.local_k = a.local_k; d.local_v = a.local_v; d.L_max = a.L_max; d.L = a.L; d.q_start = a.q_start;

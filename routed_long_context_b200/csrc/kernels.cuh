@@ -44,6 +44,32 @@ struct DqTcArgs {
 };
 msa_status launch_attn_bwd_dq_tc(DqTcArgs a, int n_q, cudaStream_t s);
 
+// dK / dV of the attention backward on tcgen05 (attn_bwd_tc.cu): the same inputs as DqTcArgs plus
+// the gradient outputs. n_rsplit row ranges per key tile; with n_rsplit > 1 each range writes its
+// partial (dK already scaled) into part_dkv [n_rsplit][n_q][key_pad][2][hkv][d] for the reduce
+// kernel, otherwise the gradients go to dmem [n_q][max_mem][2][hkv][d] and dlk / dlv
+// [n_q][L_max][hkv][d] directly.
+struct DkdvTcArgs {
+    const __nv_bfloat16* q;
+    const __nv_bfloat16* mem_kv;
+    const int32_t* mem_len;
+    int max_mem;
+    const __nv_bfloat16* local_k;
+    const __nv_bfloat16* local_v;
+    int L_max, L, q_start, T, hq, hkv, G;
+    float scale, scale_log2e;
+    const __nv_bfloat16* dout;
+    const float* lse;
+    const float* Dvec;
+    float* dmem;
+    float* dlk;
+    float* dlv;
+    int n_rsplit, key_pad;
+    float* part_dkv;
+    int* err;
+};
+msa_status launch_attn_bwd_dkdv_tc(const DkdvTcArgs& a, int n_q, cudaStream_t s);
+
 // Rotates rows of [*, heads, d] vectors. Row r of the launch belongs to segment s at offset u:
 //   uniform_len > 0: s = r / uniform_len, u = r % uniform_len,
 //                    input row s*in_stride + u, output row s*out_stride + out_off + u;
