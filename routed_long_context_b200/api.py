@@ -24,8 +24,14 @@ def _dt(t: torch.Tensor) -> int:
         raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)") from None
 
 
-def _ptr(t) -> int | None:
-    return None if t is None else t.data_ptr()
+def _ptr(t, strided: bool = False) -> int | None:
+    """Device or host address of a tensor for the C ABI, which reads every array as dense row-major;
+    a non-contiguous view is refused unless the entry point takes its stride (strided=True)."""
+    if t is None:
+        return None
+    if not strided and not t.is_contiguous():
+        raise ValueError(f"tensor of shape {tuple(t.shape)} and strides {t.stride()} must be contiguous")
+    return t.data_ptr()
 
 
 def _stream(stream) -> int:
@@ -199,10 +205,16 @@ def msa_topk_merge(cand_score, cand_idx, shard_doc_off, k: int, idx=None, score=
     n_q, k_cand = cand_score.shape[-2:]
     dev = cand_score.device
     stride = n_q * k_cand if shard_stride is None else int(shard_stride)
+    for t in (cand_score, cand_idx):
+        # each shard's [n_q, k_cand] lists dense, shards `stride` elements apart
+        if t.stride(-1) != 1 or (n_q > 1 and t.stride(-2) != k_cand) or \
+                (t.dim() >= 3 and t.shape[0] > 1 and t.stride(0) != stride):
+            raise ValueError(f"msa_topk_merge: candidate lists of strides {t.stride()} do not match "
+                             f"[n_shards, {n_q}, {k_cand}] with shards {stride} elements apart")
     idx = torch.empty((n_q, k), dtype=torch.int32, device=dev) if idx is None else idx
     score = torch.empty((n_q, k), dtype=torch.float32, device=dev) if score is None else score
-    check(lib.msa_topk_merge(_ptr(cand_score), _ptr(cand_idx), stride, n_shards, n_q, k_cand, off.ctypes.data, k,
-                             _ptr(idx), _ptr(score), _stream(stream)), "msa_topk_merge")
+    check(lib.msa_topk_merge(_ptr(cand_score, strided=True), _ptr(cand_idx, strided=True), stride, n_shards, n_q,
+                             k_cand, off.ctypes.data, k, _ptr(idx), _ptr(score), _stream(stream)), "msa_topk_merge")
     return idx, score
 
 

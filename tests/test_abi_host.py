@@ -162,3 +162,25 @@ def test_new_entry_points_validate_on_the_host(lib):
     assert lib.msa_sparse_attn_split_workspace_size(1, 64, 32, 8, 8064, 64, ctypes.byref(n)) == 0 and n.value > 0
     assert lib.msa_sparse_attn_backward_workspace_size(1, 512, 32, 8, 128, 512, ctypes.byref(n)) == 0
     assert lib.msa_route_backward_workspace_size(512, 1, 512, 8, 128, ctypes.byref(n)) == 0 and n.value > 0
+
+
+def test_binding_refuses_views_the_c_abi_would_misread(lib):
+    """The C ABI reads dense row-major arrays: a transposed or sliced view is refused before any
+    call, and the Memory Parallel merge accepts strided candidate lists only when their layout
+    matches the shard stride it is given."""
+    import torch
+
+    from routed_long_context_b200 import api
+
+    with pytest.raises(ValueError):
+        api._ptr(torch.zeros(4, 6).t())
+    with pytest.raises(ValueError):
+        api._ptr(torch.zeros(4, 6)[:, 1:3])
+    assert api._ptr(torch.zeros(4, 6)[1:3]) is not None           # a leading-dimension slice is dense
+    packed = torch.zeros(3, 2, 2, 5, dtype=torch.int32)          # [shards][score, index][n_q][k_cand]
+    bounds = np.array([0, 10, 20, 30])
+    with pytest.raises(ValueError):                               # the pair is interleaved: stride needed
+        api.msa_topk_merge(packed[:, 0].view(torch.float32), packed[:, 1], bounds, 4)
+    with pytest.raises(ValueError):                               # inner lists not dense
+        api.msa_topk_merge(torch.zeros(3, 5, 2)[:, :, 0], torch.zeros(3, 5, 2, dtype=torch.int32)[:, :, 0],
+                           bounds, 4, shard_stride=10)
