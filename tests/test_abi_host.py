@@ -184,3 +184,43 @@ def test_binding_refuses_views_the_c_abi_would_misread(lib):
     with pytest.raises(ValueError):                               # inner lists not dense
         api.msa_topk_merge(torch.zeros(3, 5, 2)[:, :, 0], torch.zeros(3, 5, 2, dtype=torch.int32)[:, :, 0],
                            bounds, 4, shard_stride=10)
+
+
+def test_too_small_workspace_is_refused_before_any_launch(lib):
+    """A caller workspace below the size the library asks for (the stand-in for an allocation that
+    failed) is refused with MSA_ERR_WORKSPACE and a message naming both sizes; nothing is launched
+    (the calls get placeholder pointers that no kernel could read)."""
+    from routed_long_context_b200 import _lib
+
+    P = ctypes.c_void_p(256)
+    f = ctypes.c_float(0.1)
+    calls = {
+        "msa_route_scores": lambda: lib.msa_route_scores(P, 1, 1000, P, 100, P, 1, 64, 8, 128, P, None, P, 16, None),
+        "msa_topk_docs": lambda: lib.msa_topk_docs(P, 1, 1000, 4, P, P, P, 0, None),
+        "msa_route_backward": lambda: lib.msa_route_backward(P, 1, 1000, P, 100, P, 1, 17, 8, 128, P, P, P, P, 16,
+                                                             None),
+        "msa_sparse_attn_split": lambda: lib.msa_sparse_attn_split(P, P, P, 64, P, P, 16, 16, 0, 1, 16, 32, 8, 128, f,
+                                                                   P, None, 1, P, 16, None),
+        "msa_sparse_attn_backward": lambda: lib.msa_sparse_attn_backward(P, P, P, 64, P, P, 16, 16, 0, 1, 16, 32, 8,
+                                                                         128, f, P, P, P, 1, P, P, P, P, P, 16, None),
+    }
+    for name, call in calls.items():
+        assert call() == _lib.MSA_ERR_WORKSPACE, name
+        msg = lib.msa_last_error().decode()
+        assert msg.startswith(name) and "workspace" in msg and re.search(r"\d+ < \d+", msg), msg
+
+    layers = (_lib.LayerArgs * 1)()
+    for fld, _ in _lib.LayerArgs._fields_:
+        setattr(layers[0], fld, 256)
+    a = _lib.InterleaveArgs()
+    a.n_layers, a.layers, a.dt = 1, layers, 1
+    a.n_chunks, a.n_docs = 10, 2
+    a.doc_chunk_off = a.doc_chunk_off_host = a.chunk_doc = a.rope_cos_sin = 256
+    a.n_q, a.H, a.d, a.hq, a.hkv, a.k = 1, 8, 128, 32, 8, 1
+    a.L_prev, a.T_new, a.new_q_stride, a.L_max, a.max_mem = 56, 8, 8, 64, 16
+    a.rope_max_pos, a.scale, a.ws, a.ws_bytes = 4096, 0.1, 256, 16
+    assert lib.msa_interleave_step(ctypes.byref(a), None, None, 1000) == _lib.MSA_ERR_WORKSPACE
+    msg = lib.msa_last_error().decode()
+    n = ctypes.c_size_t(0)
+    assert lib.msa_interleave_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0
+    assert f"16 < {n.value}" in msg, msg
