@@ -11,6 +11,10 @@ namespace msa {
 // dims[0] innermost in elements, strides[i] in bytes for dims i + 1, box in elements.
 msa_status make_tensor_map_bf16(CUtensorMap* map, const void* ptr, int rank, const uint64_t* dims,
                                 const uint64_t* strides, const uint32_t* box);
+// The same for fp32 or bf16 elements, with the 128-byte swizzle or none (a box then lands in shared
+// memory in plain row-major order).
+msa_status make_tensor_map(CUtensorMap* map, const void* ptr, bool fp32, int rank, const uint64_t* dims,
+                           const uint64_t* strides, const uint32_t* box, bool swizzle128);
 
 // The bf16 attention kernel choice of msa_attn_set_impl (0 = default: tcgen05 where it applies).
 int attn_impl_setting();

@@ -374,10 +374,11 @@ msa_status make_map(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t 
 
 // Tensor map of a bf16 array for TMA loads with the 128-byte swizzle (shared with the attention
 // kernels): dims[0] innermost (elements), strides in bytes for dims 1..rank-1.
-msa_status make_tensor_map_bf16(CUtensorMap* map, const void* ptr, int rank, const uint64_t* dims,
-                                const uint64_t* strides, const uint32_t* box) {
+msa_status make_tensor_map(CUtensorMap* map, const void* ptr, bool fp32, int rank, const uint64_t* dims,
+                           const uint64_t* strides, const uint32_t* box, bool swizzle128) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return set_error(MSA_ERR_CUDA, "tensor map: cuTensorMapEncodeTiled unavailable");
+    if (rank < 1 || rank > 5) return set_error(MSA_ERR_INVALID_ARG, "tensor map: rank %d", rank);
     cuuint64_t d[5], st[4];
     cuuint32_t b[5], e[5];
     for (int i = 0; i < rank; ++i) {
@@ -386,11 +387,17 @@ msa_status make_tensor_map_bf16(CUtensorMap* map, const void* ptr, int rank, con
         e[i] = 1;
         if (i + 1 < rank) st[i] = strides[i];
     }
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(ptr), d, st, b, e,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r = fn(map, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank,
+                    const_cast<void*>(ptr), d, st, b, e, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return set_error(MSA_ERR_CUDA, "tensor map encode failed (%d)", (int)r);
     return MSA_OK;
+}
+
+msa_status make_tensor_map_bf16(CUtensorMap* map, const void* ptr, int rank, const uint64_t* dims,
+                                const uint64_t* strides, const uint32_t* box) {
+    return make_tensor_map(map, ptr, false, rank, dims, strides, box, true);
 }
 
 namespace {

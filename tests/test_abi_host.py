@@ -107,7 +107,7 @@ def test_route_and_attention_reject_bad_shapes(lib):
                              ctypes.c_void_p(256), 0, None)
     assert st == 1
     assert lib.msa_route_set_impl(4) == 1 and lib.msa_route_set_impl(0) == 0
-    assert lib.msa_pool_set_impl(3) == 1 and lib.msa_pool_set_impl(-1) == 1 and lib.msa_pool_set_impl(0) == 0
+    assert lib.msa_pool_set_impl(4) == 1 and lib.msa_pool_set_impl(-1) == 1 and lib.msa_pool_set_impl(0) == 0
     assert lib.msa_attn_set_impl(4) == 1 and lib.msa_attn_set_impl(3) == 0 and lib.msa_attn_set_impl(0) == 0
     assert lib.msa_pool_set_pipeline(1, 0, 0) == 1         # fewer than 2 stages
     assert lib.msa_pool_set_pipeline(0, 1000, 0) == 1      # not a multiple of 1024
