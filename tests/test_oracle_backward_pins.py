@@ -184,3 +184,21 @@ def test_training_loss_gradient_through_encode_route_and_attention():
             return loss(*a)
         i = r.choice(x.size, 12, replace=False)
         np.testing.assert_allclose(g.flat[i], _fd(f, x, i), atol=1e-7)
+
+
+def test_three_term_bf16_split_of_fp32_is_exact():
+    """The tensor-core best-token search of the router backward feeds the fp32 normalised queries as
+    three bf16 terms (hi = bf16(x), mid = bf16(x - hi), lo = bf16(x - hi - mid), each difference exact
+    in fp32): their sum gives x back exactly, so the bf16 tensor cores see the fp32 operand itself.
+    Checked on normal values over several magnitudes, including the scale the folded queries have
+    (unit heads divided by H)."""
+    from msa_inputs import rng as R
+
+    r = np.random.default_rng(21)
+    for scale in (1.0, 1.0 / 8 / np.sqrt(128), 1e-3, 1e3):
+        x = (r.standard_normal(1 << 18) * scale).astype(np.float32)
+        hi = R.round_to(x, "bf16")
+        r1 = (x - hi).astype(np.float32)
+        mid = R.round_to(r1, "bf16")
+        lo = R.round_to((r1 - mid).astype(np.float32), "bf16")
+        np.testing.assert_array_equal(hi.astype(np.float64) + mid + lo, x.astype(np.float64))
