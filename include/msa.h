@@ -129,8 +129,7 @@ msa_status msa_pool_chunks(const void* k, const void* v, const void* kr, msa_dty
                            int normalize_router, void* stream);
 
 /* Selects the pooling kernel: 0 = by size (default), 1 = register streaming, 2 = bulk copy where
- * the layout allows, 3 = the bulk-copy kernel with each stage's token rows brought in by one 3D
- * tensor-map box (opt-in; not yet validated on a GPU). Process-wide. */
+ * the layout allows. Process-wide. */
 msa_status msa_pool_set_impl(int impl);
 
 /* Tuning knob of the bulk-copy pooling kernel: n_stages pipeline stages (2..16) of stage_bytes

@@ -306,3 +306,46 @@ def route_and_attend_fine(krbar, doc_chunk_off, tokbank, doc_tok_off, qr_active,
     q_rot = apply_rope(q_new, global_positions(k, L_prev, T_new), base)
     o = sparse_attention(q_rot, mem[:, 0], mem[:, 1], k_local, v_local[:L], L_prev, scale)
     return idx[0], val[0], o
+
+
+# ---------------------------------------------------------------------------------------------
+# the Memory Interleave loop for one routed layer
+# ---------------------------------------------------------------------------------------------
+def interleave_round_tokens(r: int, T0: int, T_new: int):
+    """(L_prev, n_new) of round r (0-based): round 0 brings the T0 prompt tokens into the active
+    context, every later round the T_new tokens generated in the round before."""
+    return (0, T0) if r == 0 else (T0 + T_new * (r - 1), T_new)
+
+
+def interleave(krbar, doc_chunk_off, kvbar, qr, q, k_raw, v, T0: int, T_new: int, rounds: int, k: int,
+               base: float, scale: float | None = None, select=None):
+    """Memory Interleave for one routed layer and one query: `rounds` rounds of route -> attend ->
+    append -> re-route ([P1] §组件 3 Memory Interleaving; [P5] §4 生成式檢索 -> 上下文擴展 -> 生成 ->
+    再檢索; [P2] re-route with the updated context).
+
+    qr [T_total, H, d], q [T_total, hq, d], k_raw / v [T_total, hkv, d] hold every token the query
+    ever has (T_total = T0 + T_new * (rounds - 1)); token j of the active context sits at global
+    position k + j. Round r appends its tokens (interleave_round_tokens) to the local context,
+    routes with ALL active tokens, replaces the memory set with that round's top-k, and the appended
+    tokens attend causally over [selected memory ; local context].
+
+    select: optional list of per-round document indices used for the attention in place of the
+    oracle's own top-k (for comparing against an implementation whose scores may order near-tied
+    documents differently); routing and its scores are computed either way.
+    Returns a list over rounds of (idx [k], scores of idx [k], doc_scores [D], output [n_new, hq, d]).
+    """
+    d = q.shape[-1]
+    scale = 1.0 / np.sqrt(d) if scale is None else scale
+    out = []
+    for r in range(rounds):
+        L_prev, n_new = interleave_round_tokens(r, T0, T_new)
+        L = L_prev + n_new
+        ds, _ = route(krbar, doc_chunk_off, np.asarray(qr)[None, :L])
+        idx, val = topk_docs(ds, k)
+        use = idx[0] if select is None else np.asarray(select[r])
+        mem = gather_memory(kvbar, doc_chunk_off, use)
+        k_local = apply_rope(k_raw[:L], global_positions(k, 0, L), base)
+        q_rot = apply_rope(q[L_prev:L], global_positions(k, L_prev, n_new), base)
+        o = sparse_attention(q_rot, mem[:, 0], mem[:, 1], k_local, v[:L], L_prev, scale)
+        out.append((idx[0], val[0], ds[0], o))
+    return out

@@ -126,8 +126,7 @@ def attn_set_impl(impl: int) -> None:
 
 
 def pool_set_impl(impl: int) -> None:
-    """Chunk-mean pooling: 0 = by size (default), 1 = register streaming, 2 = bulk copy where the layout allows,
-    3 = bulk-copy kernel fed by tensor-map boxes (opt-in; not yet validated on a GPU)."""
+    """Chunk-mean pooling: 0 = by size (default), 1 = register streaming, 2 = bulk copy where the layout allows."""
     check(lib.msa_pool_set_impl(impl), "msa_pool_set_impl")
 
 

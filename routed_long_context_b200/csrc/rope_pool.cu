@@ -90,7 +90,6 @@ struct PoolArgs {
     int rows_per_stage[3];   // token rows of each tensor part per pipeline stage
     int rows_per_copy[3];    // token rows of each tensor part per bulk copy (a stage takes one or more)
     int tab_bytes;           // bytes of one RoPE table row (d/2 cos/sin pairs), staged after rotated rows
-    int tiled;               // 1: token rows by 3D tensor-map boxes of a whole stage; 0: untiled bulk copies
     int n_stages;
     int stage_bytes;
 };
@@ -246,8 +245,7 @@ constexpr int kBulkMaxConsumers = 256;
 
 template <typename TIn, typename TOut>
 __global__ void __launch_bounds__(kBulkMaxConsumers + 32)
-    pool_bulk_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CUtensorMap tm1,
-                     const __grid_constant__ CUtensorMap tm2, const PoolArgs a) {
+    pool_bulk_kernel(const PoolArgs a) {
     constexpr int VEC = 16 / sizeof(TIn);
     extern __shared__ __align__(128) unsigned char pool_smem[];
     const int S = a.n_stages;
@@ -300,20 +298,12 @@ __global__ void __launch_bounds__(kBulkMaxConsumers + 32)
                         if (n_tab < 0) n_tab = 0;
                     }
                     const uint32_t stage_addr = smem_u32(ring + (size_t)p_st * a.stage_bytes);
-                    if (a.tiled) {
-                        // one box of R whole rows [R][E / inner][inner]: row-major in shared memory; rows
-                        // past the item (or the tensor, zero-filled) are copied and never read
-                        const CUtensorMap* tm = it.part == 0 ? &tm0 : (it.part == 1 ? &tm1 : &tm2);
-                        mbar_expect_tx(smem_u32(full + p_st), (uint32_t)(R * row_bytes + n_tab * a.tab_bytes));
-                        tma_load_3d(stage_addr, tm, 0, 0, (int)r0, smem_u32(full + p_st));
-                    } else {
-                        mbar_expect_tx(smem_u32(full + p_st), (uint32_t)(n * row_bytes + n_tab * a.tab_bytes));
-                        const int64_t CR = a.rows_per_copy[it.part];
-                        for (int64_t cr = 0; cr < n; cr += CR) {
-                            const int64_t m = min(CR, n - cr);
-                            bulk_load_evict_first(stage_addr + (uint32_t)(cr * row_bytes), src + (r0 + cr) * E,
-                                                  (uint32_t)(m * row_bytes), smem_u32(full + p_st), pol);
-                        }
+                    mbar_expect_tx(smem_u32(full + p_st), (uint32_t)(n * row_bytes + n_tab * a.tab_bytes));
+                    const int64_t CR = a.rows_per_copy[it.part];
+                    for (int64_t cr = 0; cr < n; cr += CR) {
+                        const int64_t m = min(CR, n - cr);
+                        bulk_load_evict_first(stage_addr + (uint32_t)(cr * row_bytes), src + (r0 + cr) * E,
+                                              (uint32_t)(m * row_bytes), smem_u32(full + p_st), pol);
                     }
                     if (n_tab > 0)
                         bulk_load_evict_first(stage_addr + (uint32_t)(R * row_bytes),
@@ -620,8 +610,7 @@ msa_status launch_pack_tokens(const PackArgs& a, msa_dtype dt, cudaStream_t s) {
 
 namespace {
 
-std::atomic<int> g_pool_impl{0};          // 0: by size, 1: register streaming, 2: bulk copy where the layout allows,
-                                          // 3: the bulk-copy kernel with tensor-map boxes (opt-in)
+std::atomic<int> g_pool_impl{0};          // 0: by size, 1: register streaming, 2: bulk copy where the layout allows
 std::atomic<int> g_pool_stages{0};        // 0: default
 std::atomic<int> g_pool_stage_bytes{0};   // 0: default
 std::atomic<int> g_pool_copy_bytes{0};    // 0: one bulk copy per stage
@@ -631,7 +620,7 @@ constexpr int kBulkStageBytesDefault = 32768;
 // Launches the bulk-copy pooling kernel when every part's row fits a stage and a row needs at most
 // kBulkMaxConsumers threads; *launched tells whether it did.
 template <typename TIn, typename TOut>
-msa_status launch_pool_bulk(PoolArgs a, cudaStream_t s, bool* launched, bool tiled) {
+msa_status launch_pool_bulk(PoolArgs a, cudaStream_t s, bool* launched) {
     constexpr int VEC = 16 / sizeof(TIn);
     *launched = false;
     a.tab_bytes = (a.d / 2) * (int)sizeof(float2);
@@ -654,29 +643,6 @@ msa_status launch_pool_bulk(PoolArgs a, cudaStream_t s, bool* launched, bool til
     if (nc > kBulkMaxConsumers) return MSA_OK;
     a.n_stages = S;
     a.stage_bytes = SB;
-    // tensor maps over each part's token rows: [n_tok][E / inner][inner] with inner = 128 bytes of
-    // elements, one box = R rows (the stage); unused parts keep a zeroed map that no copy reads
-    CUtensorMap tm[3];
-    memset(tm, 0, sizeof(tm));
-    a.tiled = 0;
-    if (tiled) {
-        constexpr int inner = 128 / (int)sizeof(TIn);
-        bool ok = true;
-        for (int i = 0; i < a.n_parts && ok; ++i) {
-            const int part = a.parts[i];
-            const int E = a.heads[part] * a.d;
-            ok = E % inner == 0 && E / inner <= 256 && a.rows_per_stage[part] <= 256;
-        }
-        for (int i = 0; i < a.n_parts && ok; ++i) {
-            const int part = a.parts[i];
-            const uint64_t E = (uint64_t)a.heads[part] * a.d;
-            const uint64_t dims[3] = {(uint64_t)inner, E / inner, (uint64_t)a.n_tok};
-            const uint64_t strides[2] = {128, E * sizeof(TIn)};
-            const uint32_t box[3] = {(uint32_t)inner, (uint32_t)(E / inner), (uint32_t)a.rows_per_stage[part]};
-            MSA_RETURN_IF(make_tensor_map(&tm[part], a.src[part], sizeof(TIn) == 4, 3, dims, strides, box, false));
-        }
-        a.tiled = ok ? 1 : 0;
-    }
     const size_t smem = (size_t)S * SB + 2 * (size_t)S * sizeof(uint64_t) + 16;
     static std::mutex mu;
     static size_t opted[64] = {0};
@@ -699,7 +665,7 @@ msa_status launch_pool_bulk(PoolArgs a, cudaStream_t s, bool* launched, bool til
     const int64_t n_items = a.n_chunks * a.n_parts;
     const int64_t cap = (int64_t)sm_count() * occ;
     const unsigned grid = (unsigned)(n_items < cap ? n_items : cap);
-    pool_bulk_kernel<TIn, TOut><<<grid, nc + 32, smem, s>>>(tm[0], tm[1], tm[2], a);
+    pool_bulk_kernel<TIn, TOut><<<grid, nc + 32, smem, s>>>(a);
     MSA_LAUNCH_CHECK();
     *launched = true;
     return MSA_OK;
@@ -801,8 +767,6 @@ msa_status msa_pool_chunks(const void* k, const void* v, const void* kr, msa_dty
     // which wait on their RoPE table reads, make a tail, and the bulk-copy kernel (table rows staged
     // with the keys, items spread over a persistent grid) is faster.
     int impl = g_pool_impl.load();
-    const bool tiled = impl == 3;
-    if (impl == 3) impl = 2;
     if (impl == 0) {
         int occ = 0;
         MSA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(
@@ -816,13 +780,13 @@ msa_status msa_pool_chunks(const void* k, const void* v, const void* kr, msa_dty
     if (impl == 2) {
         bool launched = false;
         if (in_dt == MSA_BF16 && out_dt == MSA_BF16)
-            MSA_RETURN_IF((launch_pool_bulk<__nv_bfloat16, __nv_bfloat16>(a, s, &launched, tiled)));
+            MSA_RETURN_IF((launch_pool_bulk<__nv_bfloat16, __nv_bfloat16>(a, s, &launched)));
         else if (in_dt == MSA_BF16)
-            MSA_RETURN_IF((launch_pool_bulk<__nv_bfloat16, float>(a, s, &launched, tiled)));
+            MSA_RETURN_IF((launch_pool_bulk<__nv_bfloat16, float>(a, s, &launched)));
         else if (out_dt == MSA_BF16)
-            MSA_RETURN_IF((launch_pool_bulk<float, __nv_bfloat16>(a, s, &launched, tiled)));
+            MSA_RETURN_IF((launch_pool_bulk<float, __nv_bfloat16>(a, s, &launched)));
         else
-            MSA_RETURN_IF((launch_pool_bulk<float, float>(a, s, &launched, tiled)));
+            MSA_RETURN_IF((launch_pool_bulk<float, float>(a, s, &launched)));
         if (launched) return MSA_OK;
     }
     const int64_t cap = 1 << 20;
@@ -841,7 +805,7 @@ msa_status msa_pool_chunks(const void* k, const void* v, const void* kr, msa_dty
 }
 
 msa_status msa_pool_set_impl(int impl) {
-    MSA_REQUIRE(impl >= 0 && impl <= 3, "msa_pool_set_impl: impl must be 0, 1, 2 or 3");
+    MSA_REQUIRE(impl >= 0 && impl <= 2, "msa_pool_set_impl: impl must be 0, 1 or 2");
     g_pool_impl.store(impl);
     return MSA_OK;
 }

@@ -41,12 +41,12 @@ def _rel(got, ref):
 ATTN_BWD_TOL = 1e-2
 
 
-@pytest.mark.parametrize("impl", [0, 2])
+@pytest.mark.parametrize("impl", [0, 2, 3])
 @pytest.mark.parametrize("hq,hkv", [(32, 8), (8, 8), (32, 4)])
 @pytest.mark.parametrize("T,max_mem,mem_lens,q_start", [(13, 40, (0, 5, 37), 7), (64, 140, (130, 64, 1), 0),
                                                         (100, 300, (256, 300, 77), 20)])
 def test_attention_backward_matches_oracle(m, impl, hq, hkv, T, max_mem, mem_lens, q_start):
-    """impl 0: tcgen05 (forward split and dQ), impl 2: mma.sync throughout."""
+    """impl 0: tcgen05 (forward split and dQ), impl 2: mma.sync throughout, impl 3: dK/dV on tcgen05 too."""
     n_q, d, dt = 3, 128, "bf16"
     L = q_start + T
     q = _gen(1, (n_q, T, hq, d), dt)

@@ -323,14 +323,14 @@ def test_interleave_chain_docs_selected_each_round():
         krbar = w.host_tensor(layer, "krbar")
         kv = w.host_tensor(layer, "bank")
         qr, q, kn, vn = w.qr(layer), w.q(layer), w.k_new(layer), w.v_new(layer)
-        for rnd in range(w.rounds):
-            L_prev, tn = w.round_tokens(rnd)
-            for qi in range(w.n_q):
-                idx, val, o = O.route_and_attend(krbar, w.doc_chunk_off, kv, qr[qi, :L_prev + tn],
-                                                 q[qi, L_prev:L_prev + tn], kn[qi], vn[qi], L_prev, w.k, w.rope_base)
+        for qi in range(w.n_q):
+            rounds = O.interleave(krbar, w.doc_chunk_off, kv, qr[qi], q[qi], kn[qi], vn[qi], w.T0, w.T_new, w.rounds,
+                                  w.k, w.rope_base)
+            for rnd, (idx, val, ds, o) in enumerate(rounds):
                 for doc in w.expected(layer, rnd, qi):
                     assert doc in idx, (layer, rnd, qi, doc, idx)
-                assert o.shape == (tn, w.hq, w.d)
+                assert o.shape == (w.round_tokens(rnd)[1], w.hq, w.d)
+                np.testing.assert_array_equal(val, ds[idx])
 
 
 def test_interleave_single_round_is_one_route_and_attend():
@@ -345,6 +345,69 @@ def test_interleave_single_round_is_one_route_and_attend():
     kr = O.apply_rope(kn[0, :8], np.arange(3, 11), 1e6)
     qq = O.apply_rope(q[0, :8], np.arange(3, 11), 1e6)
     np.testing.assert_allclose(o, O.sparse_attention(qq, mem[:, 0], mem[:, 1], kr, vn[0, :8], 0, 0.25), atol=1e-15)
+    # the interleave loop with one round is exactly this route-and-attend
+    (i3, v3, _, o3), = O.interleave(krbar, w.doc_chunk_off, kv, qr[0, :8], q[0, :8], kn[0, :8], vn[0, :8], 8, 4, 1,
+                                    3, 1e6)
+    np.testing.assert_array_equal(i3, idx)
+    np.testing.assert_array_equal(v3, val)
+    np.testing.assert_array_equal(o3, o)
+
+
+def _interleave_case(seed, T0=6, T_new=3, rounds=3, n_docs=30, H=2, d=16, hq=4, hkv=2):
+    r = np.random.default_rng(seed)
+    counts = r.integers(1, 5, n_docs)
+    off = np.concatenate([[0], np.cumsum(counts)])
+    C = int(off[-1])
+    T_total = T0 + T_new * (rounds - 1)
+    return (off, r.standard_normal((C, H, d)), r.standard_normal((C, 2, hkv, d)),
+            r.standard_normal((T_total, H, d)), r.standard_normal((T_total, hq, d)),
+            r.standard_normal((T_total, hkv, d)), r.standard_normal((T_total, hkv, d)))
+
+
+def test_interleave_rounds_are_prefixes_of_one_causal_pass():
+    """With every router token equal, every round selects the same documents; the appended tokens
+    then attend exactly as they would in one causal pass over the whole context: the rounds'
+    outputs, concatenated, equal a single round over all tokens. A wrong global offset, a local
+    context that does not accumulate, or a wrong causal start in a later round breaks this."""
+    off, krbar, kv, qr, q, kn, vn = _interleave_case(31)
+    qr[:] = qr[0]
+    T0, T_new, R, k = 6, 3, 3, 4
+    rounds = O.interleave(krbar, off, kv, qr, q, kn, vn, T0, T_new, R, k, 1e6)
+    (i1, _, _, whole), = O.interleave(krbar, off, kv, qr, q, kn, vn, T0 + T_new * (R - 1), 0, 1, k, 1e6)
+    for idx, _, _, _ in rounds:
+        np.testing.assert_array_equal(idx, i1)
+    np.testing.assert_allclose(np.concatenate([o for *_, o in rounds]), whole, atol=1e-13)
+    assert [o.shape[0] for *_, o in rounds] == [6, 3, 3]
+
+
+def test_interleave_routes_with_every_active_token():
+    """Round r routes with all tokens active so far (the max over tokens runs over a growing set):
+    every document's score, hence the score at each rank of the top-k, never falls from one round
+    to the next; routing with only the appended tokens would break that on random inputs, and a
+    later round's scores are the max of the earlier round's and the appended tokens' own."""
+    off, krbar, kv, qr, q, kn, vn = _interleave_case(32, rounds=4)
+    rounds = O.interleave(krbar, off, kv, qr, q, kn, vn, 6, 3, 4, 5, 1e6)
+    for (ia, va, da, _), (ib, vb, db, _) in zip(rounds[:-1], rounds[1:]):
+        assert np.all(db >= da)
+        assert np.all(vb >= va)
+    for r in range(1, 4):
+        L_prev, n = O.interleave_round_tokens(r, 6, 3)
+        new_only, _ = O.route(krbar, off, qr[None, L_prev:L_prev + n])
+        np.testing.assert_allclose(rounds[r][2], np.maximum(rounds[r - 1][2], new_only[0]), atol=1e-15)
+    assert any(np.any(rounds[r][2] > rounds[r - 1][2]) for r in range(1, 4))
+
+
+def test_interleave_select_override_keeps_routing():
+    """`select` replaces only the documents the attention reads: routing, top-k and scores stay the
+    oracle's, and attending over the oracle's own choice reproduces the default output."""
+    off, krbar, kv, qr, q, kn, vn = _interleave_case(33)
+    base = O.interleave(krbar, off, kv, qr, q, kn, vn, 6, 3, 3, 4, 1e6)
+    same = O.interleave(krbar, off, kv, qr, q, kn, vn, 6, 3, 3, 4, 1e6, select=[b[0] for b in base])
+    other = O.interleave(krbar, off, kv, qr, q, kn, vn, 6, 3, 3, 4, 1e6, select=[[0, 1, 2, 3]] * 3)
+    for b, s_, o_ in zip(base, same, other):
+        np.testing.assert_array_equal(b[3], s_[3])
+        np.testing.assert_array_equal(b[0], o_[0])
+        np.testing.assert_array_equal(b[2], o_[2])
 
 
 @pytest.mark.parametrize("name", ["tiny"])
