@@ -450,6 +450,28 @@ typedef struct msa_interleave_args {
 msa_status msa_interleave_step(const msa_interleave_args* a, void* compute, void* copy, int64_t host_wait_timeout_us);
 msa_status msa_interleave_workspace_size(const msa_interleave_args* a, size_t* bytes);
 
+/* ----------------------------------------------------------------------------------------------
+ * One workspace query for every call that takes a workspace. op names the call, cfg points to the
+ * matching configuration struct below (host memory, read only), *bytes receives the size that
+ * call needs (the same answer as its own *_workspace_size function, which stays available).
+ * Unknown op, NULL cfg or NULL bytes: MSA_ERR_INVALID_ARG; sizes the call itself would refuse:
+ * the same status as its *_workspace_size. Host-only, enqueues nothing. The pages define no
+ * interface; the query exists because the caller owns all scratch memory.
+ * ---------------------------------------------------------------------------------------------- */
+enum {
+    MSA_OP_ROUTE = 1,               /* msa_route_scores          cfg: const msa_route_ws_cfg*     */
+    MSA_OP_TOPK = 2,                /* msa_topk_docs             cfg: const msa_topk_ws_cfg*      */
+    MSA_OP_SPARSE_ATTN_SPLIT = 3,   /* msa_sparse_attn_split     cfg: const msa_attn_ws_cfg*      */
+    MSA_OP_SPARSE_ATTN_BACKWARD = 4,/* msa_sparse_attn_backward  cfg: const msa_attn_ws_cfg*      */
+    MSA_OP_ROUTE_BACKWARD = 5,      /* msa_route_backward        cfg: const msa_route_bwd_ws_cfg* */
+    MSA_OP_INTERLEAVE = 6           /* msa_interleave_step       cfg: const msa_interleave_args*  */
+};
+typedef struct { int n_q, T, H, d; msa_dtype dt; } msa_route_ws_cfg;
+typedef struct { int n_q; int64_t n_docs; int k; } msa_topk_ws_cfg;
+typedef struct { int n_q, T, hq, hkv, max_mem, L; } msa_attn_ws_cfg;
+typedef struct { int64_t n_chunks; int n_q, T, H, d; } msa_route_bwd_ws_cfg;
+msa_status msa_workspace_size(int op, const void* cfg, size_t* bytes);
+
 #ifdef __cplusplus
 }
 #endif

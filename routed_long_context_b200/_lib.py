@@ -33,6 +33,28 @@ class InterleaveArgs(ctypes.Structure):
                 ("ws", vp), ("ws_bytes", sz)]
 
 
+MSA_OP_ROUTE, MSA_OP_TOPK, MSA_OP_SPARSE_ATTN_SPLIT, MSA_OP_SPARSE_ATTN_BACKWARD, MSA_OP_ROUTE_BACKWARD, \
+    MSA_OP_INTERLEAVE = range(1, 7)
+
+
+class RouteWsCfg(ctypes.Structure):
+    _fields_ = [("n_q", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int), ("d", ctypes.c_int), ("dt", i32)]
+
+
+class TopkWsCfg(ctypes.Structure):
+    _fields_ = [("n_q", ctypes.c_int), ("n_docs", i64), ("k", ctypes.c_int)]
+
+
+class AttnWsCfg(ctypes.Structure):
+    _fields_ = [("n_q", ctypes.c_int), ("T", ctypes.c_int), ("hq", ctypes.c_int), ("hkv", ctypes.c_int),
+                ("max_mem", ctypes.c_int), ("L", ctypes.c_int)]
+
+
+class RouteBwdWsCfg(ctypes.Structure):
+    _fields_ = [("n_chunks", i64), ("n_q", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int),
+                ("d", ctypes.c_int)]
+
+
 # name -> (restype, argtypes)
 SIGNATURES = {
     "msa_last_error": (ctypes.c_char_p, []),
@@ -86,6 +108,7 @@ SIGNATURES = {
                                                 ctypes.POINTER(sz)]),
     "msa_interleave_step": (i32, [ctypes.POINTER(InterleaveArgs), vp, vp, i64]),
     "msa_interleave_workspace_size": (i32, [ctypes.POINTER(InterleaveArgs), ctypes.POINTER(sz)]),
+    "msa_workspace_size": (i32, [ctypes.c_int, vp, ctypes.POINTER(sz)]),
 }
 
 

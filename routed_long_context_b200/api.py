@@ -164,6 +164,15 @@ def msa_route_scores(kr_index, chunk_doc, n_docs: int, qr, doc_scores=None, chun
     return (doc_scores, chunk_scores) if chunk_scores is not None else doc_scores
 
 
+def msa_workspace_size(op: int, cfg) -> int:
+    """Workspace bytes of the call named by op (_lib.MSA_OP_*), cfg its ctypes configuration struct
+    (_lib.RouteWsCfg, TopkWsCfg, AttnWsCfg, RouteBwdWsCfg, or the InterleaveArgs of a round)."""
+    n = ctypes.c_size_t(0)
+    check(lib.msa_workspace_size(op, ctypes.cast(ctypes.byref(cfg), ctypes.c_void_p), ctypes.byref(n)),
+          "msa_workspace_size")
+    return n.value
+
+
 def topk_workspace_size(n_q: int, n_docs: int, k: int) -> int:
     n = ctypes.c_size_t(0)
     check(lib.msa_topk_workspace_size(n_q, n_docs, k, ctypes.byref(n)), "msa_topk_workspace_size")

@@ -104,6 +104,36 @@ msa_status msa_rope_table(int64_t max_pos, int d, double base, float* out_host) 
     return MSA_OK;
 }
 
+msa_status msa_workspace_size(int op, const void* cfg, size_t* bytes) {
+    MSA_REQUIRE(cfg != nullptr && bytes != nullptr, "msa_workspace_size: cfg and bytes must not be NULL");
+    switch (op) {
+        case MSA_OP_ROUTE: {
+            const auto* c = static_cast<const msa_route_ws_cfg*>(cfg);
+            return msa_route_workspace_size(c->n_q, c->T, c->H, c->d, c->dt, bytes);
+        }
+        case MSA_OP_TOPK: {
+            const auto* c = static_cast<const msa_topk_ws_cfg*>(cfg);
+            return msa_topk_workspace_size(c->n_q, c->n_docs, c->k, bytes);
+        }
+        case MSA_OP_SPARSE_ATTN_SPLIT: {
+            const auto* c = static_cast<const msa_attn_ws_cfg*>(cfg);
+            return msa_sparse_attn_split_workspace_size(c->n_q, c->T, c->hq, c->hkv, c->max_mem, c->L, bytes);
+        }
+        case MSA_OP_SPARSE_ATTN_BACKWARD: {
+            const auto* c = static_cast<const msa_attn_ws_cfg*>(cfg);
+            return msa_sparse_attn_backward_workspace_size(c->n_q, c->T, c->hq, c->hkv, c->max_mem, c->L, bytes);
+        }
+        case MSA_OP_ROUTE_BACKWARD: {
+            const auto* c = static_cast<const msa_route_bwd_ws_cfg*>(cfg);
+            return msa_route_backward_workspace_size(c->n_chunks, c->n_q, c->T, c->H, c->d, bytes);
+        }
+        case MSA_OP_INTERLEAVE:
+            return msa_interleave_workspace_size(static_cast<const msa_interleave_args*>(cfg), bytes);
+        default:
+            return set_error(MSA_ERR_INVALID_ARG, "msa_workspace_size: unknown op %d", op);
+    }
+}
+
 msa_status msa_chunk_doc_map(const int64_t* doc_chunk_off, int64_t n_docs, int64_t n_chunks, int32_t* chunk_doc,
                              void* stream) {
     MSA_REQUIRE(doc_chunk_off && chunk_doc, "msa_chunk_doc_map: NULL pointer");

@@ -105,6 +105,15 @@ __device__ __forceinline__ void store_f32(T* p, const float* v) {
                 u.z = *reinterpret_cast<uint32_t*>(&c); u.w = *reinterpret_cast<uint32_t*>(&d);
                 *reinterpret_cast<uint4*>(p + i) = u;
             }
+        } else if constexpr (N % 4 == 0) {
+#pragma unroll
+            for (int i = 0; i < N; i += 4) {
+                uint2 u;
+                __nv_bfloat162 a = __floats2bfloat162_rn(v[i], v[i + 1]);
+                __nv_bfloat162 b = __floats2bfloat162_rn(v[i + 2], v[i + 3]);
+                u.x = *reinterpret_cast<uint32_t*>(&a); u.y = *reinterpret_cast<uint32_t*>(&b);
+                *reinterpret_cast<uint2*>(p + i) = u;
+            }
         } else {
 #pragma unroll
             for (int i = 0; i < N; ++i) p[i] = __float2bfloat16_rn(v[i]);

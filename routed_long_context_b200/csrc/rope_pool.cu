@@ -39,6 +39,17 @@ __device__ __forceinline__ void widen(const uint4& u, float* out) {
     }
 }
 
+// Widen an 8-byte word group (4 bf16 or 2 fp32) to fp32.
+template <typename T>
+__device__ __forceinline__ void widen8(const uint2& u, float* out) {
+    if constexpr (sizeof(T) == 4) {
+        out[0] = __uint_as_float(u.x); out[1] = __uint_as_float(u.y);
+    } else {
+        out[0] = __uint_as_float(u.x << 16); out[1] = __uint_as_float(u.x & 0xFFFF0000u);
+        out[2] = __uint_as_float(u.y << 16); out[3] = __uint_as_float(u.y & 0xFFFF0000u);
+    }
+}
+
 __device__ __forceinline__ uint4 shfl_xor_u4(const uint4& u, int m) {
     uint4 r;
     r.x = __shfl_xor_sync(0xffffffffu, u.x, m);
@@ -94,6 +105,107 @@ struct PoolArgs {
     int stage_bytes;
 };
 
+// Rotated keys of one chunk, pair layout: a thread owns F = VEC/2 frequencies of one head, i.e.
+// the F elements of the head's first half and their rotate-half partners F elements later by
+// d/2, read as two 8-byte streams per token, so no lane needs another lane's data. The RoPE table
+// entries (cos, sin) of a batch's positions are loaded together with the batch's key rows, so their
+// latency overlaps the HBM loads. Per element the arithmetic is the one of every other pooling
+// path: x' = x c -+ partner s (fmaf of the product), then acc += x', tokens in order.
+template <typename TIn, typename TOut>
+__device__ __forceinline__ void pool_rotated_pairs(const PoolArgs& a, const TIn* __restrict__ src, int64_t c,
+                                                   int64_t doc_start, int64_t t0, int64_t t1, float inv_n, int E,
+                                                   int passes) {
+    constexpr int VEC = 16 / sizeof(TIn);
+    constexpr int F = VEC / 2;                 // frequencies per thread (8 bytes of keys per half)
+    constexpr int U = 4;                       // tokens per batch
+    const int d = a.d;
+    const int per_head = d / VEC;              // threads per head
+    for (int pass = 0; pass < passes; ++pass) {
+        const int pi = pass * kPoolThreads + threadIdx.x;
+        const bool active = pi * VEC < E;
+        const int h = pi / per_head;
+        const int f0 = (pi % per_head) * F;
+        const int64_t lo = (int64_t)h * d + f0, hi = lo + d / 2;
+        float acc_lo[F], acc_hi[F];
+#pragma unroll
+        for (int j = 0; j < F; ++j) acc_lo[j] = acc_hi[j] = 0.f;
+
+        auto rotate_add = [&](const uint2& rlo, const uint2& rhi, const float4* tab, bool in_table) {
+            float xl[F], xh[F];
+            widen8<TIn>(rlo, xl);
+            widen8<TIn>(rhi, xh);
+            if (in_table) {
+#pragma unroll
+                for (int j = 0; j < F; ++j) {
+                    const float4 w = tab[j / 2];
+                    const float cj = (j & 1) ? w.z : w.x, sj = (j & 1) ? w.w : w.y;
+                    const float l = fmaf(xl[j], cj, -xh[j] * sj);
+                    const float r = fmaf(xh[j], cj, xl[j] * sj);
+                    xl[j] = l;
+                    xh[j] = r;
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < F; ++j) {
+                acc_lo[j] += xl[j];
+                acc_hi[j] += xh[j];
+            }
+        };
+
+        const uint2 z2 = make_uint2(0, 0);
+        const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        int64_t t = t0;
+        for (; t + U <= t1; t += U) {
+            uint2 rl[U], rh[U];
+            float4 tb[U][F / 2];
+            bool ok[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const TIn* row = src + (t + u) * E;
+                rl[u] = active ? __ldcs(reinterpret_cast<const uint2*>(row + lo)) : z2;
+                rh[u] = active ? __ldcs(reinterpret_cast<const uint2*>(row + hi)) : z2;
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int64_t p = t + u - doc_start;
+                ok[u] = p < a.max_pos;
+                const float4* trow = reinterpret_cast<const float4*>(a.cs + p * (d / 2) + f0);
+#pragma unroll
+                for (int j = 0; j < F / 2; ++j) tb[u][j] = (active && ok[u]) ? __ldg(trow + j) : z4;
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (!ok[u] && active) record_device_error(a.err, MSA_DEV_ROPE_POSITION);
+                rotate_add(rl[u], rh[u], tb[u], ok[u]);
+            }
+        }
+        for (; t < t1; ++t) {
+            const TIn* row = src + t * E;
+            const uint2 rl = active ? __ldcs(reinterpret_cast<const uint2*>(row + lo)) : z2;
+            const uint2 rh = active ? __ldcs(reinterpret_cast<const uint2*>(row + hi)) : z2;
+            const int64_t p = t - doc_start;
+            const bool ok = p < a.max_pos;
+            float4 tb[F / 2];
+            const float4* trow = reinterpret_cast<const float4*>(a.cs + p * (d / 2) + f0);
+#pragma unroll
+            for (int j = 0; j < F / 2; ++j) tb[j] = (active && ok) ? __ldg(trow + j) : z4;
+            if (!ok && active) record_device_error(a.err, MSA_DEV_ROPE_POSITION);
+            rotate_add(rl, rh, tb, ok);
+        }
+        if (active) {
+            float ml[F], mh[F];
+#pragma unroll
+            for (int j = 0; j < F; ++j) {
+                ml[j] = acc_lo[j] * inv_n;
+                mh[j] = acc_hi[j] * inv_n;
+            }
+            TOut* dst = static_cast<TOut*>(a.kvbar) + (c * 2) * (int64_t)a.hkv * d;
+            store_f32<TOut, F>(dst + lo, ml);
+            store_f32<TOut, F>(dst + hi, mh);
+        }
+    }
+}
+
 template <typename TIn, typename TOut>
 __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const PoolArgs a) {
     constexpr int VEC = 16 / sizeof(TIn);
@@ -127,63 +239,38 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const PoolArgs a) {
         }
         const float inv_n = 1.0f / (float)(t1 - t0);
 
+        if (rope) {
+            pool_rotated_pairs<TIn, TOut>(a, src, c, doc_start, t0, t1, inv_n, E, passes);
+            continue;
+        }
         for (int pass = 0; pass < passes; ++pass) {
             const int e0 = (pass * kPoolThreads + threadIdx.x) * VEC;
             const bool active = e0 < E;
-            const int ih = e0 % d;
-            const bool first_half = ih < d / 2;
-            const int ci = first_half ? ih : ih - d / 2;
             float acc[VEC];
 #pragma unroll
             for (int j = 0; j < VEC; ++j) acc[j] = 0.f;
 
-            auto consume = [&](const uint4& raw, int64_t t) {
-                float x[VEC];
-                widen<TIn>(raw, x);
-                if (rope) {
-                    uint4 praw = shfl_xor_u4(raw, half_lanes);
-                    float px[VEC];
-                    widen<TIn>(praw, px);
-                    const int64_t p = t - doc_start;
-                    if (p < a.max_pos) {
-                        rotate<VEC>(x, px, a.cs + p * (d / 2), ci, first_half);
-                    } else if (active) {
-                        record_device_error(a.err, MSA_DEV_ROPE_POSITION);
-                    }
-                }
-#pragma unroll
-                for (int j = 0; j < VEC; ++j) acc[j] += x[j];
-            };
-
             const uint4 zero = make_uint4(0, 0, 0, 0);
             int64_t t = t0;
-            if (rope) {
-                // rotated keys: 4 tokens in flight (the rotation's table reads and registers dominate)
-                for (; t + 4 <= t1; t += 4) {
-                    uint4 r[4];
+            // plain streaming: kPoolUnroll tokens in flight
+            for (; t + kPoolUnroll <= t1; t += kPoolUnroll) {
+                uint4 r[kPoolUnroll];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) r[u] = active ? load_stream(src + (t + u) * E + e0) : zero;
+                for (int u = 0; u < kPoolUnroll; ++u) r[u] = active ? load_stream(src + (t + u) * E + e0) : zero;
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) consume(r[u], t + u);
-                }
-            } else {
-                // plain streaming: kPoolUnroll tokens in flight
-                for (; t + kPoolUnroll <= t1; t += kPoolUnroll) {
-                    uint4 r[kPoolUnroll];
+                for (int u = 0; u < kPoolUnroll; ++u) {
+                    float x[VEC];
+                    widen<TIn>(r[u], x);
 #pragma unroll
-                    for (int u = 0; u < kPoolUnroll; ++u) r[u] = active ? load_stream(src + (t + u) * E + e0) : zero;
-#pragma unroll
-                    for (int u = 0; u < kPoolUnroll; ++u) {
-                        float x[VEC];
-                        widen<TIn>(r[u], x);
-#pragma unroll
-                        for (int j = 0; j < VEC; ++j) acc[j] += x[j];
-                    }
+                    for (int j = 0; j < VEC; ++j) acc[j] += x[j];
                 }
             }
             for (; t < t1; ++t) {
                 uint4 r = active ? load_stream(src + t * E + e0) : zero;
-                consume(r, t);
+                float x[VEC];
+                widen<TIn>(r, x);
+#pragma unroll
+                for (int j = 0; j < VEC; ++j) acc[j] += x[j];
             }
 
             float mean[VEC];

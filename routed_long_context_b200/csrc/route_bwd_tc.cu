@@ -7,7 +7,10 @@
 // GEMM view (chunks on M, as in the forward router): D[m][n] = sum_k index[m][k] * qhat[n][k].
 // The fp32 qhat is split exactly into three bf16 terms (hi + mid + lo, each the bf16 rounding of
 // what the previous terms leave), so the bf16 tensor cores see the same fp32 operand the CUDA-core
-// kernel reads; products of two bf16 values are exact in the fp32 accumulator.
+// kernel reads; products of two bf16 values are exact in the fp32 accumulator. Only the operand is
+// exact: the 3 x 4 MMAs per slab add the products in another order than the CUDA-core kernel's fp32
+// dot product, so on tokens whose scores differ by a rounding error the two kernels can pick
+// different best tokens (exact ties still go to the first token in both).
 //
 // One CTA per (128 chunks, 32 tokens, query): warp 0 loads 64-element K slabs of the index tile
 // and of the three qhat terms by TMA (128-byte swizzle) into 4 stages; warp 1 owns 32 TMEM columns

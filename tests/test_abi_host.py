@@ -224,3 +224,39 @@ def test_too_small_workspace_is_refused_before_any_launch(lib):
     n = ctypes.c_size_t(0)
     assert lib.msa_interleave_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0
     assert f"16 < {n.value}" in msg, msg
+
+
+def test_generic_workspace_query_matches_every_per_call_query(lib):
+    """msa_workspace_size(op, cfg) answers what each call's own *_workspace_size answers, and refuses
+    unknown ops and NULL arguments."""
+    from routed_long_context_b200 import _lib as L
+
+    def ws(op, cfg):
+        n = ctypes.c_size_t(0)
+        st = lib.msa_workspace_size(op, ctypes.cast(ctypes.byref(cfg), ctypes.c_void_p), ctypes.byref(n))
+        return st, n.value
+
+    def own(fn, *args):
+        n = ctypes.c_size_t(0)
+        st = fn(*args, ctypes.byref(n))
+        return st, n.value
+
+    assert ws(L.MSA_OP_ROUTE, L.RouteWsCfg(3, 64, 8, 128, 1)) == own(lib.msa_route_workspace_size, 3, 64, 8, 128, 1)
+    assert ws(L.MSA_OP_TOPK, L.TopkWsCfg(32, 97657, 16)) == own(lib.msa_topk_workspace_size, 32, 97657, 16)
+    assert ws(L.MSA_OP_SPARSE_ATTN_SPLIT, L.AttnWsCfg(1, 64, 32, 8, 8064, 64)) == \
+        own(lib.msa_sparse_attn_split_workspace_size, 1, 64, 32, 8, 8064, 64)
+    assert ws(L.MSA_OP_SPARSE_ATTN_BACKWARD, L.AttnWsCfg(1, 512, 32, 8, 128, 512)) == \
+        own(lib.msa_sparse_attn_backward_workspace_size, 1, 512, 32, 8, 128, 512)
+    assert ws(L.MSA_OP_ROUTE_BACKWARD, L.RouteBwdWsCfg(512, 1, 512, 8, 128)) == \
+        own(lib.msa_route_backward_workspace_size, 512, 1, 512, 8, 128)
+    for op, cfg in ((L.MSA_OP_ROUTE, L.RouteWsCfg(3, 64, 8, 128, 1)), (L.MSA_OP_TOPK, L.TopkWsCfg(32, 97657, 16))):
+        assert ws(op, cfg)[0] == 0 and ws(op, cfg)[1] > 0
+    # a size the call itself refuses is refused the same way
+    assert ws(L.MSA_OP_TOPK, L.TopkWsCfg(1, 10, 65))[0] == own(lib.msa_topk_workspace_size, 1, 10, 65)[0] == 1
+    assert ws(L.MSA_OP_ROUTE, L.RouteWsCfg(0, 16, 8, 128, 1))[0] == 1
+    # unknown op, NULL cfg, NULL bytes
+    assert ws(99, L.TopkWsCfg(1, 10, 4))[0] == 1 and b"unknown op" in lib.msa_last_error()
+    n = ctypes.c_size_t(0)
+    assert lib.msa_workspace_size(L.MSA_OP_TOPK, None, ctypes.byref(n)) == 1
+    cfg = L.TopkWsCfg(1, 10, 4)
+    assert lib.msa_workspace_size(L.MSA_OP_TOPK, ctypes.cast(ctypes.byref(cfg), ctypes.c_void_p), None) == 1

@@ -35,10 +35,61 @@ def _rel(got, ref):
     return float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30))
 
 
-# The bf16 attention backward rounds P and dS to bf16 as tensor-core operands (2^-9 relative each)
-# and takes D = rowsum(dO * O) from the bf16 forward output; fp32 accumulation. Per gradient tensor
-# that stays within 1e-2 of the exact result in relative Frobenius norm.
+# The bf16 attention backward rounds P and dS to bf16 as tensor-core operands and takes
+# D = rowsum(dO * O) from the bf16 forward output; everything else is fp32. Per gradient tensor
+# that stays within 1e-2 of the exact result in relative Frobenius norm (the second check).
 ATTN_BWD_TOL = 1e-2
+# Per gradient row (a key's dK or dV, a (token, head)'s dq), the first check. Each bf16-rounded
+# operand (P, dS) carries a relative error of at most u = 2^-8 (bf16 keeps 8 significant bits), and
+# D_t = dO_t . O_t inherits the forward output's error: |dD_t| <= |dO_t| |O_t(GPU) - O_t| by
+# Cauchy-Schwarz (the forward's deviation from the oracle, measured in the test; plus fp32 rounding).
+# By the triangle inequality a row's error is then at most
+#   dV_j : u sum_t P_tj |dO_t|
+#   dK_j : scale sum_t (u |dS_tj| + P_tj |dD_t|) |q_t|,   dq_t : scale sum_j (u |dS_tj| + P_tj |dD_t|) |k_j|
+# (summed over the heads that share a kv head), to first order; the rows are held to twice that
+# (second-order terms, fp32 accumulation over up to ~10^4 terms).
+BF16_U = 2.0 ** -8
+
+
+def attn_bwd_row_bounds(q, mem_k, mem_v, local_k, local_v, q_start, scale, dout, d_err):
+    """First-order error bound of every gradient row of the sparse-attention backward (fp64):
+    (dq [T, hq], dmem_k [M, hkv], dmem_v, dlocal_k [L, hkv], dlocal_v); d_err [T, hq] bounds |dD|."""
+    q, dout = np.asarray(q, np.float64), np.asarray(dout, np.float64)
+    T, hq, d = q.shape
+    hkv = local_k.shape[1] if local_k.shape[0] else mem_k.shape[1]
+    G = hq // hkv
+    M, L = mem_k.shape[0], local_k.shape[0]
+    bq, bk, bv = np.zeros((T, hq)), np.zeros((M + L, hkv)), np.zeros((M + L, hkv))
+    vis = np.ones((T, M + L), dtype=bool)
+    for t in range(T):
+        vis[t, M:] = np.arange(L) <= q_start + t
+    for h in range(hq):
+        g = h // G
+        keys = np.concatenate([mem_k[:, g], local_k[:, g]]).astype(np.float64)
+        vals = np.concatenate([mem_v[:, g], local_v[:, g]]).astype(np.float64)
+        lg = np.where(vis, (q[:, h] @ keys.T) * scale, -np.inf)
+        p = np.exp(lg - lg.max(axis=1, keepdims=True))
+        p /= p.sum(axis=1, keepdims=True)
+        o, do = p @ vals, dout[:, h]
+        ds = p * (do @ vals.T - (do * o).sum(axis=1, keepdims=True))
+        wgt = BF16_U * np.abs(ds) + p * d_err[:, h][:, None]
+        bq[:, h] = scale * (wgt @ np.linalg.norm(keys, axis=1))
+        bk[:, g] += scale * (wgt.T @ np.linalg.norm(q[:, h], axis=1))
+        bv[:, g] += BF16_U * (p.T @ np.linalg.norm(do, axis=1))
+    return bq, bk[:M], bv[:M], bk[M:], bv[M:]
+
+
+def forward_d_error(out_gpu, out_ref, dout):
+    """Bound on |D_t(GPU) - D_t| per (token, head): |dO_t| |O_t(GPU) - O_t| + fp32 rounding."""
+    dn = np.linalg.norm(np.asarray(dout, np.float64), axis=-1)
+    return dn * np.linalg.norm(out_gpu - out_ref, axis=-1) + 2.0 ** -20 * dn * np.linalg.norm(out_ref, axis=-1)
+
+
+def assert_rows_within(got, ref, bound, factor, what):
+    """Every row (last axis) of got within factor * bound[row] of ref."""
+    err = np.linalg.norm(got - ref, axis=-1)
+    worst = float((err / np.maximum(bound, 1e-300)).max()) if err.size else 0.0
+    assert np.all(err <= factor * bound), (what, worst, factor)
 
 
 @pytest.mark.parametrize("impl", [0, 2, 3])
@@ -69,8 +120,13 @@ def test_attention_backward_matches_oracle(m, impl, hq, hkv, T, max_mem, mem_len
         ref = O.sparse_attention_backward(q[qi], mem[qi, :ml, 0], mem[qi, :ml, 1], lk[qi, :L], lv[qi, :L], q_start,
                                           scale, dout[qi])
         got = (_np(dq[qi]), _np(dmem[qi, :ml, 0]), _np(dmem[qi, :ml, 1]), _np(dlk[qi, :L]), _np(dlv[qi, :L]))
-        for name, g, r in zip(("dq", "dmem_k", "dmem_v", "dlocal_k", "dlocal_v"), got, ref):
+        o_ref = O.sparse_attention(q[qi], mem[qi, :ml, 0], mem[qi, :ml, 1], lk[qi, :L], lv[qi, :L], q_start, scale)
+        d_err = forward_d_error(_np(out[qi]), o_ref, dout[qi])
+        bounds = attn_bwd_row_bounds(q[qi], mem[qi, :ml, 0], mem[qi, :ml, 1], lk[qi, :L], lv[qi, :L], q_start, scale,
+                                     dout[qi], d_err)
+        for name, g, r, b in zip(("dq", "dmem_k", "dmem_v", "dlocal_k", "dlocal_v"), got, ref, bounds):
             if r.size:
+                assert_rows_within(g, r, b, 2.0, (qi, name))
                 assert _rel(g, r) <= ATTN_BWD_TOL, (qi, name, _rel(g, r))
         # log-sum-exp of the forward rows
         o_lse = []
@@ -178,6 +234,23 @@ def test_route_backward_matches_oracle(m, dt, impl, n_docs, T):
     finally:
         m.route_set_impl(0)
     rq, rk = O.route_backward(index, off, qr, ds, index_is_unit=True)
+    # fp32 on both sides from the same stored index. Per row (a query token's head, a chunk's head):
+    # the error is a few fp32 roundings of the row's terms before the normalisation's transpose, which
+    # divides by |Q^R_{t,h}| and can cancel almost all of a row (the planted chunk is token 3's own
+    # query): bound = 1e-5 x (sum of the row's |terms|) [/ |Q^R_{t,h}|] + 1e-4 x |row|; a row that
+    # no (query, document) attains stays exactly zero
+    arg_c, arg_t = O.route_argmax(index, off, qr, index_is_unit=True)
+    qh = O.unit(qr.astype(np.float64))
+    mq, mk = np.zeros(qr.shape[:3]), np.zeros(index.shape[:2])
+    for qi in range(n_q):
+        for i in range(n_docs):
+            c_, t_ = arg_c[qi, i], arg_t[qi, i]
+            if c_ >= 0:
+                mq[qi, t_] += abs(ds[qi, i]) * np.linalg.norm(index[c_], axis=-1) / H
+                mk[c_] += abs(ds[qi, i]) * np.linalg.norm(qh[qi, t_], axis=-1) / H
+    bq = 1e-5 * mq / np.linalg.norm(qr.astype(np.float64), axis=-1) + 1e-4 * np.linalg.norm(rq, axis=-1)
+    assert_rows_within(_np(dqr), rq, bq, 1.0, "dqr")
+    assert_rows_within(_np(dkh), rk, 1e-5 * mk + 1e-4 * np.linalg.norm(rk, axis=-1), 1.0, "dk_hat")
     assert _rel(_np(dqr), rq) <= 1e-4 and _rel(_np(dkh), rk) <= 1e-4
     g = _np(dqr)
     assert np.abs(g[0, 3]).max() > 0 and np.abs(g[0, 9]).max() == 0 and np.abs(g[0, T - 2]).max() == 0
@@ -219,21 +292,53 @@ def test_training_loss_gradients_on_a_64k_context(m):
     gi = idx.cpu().numpy()[0]
     assert set(evidence[0].tolist()) <= set(gi.tolist())
 
-    # the chained oracle
+    # the chained oracle; the pooled memory rows, the rotated local queries and keys and the router
+    # index enter it as stored (rounded to bf16, the storage precision of the path), so both sides
+    # attend and route over the same values
+    bf = lambda x: rng.round_to(np.asarray(x, np.float32), "bf16").astype(np.float64)
     kh, vh, krh = (w.host_tensor(0, n) for n in ("k", "v", "kr"))
     kb, vb, krb = O.encode_memory(kh, vh, krh, w.doc_tok_off, w.chunk, w.rope_base)
     qr = w.qr(0)
-    memo = O.gather_memory(np.stack([kb, vb], 1), w.doc_chunk_off, gi)
+    memo = O.gather_memory(np.stack([bf(kb), bf(vb)], 1), w.doc_chunk_off, gi)
     pos = O.global_positions(w.k, 0, T)
-    _, dmk, dmv, _, _ = O.sparse_attention_backward(O.apply_rope(w.q(0)[0], pos, w.rope_base), memo[:, 0], memo[:, 1],
-                                                    O.apply_rope(w.k_new(0)[0], pos, w.rope_base), w.v_new(0)[0], 0,
-                                                    1 / np.sqrt(w.d), W[0])
+    scale = 1 / np.sqrt(w.d)
+    attn_in = (bf(O.apply_rope(w.q(0)[0], pos, w.rope_base)), memo[:, 0], memo[:, 1],
+               bf(O.apply_rope(w.k_new(0)[0], pos, w.rope_base)), w.v_new(0)[0], 0, scale)
+    _, dmk, dmv, _, _ = O.sparse_attention_backward(*attn_in, W[0])
     dbar = O.gather_memory_backward(np.stack([dmk, dmv], 1), w.doc_chunk_off, gi, w.n_chunks)
-    _, g = O.router_aux_loss(O.route(krb, w.doc_chunk_off, qr)[0], [evidence[0].tolist()], tau)
-    stored = rng.round_to(O.unit(krb).astype(np.float32), "bf16").astype(np.float64)   # the index's stored form
+    stored = bf(O.unit(krb))                                                  # the index's stored form
+    ref_ds, _ = O.route(stored, w.doc_chunk_off, qr)
+    _, g = O.router_aux_loss(ref_ds, [evidence[0].tolist()], tau)
     _, dkh = O.route_backward(stored, w.doc_chunk_off, qr, lam * g, index_is_unit=True)
     rk, rv, rkr = O.encode_memory_backward(dbar[:, 0], dbar[:, 1], O.unit_backward(krb, dkh), w.doc_tok_off, w.chunk,
                                            w.rope_base)
     assert _rel(_np(dk), rk) <= ATTN_BWD_TOL
     assert _rel(_np(dv), rv) <= ATTN_BWD_TOL
     assert _rel(_np(dkr), rkr) <= ATTN_BWD_TOL
+
+    # per token row. dK and dV: the chunk's bound from the attention rows of its fetched copies,
+    # divided by the chunk's token count (the pooling's transpose; the rotation keeps norms)
+    d_err = forward_d_error(_np(out[0]), O.sparse_attention(*attn_in), W[0])
+    _, bmk, bmv, _, _ = attn_bwd_row_bounds(*attn_in, W[0], d_err)
+    bbar = O.gather_memory_backward(np.stack([bmk, bmv], 1)[..., None], w.doc_chunk_off, gi, w.n_chunks)[..., 0]
+    _, cb = O.chunk_layout(w.doc_tok_off, w.chunk)
+    tok_chunk = np.repeat(np.arange(len(cb)), cb[:, 1] - cb[:, 0])
+    n_c = (cb[:, 1] - cb[:, 0])[tok_chunk][:, None]
+    for name, got_, ref_, b in (("dk", dk, rk, bbar[:, 0]), ("dv", dv, rv, bbar[:, 1])):
+        assert_rows_within(_np(got_), ref_, 2 * b[tok_chunk] / n_c + 1e-5 * np.linalg.norm(ref_, axis=-1), 1.0, name)
+    # dK^R: the only difference between the sides is the forward scores (bf16 queries in the
+    # router's contraction), |ds(GPU) - ds| <= eps; through the softmax |dg_d| <= 2 p_d eps / (tau^2 n_q),
+    # a chunk's dk_hat per head moves by lam sum_q |dg| / H, the normalisation's transpose divides by
+    # |K-bar^R_{c,h}| and the pooling's by the chunk's token count (fp32 elsewhere: 1e-5 relative)
+    eps = float(np.abs(_np(ds) - ref_ds).max())
+    assert eps <= 2e-3
+    sq = ref_ds / tau
+    p_soft = np.exp(sq - sq.max(axis=1, keepdims=True))
+    p_soft /= p_soft.sum(axis=1, keepdims=True)
+    dg = 2 * p_soft * eps / (tau * tau * ref_ds.shape[0])                    # [n_q, D]
+    arg_c, _ = O.route_argmax(stored, w.doc_chunk_off, qr, index_is_unit=True)
+    bh = np.zeros(w.n_chunks)
+    for qi in range(arg_c.shape[0]):
+        np.add.at(bh, arg_c[qi][arg_c[qi] >= 0], lam * dg[qi][arg_c[qi] >= 0] / w.H)
+    bkr = bh[:, None] / np.linalg.norm(krb, axis=-1)                          # [C, H]
+    assert_rows_within(_np(dkr), rkr, 2 * bkr[tok_chunk] / n_c + 1e-5 * np.linalg.norm(rkr, axis=-1), 1.0, "dkr")

@@ -5,8 +5,9 @@ Some callers of this library cannot allocate device memory at the moment they se
 loop whose memory is reserved up front, a latency-bound loop that cannot take cudaMalloc's
 implicit synchronisation). msa_topk_docs_noalloc serves them from a fixed device array inside the
 library. This file checks, through the C ABI, that it returns what the workspace-based
-msa_topk_docs returns, on consecutive calls that reuse the array, and that it refuses sizes that do
-not fit. It sits last in collection order so a failure here never hides another test's result.
+msa_topk_docs and the oracle return, on consecutive calls that reuse the array, that calls after the
+first take no device memory, and that it refuses sizes that do not fit. It sits last in collection
+order so a failure here never hides another test's result.
 """
 import ctypes
 
@@ -14,6 +15,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle as O
 from msa_inputs import rng
 
 pytestmark = pytest.mark.gpu
@@ -51,7 +53,40 @@ def test_noalloc_topk_matches_workspace_topk_on_consecutive_calls():
         torch.cuda.synchronize()
         assert torch.equal(got_i, ref_i)                          # indices: exact
         assert torch.equal(got_v, ref_v)                          # scores are copied values: exact
+        # and the oracle's selection over the same fp32 scores: descending, ties to the lower index
+        o_i, o_v = O.topk_docs(scores.cpu().numpy().astype(np.float64), k)
+        np.testing.assert_array_equal(got_i.cpu().numpy(), o_i)
+        np.testing.assert_array_equal(got_v.cpu().numpy().astype(np.float64), o_v)
     assert m.device_status() == 0
+
+
+def test_noalloc_topk_leaves_device_memory_unchanged():
+    """After a first call (which may load the library's kernels), further calls take no device
+    memory: the free memory the driver reports is the same before and after them."""
+    from routed_long_context_b200 import _lib
+
+    lib = _lib.lib
+    n_q, n_docs, k = 4, 97657, 16
+    scores = _scores(99, n_q, n_docs)
+    idx = torch.empty((n_q, k), dtype=torch.int32, device="cuda")
+    val = torch.empty((n_q, k), dtype=torch.float32, device="cuda")
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+    def call():
+        st = lib.msa_topk_docs_noalloc(ctypes.c_void_p(scores.data_ptr()), n_q, n_docs, k,
+                                       ctypes.c_void_p(idx.data_ptr()), ctypes.c_void_p(val.data_ptr()), stream)
+        assert st == 0, lib.msa_last_error()
+
+    call()
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(5):
+        call()
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0, (free0, free1)
+    o_i, _ = O.topk_docs(scores.cpu().numpy().astype(np.float64), k)
+    np.testing.assert_array_equal(idx.cpu().numpy(), o_i)
 
 
 def test_noalloc_topk_rejects_sizes_beyond_its_array():
