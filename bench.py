@@ -47,12 +47,16 @@ def parse():
                     help="SMs the routers leave free for the overlapped selection and attention")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="100m", choices=["100m", "encode10m", "interleave", "fine1m", "train64k"],
-                    help="100m: the routing step (the reported metric); encode10m: offline encoding of the "
-                         "10M-token bank (document-wise RoPE + chunk-mean pooling); interleave: three Memory "
-                         "Interleave rounds over a 10M-token bank (tensor-bound routing); fine1m: the token-level "
-                         "fine stage on the 1M-token bank; train64k: a training step (forward + backward) on a "
-                         "64K-token context; the last four are reported separately")
+    ap.add_argument("--no-configs", action="store_true", help="headline line only (no per-configuration entries)")
+    ap.add_argument("--workload", default="100m",
+                    choices=["100m", "tiny", "1m", "encode10m", "decode10m", "interleave", "fine1m", "train64k"],
+                    help="100m: the routing step (the reported metric), with every other configuration under "
+                         "'configs' in the same line; the others print one configuration as a line of its own: "
+                         "tiny and 1m (one-layer step latency), encode10m (offline encoding of the 10M-token bank: "
+                         "document-wise RoPE + chunk-mean pooling), decode10m (32 decode queries over it), "
+                         "interleave (three Memory Interleave rounds over a 10M-token bank, tensor-bound routing), "
+                         "fine1m (the token-level fine stage on the 1M-token bank), train64k (a training step, "
+                         "forward + backward, on a 64K-token context)")
     return ap.parse_args()
 
 
@@ -164,23 +168,31 @@ def oracle_sample(seconds: float, layer: int = 0):
 
 
 def reference_arm(args, rank):
+    """The oracle as the reference arm: every step is a bounded sample of the 100M routing workload
+    (routing + top-k over leading slices of one layer), timed on the host; ms_per_step is that
+    sample's measured time, and the projection to a whole 18-layer step is reported beside it."""
     if rank != 0:
         return
     secs = max(1.0, args.cpu_seconds / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
         oracle_sample(secs)
-    vals, chunks, thr = [], 0, 1
+    vals, step_ms, chunks, thr = [], [], 0, 1
     for _ in range(args.steps):
+        t0 = time.perf_counter()
         v, c, thr = oracle_sample(secs)
+        step_ms.append((time.perf_counter() - t0) * 1e3)
         vals.append(v)
         chunks = c
     value = statistics.median(vals)
-    ms = 781250 * TOKENS_PER_CHUNK / value * 1e3 * args.layers
+    projected = 781250 * TOKENS_PER_CHUNK / value * 1e3 * args.layers
     sample = f"oracle routing + top-k of the first {chunks} chunks of one 100M layer per step (fp64, numpy)"
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.median(step_ms),
+        "ms_per_step_what": "the timed sample of each step (a bounded slice of one layer), wall clock on the host",
+        "projected_full_step_ms": projected,
+        "projected_full_step_what": f"{args.layers} layers x 781,250 chunks at the sample's rate (projection)",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": "100m-routing (781,250 chunks x 18 layers, 64 query tokens, top-16)",
                    "sample": sample},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": thr, "kind": "oracle", "sample": sample},
@@ -188,66 +200,416 @@ def reference_arm(args, rank):
     }))
 
 
-# ---------------------------------------------------------------------------------------------- encode
-def encode_bench(args, rank, world, local_rank):
-    """Offline encoding of the 10M-token configuration: 9,766 docs x 1024 tokens, chunk 256, bf16 token-level
-    K, V, K^R [10,000,384 x 8 x 128] (61.4 GB read) -> pooled K-bar/V-bar and unit-vector router index."""
+# ---------------------------------------------------------------------------------------------- configurations
+# Every configuration of the measured workload set, each reported with its own roofline, the fp64
+# oracle timed on the host cores on a bounded sample, and an end-to-end figure through the public API
+# with host buffers. The default run puts them under "configs" in the one JSON line; `--workload X`
+# prints one of them as a line of its own.
+def all_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return {"hbm": float(p["hbm_gbs"]), "bf16": float(p["bf16_tflops"]),
+                "bf16_sustained": float(p["bf16_tflops_sustained"]), "kind": "measured"}
+    except Exception:
+        return {"hbm": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "kind": "fallback"}
+
+
+def _ev():
     import torch
 
+    return torch.cuda.Event(enable_timing=True)
+
+
+def device_ms(fn, steps: int, warmup: int, stream) -> float:
+    """Mean ms per call of fn (which launches on `stream`), CUDA events around `steps` calls."""
+    import torch
+
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    a, b = _ev(), _ev()
+    a.record(stream)
+    for _ in range(steps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / steps
+
+
+def cpu_seconds(fn, min_s: float, max_reps: int) -> float:
+    """Seconds per call of fn on the host: repeated until min_s have passed or max_reps calls."""
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        fn()
+        n += 1
+        dt = time.perf_counter() - t0
+        if dt >= min_s or n >= max_reps:
+            return dt / n
+
+
+def oracle_threads() -> int:
+    from threadpoolctl import threadpool_info
+
+    return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+
+
+def _free():
+    import torch
+
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+def _pinned_like(t):
+    import torch
+
+    h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+    h.copy_(t)
+    return h
+
+
+class OneLayerRound:
+    """One routed layer of a token-level configuration as one interleave round through the public
+    API (append + global RoPE, routing, top-k, fetch from the pinned host bank, attention), plus the
+    pinned host copies of its query-side inputs and output for the end-to-end figure."""
+
+    def __init__(self, m, w, lay, index, bank, cs, fetch_mode=1):
+        import torch
+
+        from msa_inputs.device import TORCH_DT, small_tensors
+
+        dt = TORCH_DT[w.dtype]
+        self.w, self.m = w, m
+        self.dv = small_tensors(w, 0)
+        self.local = (torch.zeros((w.n_q, w.T_total, w.hkv, w.d), dtype=dt, device="cuda"),
+                      torch.zeros((w.n_q, w.T_total, w.hkv, w.d), dtype=dt, device="cuda"))
+        self.out = torch.empty((w.n_q, w.T0, w.hq, w.d), dtype=dt, device="cuda")
+        self.idx_host = torch.empty((w.n_q, w.k), dtype=torch.int32, pin_memory=True)
+        la = [dict(kr_index=index, host_bank=bank, qr=self.dv["qr"], q_new=self.dv["q"], k_new=self.dv["k_new"],
+                   v_new=self.dv["v_new"], local_k=self.local[0], local_v=self.local[1], out=self.out,
+                   topk_idx_host=self.idx_host)]
+        self.rd = m.InterleaveRound(la, n_chunks=lay.n_chunks, n_docs=lay.n_docs, doc_chunk_off=lay.doc_chunk_off,
+                                    doc_chunk_off_host=lay.doc_chunk_off_host, chunk_doc=lay.chunk_doc, n_q=w.n_q,
+                                    H=w.H, d=w.d, hq=w.hq, hkv=w.hkv, k=w.k, L_prev=0, T_new=w.T0,
+                                    new_q_stride=w.T_total, L_max=w.T_total, max_mem=w.max_mem, cos_sin=cs,
+                                    dtype=dt, fetch_mode=fetch_mode)
+        self.names = ("qr", "q", "k_new", "v_new")
+        self.h_in = [_pinned_like(self.dv[n]) for n in self.names]
+        self.h_out = torch.empty(self.out.shape, dtype=dt, pin_memory=True)
+        self.compute, self.copy = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def step(self, route_events=None):
+        self.rd.run(self.compute, self.copy, route_events=route_events)
+
+    def device(self, steps, warmup):
+        """(ms per step, router ms per launch) on the compute stream."""
+        import torch
+
+        for _ in range(warmup):
+            self.step()
+        torch.cuda.synchronize()
+        evs = [[_ev(), _ev()] for _ in range(steps)]
+        for e in evs:
+            e[0].record(self.compute)
+            e[1].record(self.compute)
+        torch.cuda.synchronize()
+        a, b = _ev(), _ev()
+        a.record(self.compute)
+        for i in range(steps):
+            self.step(route_events=evs[i])
+        b.record(self.compute)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / steps, sum(e[0].elapsed_time(e[1]) for e in evs) / steps
+
+    def e2e(self, steps, warmup):
+        """ms per step with the step's query-side inputs copied host -> device before it and its output
+        read back after it, serialised on the compute stream (latency, no overlap between steps)."""
+        import torch
+
+        def one():
+            with torch.cuda.stream(self.compute):
+                for h, n in zip(self.h_in, self.names):
+                    self.dv[n].copy_(h, non_blocking=True)
+            self.step()
+            with torch.cuda.stream(self.compute):
+                self.h_out.copy_(self.out, non_blocking=True)
+
+        ms = device_ms(one, steps, warmup, self.compute)
+        h2d = sum(h.numel() * h.element_size() for h in self.h_in)
+        d2h = self.h_out.numel() * self.h_out.element_size() + self.idx_host.numel() * 4
+        return ms, h2d, d2h
+
+
+def _oracle_pool_router(w, docs, group=64):
+    """fp64 oracle K-bar^R of the given documents' chunks (host-regenerated tokens), in doc order."""
+    import concurrent.futures as cf
+
+    import numpy as np
+
+    import oracle as O
+
+    def one(g):
+        d0, d1 = g
+        a, b = int(w.doc_tok_off[d0]), int(w.doc_tok_off[d1])
+        x = w.host_rows(0, "kr", np.arange(a, b)).reshape(b - a, w.H, w.d)
+        return O.encode_memory(None, None, x, w.doc_tok_off[d0:d1 + 1] - a, w.chunk, w.rope_base)[2]
+
+    groups = [(d0, min(docs, d0 + group)) for d0 in range(0, docs, group)]
+    with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
+        return np.concatenate(list(ex.map(one, groups)))
+
+
+def _oracle_kv_of_docs(w, docs):
+    """{doc: (K-bar, V-bar)} by the fp64 oracle (document-wise RoPE + pooling) from host tokens."""
+    import numpy as np
+
+    import oracle as O
+
+    out = {}
+    for doc in docs:
+        a, b = int(w.doc_tok_off[doc]), int(w.doc_tok_off[doc + 1])
+        t = {n: w.host_rows(0, n, np.arange(a, b)).reshape(b - a, w.hkv, w.d) for n in ("k", "v")}
+        kb, vb, _ = O.encode_memory(t["k"], t["v"], None, np.array([0, b - a]), w.chunk, w.rope_base)
+        out[int(doc)] = (kb, vb)
+    return out
+
+
+def _oracle_step_fn(w, krb, kv_of, n_chunks_scale=1.0):
+    """The oracle's one-layer step (route -> top-k -> gather -> global RoPE -> attention) for every
+    query of w over pooled router keys krb (a leading slice of the bank when n_chunks_scale > 1)."""
+    import numpy as np
+
+    import oracle as O
+
+    qr, qa, kn, vn = w.qr(0)[:, :w.T0], w.q(0), w.k_new(0), w.v_new(0)
+    off = w.doc_chunk_off[:np.searchsorted(w.doc_chunk_off, krb.shape[0]) + 1]
+    pos = O.global_positions(w.k, 0, w.T0)
+
+    def step():
+        ds, _ = O.route(krb, off, qr)
+        idx, _ = O.topk_docs(ds, w.k)
+        for q in range(w.n_q):
+            docs = [d for d in idx[q] if int(d) in kv_of] or list(kv_of)[:w.k]
+            kb = np.concatenate([kv_of[int(d)][0] for d in docs])
+            vb = np.concatenate([kv_of[int(d)][1] for d in docs])
+            O.sparse_attention(O.apply_rope(qa[q, :w.T0], pos, w.rope_base), kb, vb,
+                               O.apply_rope(kn[q, :w.T0], pos, w.rope_base), vn[q, :w.T0], 0, 1 / np.sqrt(w.d))
+    return step
+
+
+def _round_entry(name, metric, w, lay, rb, steps, warmup, pk, route_kind, notes, cpu):
+    """Entry of a one-layer round configuration: device step latency, router roofline, e2e, oracle."""
+    ms, route_ms = rb.device(steps, warmup)
+    e_ms, h2d, d2h = rb.e2e(steps, warmup)
+    elem = 4 if w.dtype == "f32" else 2
+    route_bytes = lay.n_chunks * w.H * w.d * elem
+    route_flops = 2.0 * w.H * w.d * lay.n_chunks * w.n_q * w.T0
+    if route_kind == "tensor":
+        ach = route_flops / (route_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": pk["bf16"], "unit": "TFLOP/s", "frac": ach / pk["bf16"],
+                "traffic": None, "kernel": "route_tc_kernel", "peak_kind": f"{pk['kind']} bf16 burst (cuBLAS)"}
+    else:
+        ach = route_bytes / (route_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": pk["hbm"], "unit": "GB/s", "frac": ach / pk["hbm"],
+                "traffic": None, "kernel": "route_simt_kernel" if w.dtype == "f32" else "route_tc_kernel",
+                "peak_kind": f"{pk['kind']} copy bandwidth"}
+    roof["note"] = notes
+    sel = rb.idx_host.numpy()
+    planted_ok = all(set(w.expected(0, 0, q)) <= set(sel[q].tolist()) for q in range(w.n_q))
+    return {"workload": name, "metric": metric, "value": ms * 1e3, "unit": "us per step", "higher_is_better": False,
+            "ms_per_step": ms, "steps": steps, "route_us_per_launch": route_ms * 1e3, "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e_ms * 1e3, "unit": "us per step", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "how": "public API (msa_interleave_step) with pinned host buffers: the step's query-side inputs "
+                           "copied in and its output read back inside the timed region, serialised (latency)"},
+            "checks": {"planted_docs_selected": planted_ok, "device_status": rb.m.device_status()}}
+
+
+def cfg_tiny(args, pk):
+    import numpy as np
+
+    import oracle as O
     import routed_long_context_b200 as m
     from msa_inputs import workloads
     from msa_inputs.device import memory_tensor
-    from routed_long_context_b200.bank import BankLayout, encode_tokens
+    from routed_long_context_b200.bank import BankLayout, encode_tokens, to_host_bank
 
-    torch.cuda.set_device(local_rank)
-    w = workloads.mem_10m(n_docs=9766 if args.n_docs == 97657 else args.n_docs)
+    w = workloads.tiny()
+    lay = BankLayout.from_doc_lengths(w.doc_len, w.chunk)
+    cs = m.rope_table(4096, w.d, w.rope_base)
+    k, v, kr = (memory_tensor(w, 0, n) for n in ("k", "v", "kr"))
+    kvbar, index = encode_tokens(lay, k, v, kr, w.chunk, cs)
+    del k, v, kr
+    rb = OneLayerRound(m, w, lay, index, to_host_bank(kvbar), cs, args.fetch_mode)
+    # the oracle's step on the full bank (pooling is the offline stage, outside the step)
+    kh, vh, krh = (w.host_tensor(0, n) for n in ("k", "v", "kr"))
+    kb, vb, krb = O.encode_memory(kh, vh, krh, w.doc_tok_off, w.chunk, w.rope_base)
+    kv_of = {d: (kb[w.doc_chunk_off[d]:w.doc_chunk_off[d + 1]], vb[w.doc_chunk_off[d]:w.doc_chunk_off[d + 1]])
+             for d in range(w.n_docs)}
+    cpu_s = cpu_seconds(_oracle_step_fn(w, krb, kv_of), 2.0, 200)
+    cpu = {"value": cpu_s * 1e6, "unit": "us per step", "cores": oracle_threads(), "kind": "oracle",
+           "sample": "the whole step (route over all 512 chunks, top-4, gather, attention), fp64"}
+    e = _round_entry("tiny: 64 docs x 1024 tokens (65,536), chunk 128, fp32; 1 query x 16 tokens, top-4, GQA 32/8, "
+                     "16 causal local tokens", "tiny: route + top-4 + fetch + attention, one layer", w, lay, rb,
+                     min(args.steps, 200), args.warmup, pk, "hbm",
+                     "latency-bound: a 2 MB fp32 index (L2-resident) and tens of microseconds of launches", cpu)
+    del rb, kvbar, index
+    _free()
+    return e
+
+
+def cfg_1m(args, pk):
+    import numpy as np
+
+    import oracle as O
+    import routed_long_context_b200 as m
+    from msa_inputs import workloads
+    from msa_inputs.device import memory_tensor
+    from routed_long_context_b200.bank import BankLayout, encode_tokens, to_host_bank
+
+    w = workloads.mem_1m()
+    lay = BankLayout.from_doc_lengths(w.doc_len, w.chunk)
+    cs = m.rope_table(4096, w.d, w.rope_base)
+    k, v, kr = (memory_tensor(w, 0, n) for n in ("k", "v", "kr"))
+    kvbar, index = encode_tokens(lay, k, v, kr, w.chunk, cs)
+    del k, v, kr
+    _free()
+    rb = OneLayerRound(m, w, lay, index, to_host_bank(kvbar), cs, args.fetch_mode)
+    # oracle: the pooled router index of the whole bank (untimed offline stage), K-bar/V-bar of the
+    # documents its own routing selects; the timed step routes over every chunk
+    krb = _oracle_pool_router(w, w.n_docs)
+    ds, _ = O.route(krb, w.doc_chunk_off, w.qr(0)[:, :w.T0])
+    sel, _ = O.topk_docs(ds, w.k)
+    cpu_s = cpu_seconds(_oracle_step_fn(w, krb, _oracle_kv_of_docs(w, sel[0])), 2.0, 20)
+    cpu = {"value": cpu_s * 1e6, "unit": "us per step", "cores": oracle_threads(), "kind": "oracle",
+           "sample": f"the whole step (route over all {lay.n_chunks:,} chunks, top-8, gather, attention), fp64"}
+    e = _round_entry(f"1m: {w.n_docs} docs ({w.n_tok:,} tokens, 128..1792), chunk 128, bf16; 1 query x 64 tokens, "
+                     "top-8, GQA 32/8", "1M: route + top-8 + fetch + attention, one layer", w, lay, rb,
+                     min(args.steps, 200), args.warmup, pk, "tensor",
+                     "16 MB index, L2-resident: the router runs at tensor and launch speed, not HBM", cpu)
+    del rb, kvbar, index
+    _free()
+    return e
+
+
+# DRAM bytes (read + write) of pool_kernel per launch on the 10M encode: None until an ncu capture of
+# the current kernel (a 400-document case, scaled by documents) is recorded here.
+POOL_TRAFFIC_10M = None
+
+
+def cfg_10m(args, pk):
+    """Two entries: the offline encode (61.4 GB through document-wise RoPE + pooling) and the decode
+    step (32 queries x 1 token routed over 39,064 chunks, top-16, per-query fetch of 8.4 MB from the
+    pinned host bank, attention)."""
+    import numpy as np
+
+    import oracle as O
+    import routed_long_context_b200 as m
+    from msa_inputs import workloads
+    from msa_inputs.device import memory_tensor
+    from routed_long_context_b200.bank import BankLayout, to_host_bank
+
+    import torch
+
+    w = workloads.mem_10m(n_docs=9766 if args.n_docs == 97657 else args.n_docs)    # fewer: a small capture case
     lay = BankLayout.from_doc_lengths(w.doc_len, w.chunk)
     cs = m.rope_table(4096, w.d, w.rope_base)
     k, v, kr = (memory_tensor(w, 0, n) for n in ("k", "v", "kr"))
     kvbar = torch.empty((lay.n_chunks, 2, w.hkv, w.d), dtype=torch.bfloat16, device="cuda")
     index = torch.empty((lay.n_chunks, w.H, w.d), dtype=torch.bfloat16, device="cuda")
     s = torch.cuda.current_stream()
-    for _ in range(args.warmup):
+
+    def encode():
         m.msa_pool_chunks(k, v, kr, lay.doc_tok_off, lay.doc_chunk_off, lay.chunk_doc, w.chunk, cos_sin=cs,
                           kvbar=kvbar, kr_index=index)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    with ClockSampler(local_rank) as clk:
-        e0.record(s)
-        for _ in range(args.steps):
-            m.msa_pool_chunks(k, v, kr, lay.doc_tok_off, lay.doc_chunk_off, lay.chunk_doc, w.chunk, cos_sin=cs,
-                              kvbar=kvbar, kr_index=index)
-        e1.record(s)
-        torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / args.steps
+
+    steps = max(3, min(args.steps, 10))
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        enc_ms = device_ms(encode, steps, args.warmup, s)
     read = 3 * w.n_tok * w.H * w.d * 2
     write = lay.n_chunks * 3 * w.H * w.d * 2
-    gbs = (read + write) / (ms / 1e3) / 1e9
-    peak, kind = peaks()
-    if rank == 0:
-        print(json.dumps({
-            "metric": "10M-token offline encode (doc-wise RoPE + chunk-mean pooling) throughput", "value": w.n_tok / (ms / 1e3),
-            "unit": "memory tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-            "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": f"encode10m: {w.n_docs:,} docs x 1024 tokens, chunk 256, K/V/K^R bf16 "
-                                   f"[{w.n_tok:,} x 8 x 128]"},
-            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
-                         "traffic": None, "kernel": "pool_kernel", "peak_kind": kind},
-            "clocks": clk.summary(), "device_status": m.device_status()}))
+    gbs = (read + write) / (enc_ms / 1e3) / 1e9
+    del k, v, kr
+    _free()
+    # oracle: document-wise RoPE + pooling of K, V, K^R of the first 16 documents (16,384 tokens)
+    n_s = 16
+
+    def oracle_encode():
+        a, b = 0, int(w.doc_tok_off[n_s])
+        t = {n: w.host_rows(0, n, np.arange(a, b)).reshape(b - a, -1, w.d) for n in ("k", "v", "kr")}
+        O.encode_memory(t["k"], t["v"], t["kr"], w.doc_tok_off[:n_s + 1], w.chunk, w.rope_base)
+
+    enc_cpu = cpu_seconds(oracle_encode, 3.0, 5)
+    encode_entry = {
+        "workload": f"10m encode: {w.n_docs:,} docs x 1024 tokens, chunk 256, K/V/K^R bf16 [{w.n_tok:,} x 8 x 128]",
+        "metric": "10M offline encode (document-wise RoPE + chunk-mean pooling) throughput",
+        "value": w.n_tok / (enc_ms / 1e3), "unit": "memory tokens/s", "higher_is_better": True, "ms_per_step": enc_ms,
+        "steps": steps,
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s", "frac": gbs / pk["hbm"],
+                     "traffic": POOL_TRAFFIC_10M if w.n_docs == 9766 else None, "kernel": "pool_kernel",
+                     "peak_kind": f"{pk['kind']} copy bandwidth", "bytes": read + write},
+        "cpu_baseline": {"value": n_s * 1024 / enc_cpu, "unit": "memory tokens/s", "cores": oracle_threads(),
+                         "kind": "oracle", "sample": f"fp64 oracle encode of the first {n_s} documents "
+                                                     f"({n_s * 1024:,} tokens, generation included)"},
+        "e2e": None,
+        "e2e_note": "the encode's inputs are the model's token-level K/V/K^R, produced on the device; with them "
+                    "on the host the step is the 61.4 GB host->device copy",
+        "clocks": clk.summary(), "checks": {"device_status": m.device_status()}}
+
+    # decode: one round of 32 independent queries x 1 token over the pooled bank
+    host_bank = to_host_bank(kvbar)
+    rb = OneLayerRound(m, w, lay, index, host_bank, cs, args.fetch_mode)
+    entry = _round_entry("10m decode: 39,064 chunks (chunk 256), 32 queries x 1 decode token, top-16, per-query "
+                         "fetch from the pinned host bank", "10M decode: route + top-16 + fetch + attention, "
+                         "32 queries", w, lay, rb, min(args.steps, 200), args.warmup, pk, "hbm",
+                         "80 MB index per step (32 columns: HBM-bound); the fetch reads 8.4 MB over the host link",
+                         None)
+    # the fetch alone, over the host link, against a pinned copy measured in this process
+    idx_dev = torch.from_numpy(rb.idx_host.numpy().copy()).cuda()
+    mem = torch.empty((w.n_q, w.max_mem, 2, w.hkv, w.d), dtype=torch.bfloat16, device="cuda")
+    mem_len = torch.empty(w.n_q, dtype=torch.int32, device="cuda")
+    f_ms = device_ms(lambda: m.msa_gather_kv_device(host_bank, lay.doc_chunk_off, idx_dev, w.max_mem, dev_mem_kv=mem,
+                                                    mem_len=mem_len), min(args.steps, 100), args.warmup, s)
+    f_bytes = int(mem_len.sum().item()) * 2 * w.hkv * w.d * 2
+    link = host_link_gbs()
+    entry["fetch"] = {"bound": "host-link", "achieved": f_bytes / (f_ms / 1e3) / 1e9, "peak": link, "unit": "GB/s",
+                      "frac": f_bytes / (f_ms / 1e3) / 1e9 / link, "bytes": f_bytes, "us": f_ms * 1e3,
+                      "kernel": "gather_device_kernel",
+                      "peak_kind": "pinned host->device copy of 1 GiB measured in this process"}
+    # oracle: route the 32 decode tokens over the chunks of the first 1,024 documents (4,096 chunks),
+    # projected to the whole bank by chunks, plus top-16, gather and attention for every query
+    n_d = min(1024, w.n_docs)
+    krb = _oracle_pool_router(w, n_d)
+    kv_of = _oracle_kv_of_docs(w, range(w.k))
+    step = _oracle_step_fn(w, krb, kv_of)
+    t_all = cpu_seconds(step, 2.0, 5)
+    qr = w.qr(0)[:, :1]
+    off = w.doc_chunk_off[:n_d + 1]
+    t_route = cpu_seconds(lambda: O.route(krb, off, qr), 1.0, 5)
+    proj = t_all + t_route * (lay.n_chunks / krb.shape[0] - 1)
+    entry["cpu_baseline"] = {"value": proj * 1e6, "unit": "us per step", "cores": oracle_threads(), "kind": "oracle",
+                             "sample": f"fp64 oracle step over the chunks of the first {n_d:,} documents "
+                                       f"({krb.shape[0]:,} chunks; {t_all * 1e6:.0f} us), its routing part scaled "
+                                       f"by chunks to all {lay.n_chunks:,} (projection)"}
+    del rb, mem, host_bank, kvbar, index
+    _free()
+    return encode_entry, entry
 
 
-# ---------------------------------------------------------------------------------------------- interleave
-def interleave_bench(args, rank, world, local_rank):
+def cfg_interleave(args, pk):
     """Three Memory Interleave rounds (64 + 32 + 32 tokens per query, 8 queries) over a 10M-token
     pre-pooled bank (78,128 chunks of 128) and 18 routed layers; one step = the three rounds."""
+    import numpy as np
     import torch
 
+    import oracle as O
     import routed_long_context_b200 as m
     from msa_inputs import workloads
     from msa_inputs.device import memory_tensor, small_tensors
     from routed_long_context_b200.bank import BankLayout, index_from_prepooled
 
-    torch.cuda.set_device(local_rank)
     w = workloads.interleave(layers=args.layers, n_host_banks=args.host_banks)
     lay = BankLayout(w.doc_chunks)
     cs = m.rope_table(4096, w.d, w.rope_base)
@@ -256,13 +618,9 @@ def interleave_bench(args, rank, world, local_rank):
     banks = []
     for s_ in range(w.n_host_banks):
         dev = memory_tensor(w, s_, "bank")
-        h = torch.empty(dev.shape, dtype=dt, pin_memory=True)
-        h.copy_(dev)
-        banks.append(h)
+        banks.append(_pinned_like(dev))
         del dev
     small = [small_tensors(w, l) for l in range(w.layers)]
-    qr_round = [[small[l]["qr"][:, :w.round_tokens(r)[0] + w.round_tokens(r)[1]].contiguous() for r in range(w.rounds)]
-                for l in range(w.layers)]
     local = [(torch.zeros((w.n_q, w.T_total, w.hkv, w.d), dtype=dt, device="cuda"),
               torch.zeros((w.n_q, w.T_total, w.hkv, w.d), dtype=dt, device="cuda")) for _ in range(w.layers)]
     outs = [[torch.empty((w.n_q, w.round_tokens(r)[1], w.hq, w.d), dtype=dt, device="cuda") for r in range(w.rounds)]
@@ -270,6 +628,17 @@ def interleave_bench(args, rank, world, local_rank):
     idx_host = [[torch.empty((w.n_q, w.k), dtype=torch.int32, pin_memory=True) for _ in range(w.rounds)]
                 for _ in range(w.layers)]
     compute, copy = torch.cuda.Stream(), torch.cuda.Stream()
+    # the routing queries of round r are the first L_prev + n_new tokens: a contiguous copy per round
+    qr_round = [[torch.empty((w.n_q, sum(w.round_tokens(r)), w.H, w.d), dtype=dt, device="cuda")
+                 for r in range(w.rounds)] for _ in range(w.layers)]
+
+    def refresh_qr():
+        for l in range(w.layers):
+            for r in range(w.rounds):
+                qr_round[l][r].copy_(small[l]["qr"][:, :qr_round[l][r].shape[1]])
+
+    with torch.cuda.stream(compute):
+        refresh_qr()
     rounds = []
     for r in range(w.rounds):
         L_prev, tn = w.round_tokens(r)
@@ -282,54 +651,93 @@ def interleave_bench(args, rank, world, local_rank):
                                         H=w.H, d=w.d, hq=w.hq, hkv=w.hkv, k=w.k, L_prev=L_prev, T_new=tn,
                                         new_q_stride=w.T_total, L_max=w.T_total, max_mem=w.max_mem, cos_sin=cs,
                                         dtype=dt, fetch_mode=args.fetch_mode))
+    steps = max(3, min(args.steps, 20))
     for _ in range(args.warmup):
         for rd in rounds:
             rd.run(compute, copy)
     torch.cuda.synchronize()
     chain_ok = all(set(w.expected(l, r, q)) <= set(idx_host[l][r][q].tolist())
                    for l in range(w.layers) for r in range(w.rounds) for q in range(w.n_q))
-    route_ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(2 * w.layers)] for _ in range(w.rounds)]
-                for _ in range(args.steps)]
+    route_ev = [[[_ev() for _ in range(2 * w.layers)] for _ in range(w.rounds)] for _ in range(steps)]
     for a in route_ev:
         for b in a:
             for e in b:
                 e.record(compute)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0, e1 = _ev(), _ev()
     torch.cuda.synchronize()
-    with ClockSampler(local_rank) as clk:
+    with ClockSampler(torch.cuda.current_device()) as clk:
         e0.record(compute)
-        for i in range(args.steps):
+        for i in range(steps):
             for r, rd in enumerate(rounds):
                 rd.run(compute, copy, route_events=route_ev[i][r])
         e1.record(compute)
         torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / args.steps
-    # router FLOPs per launch: 2 * (H*d) * chunks * (n_q * routing tokens of the round)
+    ms = e0.elapsed_time(e1) / steps
     flops = [2.0 * w.H * w.d * lay.n_chunks * w.n_q * sum(w.round_tokens(r)) for r in range(w.rounds)]
-    rms = [sum(route_ev[i][r][2 * l].elapsed_time(route_ev[i][r][2 * l + 1]) for i in range(args.steps)
-               for l in range(w.layers)) / (args.steps * w.layers) for r in range(w.rounds)]
+    rms = [sum(route_ev[i][r][2 * l].elapsed_time(route_ev[i][r][2 * l + 1]) for i in range(steps)
+               for l in range(w.layers)) / (steps * w.layers) for r in range(w.rounds)]
     tflops = [f / (t / 1e3) / 1e12 for f, t in zip(flops, rms)]
-    try:
-        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-            peak, kind = float(json.load(f)["bf16_tflops_sustained"]), "measured sustained bf16 (cuBLAS)"
-    except Exception:
-        peak, kind = 1400.0, "fallback sustained bf16"
-    if rank == 0:
-        tokens = lay.n_chunks * TOKENS_PER_CHUNK * w.layers * w.rounds
-        print(json.dumps({
-            "metric": "Memory Interleave: memory tokens routed/s (3 rounds x 18 layers over a 10M-token bank)",
-            "value": tokens / (ms / 1e3), "unit": "memory tokens/s", "n_gpus": 1, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "interleave: 78,128 chunks x 18 layers, 8 queries, 64/96/128 routing tokens, top-12"},
-            "route_ms_per_layer_by_round": rms, "route_tflops_by_round": tflops,
-            "roofline": {"bound": "tensor", "achieved": tflops[-1], "peak": peak, "unit": "TFLOP/s",
-                         "frac": tflops[-1] / peak, "traffic": None, "kernel": "route_tc_kernel, round 3 (1,024 columns)",
-                         "peak_kind": kind},
-            "checks": {"chain_docs_selected": chain_ok, "device_status": m.device_status()},
-            "clocks": clk.summary()}))
+    peak = pk["bf16_sustained"]
+
+    # end to end: every step copies all layers' query-side inputs (pinned host) in, runs the three
+    # rounds and reads every round's attention output back, serialised on the compute stream
+    names = ("qr", "q", "k_new", "v_new")
+    h_in = [[_pinned_like(small[l][n]) for n in names] for l in range(w.layers)]
+    h_out = [[_pinned_like(outs[l][r]) for r in range(w.rounds)] for l in range(w.layers)]
+
+    def e2e_step():
+        with torch.cuda.stream(compute):
+            for l in range(w.layers):
+                for h, n in zip(h_in[l], names):
+                    small[l][n].copy_(h, non_blocking=True)
+            refresh_qr()
+        for rd in rounds:
+            rd.run(compute, copy)
+        with torch.cuda.stream(compute):
+            for l in range(w.layers):
+                for r in range(w.rounds):
+                    h_out[l][r].copy_(outs[l][r], non_blocking=True)
+
+    e_ms = device_ms(e2e_step, steps, 1, compute)
+    h2d = sum(h.numel() * h.element_size() for hl in h_in for h in hl)
+    d2h = sum(h.numel() * h.element_size() for hl in h_out for h in hl) + \
+        sum(t.numel() * 4 for tl in idx_host for t in tl)
+    tokens = lay.n_chunks * TOKENS_PER_CHUNK * w.layers * w.rounds
+
+    # oracle: routing of one query's round-3 tokens (128) over leading slices of layer 0's bank for
+    # ~3 s (the dominant cost of a round), memory tokens routed per second
+    qr3 = w.qr(0)[:1, :sum(w.round_tokens(w.rounds - 1))]
+    done, t0 = 0, time.perf_counter()
+    while done < w.n_docs and time.perf_counter() - t0 < 3.0:
+        d1 = min(w.n_docs, done + 512)
+        a, b = int(w.doc_chunk_off[done]), int(w.doc_chunk_off[d1])
+        rows = w.host_rows(0, "krbar", np.arange(a, b)).reshape(b - a, w.H, w.d)
+        O.topk_docs(O.route(rows, w.doc_chunk_off[done:d1 + 1] - a, qr3)[0], w.k)
+        done = d1
+    cpu_rate = int(w.doc_chunk_off[done]) * TOKENS_PER_CHUNK / (time.perf_counter() - t0)
+    entry = {
+        "workload": "interleave: 78,128 chunks x 18 layers, 8 queries, 3 rounds (64/96/128 routing tokens), top-12",
+        "metric": "Memory Interleave: memory tokens routed/s (3 rounds x 18 layers over a 10M-token bank)",
+        "value": tokens / (ms / 1e3), "unit": "memory tokens/s", "higher_is_better": True, "ms_per_step": ms,
+        "steps": steps, "route_ms_per_layer_by_round": rms, "route_tflops_by_round": tflops,
+        "roofline": {"bound": "tensor", "achieved": tflops[-1], "peak": peak, "unit": "TFLOP/s",
+                     "frac": tflops[-1] / peak, "frac_by_round": [t / peak for t in tflops], "traffic": None,
+                     "kernel": "route_tc_kernel, round 3 (1,024 columns)",
+                     "peak_kind": f"{pk['kind']} sustained bf16 (cuBLAS)"},
+        "cpu_baseline": {"value": cpu_rate, "unit": "memory tokens/s", "cores": oracle_threads(), "kind": "oracle",
+                         "sample": f"fp64 oracle routing + top-12 of one query's 128 round-3 tokens over the first "
+                                   f"{int(w.doc_chunk_off[done]):,} chunks of one layer"},
+        "e2e": {"value": tokens / (e_ms / 1e3), "unit": "memory tokens/s", "ms_per_step": e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "how": "public API (msa_interleave_step per round) with pinned host buffers: all layers' query-side "
+                       "inputs in and every round's output back inside the timed region, serialised"},
+        "clocks": clk.summary(),
+        "checks": {"chain_docs_selected": chain_ok, "device_status": m.device_status()}}
+    del rounds, index, banks, small, local, outs
+    _free()
+    return entry
 
 
-# ---------------------------------------------------------------------------------------------- fine stage
 def host_link_gbs(nbytes: int = 1 << 30, reps: int = 5) -> float:
     """Pinned host -> device copy bandwidth measured in this process (best of reps, CUDA events)."""
     import torch
@@ -338,7 +746,7 @@ def host_link_gbs(nbytes: int = 1 << 30, reps: int = 5) -> float:
     d = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
     best = float("inf")
     for _ in range(reps):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a, b = _ev(), _ev()
         a.record()
         d.copy_(h, non_blocking=True)
         b.record()
@@ -348,19 +756,19 @@ def host_link_gbs(nbytes: int = 1 << 30, reps: int = 5) -> float:
     return nbytes / (best / 1e3) / 1e9
 
 
-def fine_bench(args, rank, world, local_rank):
+def cfg_fine1m(args, pk):
     """Token-level fine stage on the 1M-token bank: one step = route (pooled index) + top-8 + fetch of
     the selected documents' token K/V from the pinned token bank + global RoPE of the local context +
     split-key attention of 64 query tokens over those rows."""
     import numpy as np
     import torch
 
+    import oracle as O
     import routed_long_context_b200 as m
     from msa_inputs import workloads
     from msa_inputs.device import memory_tensor, small_tensors
     from routed_long_context_b200.bank import BankLayout, to_host_bank
 
-    torch.cuda.set_device(local_rank)
     w = workloads.mem_1m()
     lay = BankLayout.from_doc_lengths(w.doc_len, w.chunk)
     cs = m.rope_table(4096, w.d, w.rope_base)
@@ -370,7 +778,7 @@ def fine_bench(args, rank, world, local_rank):
     del k, v, kr
     host_tok = to_host_bank(tok)
     del tok
-    torch.cuda.empty_cache()
+    _free()
     dv = small_tensors(w, 0)
     T, max_mem = w.T0, w.k * int(w.doc_len.max())
     seg = torch.tensor([0, T], dtype=torch.int64, device="cuda")
@@ -411,10 +819,10 @@ def fine_bench(args, rank, world, local_rank):
     rows = int(mem_len.cpu().sum())
     gi = idx.cpu().numpy()[0]
     planted_ok = set(w.expected(0, 0, 0)) <= set(gi.tolist())
-    steps = min(args.steps, 100)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    steps = max(3, min(args.steps, 100))
+    evs = [[_ev() for _ in range(4)] for _ in range(steps)]
     torch.cuda.synchronize()
-    with ClockSampler(local_rank) as clk:
+    with ClockSampler(torch.cuda.current_device()) as clk:
         for i in range(steps):
             step(evs[i])
         torch.cuda.synchronize()
@@ -425,25 +833,97 @@ def fine_bench(args, rank, world, local_rank):
     fetch_bytes = rows * 2 * w.hkv * w.d * 2
     link = host_link_gbs()
     fetch_gbs = fetch_bytes / (fetch_ms / 1e3) / 1e9
-    G = w.hq // w.hkv
     attn_flops = 4.0 * w.n_q * T * w.hq * w.d * (rows + T / 2)
-    if rank == 0:
-        print(json.dumps({
-            "metric": "1M fine stage: token rows fetched and attended per second (route + top-8 + token fetch + "
-                      "split attention)",
-            "value": rows / (ms / 1e3), "unit": "memory token rows/s", "n_gpus": 1, "steps": steps,
-            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": f"fine1m: {w.n_docs} docs ({w.n_tok:,} tokens), token bank "
-                                   f"{w.n_tok * 4096 / 1e9:.1f} GB pinned host, 64 query tokens, top-8 -> {rows} rows",
-                       "fetch_mode": args.fetch_mode},
-            "route_topk_ms": route_ms, "fetch_ms": fetch_ms, "attn_ms": attn_ms, "attn_tflops": attn_flops / attn_ms / 1e9,
-            "roofline": {"bound": "host-link", "achieved": fetch_gbs, "peak": link, "unit": "GB/s",
-                         "frac": fetch_gbs / link, "traffic": None,
-                         "kernel": "gather_device_kernel" if args.fetch_mode == 1 else "cudaMemcpyAsync per document",
-                         "peak_kind": "pinned host->device copy measured in this process", "bytes": fetch_bytes},
-            "checks": {"planted_docs_selected": planted_ok, "device_status": m.device_status(), "G": G},
-            "clocks": clk.summary()}))
+    attn_tflops = attn_flops / attn_ms / 1e9
 
+    # end to end: query-side inputs in, the step, the attention output back, serialised
+    names = ("qr", "q", "k_new", "v_new")
+    h_in = [_pinned_like(dv[n]) for n in names]
+    h_out = _pinned_like(out)
+
+    def e2e_step():
+        for h, n in zip(h_in, names):
+            dv[n].copy_(h, non_blocking=True)
+        step()
+        h_out.copy_(out, non_blocking=True)
+
+    e_ms = device_ms(e2e_step, steps, 1, s)
+    # oracle: routing over the first 125 documents' chunks (projected by chunks to the whole bank)
+    # and the token-level attention of the 64 query tokens over the rows of the 8 planted documents
+    krb = _oracle_pool_router(w, 125)
+    t_route = cpu_seconds(lambda: O.topk_docs(O.route(krb, w.doc_chunk_off[:126], w.qr(0)[:, :T])[0], w.k), 1.0, 5)
+    pdocs = w.expected(0, 0, 0)
+    trows = np.concatenate([np.arange(w.doc_tok_off[d], w.doc_tok_off[d + 1]) for d in pdocs])
+    kt = w.host_rows(0, "k", trows).reshape(len(trows), w.hkv, w.d)
+    vt = w.host_rows(0, "v", trows).reshape(len(trows), w.hkv, w.d)
+    tb = O.token_bank(kt, vt, np.concatenate([[0], np.cumsum(w.doc_len[pdocs])]), w.rope_base)
+    pos = O.global_positions(w.k, 0, T)
+    qo = O.apply_rope(w.q(0)[0], pos, w.rope_base)
+    kl = O.apply_rope(w.k_new(0)[0], pos, w.rope_base)
+    t_attn = cpu_seconds(lambda: O.sparse_attention(qo, tb[:, 0], tb[:, 1], kl, w.v_new(0)[0], 0, 1 / np.sqrt(w.d)),
+                         1.0, 5)
+    cpu_step = t_route * lay.n_chunks / krb.shape[0] + t_attn * rows / len(trows)
+    entry = {
+        "workload": f"fine1m: {w.n_docs} docs ({w.n_tok:,} tokens), token bank {w.n_tok * 4096 / 1e9:.1f} GB pinned "
+                    f"host, 64 query tokens, top-8 -> {rows} token rows",
+        "metric": "1M fine stage: token rows fetched and attended per second (route + top-8 + token fetch + split "
+                  "attention)",
+        "value": rows / (ms / 1e3), "unit": "memory token rows/s", "higher_is_better": True, "ms_per_step": ms,
+        "steps": steps, "fetch_mode": args.fetch_mode,
+        "route_topk_ms": route_ms, "fetch_ms": fetch_ms, "attn_ms": attn_ms, "attn_tflops": attn_tflops,
+        "attn_roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": pk["bf16"], "unit": "TFLOP/s",
+                          "frac": attn_tflops / pk["bf16"], "kernel": "attn_tc_kernel + attn_combine_kernel",
+                          "peak_kind": f"{pk['kind']} bf16 burst (cuBLAS)"},
+        "roofline": {"bound": "host-link", "achieved": fetch_gbs, "peak": link, "unit": "GB/s",
+                     "frac": fetch_gbs / link, "traffic": None,
+                     "kernel": "gather_device_kernel" if args.fetch_mode == 1 else "cudaMemcpyAsync per document",
+                     "peak_kind": "pinned host->device copy of 1 GiB measured in this process",
+                     "bytes": fetch_bytes},
+        "cpu_baseline": {"value": rows / cpu_step, "unit": "memory token rows/s", "cores": oracle_threads(),
+                         "kind": "oracle",
+                         "sample": "fp64 oracle routing over the first 125 documents' chunks scaled by chunks to the "
+                                   "bank, plus token-level attention over the 8 planted documents' rows scaled by "
+                                   "rows to the step's (projection)"},
+        "e2e": {"value": rows / (e_ms / 1e3), "unit": "memory token rows/s", "ms_per_step": e_ms,
+                "h2d_bytes_per_step": sum(h.numel() * h.element_size() for h in h_in),
+                "d2h_bytes_per_step": h_out.numel() * h_out.element_size(),
+                "how": "public API calls with pinned host buffers: query-side inputs in and the output back inside "
+                       "the timed region, serialised"},
+        "clocks": clk.summary(),
+        "checks": {"planted_docs_selected": planted_ok, "device_status": m.device_status()}}
+    del host_tok, mem, index
+    _free()
+    return entry
+
+
+def run_configs(args, pk):
+    """Every configuration, one after the other (each frees its device memory before the next)."""
+    out = {}
+    for name, fn in (("tiny", cfg_tiny), ("1m", cfg_1m), ("10m", cfg_10m), ("interleave", cfg_interleave),
+                     ("fine1m", cfg_fine1m)):
+        t0 = time.perf_counter()
+        try:
+            r = fn(args, pk)
+        except Exception as e:  # one configuration failing must not hide the others: report it
+            out[name] = {"error": repr(e)[:500]}
+            continue
+        if name == "10m":
+            out["10m_encode"], out["10m_decode"] = r
+        else:
+            out[name] = r
+        out.setdefault("_wall_s", {})[name] = time.perf_counter() - t0
+    return out
+
+
+def workload_line(args, entry, world):
+    """A configuration entry printed as a line of its own (`--workload X`)."""
+    line = {"metric": entry["metric"], "value": entry["value"], "unit": entry["unit"], "n_gpus": world,
+            "steps": entry.get("steps", args.steps), "warmup": args.warmup, "ms_per_step": entry["ms_per_step"],
+            "higher_is_better": entry.get("higher_is_better", True), "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32" if entry["workload"].startswith("tiny") else "bf16", "data": "synthetic",
+            "config": {"workload": entry["workload"]}}
+    line.update({k: v for k, v in entry.items() if k not in line and k not in ("workload",)})
+    print(json.dumps(line))
 
 # ---------------------------------------------------------------------------------------------- training step
 def train_bench(args, rank, world, local_rank):
@@ -571,15 +1051,42 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
     if args.impl == "reference":
         return reference_arm(args, rank)
-    if args.workload == "encode10m":
-        return encode_bench(args, rank, world, local_rank)
-    if args.workload == "interleave":
-        return interleave_bench(args, rank, world, local_rank)
-    if args.workload == "fine1m":
-        return fine_bench(args, rank, world, local_rank)
+    if args.workload in ("tiny", "1m", "encode10m", "decode10m", "interleave", "fine1m"):
+        import torch
+
+        torch.cuda.set_device(local_rank)
+        pk = all_peaks()
+        fn = {"tiny": cfg_tiny, "1m": cfg_1m, "encode10m": cfg_10m, "decode10m": cfg_10m,
+              "interleave": cfg_interleave, "fine1m": cfg_fine1m}[args.workload]
+        entry = fn(args, pk)
+        if args.workload in ("encode10m", "decode10m"):
+            entry = entry[0] if args.workload == "encode10m" else entry[1]
+        if rank == 0:
+            workload_line(args, entry, world)
+        return
     if args.workload == "train64k":
         return train_bench(args, rank, world, local_rank)
 
+    import torch
+    import torch.distributed as dist
+
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local_rank))
+    line = headline(args, rank, world, local_rank)
+    _free()                                            # the headline's 30 GB are released here
+    if world == 1 and not args.no_configs:
+        line["configs"] = run_configs(args, all_peaks())
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def headline(args, rank, world, local_rank):
+    """The 100M routing step: 18 routed layers per step (the reported metric); returns the JSON line."""
     import numpy as np
     import torch
     import torch.distributed as dist
@@ -589,12 +1096,7 @@ def main():
     from msa_inputs.device import memory_tensor, small_tensors
     from routed_long_context_b200.bank import BankLayout, index_from_prepooled
 
-    torch.cuda.set_device(local_rank)
     m.api.route_set_max_stages(args.router_stages)
-    if world > 1:
-        from datetime import timedelta
-
-        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local_rank))
 
     def barrier():
         if world > 1:
@@ -726,7 +1228,7 @@ def main():
         read[b_].record(s_out)
     for b_ in range(2):                                        # warm the second set's round
         sets[b_][2].run(compute, copy)
-    e_steps = max(4, args.steps // 4)
+    e_steps = args.steps
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
@@ -754,8 +1256,24 @@ def main():
     e2e_ms = e0.elapsed_time(e1) / e_steps
     assert torch.equal(sets[(e_steps - 1) % 2][3][0].cuda(), sets[(e_steps - 1) % 2][1][0])
 
+    # the same end to end, one step at a time: inputs in, the round, outputs back, all on the compute
+    # stream, so each step's copies and compute are serialised (per-step latency, no overlap)
+    dev_in, dev_out, rd, host_out = sets[0]
+
+    def serial_step():
+        with torch.cuda.stream(compute):
+            dev_in.copy_(host_in, non_blocking=True)
+        rd.run(compute, copy)
+        with torch.cuda.stream(compute):
+            host_out.copy_(dev_out, non_blocking=True)
+
+    barrier()
+    e2e_serial_ms = device_ms(serial_step, args.steps, 1, compute)
+    barrier()
+
     # ---- max over ranks
-    ms_step, e2e_ms, route_ms, route_ms_live = max_over_ranks([ms_step, e2e_ms, route_ms, route_ms_live], "cuda")
+    ms_step, e2e_ms, e2e_serial_ms, route_ms, route_ms_live = max_over_ranks(
+        [ms_step, e2e_ms, e2e_serial_ms, route_ms, route_ms_live], "cuda")
     tokens_per_step = lay.n_chunks * TOKENS_PER_CHUNK * w.layers
     value = whole_job_rate(tokens_per_step, world, ms_step)
     e2e_value = whole_job_rate(tokens_per_step, world, e2e_ms)
@@ -771,8 +1289,7 @@ def main():
                "sample": f"fp64 oracle routing + top-k over the first {chunks} chunks of one 100M layer "
                          f"({chunks * TOKENS_PER_CHUNK} memory tokens), 64 query tokens"}
 
-    if rank == 0:
-        print(json.dumps({
+    return {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded counter-based generator)",
@@ -792,17 +1309,20 @@ def main():
                          "peak_kind": f"{peak_kind} (copy bandwidth)"},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "ms_per_step": e2e_ms,
-                    "how": "public API with pinned host buffers; double-buffered: each step's H2D and D2H on their "
-                           "own streams overlap the neighbouring steps' compute, all inside the timed region"},
+                    "ms_per_step": e2e_ms, "steps": e_steps,
+                    "how": "pipelined throughput through the public API with pinned host buffers: double-buffered, "
+                           "each step's H2D and D2H on their own streams overlap the neighbouring steps' compute, "
+                           "all inside the timed region",
+                    "serial_ms_per_step": e2e_serial_ms,
+                    "serial_value": whole_job_rate(tokens_per_step, world, e2e_serial_ms),
+                    "serial_how": "per-step latency: the step's H2D, its round and its D2H serialised on one "
+                                  "stream, no overlap between steps"},
             # per layer: prepass, router, top-k, fetch kernel (mode 1) or memory lengths (mode 0),
             # attention; per step: one fused append for every layer
             "gpu_launches": (5 * w.layers + (w.layers + 23) // 24) * args.steps,
             "clocks": clk.summary(),
             "checks": {"planted_docs_selected": planted_ok, "device_status": status},
-        }))
-    if world > 1:
-        dist.destroy_process_group()
+    }
 
 
 if __name__ == "__main__":
