@@ -494,9 +494,10 @@ def cfg_1m(args, pk):
     return e
 
 
-# DRAM bytes (read + write) of pool_kernel per launch on the 10M encode: None until an ncu capture of
-# the current kernel (a 400-document case, scaled by documents) is recorded here.
-POOL_TRAFFIC_10M = None
+# DRAM bytes (read + write) of pool_kernel per launch on the 10M encode: ncu --set full on a
+# 400-document case of the current kernel (2,517.15 MB read + 7.77 MB written), scaled by documents
+# to the 9,766-document bank (traffic grows with the tokens pooled).
+POOL_TRAFFIC_10M = (2517.153e6 + 7.774e6) * 9766 / 400
 
 
 def cfg_10m(args, pk):
@@ -810,8 +811,9 @@ def cfg_fine1m(args, pk):
         if ev: ev[2].record(s)
         m.msa_rope_doc(dv["k_new"][0], seg, w.k, cs, out=lk)
         m.msa_rope_doc(dv["q"][0], seg, w.k, cs, out=qq)
-        m.msa_sparse_attn_split(qq[None], mem, mem_len, lk[None], dv["v_new"], T, 0, out=out, ws=aws)
         if ev: ev[3].record(s)
+        m.msa_sparse_attn_split(qq[None], mem, mem_len, lk[None], dv["v_new"], T, 0, out=out, ws=aws)
+        if ev: ev[4].record(s)
 
     for _ in range(args.warmup):
         step()
@@ -820,7 +822,7 @@ def cfg_fine1m(args, pk):
     gi = idx.cpu().numpy()[0]
     planted_ok = set(w.expected(0, 0, 0)) <= set(gi.tolist())
     steps = max(3, min(args.steps, 100))
-    evs = [[_ev() for _ in range(4)] for _ in range(steps)]
+    evs = [[_ev() for _ in range(5)] for _ in range(steps)]
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device()) as clk:
         for i in range(steps):
@@ -828,8 +830,9 @@ def cfg_fine1m(args, pk):
         torch.cuda.synchronize()
     route_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / steps
     fetch_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / steps
-    attn_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / steps
-    ms = sum(e[0].elapsed_time(e[3]) for e in evs) / steps
+    rope_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / steps
+    attn_ms = sum(e[3].elapsed_time(e[4]) for e in evs) / steps
+    ms = sum(e[0].elapsed_time(e[4]) for e in evs) / steps
     fetch_bytes = rows * 2 * w.hkv * w.d * 2
     link = host_link_gbs()
     fetch_gbs = fetch_bytes / (fetch_ms / 1e3) / 1e9
@@ -870,7 +873,9 @@ def cfg_fine1m(args, pk):
                   "attention)",
         "value": rows / (ms / 1e3), "unit": "memory token rows/s", "higher_is_better": True, "ms_per_step": ms,
         "steps": steps, "fetch_mode": args.fetch_mode,
-        "route_topk_ms": route_ms, "fetch_ms": fetch_ms, "attn_ms": attn_ms, "attn_tflops": attn_tflops,
+        "route_topk_ms": route_ms, "fetch_ms": fetch_ms, "rope_ms": rope_ms, "attn_ms": attn_ms,
+        "attn_tflops": attn_tflops, "attn_what": "split-key attention + combine (the two RoPE launches of the "
+                                                "local context are rope_ms)",
         "attn_roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": pk["bf16"], "unit": "TFLOP/s",
                           "frac": attn_tflops / pk["bf16"], "kernel": "attn_tc_kernel + attn_combine_kernel",
                           "peak_kind": f"{pk['kind']} bf16 burst (cuBLAS)"},

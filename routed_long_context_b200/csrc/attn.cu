@@ -448,7 +448,9 @@ __global__ void __launch_bounds__(128, SPLIT ? 3 : 1) attn_mma_kernel(const Attn
 
 // Merge of the split-KV partial results: one warp per (query, token, head) row, lane l owning dims
 // 4l..4l+3. out = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s with M = max_s m_s; a row whose
-// ranges saw no visible key (all m_s = -inf) is 0.
+// ranges saw no visible key (all m_s = -inf) is 0. Lane s reads range s's (m, l) (ranges in groups
+// of 32) and the max and the weights go round the warp by shuffles, so every range's loads are in
+// flight together instead of one dependent round trip per range; the sums run in range order.
 __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restrict__ part_o,
                                                            const float2* __restrict__ part_ml, int n_split,
                                                            int64_t rows, __nv_bfloat16* __restrict__ out,
@@ -458,19 +460,38 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
     if (row >= rows) return;
     const float ninf = -__int_as_float(0x7f800000);
     float M = ninf;
-    for (int s = 0; s < n_split; ++s) M = fmaxf(M, part_ml[(int64_t)s * rows + row].x);
+    for (int s0 = 0; s0 < n_split; s0 += 32) {
+        const float m = s0 + lane < n_split ? part_ml[(int64_t)(s0 + lane) * rows + row].x : ninf;
+        M = fmaxf(M, m);
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float acc[4] = {0.f, 0.f, 0.f, 0.f}, L = 0.f;
     if (M != ninf) {
-        for (int s = 0; s < n_split; ++s) {
-            const float2 ml = part_ml[(int64_t)s * rows + row];
-            if (ml.x == ninf) continue;
-            const float w = exp2f(ml.x - M);
-            L = fmaf(w, ml.y, L);
-            const float4 o = *reinterpret_cast<const float4*>(part_o + ((int64_t)s * rows + row) * kD + lane * 4);
-            acc[0] = fmaf(w, o.x, acc[0]);
-            acc[1] = fmaf(w, o.y, acc[1]);
-            acc[2] = fmaf(w, o.z, acc[2]);
-            acc[3] = fmaf(w, o.w, acc[3]);
+        for (int s0 = 0; s0 < n_split; s0 += 32) {
+            const int n = min(32, n_split - s0);
+            const float2 ml = lane < n ? part_ml[(int64_t)(s0 + lane) * rows + row] : make_float2(ninf, 0.f);
+            const float w_l = ml.x == ninf ? 0.f : exp2f(ml.x - M);
+            float4 o[8];
+            for (int b = 0; b < n; b += 8) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    o[i] = b + i < n ? *reinterpret_cast<const float4*>(part_o + ((int64_t)(s0 + b + i) * rows + row) *
+                                                                                     kD + lane * 4)
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float w = __shfl_sync(0xffffffffu, w_l, (b + i) & 31);
+                    const float ls = __shfl_sync(0xffffffffu, ml.y, (b + i) & 31);
+                    if (b + i < n && w != 0.f) {
+                        L = fmaf(w, ls, L);
+                        acc[0] = fmaf(w, o[i].x, acc[0]);
+                        acc[1] = fmaf(w, o[i].y, acc[1]);
+                        acc[2] = fmaf(w, o[i].z, acc[2]);
+                        acc[3] = fmaf(w, o[i].w, acc[3]);
+                    }
+                }
+            }
         }
     }
     const float inv = L > 0.f ? 1.f / L : 0.f;

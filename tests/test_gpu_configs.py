@@ -23,11 +23,14 @@ def _np(t):
     return t.float().cpu().numpy().astype(np.float64)
 
 
-def assert_topk_matches(gpu_idx, ref_scores_row, k, tol=2e-3):
+def assert_topk_matches(gpu_idx, ref_scores_row, k, tol=2e-3, gpu_scores_row=None):
     """The selected set equals the oracle's, excused only where the oracle's k-th and (k+1)-th scores
-    lie within tol (then every GPU pick must score within tol of the oracle's k-th score). The order
-    inside the set is unique only up to score differences the precision resolves: along the GPU's
-    ranking the oracle scores may never rise by more than 2 * tol."""
+    lie within tol (then every GPU pick must score within tol of the oracle's k-th score).
+
+    With the GPU's own document scores (gpu_scores_row), the selection must be exactly their top-k
+    (descending, ties to the lower index), and the order is held to the observed score error
+    err = max |GPU - oracle|: a document ranked before another by the GPU cannot score more than
+    2 err below it in the oracle. Without them, the order is held to 2 * tol."""
     ref_idx, ref_val = O.topk_docs(ref_scores_row[None], min(k + 1, len(ref_scores_row)))
     ref_idx, ref_val = ref_idx[0], ref_val[0]
     gpu_idx = np.asarray(gpu_idx)
@@ -35,9 +38,14 @@ def assert_topk_matches(gpu_idx, ref_scores_row, k, tol=2e-3):
     if set(gpu_idx.tolist()) != set(ref_idx[:k].tolist()):
         assert len(ref_val) > k and ref_val[k - 1] - ref_val[k] <= tol, (gpu_idx, ref_idx[:k], ref_val[:k + 1])
         assert np.all(ref_scores_row[gpu_idx] >= ref_val[k - 1] - tol)
+    slack = 2 * tol
+    if gpu_scores_row is not None:
+        g = np.asarray(gpu_scores_row, dtype=np.float64)
+        np.testing.assert_array_equal(gpu_idx, O.topk_docs(g[None], k)[0][0])
+        slack = 2 * float(np.abs(g - ref_scores_row).max()) + 1e-7
     s = ref_scores_row[gpu_idx]
     for i in range(k - 1):
-        assert s[i] >= s[i + 1:].max() - 2 * tol, (i, s)
+        assert s[i] >= s[i + 1:].max() - slack, (i, s, slack)
 
 
 def _row_rel_err(got, ref):
@@ -107,7 +115,7 @@ def test_tiny_end_to_end(m, fetch_mode):
     assert np.abs(_np(ds) - ref_ds).max() <= 1e-5
     # selection, then the oracle's attention over the documents the GPU selected
     got_idx = idx_host[0][0].numpy()[0]
-    assert_topk_matches(got_idx, ref_ds[0], w.k)
+    assert_topk_matches(got_idx, ref_ds[0], w.k, gpu_scores_row=_np(ds)[0])
     assert set(got_idx[:2].tolist()) == {17, 42}
     mem = O.gather_memory(np.stack([kb, vb], 1), w.doc_chunk_off, got_idx)
     kl = O.apply_rope(w.k_new(0)[0], O.global_positions(w.k, 0, w.T0), w.rope_base)
@@ -191,7 +199,7 @@ def test_1m_end_to_end(m):
     assert np.abs(ds_gpu - ref_ds).max() <= 2e-3
     np.testing.assert_allclose(_np(index), O.unit(krb).reshape(_np(index).shape), atol=2.0 ** -8)
     gi = idx_host[0][0].numpy()[0]
-    assert_topk_matches(gi, ref_ds[0], w.k)
+    assert_topk_matches(gi, ref_ds[0], w.k, gpu_scores_row=ds_gpu[0])
     assert set(w.expected(0, 0, 0)) <= set(gi.tolist())
     # pooled K-bar / V-bar of the selected documents, then attention over them
     enc = oracle_encode_docs(w, 0, gi, ("k", "v"))
@@ -292,7 +300,7 @@ def test_10m_encode_and_decode_routing(m):
     err = np.abs(ds_gpu - ref_ds)
     assert err.max() <= 2e-3, float(err.max())
     for q in range(w.n_q):
-        assert_topk_matches(gi[q], ref_ds[q], w.k)
+        assert_topk_matches(gi[q], ref_ds[q], w.k, gpu_scores_row=ds_gpu[q])
         assert set(w.expected(0, 0, q)) <= set(gi[q].tolist())
 
     # pooled K-bar / V-bar: selected, planted and a seeded sample of documents
@@ -352,7 +360,7 @@ def test_100m_two_layers_full_routing(m, fetch_mode):
         ref = oracle_route_prepooled(w, l, w.qr(l))
         assert np.abs(ds_gpu - ref).max() <= 2e-3
         gi = idx_host[l][0].numpy()[0]
-        assert_topk_matches(gi, ref[0], w.k)
+        assert_topk_matches(gi, ref[0], w.k, gpu_scores_row=ds_gpu[0])
         assert set(w.expected(l, 0, 0)) <= set(gi.tolist())
         mem = oracle_bank_rows(w, l, gi)
         kl = O.apply_rope(w.k_new(l)[0], O.global_positions(w.k, 0, w.T0), w.rope_base)
@@ -390,12 +398,15 @@ def test_interleave_three_rounds(m):
         krbar = w.host_tensor(l, "krbar")
         bank = _BankRows(w, w.host_bank_slot(l))
         qr, qa, kn, vn = w.qr(l), w.q(l), w.k_new(l), w.v_new(l)
+        ds_gpu = [_np(m.msa_route_scores(index[l], lay.chunk_doc, lay.n_docs,
+                                         dvs[l]["qr"][:, :sum(w.round_tokens(r))].contiguous()))
+                  for r in range(w.rounds)]
         for q in range(w.n_q):
             gpu_sel = [idx_host[l][r].numpy()[q] for r in range(w.rounds)]
             ref = O.interleave(krbar, w.doc_chunk_off, bank, qr[q], qa[q], kn[q], vn[q], w.T0, w.T_new, w.rounds,
                                w.k, w.rope_base, select=gpu_sel)
             for r, (_, _, ds, o) in enumerate(ref):
-                assert_topk_matches(gpu_sel[r], ds, w.k)
+                assert_topk_matches(gpu_sel[r], ds, w.k, gpu_scores_row=ds_gpu[r][q])
                 assert set(w.expected(l, r, q)) <= set(gpu_sel[r].tolist()), (l, r, q)
                 assert _row_rel_err(_np(outs[l][r])[q], o) <= 2e-2, (l, r, q)
     del index

@@ -160,6 +160,46 @@ def test_pool_document_translation_invariance_bitwise(m):
     assert torch.equal(got[0], got[1])
 
 
+@pytest.mark.parametrize("in_dt,out_dt", [("bf16", "bf16"), ("f32", "f32"), ("bf16", "f32")])
+def test_pool_and_route_with_large_magnitude_values(m, in_dt, out_dt):
+    """The seeded generator stops at +-3.46 sigma; here 1% of the token elements (and of the router
+    queries) are replaced by spikes of +-6 to +-1024 (exact in bf16), so pooling, the rotation, the
+    index normalisation and the router's contraction are checked against the oracle over a wide
+    range of magnitudes, on ragged documents."""
+    from routed_long_context_b200.bank import BankLayout
+
+    chunk = 128
+    lay = BankLayout.from_doc_lengths(RAGGED, chunk)
+    n_tok = sum(RAGGED)
+
+    def spiked(tid, shape, dt):
+        x = _gen(tid, shape, dt).reshape(-1)
+        n = x.size // 100
+        pos = rng.uniform_int(SEED, 5000 + tid, n, x.size).astype(np.int64)
+        mag = np.array([6.0, 12.0, 100.0, 1024.0], dtype=np.float32)[rng.uniform_int(SEED, 6000 + tid, n, 4)]
+        sign = np.where(rng.uniform_int(SEED, 7000 + tid, n, 2) == 0, -1.0, 1.0).astype(np.float32)
+        x[pos] = mag * sign
+        return x.reshape(shape)
+
+    k, v, kr = (spiked(70 + i, (n_tok, 8, 128), in_dt) for i in range(3))
+    cs = m.rope_table(2048, 128, 1e6)
+    odt = torch.float32 if out_dt == "f32" else torch.bfloat16
+    kvbar, idx = m.msa_pool_chunks(upload(k, in_dt), upload(v, in_dt), upload(kr, in_dt), lay.doc_tok_off,
+                                   lay.doc_chunk_off, lay.chunk_doc, chunk, cos_sin=cs, out_dtype=odt)
+    kb, vb, krb = O.encode_memory(k, v, kr, lay.doc_tok_off_host, chunk, 1e6)
+    _close(_np(kvbar[:, 0]), kb, out_dt, "K-bar")
+    _close(_np(kvbar[:, 1]), vb, out_dt, "V-bar")
+    _close(_np(idx), O.unit(krb), out_dt, "router index")
+    qr = spiked(80, (2, 7, 8, 128), out_dt)
+    ds = m.msa_route_scores(idx, lay.chunk_doc, lay.n_docs, upload(qr, out_dt))
+    # the oracle scores the index as stored (each head a unit vector up to its rounding)
+    ref, _ = O.route(_np(idx), lay.doc_chunk_off_host, qr)
+    tol = 1e-5 if out_dt == "f32" else 2e-3
+    assert np.nanmax(np.abs(np.where(np.isfinite(ref), _np(ds) - ref, 0.0))) <= tol
+    assert np.array_equal(np.isfinite(ref), np.isfinite(_np(ds)))
+    _status(m)
+
+
 # -------------------------------------------------------------------------------------- routing
 def _route_case(C_docs_seed, n_q, T, dtype, n_docs=140):
     counts = 1 + rng.uniform_int(SEED, 900 + C_docs_seed, n_docs, 12).astype(np.int64)   # 1..12 chunks per doc
