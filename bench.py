@@ -873,6 +873,7 @@ def cfg_fine1m(args, pk):
                   "attention)",
         "value": rows / (ms / 1e3), "unit": "memory token rows/s", "higher_is_better": True, "ms_per_step": ms,
         "steps": steps, "fetch_mode": args.fetch_mode,
+        "attn_plan": m.api.sparse_attn_split_plan(w.n_q, T, w.hq, w.hkv, max_mem, T),
         "route_topk_ms": route_ms, "fetch_ms": fetch_ms, "rope_ms": rope_ms, "attn_ms": attn_ms,
         "attn_tflops": attn_tflops, "attn_what": "split-key attention + combine (the two RoPE launches of the "
                                                 "local context are rope_ms)",

@@ -309,6 +309,14 @@ msa_status msa_sparse_attn_split(const void* q, const void* mem_kv, const int32_
                                  void* ws, size_t ws_bytes, void* stream);
 msa_status msa_sparse_attn_split_workspace_size(int n_q, int T, int hq, int hkv, int max_mem, int L, size_t* bytes);
 
+/* The launch plan msa_sparse_attn_split would use on the current device for these sizes (a query:
+ * enqueues nothing). *row_blocks: 128-row blocks per tensor-core CTA (1 or 2; 0 on the mma.sync
+ * path); *key_ranges: key ranges per (row blocks, kv head, query); *cluster: when >= 1, the ranges
+ * form a thread-block cluster of that many CTAs and are merged in distributed shared memory (no
+ * combine pass), 0 when partial results are combined through the workspace. */
+msa_status msa_sparse_attn_split_plan(int n_q, int T, int hq, int hkv, int max_mem, int L, int* row_blocks,
+                                      int* key_ranges, int* cluster);
+
 /* ---------------------------------------------------------------------------------------------
  * Backward pass (end-to-end training: [P1] 核心创新 端到端可训练性 — routing, compression and
  * attention are optimised in one gradient flow; [P1] §训练策略 and [P2] §训练层面 — a weighted

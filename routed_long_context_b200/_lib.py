@@ -109,6 +109,9 @@ SIGNATURES = {
     "msa_interleave_step": (i32, [ctypes.POINTER(InterleaveArgs), vp, vp, i64]),
     "msa_interleave_workspace_size": (i32, [ctypes.POINTER(InterleaveArgs), ctypes.POINTER(sz)]),
     "msa_workspace_size": (i32, [ctypes.c_int, vp, ctypes.POINTER(sz)]),
+    "msa_sparse_attn_split_plan": (i32, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_int, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int),
+                                         ctypes.POINTER(ctypes.c_int)]),
 }
 
 

@@ -282,6 +282,15 @@ def sparse_attn_split_workspace_size(n_q: int, T: int, hq: int, hkv: int, max_me
     return n.value
 
 
+def sparse_attn_split_plan(n_q: int, T: int, hq: int, hkv: int, max_mem: int, L: int) -> dict:
+    """The launch plan of msa_sparse_attn_split on the current device: row blocks per CTA, key ranges,
+    and the cluster size when the ranges are merged in distributed shared memory (0: combine pass)."""
+    rb, kr, cl = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    check(lib.msa_sparse_attn_split_plan(n_q, T, hq, hkv, max_mem, L, ctypes.byref(rb), ctypes.byref(kr),
+                                         ctypes.byref(cl)), "msa_sparse_attn_split_plan")
+    return {"row_blocks": rb.value, "key_ranges": kr.value, "cluster": cl.value}
+
+
 def msa_sparse_attn_split(q, mem_kv, mem_len, local_k, local_v, L: int, q_start: int, scale: float | None = None,
                           out=None, ws=None, lse=None, stream=None):
     """msa_sparse_attn for long memories (token-level fine stage): keys split into ranges that run as

@@ -16,8 +16,10 @@ namespace msa {
 
 msa_status launch_attn_tc(const void* q, const void* mem_kv, const int32_t* mem_len, int max_mem, const void* local_k,
                           const void* local_v, int L_max, int L, int q_start, int n_q, int T, int hq, int hkv,
-                          float scale_log2e, int n_split, float* part_o, float2* part_ml, cudaStream_t s);
+                          float scale_log2e, int n_split, float* part_o, float2* part_ml, void* out, float* lse,
+                          bool try_cluster, bool* merged, cudaStream_t s);
 int attn_tc_splits(int n_q, int T, int hq, int hkv, int max_mem, int L);
+msa_status attn_tc_plan(int n_q, int T, int hq, int hkv, int n_split, int* blocks, int* cluster);
 
 namespace {
 
@@ -612,6 +614,26 @@ msa_status msa_sparse_attn_split_workspace_size(int n_q, int T, int hq, int hkv,
     return MSA_OK;
 }
 
+msa_status msa_sparse_attn_split_plan(int n_q, int T, int hq, int hkv, int max_mem, int L, int* row_blocks,
+                                      int* key_ranges, int* cluster) {
+    MSA_REQUIRE(row_blocks && key_ranges && cluster, "msa_sparse_attn_split_plan: NULL output");
+    MSA_REQUIRE(n_q > 0 && T > 0 && hq > 0 && hkv > 0 && hq % hkv == 0 && max_mem >= 0 && L >= 0,
+                "msa_sparse_attn_split_plan: bad sizes");
+    const bool tc = g_attn_impl.load() == 0 || g_attn_impl.load() == 3;
+    *row_blocks = 0;
+    *cluster = 0;
+    *key_ranges = tc ? attn_tc_splits(n_q, T, hq, hkv, max_mem, L) : pick_splits(n_q, T, hq, hkv, max_mem, L);
+    if (!tc) return MSA_OK;
+    int blocks = 1, cs = 0;
+    MSA_RETURN_IF(attn_tc_plan(n_q, T, hq, hkv, *key_ranges, &blocks, &cs));
+    *row_blocks = blocks;
+    if (g_attn_impl.load() == 0 && cs >= 1) {
+        *key_ranges = cs;
+        *cluster = cs;
+    }
+    return MSA_OK;
+}
+
 msa_status msa_sparse_attn_split(const void* q, const void* mem_kv, const int32_t* mem_len, int max_mem,
                                  const void* local_k, const void* local_v, int L_max, int L, int q_start, int n_q,
                                  int T, int hq, int hkv, int d, float scale, void* out, float* lse, msa_dtype dt,
@@ -648,8 +670,13 @@ msa_status msa_sparse_attn_split(const void* q, const void* mem_kv, const int32_
                                           align_up((size_t)n_split * n_q * T * hq * kD * 4, 256));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (tc) {
+        // impl 0: key ranges merged inside a thread-block cluster when the grid fits one wave of
+        // clusters; impl 3 (and any shape that does not fit) writes partial results and combines them
+        bool merged = false;
         MSA_RETURN_IF(launch_attn_tc(q, mem_kv, mem_len, max_mem, local_k, local_v, L_max, L, q_start, n_q, T, hq, hkv,
-                                     a.scale_log2e, n_split, a.part_o, a.part_ml, st));
+                                     a.scale_log2e, n_split, a.part_o, a.part_ml, out, lse, g_attn_impl.load() == 0,
+                                     &merged, st));
+        if (merged) return MSA_OK;
         return launch_combine(a, n_q, st);
     }
     return launch_mma<true>(a, n_q, st);

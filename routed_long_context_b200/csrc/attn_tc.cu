@@ -27,6 +27,8 @@
 // CTA records MSA_DEV_WAIT_TIMEOUT, leaves its loops, waits (bounded) for its own copies and MMAs
 // and frees TMEM.
 #include <algorithm>
+#include <map>
+#include <mutex>
 
 #include "common.cuh"
 #include "kernels.cuh"
@@ -37,25 +39,34 @@ namespace msa {
 
 msa_status launch_attn_tc(const void* q, const void* mem_kv, const int32_t* mem_len, int max_mem, const void* local_k,
                           const void* local_v, int L_max, int L, int q_start, int n_q, int T, int hq, int hkv,
-                          float scale_log2e, int n_split, float* part_o, float2* part_ml, cudaStream_t s);
+                          float scale_log2e, int n_split, float* part_o, float2* part_ml, void* out, float* lse,
+                          bool try_cluster, bool* merged, cudaStream_t s);
 int attn_tc_splits(int n_q, int T, int hq, int hkv, int max_mem, int L);
+msa_status attn_tc_plan(int n_q, int T, int hq, int hkv, int n_split, int* blocks, int* cluster);
 
 namespace {
 
-constexpr int kRows = 128;                     // MMA M, TMEM lanes
+constexpr int kRows = 128;                     // MMA M, TMEM lanes: the rows of one row block
 constexpr int kKeys = 64;                      // keys per tile, MMA N of S
-constexpr int kHalfKeys = kKeys / 2;           // keys of a tile per softmax warp
 constexpr int kD = 128;
-constexpr int kStages = 5;
 constexpr int kThreads = 64 + 256;             // loader, MMA issuer, 8 softmax warps
 constexpr int kHalfQ = kRows * 128;            // one 64-element K block of Q: 128 rows x 128 B
 constexpr int kHalfKV = kKeys * 128;           // 64 rows x 128 B
 constexpr int kStageBytes = 4 * kHalfKV;       // K (2 halves) + V (2 halves)
 constexpr int kPBytes = kRows * 128;           // one P buffer: 128 rows x 64 keys bf16
-constexpr int kTmemCols = 256;                 // S buffers at 0 and 64, O at 128
-constexpr int kColO = 2 * kKeys;
-constexpr int kRedBytes = 2 * 2 * kRows * 4;   // [tile parity][key half][row] partial maxima / sums
-constexpr int kSmemBytes = 1024 + 2 * kHalfQ + kStages * kStageBytes + kPBytes + kRedBytes + 256;
+// NH row blocks of 128 rows per CTA. NH = 1: two softmax warps per row (each on 32 keys of a tile,
+// exchanging the row max); NH = 2: one softmax warp per row and both row blocks of a kv head in one
+// CTA, so each K/V tile is loaded once for 256 rows.
+template <int NH> struct TcShape {
+    static constexpr int kSplitKeys = 3 - NH;                  // softmax warps per row
+    static constexpr int kKW = kKeys / kSplitKeys;             // keys of a tile per softmax warp
+    static constexpr int kOW = kD / kSplitKeys;                // O columns per softmax warp
+    static constexpr int kStages = NH == 1 ? 5 : 4;
+    static constexpr int kTmemCols = 256 * NH;                 // S (row block r, buffer b) at (2r + b) * 64
+    static constexpr int kColO = 128 * NH;                     // O of row block r at kColO + 128 r
+    static constexpr int kRedBytes = NH == 1 ? 2 * 2 * kRows * 4 : 0;   // [parity][key half][row]
+    static constexpr int kSmemBytes = 1024 + NH * 2 * kHalfQ + kStages * kStageBytes + NH * kPBytes + kRedBytes + 256;
+};
 // A row's O is rescaled only when its running max grows by more than this (log2 units); otherwise
 // the probabilities are taken against the older, smaller max (at most 2^8, exact in fp32 and as
 // bf16 operands) and the final normalisation uses the same reference.
@@ -73,24 +84,36 @@ struct AttnTcArgs {
     int n_split;
     float* part_o;
     float2* part_ml;
+    __nv_bfloat16* out;    // merged in the cluster: the normalised output [n_q][T][hq][d]
+    float* lse;            // merged in the cluster, optional: natural-log log-sum-exp [n_q][T][hq]
     int* err;
     int use_tma;           // memory tiles by TMA from tm_mem (otherwise every tile by cp.async)
     int use_tma_loc;       // local-key tiles by TMA from tm_lk / tm_lv
 };
 
+// CL: the n_split CTAs of a (row blocks, kv head, query) form one thread-block cluster and merge
+// their key ranges through distributed shared memory into the final output (no partial results in
+// global memory, no combine kernel); otherwise each CTA writes its range's partial result.
+template <int NH, bool CL>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                                                               const __grid_constant__ CUtensorMap tm_mem,
                                                               const __grid_constant__ CUtensorMap tm_lk,
                                                               const __grid_constant__ CUtensorMap tm_lv,
                                                               const AttnTcArgs a) {
+    using Sh = TcShape<NH>;
+    constexpr int kStages = Sh::kStages;
+    constexpr int kKW = Sh::kKW;
+    constexpr int kOW = Sh::kOW;
+    constexpr int kColO = Sh::kColO;
+    constexpr int kTmemCols = Sh::kTmemCols;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = a.G;
     const int split = blockIdx.x % a.n_split;
-    const int r0 = (blockIdx.x / a.n_split) * kRows;
+    const int r0 = (blockIdx.x / a.n_split) * (kRows * NH);
     const int qi = blockIdx.z, g = blockIdx.y;
     const int n_rows = a.T * G;
     const int mem_len = max(min(a.mem_len[qi], a.max_mem), 0);
-    const int r_last = min(r0 + kRows, n_rows) - 1;
+    const int r_last = min(r0 + kRows * NH, n_rows) - 1;
     const int n_local = max(min(a.L, a.q_start + r_last / G + 1), 0);
     const int n_keys = mem_len + n_local;
     const int tiles = (n_keys + kKeys - 1) / kKeys;
@@ -101,14 +124,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     const int64_t rows_total = (int64_t)gridDim.z * a.T * a.hq;
     const float ninf = -__int_as_float(0x7f800000);
 
-    if (n_t == 0) {   // an empty key range: the partial result of nothing
+    if (!CL && n_t == 0) {   // an empty key range: the partial result of nothing
         if (warp >= 2) {
-            const int ch = (warp - 2) >> 2;   // half of the O row this warp writes
-            const int row = r0 + (warp & 3) * 32 + lane;
+            const int sw = (warp - 2) >> 2;
+            const int rh = NH == 2 ? sw : 0, ch = NH == 1 ? sw : 0;
+            const int row = r0 + rh * kRows + (warp & 3) * 32 + lane;
             if (row < n_rows) {
                 const int64_t gr = ((int64_t)qi * a.T + row / G) * a.hq + g * G + row % G;
                 float4* po = reinterpret_cast<float4*>(a.part_o + ((int64_t)split * rows_total + gr) * kD);
-                for (int i = 0; i < kD / 8; ++i) po[ch * (kD / 8) + i] = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int i = 0; i < kOW / 4; ++i) po[ch * (kOW / 4) + i] = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (ch == 0) a.part_ml[(int64_t)split * rows_total + gr] = make_float2(ninf, 0.f);
             }
         }
@@ -117,11 +141,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* sQ = base;                                   // 2 d-halves x 16 KB
-    uint8_t* sKV = sQ + 2 * kHalfQ;                       // kStages x (K 2 halves, V 2 halves)
-    uint8_t* sP = sKV + kStages * kStageBytes;            // one 16 KB P buffer
-    float* sRed = reinterpret_cast<float*>(sP + kPBytes);  // [2][2][128]
-    uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sRed) + kRedBytes);
+    uint8_t* sQ = base;                                   // NH row blocks x 2 d-halves x 16 KB
+    uint8_t* sKV = sQ + NH * 2 * kHalfQ;                  // kStages x (K 2 halves, V 2 halves)
+    uint8_t* sP = sKV + kStages * kStageBytes;            // one 16 KB P buffer per row block
+    float* sRed = reinterpret_cast<float*>(sP + NH * kPBytes);  // NH = 1: [2][2][128]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sRed) + Sh::kRedBytes);
     uint64_t* kv_full = bars;                             // [kStages] loader arrival (+ TMA bytes)
     uint64_t* kv_empty = bars + kStages;                  // [kStages] MMA commit
     uint64_t* q_full = bars + 2 * kStages;                // TMA bytes of Q
@@ -161,6 +185,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // a CTA of a cluster whose key range is empty takes part in the merge with an empty partial
+    const bool work = n_t > 0;
 
     if (warp == 0) {
         // ------------------------------------------------------------------ loader
@@ -173,16 +199,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         const int c = lane & 15, rsub = lane >> 4;
         const int cc = c & 7;
         const int hq_off = (c >> 3);
-        if (lane == 0) {
+        if (lane == 0 && work) {
             // Q: per d half one box [128 / G tokens][G heads][64 d] of the 4D map over q [n_q][T][hq][d]
             // (rows r = t * G + h' land in the swizzled K-major layout; tokens past T are zero-filled);
             // issued first, so its latency overlaps the first K/V tiles'
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_q)) : "memory");
             if (a.use_tma) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_mem)) : "memory");
-            mbar_expect_tx(smem_u32(q_full), (uint32_t)(2 * kHalfQ));
+            mbar_expect_tx(smem_u32(q_full), (uint32_t)(NH * 2 * kHalfQ));
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
-                tma_load_4d(smem_u32(sQ) + (uint32_t)(h * kHalfQ), &tm_q, h * 64, g * G, r0 / G, qi, smem_u32(q_full));
+            for (int rh = 0; rh < NH; ++rh)
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+                    tma_load_4d(smem_u32(sQ) + (uint32_t)((rh * 2 + h) * kHalfQ), &tm_q, h * 64, g * G,
+                                (r0 + rh * kRows) / G, qi, smem_u32(q_full));
         }
         const int64_t mstride = 2LL * a.hkv * kD;                         // elements between memory rows
         const int64_t lstride = (int64_t)a.hkv * kD;                      // elements between local rows
@@ -252,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             if (lane == 0) mbar_arrive(full);
             tma_phase[st] = -1;
         }
-        if (lane == 0 && *abort_flag) {
+        if (lane == 0 && work && *abort_flag) {
             // leave no TMA copy in flight: wait (bounded, ignoring the abort flag) for Q and the last tiles
             const uint64_t t0 = globaltimer();
             while (!mbar_try_wait(smem_u32(q_full), 0) && globaltimer() - t0 < kWaitNs) {
@@ -264,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        if (lane == 0 && work) {
             // M = 128, bf16 x bf16 -> fp32; S: N = 64, both K-major; P V: N = 128, B (V) MN-major
             const uint32_t idesc_s = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kKeys >> 3) << 17) |
                                      ((uint32_t)(kRows >> 4) << 24);
@@ -277,14 +306,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 if (!mbar_wait(smem_u32(&kv_full[st]), (uint32_t)(j / kStages) & 1u, abort_flag)) return false;
                 tc_fence_after();
                 const uint32_t sb = smem_u32(sKV + st * kStageBytes);
-                const uint32_t d_tmem = tmem_base + (uint32_t)((j & 1) * kKeys);
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const uint64_t ad = sw128_desc(smem_u32(sQ) + h * kHalfQ);
-                    const uint64_t bd = sw128_desc(sb + h * kHalfKV);
+                for (int rh = 0; rh < NH; ++rh) {
+                    const uint32_t d_tmem = tmem_base + (uint32_t)((2 * rh + (j & 1)) * kKeys);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_bf16(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc_s, (h | kk) ? 1u : 0u);
+                    for (int h = 0; h < 2; ++h) {
+                        const uint64_t ad = sw128_desc(smem_u32(sQ) + (rh * 2 + h) * kHalfQ);
+                        const uint64_t bd = sw128_desc(sb + h * kHalfKV);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_bf16(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc_s,
+                                      (h | kk) ? 1u : 0u);
+                    }
                 }
                 pending = true;
                 umma_commit(smem_u32(&s_full[j & 1]));
@@ -300,13 +333,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 tc_fence_after();
                 const int st = j % kStages;
                 const uint32_t vb = smem_u32(sKV + st * kStageBytes + 2 * kHalfKV);
-                const uint64_t pd = sw128_desc(smem_u32(sP));
                 const uint64_t vd = sw128_mn_desc(vb, kHalfKV);
-                const uint32_t o_tmem = tmem_base + kColO;
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)   // 16 keys per step: +32 B along P's rows, +2 KB (16 V rows)
-                    umma_bf16(o_tmem, pd + (uint64_t)(kk * 2), vd + (uint64_t)(kk * (2048 >> 4)), idesc_o,
-                              (j > 0 || kk > 0) ? 1u : 0u);
+                for (int rh = 0; rh < NH; ++rh) {
+                    const uint64_t pd = sw128_desc(smem_u32(sP + rh * kPBytes));
+                    const uint32_t o_tmem = tmem_base + kColO + rh * 128;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)   // 16 keys per step: +32 B along P's rows, +2 KB (16 V rows)
+                        umma_bf16(o_tmem, pd + (uint64_t)(kk * 2), vd + (uint64_t)(kk * (2048 >> 4)), idesc_o,
+                                  (j > 0 || kk > 0) ? 1u : 0u);
+                }
                 umma_commit(smem_u32(&kv_empty[st]));
                 umma_commit(smem_u32(&o_done[j & 1]));
                 pending = false;
@@ -328,13 +364,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         // decision; each keeps the sum of its own keys (added at the end) and rescales its half of
         // the O row.
         const int quarter = warp & 3;
-        const int ch = (warp - 2) >> 2;
+        const int sw = (warp - 2) >> 2;
+        const int rh = NH == 2 ? sw : 0;                 // row block of this warp
+        const int ch = NH == 1 ? sw : 0;                 // key half of this warp (NH = 1)
         const int rl = quarter * 32 + lane;
-        const int row = r0 + rl;
+        const int row = r0 + rh * kRows + rl;
         const bool rvalid = row < n_rows;
         const int t = rvalid ? row / G : 0;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-        const uint32_t o_tmem = tmem_base + lane_off + kColO + ch * (kD / 2);
+        const uint32_t o_tmem = tmem_base + lane_off + kColO + rh * 128 + ch * kOW;
         float m = ninf, l = 0.f;      // reference max of the accumulated O row (log2 units), own keys' sum
         bool ok = true;
         // waits (lane 0, broadcast) on an mbarrier phase
@@ -359,36 +397,38 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             *theirs = sRed[((e & 1) * 2 + (ch ^ 1)) * kRows + rl];
             return true;
         };
-        for (int j = 0; j < n_t; ++j) {
+        for (int j = 0; j < n_t; ++j) {   // no tile (and no wait) when the range is empty
             if (!wait_bar(&s_full[j & 1], ((uint32_t)j >> 1) & 1u)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            float s[kHalfKeys];
-            tmem_ld32(tmem_base + lane_off + (uint32_t)((j & 1) * kKeys + ch * kHalfKeys), s);
-            const int kb = k_begin + j * kKeys + ch * kHalfKeys;
+            float s[kKW];
+#pragma unroll
+            for (int c0 = 0; c0 < kKW; c0 += 32)
+                tmem_ld32(tmem_base + lane_off + (uint32_t)((2 * rh + (j & 1)) * kKeys + ch * kKW + c0), s + c0);
+            const int kb = k_begin + j * kKeys + ch * kKW;
             // masked keys to -inf where the tile needs it: inside the range and (a memory row or a
             // causal local key)
-            if (!(__all_sync(0xffffffffu, rvalid) && kb + kHalfKeys <= k_end && kb + kHalfKeys <= mem_len)) {
+            if (!(__all_sync(0xffffffffu, rvalid) && kb + kKW <= k_end && kb + kKW <= mem_len)) {
                 const int lim = mem_len + a.q_start + t;
 #pragma unroll
-                for (int c = 0; c < kHalfKeys; ++c) {
+                for (int c = 0; c < kKW; ++c) {
                     const int kk = kb + c;
                     const bool vis = rvalid & (kk < k_end) & ((kk < mem_len) | (kk <= lim));
                     s[c] = vis ? s[c] : ninf;
                 }
             }
-            // the half tile's max over the raw scores in four chains (scale > 0 commutes with max and
-            // with its rounding), then the pair's
+            // the max over this warp's raw scores in four chains (scale > 0 commutes with max and with
+            // its rounding), then (NH = 1) the pair's
             float mx[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) mx[i] = s[i];
 #pragma unroll
-            for (int c = 4; c < kHalfKeys; ++c) mx[c & 3] = fmaxf(mx[c & 3], s[c]);
+            for (int c = 4; c < kKW; ++c) mx[c & 3] = fmaxf(mx[c & 3], s[c]);
             mx[0] = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
             float other = ninf;
-            if (!exchange(mx[0], j, &other)) {
+            if (NH == 1 && !exchange(mx[0], j, &other)) {
                 ok = false;
                 break;
             }
@@ -405,7 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             const float nref = m == ninf ? 0.f : -m;
             float psum[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int c = 0; c < kHalfKeys; ++c) {
+            for (int c = 0; c < kKW; ++c) {
                 s[c] = ex2(fmaf(s[c], a.scale_log2e, nref));
                 psum[c & 3] += s[c];
             }
@@ -417,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                     break;
                 }
 #pragma unroll
-                for (int part = 0; part < kD / 64; ++part) {
+                for (int part = 0; part < kOW / 32; ++part) {
                     float o[32];
                     tmem_ld32(o_tmem + (uint32_t)(part * 32), o);
 #pragma unroll
@@ -430,37 +470,76 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 ok = false;
                 break;
             }
-            uint8_t* prow = sP + rl * 128;
+            uint8_t* prow = sP + rh * kPBytes + rl * 128;
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
+            for (int c4 = 0; c4 < kKW / 8; ++c4) {
                 uint4 u;
                 u.x = pack_bf16(s[c4 * 8 + 0], s[c4 * 8 + 1]);
                 u.y = pack_bf16(s[c4 * 8 + 2], s[c4 * 8 + 3]);
                 u.z = pack_bf16(s[c4 * 8 + 4], s[c4 * 8 + 5]);
                 u.w = pack_bf16(s[c4 * 8 + 6], s[c4 * 8 + 7]);
-                const int cc = ch * 4 + c4;
+                const int cc = ch * (kKW / 8) + c4;
                 *reinterpret_cast<uint4*>(prow + ((cc ^ (rl & 7)) << 4)) = u;
             }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             tc_fence_before();
             mbar_arrive(smem_u32(&p_full[j & 1]));
         }
-        if (ok) ok = wait_pv(n_t - 1);
+        if (ok && work) ok = wait_pv(n_t - 1);
         float l_other = 0.f;
-        if (ok) ok = exchange(l, n_t, &l_other);
-        if (ok) {
-            const int64_t gr = ((int64_t)qi * a.T + t) * a.hq + g * G + (rvalid ? row % G : 0);
-            float4* po = reinterpret_cast<float4*>(a.part_o + ((int64_t)split * rows_total + gr) * kD);
+        if (NH == 1 && ok) ok = exchange(l, n_t, &l_other);
+        if (CL) {
+            // stage this range's partial in shared memory for the cluster's merge: O rows (fp32,
+            // 512 B, 16-byte chunk c stored at chunk c ^ (row % 32), so the 32 lanes' rows of a warp
+            // store hit distinct banks) in the idle K/V ring, (max, sum) per row in the idle P
+            // buffer; an empty or abandoned range stages (-inf, 0) and no O
+            const int rr = rh * kRows + rl;
+            float* st_row = reinterpret_cast<float*>(sKV) + rr * kD;
+            if (ok && work) {
 #pragma unroll
-            for (int part = 0; part < kD / 64; ++part) {
+                for (int part = 0; part < kOW / 32; ++part) {
+                    float o[32];
+                    tmem_ld32(o_tmem + (uint32_t)(part * 32), o);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int chunk = (ch * kOW + part * 32) / 4 + i;
+                        *reinterpret_cast<float4*>(st_row + ((chunk ^ (rr & 31)) << 2)) =
+                            make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+                    }
+                }
+            }
+            if (ch == 0)
+                reinterpret_cast<float2*>(sP)[rr] = (ok && work) ? make_float2(m, l + l_other) : make_float2(ninf, 0.f);
+        } else if (ok) {
+            // The range's unnormalised O rows, 32 columns at a time: TMEM -> registers (a row per
+            // lane) -> this warp's slot of the (now idle) K/V ring, [32 rows][36 floats] -> global,
+            // eight lanes per 128-byte row piece, so each store instruction writes four whole
+            // 128-byte pieces instead of 32 scattered 16-byte ones.
+            float* slot = reinterpret_cast<float*>(sKV) + (warp - 2) * (32 * 36);
+            const int rsub = lane >> 3, c4 = lane & 7;
+#pragma unroll
+            for (int part = 0; part < kOW / 32; ++part) {
                 float o[32];
                 tmem_ld32(o_tmem + (uint32_t)(part * 32), o);
-                if (rvalid)
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        po[(ch * 2 + part) * 8 + i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+                for (int i = 0; i < 8; ++i)
+                    *reinterpret_cast<float4*>(slot + lane * 36 + 4 * i) =
+                        make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+                __syncwarp();
+#pragma unroll
+                for (int it = 0; it < 8; ++it) {
+                    const int r = it * 4 + rsub;                          // row of this warp's 32
+                    const int row_r = r0 + rh * kRows + quarter * 32 + r;
+                    if (row_r < n_rows) {
+                        const int64_t gr_r = ((int64_t)qi * a.T + row_r / G) * a.hq + g * G + row_r % G;
+                        float* dst = a.part_o + ((int64_t)split * rows_total + gr_r) * kD + ch * kOW + part * 32;
+                        *reinterpret_cast<float4*>(dst + 4 * c4) = *reinterpret_cast<const float4*>(slot + r * 36 + 4 * c4);
+                    }
+                }
+                __syncwarp();
             }
             // both warps hold the same m; the row's sum is the two halves' (added in key-half order)
+            const int64_t gr = ((int64_t)qi * a.T + t) * a.hq + g * G + (rvalid ? row % G : 0);
             if (rvalid && ch == 0) a.part_ml[(int64_t)split * rows_total + gr] = make_float2(m, l + l_other);
         }
     }
@@ -472,24 +551,206 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
                      : "memory");
     }
+    if constexpr (CL) {
+        // ---------------------------------------------------------------- merge of the cluster's ranges
+        // Every thread of every CTA passes both cluster barriers (no early exit above in this
+        // variant). CTA rank k merges rows [k R, (k + 1) R) of the block: a warp per row, lane l on
+        // O dims 4l .. 4l + 3, reading each range's (max, sum) and O row from that CTA's shared
+        // memory: out = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s, M = max_s m_s (ranges with
+        // m_s = -inf skipped, a row no range saw is 0), in range order.
+        __syncwarp();
+        cluster_sync_all();
+        const int n_cl = a.n_split;
+        const int rank = (int)cluster_ctarank();
+        const int R = (NH * kRows + n_cl - 1) / n_cl;
+        const int rr_end = min(NH * kRows, (rank + 1) * R);
+        const uint32_t st_base = smem_u32(sKV), ml_base = smem_u32(sP);
+        for (int rr = rank * R + warp; rr < rr_end; rr += kThreads / 32) {
+            const int row_g = r0 + rr;
+            if (row_g >= n_rows) break;                   // rows only grow with rr
+            float M = ninf;
+            for (int s0 = 0; s0 < n_cl; ++s0) M = fmaxf(M, ld_cluster_f2(cluster_map(ml_base + rr * 8, s0)).x);
+            float acc[4] = {0.f, 0.f, 0.f, 0.f}, L = 0.f;
+            if (M != ninf) {
+                const uint32_t off = st_base + (uint32_t)(rr * kD * 4 + ((lane ^ (rr & 31)) << 4));
+                for (int s0 = 0; s0 < n_cl; ++s0) {
+                    const float2 ml = ld_cluster_f2(cluster_map(ml_base + rr * 8, s0));
+                    if (ml.x == ninf) continue;
+                    const float w = exp2f(ml.x - M);
+                    const float4 o = ld_cluster_f4(cluster_map(off, s0));
+                    L = fmaf(w, ml.y, L);
+                    acc[0] = fmaf(w, o.x, acc[0]);
+                    acc[1] = fmaf(w, o.y, acc[1]);
+                    acc[2] = fmaf(w, o.z, acc[2]);
+                    acc[3] = fmaf(w, o.w, acc[3]);
+                }
+            }
+            const float inv = L > 0.f ? 1.f / L : 0.f;
+            const int64_t gr = ((int64_t)qi * a.T + row_g / G) * a.hq + g * G + row_g % G;
+            uint2 u;
+            u.x = pack_bf16(acc[0] * inv, acc[1] * inv);
+            u.y = pack_bf16(acc[2] * inv, acc[3] * inv);
+            *reinterpret_cast<uint2*>(a.out + gr * kD + lane * 4) = u;
+            if (a.lse && lane == 0) a.lse[gr] = L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : ninf;
+        }
+        __syncwarp();
+        cluster_sync_all();   // no CTA leaves while another still reads its shared memory
+    }
 }
 
 }  // namespace
 
-// Key ranges per (128-row block, kv head, query): one wave of one CTA per SM (148), at least four
+// Row blocks per CTA: both of a kv head when it has more than 128 rows.
+int attn_tc_blocks(int T, int hq, int hkv) { return T * (hq / hkv) > kRows ? 2 : 1; }
+
+// Key ranges per (row blocks, kv head, query): one wave of one CTA per SM (148), at least four
 // 64-key tiles per range.
 int attn_tc_splits(int n_q, int T, int hq, int hkv, int max_mem, int L) {
     const int G = hq / hkv;
-    const int64_t base = (int64_t)((T * G + kRows - 1) / kRows) * hkv * n_q;
+    const int rows = kRows * attn_tc_blocks(T, hq, hkv);
+    const int64_t base = (int64_t)((T * G + rows - 1) / rows) * hkv * n_q;
     const int tiles = (max_mem + L + kKeys - 1) / kKeys;
     const int64_t want = 148 / std::max<int64_t>(base, 1);
     return (int)std::max<int64_t>(1, std::min<int64_t>(want, std::max(1, tiles / 4)));
 }
 
+namespace {
+
+// Largest cluster (1, 2, 4, 8 or 16 CTAs, one per key range) such that the whole grid of clusters
+// is resident at once (one wave), or 0 when no cluster launch of this kernel fits.
+// Opts both variants of row-block count NH into their dynamic shared memory and the cluster variant
+// into clusters of up to 16 CTAs, once per device.
+template <int NH>
+msa_status opt_in_tc() {
+    constexpr int smem = TcShape<NH>::kSmemBytes;
+    static std::mutex mu;
+    static int opted[64] = {0};
+    int dev = 0;
+    MSA_CUDA_TRY(cudaGetDevice(&dev));
+    std::lock_guard<std::mutex> lk(mu);
+    if (dev >= 0 && dev < 64 && opted[dev]) return MSA_OK;
+    MSA_CUDA_TRY(cudaFuncSetAttribute(attn_tc_kernel<NH, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    MSA_CUDA_TRY(cudaFuncSetAttribute(attn_tc_kernel<NH, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    MSA_CUDA_TRY(cudaFuncSetAttribute(attn_tc_kernel<NH, true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+    if (dev >= 0 && dev < 64) opted[dev] = 1;
+    return MSA_OK;
+}
+
+template <int NH>
+int pick_cluster_uncached(int64_t base);
+
+// pick_cluster_uncached asks the driver for cluster occupancy: remembered per (device, NH, base)
+template <int NH>
+int pick_cluster(int64_t base) {
+    static std::mutex mu;
+    static std::map<std::pair<int, int64_t>, int> memo;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return 0;
+    }
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        auto it = memo.find({dev, base});
+        if (it != memo.end()) return it->second;
+    }
+    const int cs = pick_cluster_uncached<NH>(base);
+    std::lock_guard<std::mutex> lk(mu);
+    memo[{dev, base}] = cs;
+    return cs;
+}
+
+template <int NH>
+int pick_cluster_uncached(int64_t base) {
+    constexpr int smem = TcShape<NH>::kSmemBytes;
+    if (opt_in_tc<NH>() != MSA_OK) return 0;
+    for (int cs = 16; cs >= 1; cs >>= 1) {
+        if ((int64_t)cs * base > 148) continue;
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)cs;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3((unsigned)(cs * base), 1, 1);
+        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, attn_tc_kernel<NH, true>, &cfg) != cudaSuccess) {
+            (void)cudaGetLastError();
+            continue;
+        }
+        if ((int64_t)n >= base) return cs;
+    }
+    return 0;
+}
+
+template <int NH>
+msa_status launch_tc(const CUtensorMap& tq, const CUtensorMap& tm, const CUtensorMap& tlk, const CUtensorMap& tlv,
+                     AttnTcArgs a, int n_q, int n_split, int cs, bool* merged, cudaStream_t s) {
+    constexpr int smem = TcShape<NH>::kSmemBytes;
+    const int row_blocks = (a.T * a.G + NH * kRows - 1) / (NH * kRows);
+    MSA_RETURN_IF(opt_in_tc<NH>());
+    *merged = false;
+    if (cs >= 1) {
+        a.n_split = cs;
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)cs;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3((unsigned)(row_blocks * cs), (unsigned)a.hkv, (unsigned)n_q);
+        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = s;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        MSA_CUDA_TRY(cudaLaunchKernelEx(&cfg, attn_tc_kernel<NH, true>, tq, tm, tlk, tlv, a));
+        *merged = true;
+        return MSA_OK;
+    }
+    attn_tc_kernel<NH, false><<<dim3(row_blocks * n_split, a.hkv, n_q), kThreads, smem, s>>>(tq, tm, tlk, tlv, a);
+    MSA_LAUNCH_CHECK();
+    return MSA_OK;
+}
+
+}  // namespace
+
+// The launch plan: row blocks per CTA (NH) and cluster size (0: partial results + combine). A
+// cluster layout is taken when the whole grid of clusters is resident in one wave and keeps at least
+// min(96, the combine layout's CTA count) SMs busy; the kv head's natural NH first (2 when it has
+// more than 128 rows), then one row block per CTA, whose clusters are half as wide.
+void choose_tc_plan(int n_q, int T, int hq, int hkv, int n_split, int* nh, int* cs_out) {
+    const int G = hq / hkv;
+    const int nh_pref = attn_tc_blocks(T, hq, hkv);
+    const int64_t fallback_ctas =
+        (int64_t)((T * G + nh_pref * kRows - 1) / (nh_pref * kRows)) * hkv * n_q * n_split;
+    for (int NH = nh_pref; NH >= 1; --NH) {
+        const int64_t base = (int64_t)((T * G + NH * kRows - 1) / (NH * kRows)) * hkv * n_q;
+        const int cs = NH == 2 ? pick_cluster<2>(base) : pick_cluster<1>(base);
+        if (cs >= 1 && (int64_t)cs * base >= std::min<int64_t>(96, fallback_ctas)) {
+            *nh = NH;
+            *cs_out = cs;
+            return;
+        }
+    }
+    *nh = nh_pref;
+    *cs_out = 0;
+}
+
+msa_status attn_tc_plan(int n_q, int T, int hq, int hkv, int n_split, int* blocks, int* cluster) {
+    choose_tc_plan(n_q, T, hq, hkv, n_split, blocks, cluster);
+    return MSA_OK;
+}
+
 msa_status launch_attn_tc(const void* q, const void* mem_kv, const int32_t* mem_len, int max_mem, const void* local_k,
                           const void* local_v, int L_max, int L, int q_start, int n_q, int T, int hq, int hkv,
-                          float scale_log2e, int n_split, float* part_o, float2* part_ml, cudaStream_t s) {
-    static_assert(kSmemBytes <= 232448, "shared memory");
+                          float scale_log2e, int n_split, float* part_o, float2* part_ml, void* out, float* lse,
+                          bool try_cluster, bool* merged, cudaStream_t s) {
+    static_assert(TcShape<1>::kSmemBytes <= 232448 && TcShape<2>::kSmemBytes <= 232448, "shared memory");
     AttnTcArgs a{};
     a.q = static_cast<const __nv_bfloat16*>(q);
     a.mem_kv = static_cast<const __nv_bfloat16*>(mem_kv);
@@ -498,6 +759,7 @@ msa_status launch_attn_tc(const void* q, const void* mem_kv, const int32_t* mem_
     a.local_v = static_cast<const __nv_bfloat16*>(local_v);
     a.L_max = L_max; a.L = L; a.q_start = q_start; a.T = T; a.hq = hq; a.hkv = hkv; a.G = hq / hkv;
     a.scale_log2e = scale_log2e; a.n_split = n_split; a.part_o = part_o; a.part_ml = part_ml;
+    a.out = static_cast<__nv_bfloat16*>(out); a.lse = lse;
     a.err = device_error_word();
     // queries [n_q][T][hq][d]: dims (d, head, token, query), box (64, G, 128 / G, 1): one box is 128 rows
     // r = t * G + h' of kv head g in the swizzled K-major layout
@@ -529,11 +791,10 @@ msa_status launch_attn_tc(const void* q, const void* mem_kv, const int32_t* mem_
         MSA_RETURN_IF(make_tensor_map_bf16(&tlv, local_v, 3, dims, strides, box));
         a.use_tma_loc = 1;
     }
-    MSA_CUDA_TRY(cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes));
-    const int row_blocks = (T * a.G + kRows - 1) / kRows;
-    attn_tc_kernel<<<dim3(row_blocks * n_split, hkv, n_q), kThreads, kSmemBytes, s>>>(tq, tm, tlk, tlv, a);
-    MSA_LAUNCH_CHECK();
-    return MSA_OK;
+    int NH = attn_tc_blocks(T, hq, hkv), cs = 0;
+    if (try_cluster && out) choose_tc_plan(n_q, T, hq, hkv, n_split, &NH, &cs);
+    if (NH == 2) return launch_tc<2>(tq, tm, tlk, tlv, a, n_q, n_split, cs, merged, s);
+    return launch_tc<1>(tq, tm, tlk, tlv, a, n_q, n_split, cs, merged, s);
 }
 
 }  // namespace msa

@@ -412,14 +412,16 @@ def test_device_gather_token_rows_over_many_blocks(m):
     _status(m)
 
 
-@pytest.mark.parametrize("impl", [0, 2])
+@pytest.mark.parametrize("impl", [0, 2, 3])
 @pytest.mark.parametrize("hq,hkv", [(32, 8), (8, 8), (32, 4)])
 @pytest.mark.parametrize("T,mem_lens,q_start", [(64, (0, 700, 1537), 0), (24, (4099, 1, 64), 40),
                                                 (300, (130, 2200, 64), 5)])
 def test_sparse_attention_split_long_memory(m, impl, hq, hkv, T, mem_lens, q_start):
-    """Split-key attention over long memories, on tcgen05 (impl 0) and on mma.sync (impl 2): several
-    key ranges per block (some empty), ragged tails, empty memory, causal local keys, several
-    128-row blocks; against the oracle within the bf16 bound."""
+    """Split-key attention over long memories, on tcgen05 with the key ranges merged in a thread-block
+    cluster where the grid allows it (impl 0), on tcgen05 with partial results and a combine pass
+    (impl 3), and on mma.sync (impl 2): several key ranges per block (some empty), ragged tails,
+    empty memory, causal local keys, one and two 128-row blocks per CTA; against the oracle within
+    the bf16 bound."""
     n_q, d, dtype = 3, 128, "bf16"
     max_mem = max(mem_lens) + 5
     L = q_start + T
@@ -432,17 +434,38 @@ def test_sparse_attention_split_long_memory(m, impl, hq, hkv, T, mem_lens, q_sta
         assert m.sparse_attn_split_workspace_size(n_q, T, hq, hkv, max_mem, L) >= 2 * rows * (d * 4 + 8)
     m.attn_set_impl(impl)
     try:
+        plan = m.api.sparse_attn_split_plan(n_q, T, hq, hkv, max_mem, L)
+        natural = 2 if T * (hq // hkv) > 128 else 1
+        if impl == 2:
+            assert plan["row_blocks"] == 0 and plan["cluster"] == 0
+        elif impl == 3 or plan["cluster"] == 0:
+            assert plan["row_blocks"] == natural and plan["cluster"] == 0 if impl == 3 else plan["row_blocks"] == natural
+        else:
+            assert plan["row_blocks"] in (1, natural) and plan["key_ranges"] == plan["cluster"]
+        lse = torch.empty((n_q, T, hq), dtype=torch.float32, device="cuda")
         out = m.msa_sparse_attn_split(upload(q, dtype), upload(mem, dtype), torch.from_numpy(mem_len).cuda(),
-                                      upload(lk, dtype), upload(lv, dtype), L, q_start)
+                                      upload(lk, dtype), upload(lv, dtype), L, q_start, lse=lse)
     finally:
         m.attn_set_impl(0)
     _status(m)
     got = _np(out)
+    scale = 1 / np.sqrt(d)
     for qi in range(n_q):
         ml = mem_len[qi]
-        ref = O.sparse_attention(q[qi], mem[qi, :ml, 0], mem[qi, :ml, 1], lk[qi, :L], lv[qi, :L], q_start,
-                                 1 / np.sqrt(d))
+        ref = O.sparse_attention(q[qi], mem[qi, :ml, 0], mem[qi, :ml, 1], lk[qi, :L], lv[qi, :L], q_start, scale)
         assert _row_rel_err(got[qi], ref) <= 2e-2
+        # the log-sum-exp of each row's logits (merged in the cluster or by the combine pass)
+        ref_lse = np.empty((T, hq))
+        for h in range(hq):
+            g_ = h // (hq // hkv)
+            keys = np.concatenate([mem[qi, :ml, 0, g_], lk[qi, :L, g_]])
+            lg = (q[qi, :, h].astype(np.float64) @ keys.T.astype(np.float64)) * scale
+            vis = np.ones_like(lg, dtype=bool)
+            vis[:, ml:] = np.arange(L)[None, :] <= q_start + np.arange(T)[:, None]
+            lg = np.where(vis, lg, -np.inf)
+            mx = lg.max(axis=1)
+            ref_lse[:, h] = mx + np.log(np.exp(lg - mx[:, None]).sum(axis=1))
+        np.testing.assert_allclose(_np(lse[qi]), ref_lse, atol=2e-3)
 
 
 def test_sparse_attention_split_no_keys_gives_zero_and_rejects_fp32(m):
