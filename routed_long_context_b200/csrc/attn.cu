@@ -457,6 +457,9 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
                                                            const float2* __restrict__ part_ml, int n_split,
                                                            int64_t rows, __nv_bfloat16* __restrict__ out,
                                                            float* __restrict__ lse) {
+    // launched as a programmatic dependent of the split kernel: its blocks may start while the split
+    // kernel finishes; the partial results are read only after it has completed and they are visible
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= rows) return;
@@ -507,9 +510,19 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
 
 msa_status launch_combine(const AttnArgs& a, int n_q, cudaStream_t s) {
     const int64_t rows = (int64_t)n_q * a.T * a.hq;
-    attn_combine_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(a.part_o, a.part_ml, a.n_split, rows,
-                                                                   static_cast<__nv_bfloat16*>(a.out), a.lse);
-    MSA_LAUNCH_CHECK();
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3((unsigned)((rows + 7) / 8), 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    MSA_CUDA_TRY(cudaLaunchKernelEx(&cfg, attn_combine_kernel, static_cast<const float*>(a.part_o),
+                                    static_cast<const float2*>(a.part_ml), a.n_split, rows,
+                                    static_cast<__nv_bfloat16*>(a.out), a.lse));
     return MSA_OK;
 }
 

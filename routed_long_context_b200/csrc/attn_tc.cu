@@ -136,6 +136,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 if (ch == 0) a.part_ml[(int64_t)split * rows_total + gr] = make_float2(ninf, 0.f);
             }
         }
+        asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
         return;
     }
 
@@ -404,9 +405,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             }
             tc_fence_after();
             float s[kKW];
-#pragma unroll
-            for (int c0 = 0; c0 < kKW; c0 += 32)
-                tmem_ld32(tmem_base + lane_off + (uint32_t)((2 * rh + (j & 1)) * kKeys + ch * kKW + c0), s + c0);
+            if constexpr (kKW == 64)
+                tmem_ld64(tmem_base + lane_off + (uint32_t)((2 * rh + (j & 1)) * kKeys), s);
+            else
+                tmem_ld32(tmem_base + lane_off + (uint32_t)((2 * rh + (j & 1)) * kKeys + ch * kKW), s);
             const int kb = k_begin + j * kKeys + ch * kKW;
             // masked keys to -inf where the tile needs it: inside the range and (a memory row or a
             // causal local key)
@@ -496,16 +498,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             const int rr = rh * kRows + rl;
             float* st_row = reinterpret_cast<float*>(sKV) + rr * kD;
             if (ok && work) {
+                float o[kOW];
+                if constexpr (kOW == 128) tmem_ld128(o_tmem, o); else tmem_ld64(o_tmem, o);
 #pragma unroll
-                for (int part = 0; part < kOW / 32; ++part) {
-                    float o[32];
-                    tmem_ld32(o_tmem + (uint32_t)(part * 32), o);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int chunk = (ch * kOW + part * 32) / 4 + i;
-                        *reinterpret_cast<float4*>(st_row + ((chunk ^ (rr & 31)) << 2)) =
-                            make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
-                    }
+                for (int i = 0; i < kOW / 4; ++i) {
+                    const int chunk = ch * (kOW / 4) + i;
+                    *reinterpret_cast<float4*>(st_row + ((chunk ^ (rr & 31)) << 2)) =
+                        make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
                 }
             }
             if (ch == 0)
@@ -517,10 +516,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             // 128-byte pieces instead of 32 scattered 16-byte ones.
             float* slot = reinterpret_cast<float*>(sKV) + (warp - 2) * (32 * 36);
             const int rsub = lane >> 3, c4 = lane & 7;
+            float oall[kOW];
+            if constexpr (kOW == 128) tmem_ld128(o_tmem, oall); else tmem_ld64(o_tmem, oall);
 #pragma unroll
             for (int part = 0; part < kOW / 32; ++part) {
-                float o[32];
-                tmem_ld32(o_tmem + (uint32_t)(part * 32), o);
+                const float* o = oall + part * 32;
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
                     *reinterpret_cast<float4*>(slot + lane * 36 + 4 * i) =
@@ -545,6 +545,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     }
 
     __syncthreads();
+    // the combine pass (a programmatic dependent of this grid) may be scheduled now; it reads the
+    // partial results only after this grid has completed
+    if constexpr (!CL) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (threadIdx.x == 0 && *abort_flag) record_device_error(a.err, MSA_DEV_WAIT_TIMEOUT);
     if (warp == 1) {
         tc_fence_after();
@@ -616,8 +619,8 @@ int attn_tc_splits(int n_q, int T, int hq, int hkv, int max_mem, int L) {
 
 namespace {
 
-// Largest cluster (1, 2, 4, 8 or 16 CTAs, one per key range) such that the whole grid of clusters
-// is resident at once (one wave), or 0 when no cluster launch of this kernel fits.
+// Largest cluster (1 to 16 CTAs, one per key range) such that the whole grid of clusters is
+// resident at once (one wave), or 0 when no cluster launch of this kernel fits.
 // Opts both variants of row-block count NH into their dynamic shared memory and the cluster variant
 // into clusters of up to 16 CTAs, once per device.
 template <int NH>
@@ -664,7 +667,7 @@ template <int NH>
 int pick_cluster_uncached(int64_t base) {
     constexpr int smem = TcShape<NH>::kSmemBytes;
     if (opt_in_tc<NH>() != MSA_OK) return 0;
-    for (int cs = 16; cs >= 1; cs >>= 1) {
+    for (int cs = 16; cs >= 1; --cs) {   // any size: the GPCs hold e.g. 7 clusters of 16 but 8 of 14
         if ((int64_t)cs * base > 148) continue;
         cudaLaunchConfig_t cfg = {};
         cudaLaunchAttribute attr[1];
@@ -719,26 +722,18 @@ msa_status launch_tc(const CUtensorMap& tq, const CUtensorMap& tm, const CUtenso
 
 }  // namespace
 
-// The launch plan: row blocks per CTA (NH) and cluster size (0: partial results + combine). A
-// cluster layout is taken when the whole grid of clusters is resident in one wave and keeps at least
-// min(96, the combine layout's CTA count) SMs busy; the kv head's natural NH first (2 when it has
-// more than 128 rows), then one row block per CTA, whose clusters are half as wide.
+// The launch plan: row blocks per CTA (NH: 2 when the kv head has more than 128 rows) and cluster
+// size (0: partial results + combine). The ranges are merged in a cluster when the whole grid of
+// clusters is resident in one wave with at least 60 % of the combine layout's ranges per row block
+// (measured: clusters of 2 to 5 ranges beat partials + combine by 7-13 %; on the fine stage's 8 kv
+// heads the largest co-resident clusters hold 6 of its 18 ranges and lose to the combine, 37 vs 31 us).
 void choose_tc_plan(int n_q, int T, int hq, int hkv, int n_split, int* nh, int* cs_out) {
     const int G = hq / hkv;
-    const int nh_pref = attn_tc_blocks(T, hq, hkv);
-    const int64_t fallback_ctas =
-        (int64_t)((T * G + nh_pref * kRows - 1) / (nh_pref * kRows)) * hkv * n_q * n_split;
-    for (int NH = nh_pref; NH >= 1; --NH) {
-        const int64_t base = (int64_t)((T * G + NH * kRows - 1) / (NH * kRows)) * hkv * n_q;
-        const int cs = NH == 2 ? pick_cluster<2>(base) : pick_cluster<1>(base);
-        if (cs >= 1 && (int64_t)cs * base >= std::min<int64_t>(96, fallback_ctas)) {
-            *nh = NH;
-            *cs_out = cs;
-            return;
-        }
-    }
-    *nh = nh_pref;
-    *cs_out = 0;
+    const int NH = attn_tc_blocks(T, hq, hkv);
+    const int64_t base = (int64_t)((T * G + NH * kRows - 1) / (NH * kRows)) * hkv * n_q;
+    const int cs = NH == 2 ? pick_cluster<2>(base) : pick_cluster<1>(base);
+    *nh = NH;
+    *cs_out = (cs >= 1 && 10 * cs >= 6 * n_split) ? cs : 0;
 }
 
 msa_status attn_tc_plan(int n_q, int T, int hq, int hkv, int n_split, int* blocks, int* cluster) {
