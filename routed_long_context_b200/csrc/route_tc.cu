@@ -62,6 +62,19 @@ struct TcParams {
 };
 
 // ------------------------------------------------------------------------------------- kernel
+// Max over each of the 32 / T whole queries of one 32-column piece (T static), then the query's
+// flush; every step is unrolled, so the queries' shuffle chains interleave.
+template <int T, typename Flush>
+__device__ __forceinline__ void flush_queries(const float (&v)[32], int q0, int q_end, Flush& flush) {
+#pragma unroll
+    for (int qi = 0; qi < 32 / T; ++qi) {
+        float m = v[qi * T];
+#pragma unroll
+        for (int j = 1; j < T; ++j) m = fmaxf(m, v[qi * T + j]);
+        flush(q0 + qi, m, q0 + qi < q_end);
+    }
+}
+
 template <bool RESIDENT>
 __global__ void __launch_bounds__(kThreads, 1)
     route_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const TcParams p) {
@@ -273,32 +286,66 @@ __global__ void __launch_bounds__(kThreads, 1)
             // 32-column reads stay inside this accumulator's acc_stride columns
             const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * p.acc_stride);
 
-            auto flush = [&](int q, float m) {
-                // segmented max over runs of equal doc among the warp's 32 consecutive chunks
+            // The warp's 32 consecutive chunks form runs of equal document. Which lanes a
+            // segmented max may combine is the same for every query column: bit i of `same` says
+            // lane + 2^i holds this lane's document; `head` marks the first lane of each run.
+            unsigned same = 0;
+#pragma unroll
+            for (int i = 0; i < 5; ++i) {
+                const int od = __shfl_down_sync(0xffffffffu, doc, 1 << i);
+                if (lane + (1 << i) < 32 && od == doc) same |= 1u << i;
+            }
+            const int prev = __shfl_up_sync(0xffffffffu, doc, 1);
+            const bool head = doc >= 0 && (lane == 0 || prev != doc);
+
+            // segmented max of m over the lane's document run, one float atomic max per run
+            auto flush = [&](int q, float m, bool real) {
                 float v = doc >= 0 ? m : ninf;
 #pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const float ov = __shfl_down_sync(0xffffffffu, v, off);
-                    const int od = __shfl_down_sync(0xffffffffu, doc, off);
-                    if (lane + off < 32 && od == doc) v = fmaxf(v, ov);
+                for (int i = 0; i < 5; ++i) {
+                    const float ov = __shfl_down_sync(0xffffffffu, v, 1 << i);
+                    if ((same >> i) & 1u) v = fmaxf(v, ov);
                 }
-                const int prev = __shfl_up_sync(0xffffffffu, doc, 1);
-                if (doc >= 0 && (lane == 0 || prev != doc)) atomic_max_f32(p.doc_scores + (int64_t)q * p.n_docs + doc, v);
-                if (p.chunk_scores && doc >= 0) atomic_max_f32(p.chunk_scores + (int64_t)q * p.n_chunks + c, m);
+                if (real && head) atomic_max_f32(p.doc_scores + (int64_t)q * p.n_docs + doc, v);
+                if (real && p.chunk_scores && doc >= 0) atomic_max_f32(p.chunk_scores + (int64_t)q * p.n_chunks + c, m);
             };
+
+            const int pieces = (max(col_end - n0, 0) + 31) / 32;
+            auto release = [&]() {
+                // every TMEM read of this accumulator is done: hand it back to the MMA warp
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));
+            };
+            if (32 % p.T == 0) {
+                // a query's T columns never straddle a 32-column piece (pieces start at multiples of
+                // 32 and N is a multiple of T): each piece holds 32 / T whole queries, reduced and
+                // flushed without branches; queries past col_end are padding and issue no atomics
+                const int q_end = col_end / p.T;
+                for (int pc = 0; pc < pieces; ++pc) {
+                    float v[32];
+                    tmem_ld32(trow + (uint32_t)(pc * 32), v);
+                    if (pc == pieces - 1) release();
+                    const int q0 = (n0 + pc * 32) / p.T;
+                    switch (p.T) {
+                        case 1: flush_queries<1>(v, q0, q_end, flush); break;
+                        case 2: flush_queries<2>(v, q0, q_end, flush); break;
+                        case 4: flush_queries<4>(v, q0, q_end, flush); break;
+                        case 8: flush_queries<8>(v, q0, q_end, flush); break;
+                        case 16: flush_queries<16>(v, q0, q_end, flush); break;
+                        default: flush_queries<32>(v, q0, q_end, flush); break;
+                    }
+                }
+                if (pieces == 0) release();
+                continue;
+            }
 
             int run_q = -1;
             float run_max = ninf;
-            const int pieces = (max(col_end - n0, 0) + 31) / 32;
             for (int pc = 0; pc < pieces; ++pc) {
                 float v[32];
                 tmem_ld32(trow + (uint32_t)(pc * 32), v);
-                if (pc == pieces - 1) {
-                    // every TMEM read of this accumulator is done: hand it back to the MMA warp
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));
-                }
+                if (pc == pieces - 1) release();
                 const int base_col = n0 + pc * 32;
                 const int hi_col = min(base_col + 32, col_end);
                 for (int q = base_col / p.T; q * p.T < hi_col; ++q) {
@@ -311,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // the query's columns in this tile are complete once they end inside this
                     // piece or the tile's real columns end here; otherwise carry the running max
                     if ((q + 1) * p.T <= hi_col || hi_col == col_end) {
-                        flush(q, m);
+                        flush(q, m, true);
                         run_q = -1;
                     } else {
                         run_q = q;
@@ -319,12 +366,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            if (pieces == 0) {
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));
-            }
-            if (run_q >= 0) flush(run_q, run_max);
+            if (pieces == 0) release();
+            if (run_q >= 0) flush(run_q, run_max, true);
         }
     }
 

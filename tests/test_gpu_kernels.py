@@ -230,7 +230,10 @@ def test_route_fp32_cuda_cores(m, n_q, T):
     _status(m)
 
 
-@pytest.mark.parametrize("n_q,T", [(1, 16), (1, 64), (2, 48), (3, 100), (32, 1), (8, 128), (1, 3)])
+# (n_q, T) with T dividing 32 take the epilogue that reduces whole queries per 32-column piece:
+# padded column blocks (N = 3, 20), two query-column tiles (N = 288, 300, 320) and T = 1..32
+@pytest.mark.parametrize("n_q,T", [(1, 16), (1, 64), (2, 48), (3, 100), (32, 1), (8, 128), (1, 3), (3, 1), (5, 4),
+                                   (7, 2), (9, 32), (20, 16), (300, 1), (4, 8)])
 @pytest.mark.parametrize("impl", [2, 1, 3])
 def test_route_bf16_tensor_cores_and_cuda_cores(m, n_q, T, impl):
     from routed_long_context_b200.bank import BankLayout
