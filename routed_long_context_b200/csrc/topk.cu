@@ -7,10 +7,12 @@
 // (warp arg-max over list heads, the winner's lane pops its head), and write their KT best to
 // the workspace. The last block of a query to finish (an atomic ticket, no spinning) merges the
 // P lists and writes the first k. Reading the partial lists goes through L2 (__ldcg).
+#include <algorithm>
 #include <climits>
 #include <mutex>
 
 #include "common.cuh"
+#include "tc.cuh"
 
 namespace msa {
 namespace {
@@ -165,10 +167,13 @@ int pick_blocks(int64_t n_docs) {
 
 // ------------------------------------------------------------------------------------------------
 // k <= 32: warp-distributed lists. Lane i of a warp holds rank i of the warp's sorted list
-// (lanes >= k hold sentinels). A batch of 32 candidates (one per lane) is filtered against the
-// list's k-th entry with one ballot; each survivor is inserted by a rank count (popc of a ballot)
-// and a one-lane shift. Per block: each warp scans a strided slice, then warp 0 folds the other
-// warps' lists in; the last block of a query (atomic ticket) folds the per-block lists.
+// (lanes >= k hold sentinels). A warp loads 16 batches of 32 docs (one per lane each) at a time
+// and keeps only the entries not worse than a threshold that already has k entries at least as
+// good as it; those survivors (few, once the list has filled) go in 32 at a time: filtered against
+// the list's k-th entry with one ballot, each one inserted by a rank count (popc of a ballot) and a
+// one-lane shift, or, when more than two survive, sorted and merged in one go. Per block warp 0
+// folds the other warps' lists in; with one block per query that is the result, otherwise the
+// last block of a query (atomic ticket) folds the per-block lists.
 // ------------------------------------------------------------------------------------------------
 struct WList {
     float s;
@@ -251,49 +256,148 @@ __device__ __forceinline__ void wl_insert_batch(WList& w, int k, float cv, int c
     }
 }
 
-constexpr int kWarpTopkThreads = 256;
+// One out-of-line copy of the batch insert for the scan's many call sites (the inlined copies
+// would not fit the instruction cache).
+__device__ __noinline__ WList wl_insert_batch_call(WList w, int k, float cv, int ci, bool valid) {
+    wl_insert_batch(w, k, cv, ci, valid);
+    return w;
+}
 
+constexpr int kWarpTopkThreads = 256;
+constexpr int kRoundBatches = 16;   // batches of 32 docs a warp loads before filtering them
+
+// CL: the P blocks of a query form one thread-block cluster and fold their lists over distributed
+// shared memory (no partial lists in global memory, no ticket); otherwise the last block to finish
+// folds the partial lists.
+template <bool CL>
 __global__ void __launch_bounds__(kWarpTopkThreads) topk_warp_kernel(const float* __restrict__ scores, int64_t n_docs,
                                                                       int k, int P, float* part_s, int* part_i,
                                                                       int* counters, int32_t* out_idx, float* out_score) {
     constexpr int W = kWarpTopkThreads / 32;
-    __shared__ float ls[W][32];
-    __shared__ int li[W][32];
+    // per warp: staged candidates during the scan, then its list for the block's fold
+    __shared__ float stage_s[W][64];
+    __shared__ int stage_i[W][64];
+    __shared__ float2 cl_list[32];     // the block's list, read by the cluster's first block
     __shared__ int is_last;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int q = blockIdx.y;
     const float* row = scores + (int64_t)q * n_docs;
     WList w;
     wl_clear(w);
-    // this warp's slice: chunks of 32 consecutive docs, strided over all warps of all blocks
+    // this warp's slice: batches of 32 consecutive docs, strided over all warps of all blocks,
+    // taken kRoundBatches at a time. Per round only the candidates that can still be among the k
+    // best reach the list: those not worse than a threshold that has at least k seen entries at
+    // least as good as it (the list's k-th entry, tightened, when that leaves more than one batch,
+    // by the k-th best of the lanes' own best entries). Survivors are staged in shared memory
+    // (at most 63 at a time) and go in 32 at a time.
     const int64_t gw = (int64_t)blockIdx.x * W + warp, nw = (int64_t)P * W;
-    for (int64_t base = gw * 32; base < n_docs; base += nw * 32 * 8) {
-        float v[8];
+    float* st_s = stage_s[warp];
+    int* st_i = stage_i[warp];
+    for (int64_t base = gw * 32; base < n_docs; base += nw * 32 * kRoundBatches) {
+        float v[kRoundBatches];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
+        for (int u = 0; u < kRoundBatches; ++u) {
             const int64_t i = base + u * nw * 32 + lane;
             v[u] = i < n_docs ? __ldg(row + i) : -__int_as_float(0x7f800000);
         }
+        float ts = __shfl_sync(0xffffffffu, w.s, k - 1);
+        int ti = __shfl_sync(0xffffffffu, w.i, k - 1);
+        int count = 0;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
+        for (int u = 0; u < kRoundBatches; ++u) {
             const int64_t i = base + u * nw * 32 + lane;
-            wl_insert_batch(w, k, v[u], (int)i, i < n_docs);
+            count += __popc(__ballot_sync(0xffffffffu, i < n_docs && !better(ts, ti, v[u], (int)i)));
+        }
+        if (count > 32) {
+            float bs = -__int_as_float(0x7f800000);
+            int bi = INT_MAX;
+#pragma unroll
+            for (int u = 0; u < kRoundBatches; ++u) {
+                const int64_t i = base + u * nw * 32 + lane;
+                if (i < n_docs && better(v[u], (int)i, bs, bi)) bs = v[u], bi = (int)i;
+            }
+            warp_sort32(bs, bi);
+            const float ks = __shfl_sync(0xffffffffu, bs, k - 1);
+            const int ki = __shfl_sync(0xffffffffu, bi, k - 1);
+            if (better(ks, ki, ts, ti)) ts = ks, ti = ki;
+        }
+        int n_st = 0;
+#pragma unroll
+        for (int u = 0; u < kRoundBatches; ++u) {
+            const int64_t i = base + u * nw * 32 + lane;
+            const bool keep = i < n_docs && !better(ts, ti, v[u], (int)i);
+            const unsigned mk = __ballot_sync(0xffffffffu, keep);
+            if (keep) {
+                const int pos = n_st + __popc(mk & ((1u << lane) - 1u));
+                st_s[pos] = v[u];
+                st_i[pos] = (int)i;
+            }
+            n_st += __popc(mk);
+            if (n_st >= 32) {
+                // a full batch goes in; the rest (at most 31) moves to the front
+                __syncwarp();
+                const float cs = st_s[lane];
+                const int ci = st_i[lane];
+                const bool more = lane + 32 < n_st;
+                const float ms = more ? st_s[lane + 32] : 0.0f;
+                const int mi = more ? st_i[lane + 32] : 0;
+                __syncwarp();
+                if (more) st_s[lane] = ms, st_i[lane] = mi;
+                n_st -= 32;
+                w = wl_insert_batch_call(w, k, cs, ci, true);
+                __syncwarp();
+            }
+        }
+        if (n_st > 0) {
+            __syncwarp();
+            const bool ok = lane < n_st;
+            const float cs = ok ? st_s[lane] : -__int_as_float(0x7f800000);
+            const int ci = ok ? st_i[lane] : INT_MAX;
+            __syncwarp();
+            w = wl_insert_batch_call(w, k, cs, ci, ok);
         }
     }
     // fold the block's warp lists (sorted) into warp 0's
-    ls[warp][lane] = w.s;
-    li[warp][lane] = w.i;
+    stage_s[warp][lane] = w.s;
+    stage_i[warp][lane] = w.i;
     __syncthreads();
     if (warp == 0) {
-        for (int o = 1; o < W; ++o) warp_merge32(w, ls[o][lane], li[o][lane]);
-        part_s[((int64_t)q * P + blockIdx.x) * 32 + lane] = w.s;
-        part_i[((int64_t)q * P + blockIdx.x) * 32 + lane] = w.i;
-        __threadfence();
-        __syncwarp();
-        if (lane == 0) is_last = (atomicAdd(counters + q, 1) == P - 1);
+        for (int o = 1; o < W; ++o) warp_merge32(w, stage_s[o][lane], stage_i[o][lane]);
+        if (P == 1) {
+            // one block per query: its list is the result (no partial lists, no ticket)
+            if (lane < k) {
+                out_idx[(int64_t)q * k + lane] = w.i;
+                if (out_score) out_score[(int64_t)q * k + lane] = w.s;
+            }
+        } else if (CL) {
+            cl_list[lane] = make_float2(w.s, __int_as_float(w.i));
+        } else {
+            part_s[((int64_t)q * P + blockIdx.x) * 32 + lane] = w.s;
+            part_i[((int64_t)q * P + blockIdx.x) * 32 + lane] = w.i;
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) is_last = (atomicAdd(counters + q, 1) == P - 1);
+        }
+    }
+    if (CL) {
+        // every block's list is in its shared memory after the first barrier; the cluster's first
+        // block folds them in, and the second barrier keeps them in place until it has
+        cluster_sync_all();
+        if (cluster_ctarank() == 0 && warp == 0 && P > 1) {
+            for (int r = 1; r < P; ++r) {
+                const float2 e = ld_cluster_f2(cluster_map(smem_u32(&cl_list[lane]), (uint32_t)r));
+                warp_merge32(w, e.x, __float_as_int(e.y));
+            }
+            if (lane < k) {
+                out_idx[(int64_t)q * k + lane] = w.i;
+                if (out_score) out_score[(int64_t)q * k + lane] = w.s;
+            }
+        }
+        cluster_sync_all();
+        return;
     }
     __syncthreads();
-    if (!is_last) return;
+    if (P == 1 || !is_last) return;
     // last block: warp w folds partial lists w, w + W, ... (loads first), then warp 0 folds the warps
     __threadfence();
     wl_clear(w);
@@ -312,11 +416,11 @@ __global__ void __launch_bounds__(kWarpTopkThreads) topk_warp_kernel(const float
             if (b0 + u * W < P) warp_merge32(w, cv[u], ci[u]);
     }
     __syncthreads();
-    ls[warp][lane] = w.s;
-    li[warp][lane] = w.i;
+    stage_s[warp][lane] = w.s;
+    stage_i[warp][lane] = w.i;
     __syncthreads();
     if (warp == 0) {
-        for (int o = 1; o < W; ++o) warp_merge32(w, ls[o][lane], li[o][lane]);
+        for (int o = 1; o < W; ++o) warp_merge32(w, stage_s[o][lane], stage_i[o][lane]);
         if (lane < k) {
             out_idx[(int64_t)q * k + lane] = w.i;
             if (out_score) out_score[(int64_t)q * k + lane] = w.s;
@@ -325,13 +429,102 @@ __global__ void __launch_bounds__(kWarpTopkThreads) topk_warp_kernel(const float
 }
 
 int pick_blocks_warp(int64_t n_docs) {
-    // about 16 batches of 32 docs per warp: few partial lists for the last block to fold
-    int64_t p = (n_docs + kWarpTopkThreads * 16 - 1) / (kWarpTopkThreads * 16);
+    // two rounds of kRoundBatches batches of 32 docs per warp: up to 8,192 docs take one block
+    // per query (no ticket), and few partial lists are left for the last block to fold
+    const int64_t per_block = (int64_t)kWarpTopkThreads * kRoundBatches * 2;
+    int64_t p = (n_docs + per_block - 1) / per_block;
     const int64_t cap = (int64_t)sm_count() * 2;
     if (p > cap) p = cap;
     if (p < 1) p = 1;
     return (int)p;
 }
+constexpr int kMaxTopkCluster = 16;   // above 8 a non-portable cluster size
+
+// k <= 32: up to 8,192 docs take one block per query; up to 131,072 the query's blocks (at most
+// 16, each on at most 8,192 docs: two rounds per warp) form one cluster; beyond that the ticket
+// fold (measured faster there than clusters whose warps take more rounds).
+void warp_plan(int64_t n_docs, int* P, bool* cluster) {
+    const int64_t per_block = (int64_t)kWarpTopkThreads * kRoundBatches * 2;
+    const int64_t pc = (n_docs + per_block - 1) / per_block;
+    if (pc <= 1) {
+        *P = 1;
+        *cluster = false;
+    } else if (pc <= kMaxTopkCluster) {
+        *P = (int)pc;
+        *cluster = true;
+    } else {
+        *P = pick_blocks_warp(n_docs);
+        *cluster = false;
+    }
+}
+
+// Clusters of more than 8 blocks need the kernel's opt-in, set once per device.
+msa_status allow_large_topk_cluster() {
+    static std::mutex mu;
+    static bool done[64] = {false};
+    int dev = 0;
+    MSA_CUDA_TRY(cudaGetDevice(&dev));
+    std::lock_guard<std::mutex> lk(mu);
+    if (dev >= 0 && dev < 64 && done[dev]) return MSA_OK;
+    MSA_CUDA_TRY(cudaFuncSetAttribute(topk_warp_kernel<true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+    if (dev >= 0 && dev < 64) done[dev] = true;
+    return MSA_OK;
+}
+
+// Launches the selection with the workspace (or scratch) w laid out as msa_topk_workspace_size
+// sizes it: partial scores, partial indices, one ticket per query.
+msa_status launch_topk(const float* doc_scores, int n_q, int64_t n_docs, int k, int32_t* idx, float* score, char* w,
+                       cudaStream_t s) {
+    const bool warp_lists = k <= 32;
+    const int P_ws = warp_lists ? pick_blocks_warp(n_docs) : pick_blocks(n_docs);
+    const int KT = warp_lists ? 32 : pick_kt(k);
+    const size_t lists = (size_t)n_q * P_ws * KT;
+    float* part_s = reinterpret_cast<float*>(w);
+    int* part_i = reinterpret_cast<int*>(w + align_up(lists * 4, 256));
+    int* counters = reinterpret_cast<int*>(w + 2 * align_up(lists * 4, 256));
+    if (warp_lists) {
+        int P = 1;
+        bool cluster = false;
+        warp_plan(n_docs, &P, &cluster);
+        if (cluster) {
+            cudaLaunchConfig_t cfg{};
+            cfg.gridDim = dim3((unsigned)P, (unsigned)n_q);
+            cfg.blockDim = dim3(kWarpTopkThreads);
+            cfg.dynamicSmemBytes = 0;
+            cfg.stream = s;
+            cudaLaunchAttribute at[1];
+            at[0].id = cudaLaunchAttributeClusterDimension;
+            at[0].val.clusterDim.x = (unsigned)P;
+            at[0].val.clusterDim.y = 1;
+            at[0].val.clusterDim.z = 1;
+            cfg.attrs = at;
+            cfg.numAttrs = 1;
+            if (P > 8) MSA_RETURN_IF(allow_large_topk_cluster());
+            MSA_CUDA_TRY(cudaLaunchKernelEx(&cfg, topk_warp_kernel<true>, doc_scores, n_docs, k, P, part_s, part_i,
+                                            counters, idx, score));
+            MSA_LAUNCH_CHECK();
+            return MSA_OK;
+        }
+        // tickets start at zero (one block per query takes none)
+        if (P > 1) MSA_CUDA_TRY(cudaMemsetAsync(counters, 0, (size_t)n_q * sizeof(int), s));
+        topk_warp_kernel<false><<<dim3(P, n_q), kWarpTopkThreads, 0, s>>>(doc_scores, n_docs, k, P, part_s, part_i,
+                                                                          counters, idx, score);
+        MSA_LAUNCH_CHECK();
+        return MSA_OK;
+    }
+    const int P = P_ws;
+    MSA_CUDA_TRY(cudaMemsetAsync(counters, 0, (size_t)n_q * sizeof(int), s));
+    dim3 grid(P, n_q);
+    switch (KT) {
+        case 8: topk_kernel<8><<<grid, kTopkThreads, 0, s>>>(doc_scores, n_docs, k, P, part_s, part_i, counters, idx, score); break;
+        case 16: topk_kernel<16><<<grid, kTopkThreads, 0, s>>>(doc_scores, n_docs, k, P, part_s, part_i, counters, idx, score); break;
+        case 32: topk_kernel<32><<<grid, kTopkThreads, 0, s>>>(doc_scores, n_docs, k, P, part_s, part_i, counters, idx, score); break;
+        default: topk_kernel<64><<<grid, kTopkThreads, 0, s>>>(doc_scores, n_docs, k, P, part_s, part_i, counters, idx, score); break;
+    }
+    MSA_LAUNCH_CHECK();
+    return MSA_OK;
+}
+
 }  // namespace
 }  // namespace msa
 
@@ -359,30 +552,7 @@ msa_status msa_topk_docs(const float* doc_scores, int n_q, int64_t n_docs, int k
     size_t need = 0;
     MSA_RETURN_IF(msa_topk_workspace_size(n_q, n_docs, k, &need));
     if (ws_bytes < need) return set_error(MSA_ERR_WORKSPACE, "msa_topk_docs: workspace %zu < %zu", ws_bytes, need);
-    const bool warp_lists = k <= 32;
-    const int P = warp_lists ? pick_blocks_warp(n_docs) : pick_blocks(n_docs);
-    const int KT = warp_lists ? 32 : pick_kt(k);
-    const size_t lists = (size_t)n_q * P * KT;
-    char* w = static_cast<char*>(ws);
-    float* part_s = reinterpret_cast<float*>(w);
-    int* part_i = reinterpret_cast<int*>(w + align_up(lists * 4, 256));
-    int* counters = reinterpret_cast<int*>(w + 2 * align_up(lists * 4, 256));
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    MSA_CUDA_TRY(cudaMemsetAsync(counters, 0, (size_t)n_q * sizeof(int), s));
-    dim3 grid(P, n_q);
-    if (warp_lists) {
-        topk_warp_kernel<<<grid, kWarpTopkThreads, 0, s>>>(doc_scores, n_docs, k, P, part_s, part_i, counters, idx, score);
-        MSA_LAUNCH_CHECK();
-        return MSA_OK;
-    }
-    switch (KT) {
-        case 8: topk_kernel<8><<<grid, kTopkThreads, 0, s>>>(doc_scores, n_docs, k, P, part_s, part_i, counters, idx, score); break;
-        case 16: topk_kernel<16><<<grid, kTopkThreads, 0, s>>>(doc_scores, n_docs, k, P, part_s, part_i, counters, idx, score); break;
-        case 32: topk_kernel<32><<<grid, kTopkThreads, 0, s>>>(doc_scores, n_docs, k, P, part_s, part_i, counters, idx, score); break;
-        default: topk_kernel<64><<<grid, kTopkThreads, 0, s>>>(doc_scores, n_docs, k, P, part_s, part_i, counters, idx, score); break;
-    }
-    MSA_LAUNCH_CHECK();
-    return MSA_OK;
+    return launch_topk(doc_scores, n_q, n_docs, k, idx, score, static_cast<char*>(ws), static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"
@@ -449,31 +619,8 @@ msa_status msa_topk_docs_noalloc(const float* doc_scores, int n_q, int64_t n_doc
                          n_q, (long long)n_docs, k, need, kNoAllocScratchBytes);
     void* ws = nullptr;
     MSA_RETURN_IF(scratch_address(&ws));
-    const bool warp_lists = k <= 32;
-    const int P = warp_lists ? pick_blocks_warp(n_docs) : pick_blocks(n_docs);
-    const int KT = warp_lists ? 32 : pick_kt(k);
-    const size_t lists = (size_t)n_q * P * KT;
-    char* w = static_cast<char*>(ws);
-    float* part_s = reinterpret_cast<float*>(w);
-    int* part_i = reinterpret_cast<int*>(w + align_up(lists * 4, 256));
-    int* counters = reinterpret_cast<int*>(w + 2 * align_up(lists * 4, 256));
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // the array keeps the previous call's contents: the tickets must start at zero
-    MSA_CUDA_TRY(cudaMemsetAsync(counters, 0, (size_t)n_q * sizeof(int), s));
-    dim3 grid(P, n_q);
-    if (warp_lists) {
-        topk_warp_kernel<<<grid, kWarpTopkThreads, 0, s>>>(doc_scores, n_docs, k, P, part_s, part_i, counters, idx, score);
-        MSA_LAUNCH_CHECK();
-        return MSA_OK;
-    }
-    switch (KT) {
-        case 8: topk_kernel<8><<<grid, kTopkThreads, 0, s>>>(doc_scores, n_docs, k, P, part_s, part_i, counters, idx, score); break;
-        case 16: topk_kernel<16><<<grid, kTopkThreads, 0, s>>>(doc_scores, n_docs, k, P, part_s, part_i, counters, idx, score); break;
-        case 32: topk_kernel<32><<<grid, kTopkThreads, 0, s>>>(doc_scores, n_docs, k, P, part_s, part_i, counters, idx, score); break;
-        default: topk_kernel<64><<<grid, kTopkThreads, 0, s>>>(doc_scores, n_docs, k, P, part_s, part_i, counters, idx, score); break;
-    }
-    MSA_LAUNCH_CHECK();
-    return MSA_OK;
+    // the array keeps the previous call's contents: launch_topk zeroes the tickets it uses
+    return launch_topk(doc_scores, n_q, n_docs, k, idx, score, static_cast<char*>(ws), static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

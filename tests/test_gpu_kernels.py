@@ -284,6 +284,34 @@ def test_topk_exact_with_ties(m, n_q, D, k):
     np.testing.assert_array_equal(val.cpu().numpy(), ref_v.astype(np.float32))
 
 
+@pytest.mark.parametrize("pattern", ["ascending", "descending", "all_equal", "few_finite", "sawtooth"])
+@pytest.mark.parametrize("n_q,D,k", [(1, 97657, 16), (2, 8192, 32), (3, 8193, 1), (1, 16385, 7), (4, 600, 5),
+                                     (1, 131072, 32), (2, 131073, 16)])
+def test_topk_exact_on_adversarial_orders(m, pattern, n_q, D, k):
+    """Orders that defeat a pruning threshold: the best entries last (every round brings better
+    candidates), all scores equal (ties decided by index alone), nearly all -inf, and a sawtooth
+    whose teeth all reach the same maximum. One block per query up to 8,192 docs, a cluster of up to
+    16 blocks up to 131,072, the ticket fold above."""
+    base = np.arange(D, dtype=np.float64)
+    if pattern == "ascending":
+        row = base / D
+    elif pattern == "descending":
+        row = 1.0 - base / D
+    elif pattern == "all_equal":
+        row = np.zeros(D)
+    elif pattern == "few_finite":
+        row = np.full(D, -np.inf)
+        row[(np.arange(k + 3) * 7919) % D] = np.linspace(0.0, 1.0, k + 3)
+    else:
+        row = (base % 97) / 96.0
+    s = np.stack([np.roll(row, 13 * q) for q in range(n_q)]).astype(np.float32)
+    idx, val = m.msa_topk_docs(torch.from_numpy(s).cuda(), k)
+    ref_i, ref_v = O.topk_docs(s, k)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ref_i)
+    np.testing.assert_array_equal(val.cpu().numpy(), ref_v.astype(np.float32))
+    _status(m)
+
+
 def test_topk_repeatable(m):
     s = torch.from_numpy((np.round(_gen(70, (4, 50000)) * 8) / 8).astype(np.float32)).cuda()
     a, _ = m.msa_topk_docs(s, 16)
