@@ -43,6 +43,11 @@ constexpr int kSmemBudget = 188 * 1024;
 std::atomic<int> g_max_stages{0};     // testing knob: 0 = as many stages as the budget allows
 std::atomic<int> g_inject_stall{0};   // testing knob: make the next launches' waits time out
 constexpr int kStageA = BM * BK * 2;  // 16 KB
+constexpr int kBarBytes = 512;       // mbarriers, TMEM slot, abort flag, tile queue
+// T = 1 epilogue: each epilogue warp's 32 x 32 score block, transposed through shared memory
+// (row stride 33 floats: conflict-free both ways), and its 32 chunks' documents
+constexpr int kEpiStride = 33;
+constexpr int kEpiBytes = 4 * 32 * kEpiStride * 4 + 4 * 32 * 4;
 
 struct TcParams {
     int64_t n_chunks;
@@ -59,6 +64,7 @@ struct TcParams {
     int* err;
     int* tile_counter;     // zero at launch; tiles are handed out in order by atomicAdd
     int inject_stall;      // testing: the producer never publishes a tile, so every other wait times out
+    int transpose;         // T = 1: the epilogue walks each query's column (kEpiBytes after the barriers)
 };
 
 // ------------------------------------------------------------------------------------- kernel
@@ -96,6 +102,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tqe + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     volatile int* tile_q = abort_flag + 1;    // [2] tile index per queue entry, -1 = no more tiles
+    float* epi_buf = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + kBarBytes);   // [4][32][33]
+    int* epi_doc = reinterpret_cast<int*>(epi_buf + 4 * 32 * kEpiStride);                      // [4][32]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -286,6 +294,56 @@ __global__ void __launch_bounds__(kThreads, 1)
             // 32-column reads stay inside this accumulator's acc_stride columns
             const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * p.acc_stride);
 
+            if (p.transpose) {
+                // T = 1: lane = chunk on the way in, lane = query on the way out. The warp's 32 x 32
+                // block goes through shared memory transposed; each lane then walks its query's
+                // column down the 32 chunks, whose document runs are the same for every lane
+                // (uniform branches), and one atomic per run covers 32 queries.
+                float* tb = epi_buf + quarter * (32 * kEpiStride);
+                int* td = epi_doc + quarter * 32;
+                td[lane] = doc;
+                const int pieces = (max(col_end - n0, 0) + 31) / 32;
+                for (int pc = 0; pc < pieces; ++pc) {
+                    float v[32];
+                    tmem_ld32(trow + (uint32_t)(pc * 32), v);
+                    if (pc == pieces - 1) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));
+                    }
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) tb[j * kEpiStride + lane] = v[j];
+                    __syncwarp();
+                    const int q = n0 + pc * 32 + lane;
+                    const bool real = q < col_end;
+                    float* qrow = p.doc_scores + (int64_t)q * p.n_docs;
+                    float m = ninf;
+                    int run_doc = -1;
+#pragma unroll
+                    for (int cc = 0; cc < 32; ++cc) {
+                        const int dc = td[cc];
+                        const float x = tb[lane * kEpiStride + cc];
+                        if (dc != run_doc) {
+                            if (run_doc >= 0 && real) atomic_max_f32(qrow + run_doc, m);
+                            run_doc = dc;
+                            m = x;
+                        } else {
+                            m = fmaxf(m, x);
+                        }
+                        if (p.chunk_scores && dc >= 0 && real)
+                            atomic_max_f32(p.chunk_scores + (int64_t)q * p.n_chunks + (m0 + quarter * 32 + cc), x);
+                    }
+                    if (run_doc >= 0 && real) atomic_max_f32(qrow + run_doc, m);
+                    __syncwarp();
+                }
+                if (pieces == 0) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));
+                }
+                continue;
+            }
+
             // The warp's 32 consecutive chunks form runs of equal document. Which lanes a
             // segmented max may combine is the same for every query column: bit i of `same` says
             // lane + 2^i holds this lane's document; `head` marks the first lane of each run.
@@ -454,11 +512,11 @@ struct Plan {
 // Streamed qhat is the default: the query block is re-read from L2 with every index tile, which
 // leaves shared memory for more index stages in flight (measured faster than keeping qhat
 // resident at 64 columns). `resident` asks for qhat held in shared memory when it fits.
-bool make_plan(int N, int K, Plan* pl, bool resident = false) {
+bool make_plan(int N, int K, Plan* pl, bool resident = false, bool transpose = false) {
     if (N <= 0 || K <= 0 || K % BK != 0 || K > 8192) return false;
     const int kblocks = K / BK;
     const int n16 = (N + 15) / 16 * 16;
-    const size_t fixed = 1024 + 512;
+    const size_t fixed = 1024 + kBarBytes + (transpose ? kEpiBytes : 0);
     if (resident && n16 <= 64) {
         const size_t b = (size_t)kblocks * n16 * BK * 2;
         if (fixed + b + 4 * kStageA <= (size_t)kSmemLimit) {
@@ -507,7 +565,8 @@ int route_tc_pad_rows(int N, int K, bool resident) {
 
 msa_status launch_route_tc(const RouteTcArgs& a, cudaStream_t s) {
     Plan pl;
-    if (!make_plan(a.N, a.K, &pl, a.resident) || pl.n_pad != a.n_pad)
+    const bool transpose = a.T == 1;
+    if (!make_plan(a.N, a.K, &pl, a.resident, transpose) || pl.n_pad != a.n_pad)
         return set_error(MSA_ERR_UNSUPPORTED, "route (tensor cores): unsupported shape N=%d K=%d", a.N, a.K);
     CUtensorMap tmA, tmB;
     MSA_RETURN_IF(make_map(&tmA, a.index, (uint64_t)a.K, (uint64_t)a.n_chunks, BM, true));
@@ -532,6 +591,7 @@ msa_status launch_route_tc(const RouteTcArgs& a, cudaStream_t s) {
     p.err = a.err;
     p.tile_counter = a.tile_counter;
     p.inject_stall = g_inject_stall.load();
+    p.transpose = transpose ? 1 : 0;
     if (!p.tile_counter) return set_error(MSA_ERR_INVALID_ARG, "route (tensor cores): no tile counter");
     int64_t grid = p.n_tiles < (int64_t)sm_count() ? p.n_tiles : (int64_t)sm_count();
     if (a.grid_cap > 0 && grid > a.grid_cap) grid = a.grid_cap;
