@@ -26,8 +26,8 @@ METRIC = "memory tokens routed/s per layer at 100M (frac of HBM peak); route+att
 UNIT = "memory tokens/s"
 TOKENS_PER_CHUNK = 128
 # DRAM bytes (read + write) of one full-size router launch: ncu --set full on a 99,994-chunk case of
-# the current kernel (205.48 MB read + 3.63 MB written), scaled by the chunk count to 781,250 chunks.
-ROUTER_TRAFFIC_BYTES = (205.48e6 + 3.63e6) * 781250 / 99994
+# the current kernel (205.53 MB read + 3.54 MB written), scaled by the chunk count to 781,250 chunks.
+ROUTER_TRAFFIC_BYTES = (205.53e6 + 3.54e6) * 781250 / 99994
 
 
 def parse():
@@ -323,16 +323,31 @@ class OneLayerRound:
         torch.cuda.synchronize()
         return a.elapsed_time(b) / steps, sum(e[0].elapsed_time(e[1]) for e in evs) / steps
 
+    def graph_device(self, steps, warmup):
+        """ms per step of the round captured once into a CUDA graph (msa_interleave_graph_*) and
+        replayed on the compute stream; None with host-issued copies (fetch_mode 0), which wait on
+        the host and cannot be captured."""
+        if self.rd.args.fetch_mode != 1:
+            return None
+        self.graph = self.rd.capture(self.compute)
+        return device_ms(lambda: self.graph.launch(self.compute), steps, warmup, self.compute)
+
     def e2e(self, steps, warmup):
         """ms per step with the step's query-side inputs copied host -> device before it and its output
-        read back after it, serialised on the compute stream (latency, no overlap between steps)."""
+        read back after it, serialised on the compute stream (latency, no overlap between steps); the
+        round itself is the graph replay when one was captured."""
         import torch
+
+        graph = getattr(self, "graph", None)
 
         def one():
             with torch.cuda.stream(self.compute):
                 for h, n in zip(self.h_in, self.names):
                     self.dv[n].copy_(h, non_blocking=True)
-            self.step()
+            if graph is not None:
+                graph.launch(self.compute)
+            else:
+                self.step()
             with torch.cuda.stream(self.compute):
                 self.h_out.copy_(self.out, non_blocking=True)
 
@@ -401,7 +416,9 @@ def _oracle_step_fn(w, krb, kv_of, n_chunks_scale=1.0):
 
 def _round_entry(name, metric, w, lay, rb, steps, warmup, pk, route_kind, notes, cpu):
     """Entry of a one-layer round configuration: device step latency, router roofline, e2e, oracle."""
-    ms, route_ms = rb.device(steps, warmup)
+    eager_ms, route_ms = rb.device(steps, warmup)
+    graph_ms = rb.graph_device(steps, warmup)
+    ms = graph_ms if graph_ms is not None else eager_ms
     e_ms, h2d, d2h = rb.e2e(steps, warmup)
     elem = 4 if w.dtype == "f32" else 2
     route_bytes = lay.n_chunks * w.H * w.d * elem
@@ -418,12 +435,16 @@ def _round_entry(name, metric, w, lay, rb, steps, warmup, pk, route_kind, notes,
     roof["note"] = notes
     sel = rb.idx_host.numpy()
     planted_ok = all(set(w.expected(0, 0, q)) <= set(sel[q].tolist()) for q in range(w.n_q))
+    launch = ("one CUDA graph replay of the captured round (msa_interleave_graph_launch)" if graph_ms is not None
+              else "msa_interleave_step (host-issued copies: not capturable)")
     return {"workload": name, "metric": metric, "value": ms * 1e3, "unit": "us per step", "higher_is_better": False,
-            "ms_per_step": ms, "steps": steps, "route_us_per_launch": route_ms * 1e3, "roofline": roof,
+            "ms_per_step": ms, "steps": steps, "launch": launch, "eager_us_per_step": eager_ms * 1e3,
+            "route_us_per_launch": route_ms * 1e3, "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": {"value": e_ms * 1e3, "unit": "us per step", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "how": "public API (msa_interleave_step) with pinned host buffers: the step's query-side inputs "
-                           "copied in and its output read back inside the timed region, serialised (latency)"},
+                    "how": "public API (msa_interleave_graph_launch, or msa_interleave_step without a graph) with "
+                           "pinned host buffers: the step's query-side inputs copied in and its output read back "
+                           "inside the timed region, serialised (latency)"},
             "checks": {"planted_docs_selected": planted_ok, "device_status": rb.m.device_status()}}
 
 

@@ -601,3 +601,32 @@ def test_new_kernels_write_nothing_past_their_outputs(m):
         assert _tail_intact(b_, n_, 0x7FC0BEEF)
     assert _tail_intact(bb, bn, 0x3C5A)
     assert _tail_intact(mb, mn, 0x5A5A5A5A) and _tail_intact(sb, sn, 0x7FC0DEAD)
+
+
+@pytest.mark.parametrize("D", [600, 20000, 140000])
+def test_topk_and_router_write_nothing_past_their_outputs(m, D):
+    """Canary words after the top-k outputs (one block per query, one cluster per query, the ticket
+    fold) and after the router's document and chunk scores at T = 1 (the transposed epilogue) with a
+    ragged last tile stay untouched."""
+    from routed_long_context_b200.bank import BankLayout
+
+    f32 = torch.float32
+    s = torch.rand((3, D), device="cuda")
+    idx, ib, in_ = _canaried((3, 16), torch.int32, 0x5A5A5A5A)
+    sc, sb, sn = _canaried((3, 16), f32, 0x7FC0DEAD)
+    m.msa_topk_docs(s, 16, idx=idx, score=sc)
+    counts = 1 + rng.uniform_int(SEED, 990, 100, 7).astype(np.int64)     # 1..7 chunks per doc
+    lay = BankLayout(counts)
+    C = int(counts.sum())
+    index = upload(rng.round_to(O.unit(_gen(991, (C, 8, 128))).astype(np.float32), "bf16").reshape(C, 8, 128),
+                   "bf16")
+    qr = upload(_gen(992, (33, 1, 8, 128), "bf16"), "bf16")
+    ds, db, dn = _canaried((33, lay.n_docs), f32, 0x7FC0DEAD)
+    cs_, cb, cn = _canaried((33, C), f32, 0x7FC0DEAD)
+    m.msa_route_scores(index, lay.chunk_doc, lay.n_docs, qr, doc_scores=ds, chunk_scores=cs_)
+    torch.cuda.synchronize()
+    _status(m)
+    assert _tail_intact(ib, in_, 0x5A5A5A5A) and _tail_intact(sb, sn, 0x7FC0DEAD)
+    assert _tail_intact(db, dn, 0x7FC0DEAD) and _tail_intact(cb, cn, 0x7FC0DEAD)
+    ref_i, _ = O.topk_docs(s.cpu().numpy(), 16)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ref_i)
