@@ -458,6 +458,25 @@ typedef struct msa_interleave_args {
 msa_status msa_interleave_step(const msa_interleave_args* a, void* compute, void* copy, int64_t host_wait_timeout_us);
 msa_status msa_interleave_workspace_size(const msa_interleave_args* a, size_t* bytes);
 
+/* The same round captured once into a CUDA graph and replayed: the launches, copies and stream
+ * fork/join of msa_interleave_step with fetch_mode 1 (the only mode without host waits), recorded
+ * against the buffers and sizes that `a` names at creation. A replay reads whatever those buffers
+ * hold when it runs, so a caller refills the round's inputs (qr, q_new, k_new, v_new) in place
+ * between replays; everything else in `a` is fixed for the graph's lifetime. Replaying replaces
+ * the round's per-launch host work (argument checks, tensor maps, plans, about 10 launches per
+ * layer) with one graph launch, which is what bounds short rounds.
+ * create: a->fetch_mode must be 1 and a->route_events NULL (MSA_ERR_INVALID_ARG otherwise);
+ * `stream` must be a created stream, not the legacy default stream (MSA_ERR_INVALID_ARG). It runs
+ * the round once on `stream` (settling one-time set-up: library streams, events, kernel
+ * attributes), waits for it, then captures a second pass without executing it. On failure nothing
+ * is returned in *out and the capture is ended. The graph is tied to the device current at
+ * creation. launch: enqueues one replay on `stream`; `stream` is ordered after all of it when the
+ * call returns. destroy: releases the graph; call it once no replay is pending (NULL is a no-op). */
+typedef struct msa_interleave_graph msa_interleave_graph;
+msa_status msa_interleave_graph_create(const msa_interleave_args* a, void* stream, msa_interleave_graph** out);
+msa_status msa_interleave_graph_launch(msa_interleave_graph* g, void* stream);
+msa_status msa_interleave_graph_destroy(msa_interleave_graph* g);
+
 /* ----------------------------------------------------------------------------------------------
  * One workspace query for every call that takes a workspace. op names the call, cfg points to the
  * matching configuration struct below (host memory, read only), *bytes receives the size that

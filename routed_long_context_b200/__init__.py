@@ -5,4 +5,4 @@ sparse GQA attention and the Memory Interleave round — behind the C ABI of inc
 Importing this package loads libmsa.so and raises if it is missing: there is no fallback path.
 """
 from .api import *  # noqa: F401,F403
-from .api import InterleaveRound, MSAError, device_status, rope_table, chunk_doc_map, version  # noqa: F401
+from .api import InterleaveGraph, InterleaveRound, MSAError, device_status, rope_table, chunk_doc_map, version  # noqa: F401

@@ -108,6 +108,9 @@ SIGNATURES = {
                                                 ctypes.POINTER(sz)]),
     "msa_interleave_step": (i32, [ctypes.POINTER(InterleaveArgs), vp, vp, i64]),
     "msa_interleave_workspace_size": (i32, [ctypes.POINTER(InterleaveArgs), ctypes.POINTER(sz)]),
+    "msa_interleave_graph_create": (i32, [ctypes.POINTER(InterleaveArgs), vp, ctypes.POINTER(vp)]),
+    "msa_interleave_graph_launch": (i32, [vp, vp]),
+    "msa_interleave_graph_destroy": (i32, [vp]),
     "msa_workspace_size": (i32, [ctypes.c_int, vp, ctypes.POINTER(sz)]),
     "msa_sparse_attn_split_plan": (i32, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                          ctypes.c_int, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int),

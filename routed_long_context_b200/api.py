@@ -455,6 +455,38 @@ class InterleaveRound:
         del arr
 
 
+    def capture(self, stream) -> "InterleaveGraph":
+        """The round captured into a CUDA graph on `stream` (a created stream; fetch_mode 1): see
+        msa_interleave_graph_create. Refill the round's inputs in place between replays."""
+        return InterleaveGraph(self, stream)
+
+
+class InterleaveGraph:
+    """A captured interleave round (msa_interleave_graph_*): launch(stream) replays it."""
+
+    def __init__(self, rnd: InterleaveRound, stream):
+        self._round = rnd                  # keeps the marshalled arguments and buffers alive
+        self._g = ctypes.c_void_p(None)
+        rnd.args.route_events = None
+        check(lib.msa_interleave_graph_create(ctypes.byref(rnd.args), _stream(stream), ctypes.byref(self._g)),
+              "msa_interleave_graph_create")
+
+    def launch(self, stream=None) -> None:
+        check(lib.msa_interleave_graph_launch(self._g, _stream(stream)), "msa_interleave_graph_launch")
+
+    def close(self) -> None:
+        if self._g:
+            check(lib.msa_interleave_graph_destroy(self._g), "msa_interleave_graph_destroy")
+            self._g = ctypes.c_void_p(None)
+
+    def __del__(self):
+        try:
+            if self._g:
+                lib.msa_interleave_graph_destroy(self._g)
+        except Exception:
+            pass
+
+
 def msa_interleave_step(layers, compute=None, copy=None, timeout_us: int = 30_000_000, **kw) -> InterleaveRound:
     """One Memory Interleave round over every routed layer (see include/msa.h). Returns the marshalled
     round so it can be re-run."""

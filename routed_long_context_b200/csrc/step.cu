@@ -15,6 +15,7 @@
 // layers l+1.. (on SMs the routers leave free and in the copy engines).
 #include <algorithm>
 #include <chrono>
+#include <new>
 #include <mutex>
 #include <thread>
 #include <vector>
@@ -278,6 +279,73 @@ msa_status msa_interleave_step(const msa_interleave_args* a, void* compute, void
     MSA_CUDA_TRY(cudaEventRecord(ev_join_a, sA));
     MSA_CUDA_TRY(cudaStreamWaitEvent(sR, ev_join_s, 0));
     MSA_CUDA_TRY(cudaStreamWaitEvent(sR, ev_join_a, 0));
+    return MSA_OK;
+}
+
+struct msa_interleave_graph {
+    cudaGraph_t graph;
+    cudaGraphExec_t exec;
+    int device;
+};
+
+msa_status msa_interleave_graph_create(const msa_interleave_args* a, void* stream, msa_interleave_graph** out) {
+    MSA_REQUIRE(a && out, "msa_interleave_graph_create: NULL argument");
+    *out = nullptr;
+    MSA_REQUIRE(a->fetch_mode == 1, "msa_interleave_graph_create: fetch_mode must be 1 (fetch_mode 0 waits on the host)");
+    MSA_REQUIRE(a->route_events == nullptr, "msa_interleave_graph_create: route_events must be NULL");
+    MSA_REQUIRE(stream != nullptr && stream != static_cast<void*>(cudaStreamLegacy) &&
+                    stream != static_cast<void*>(cudaStreamPerThread),
+                "msa_interleave_graph_create: needs a created stream, not a default stream");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int dev = 0;
+    MSA_CUDA_TRY(cudaGetDevice(&dev));
+    // one eager pass: every one-time set-up (library streams, events, kernel attributes, cached
+    // plans) happens outside the capture
+    MSA_RETURN_IF(msa_interleave_step(a, stream, stream, 0));
+    MSA_CUDA_TRY(cudaStreamSynchronize(s));
+    MSA_CUDA_TRY(cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal));
+    const msa_status st = msa_interleave_step(a, stream, stream, 0);
+    cudaGraph_t graph = nullptr;
+    const cudaError_t e = cudaStreamEndCapture(s, &graph);
+    if (st != MSA_OK || e != cudaSuccess) {
+        if (graph) cudaGraphDestroy(graph);
+        if (st != MSA_OK) return st;
+        return set_error(MSA_ERR_CUDA, "msa_interleave_graph_create: capture failed: %s", cudaGetErrorString(e));
+    }
+    cudaGraphExec_t exec = nullptr;
+    const cudaError_t ie = cudaGraphInstantiate(&exec, graph, 0);
+    if (ie != cudaSuccess) {
+        cudaGraphDestroy(graph);
+        return set_error(MSA_ERR_CUDA, "msa_interleave_graph_create: instantiate failed: %s", cudaGetErrorString(ie));
+    }
+    msa_interleave_graph* g = new (std::nothrow) msa_interleave_graph{graph, exec, dev};
+    if (!g) {
+        cudaGraphExecDestroy(exec);
+        cudaGraphDestroy(graph);
+        return set_error(MSA_ERR_CUDA, "msa_interleave_graph_create: out of host memory");
+    }
+    *out = g;
+    return MSA_OK;
+}
+
+msa_status msa_interleave_graph_launch(msa_interleave_graph* g, void* stream) {
+    MSA_REQUIRE(g != nullptr, "msa_interleave_graph_launch: graph is NULL");
+    int dev = 0;
+    MSA_CUDA_TRY(cudaGetDevice(&dev));
+    MSA_REQUIRE(dev == g->device, "msa_interleave_graph_launch: graph of device %d launched on device %d", g->device,
+                dev);
+    MSA_CUDA_TRY(cudaGraphLaunch(g->exec, static_cast<cudaStream_t>(stream)));
+    return MSA_OK;
+}
+
+msa_status msa_interleave_graph_destroy(msa_interleave_graph* g) {
+    if (!g) return MSA_OK;
+    const cudaError_t a = cudaGraphExecDestroy(g->exec);
+    const cudaError_t b = cudaGraphDestroy(g->graph);
+    delete g;
+    if (a != cudaSuccess || b != cudaSuccess)
+        return set_error(MSA_ERR_CUDA, "msa_interleave_graph_destroy: %s",
+                         cudaGetErrorString(a != cudaSuccess ? a : b));
     return MSA_OK;
 }
 

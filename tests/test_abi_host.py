@@ -260,3 +260,28 @@ def test_generic_workspace_query_matches_every_per_call_query(lib):
     assert lib.msa_workspace_size(L.MSA_OP_TOPK, None, ctypes.byref(n)) == 1
     cfg = L.TopkWsCfg(1, 10, 4)
     assert lib.msa_workspace_size(L.MSA_OP_TOPK, ctypes.cast(ctypes.byref(cfg), ctypes.c_void_p), None) == 1
+
+
+def test_interleave_graph_validates_before_any_capture(lib):
+    """The captured round takes fetch_mode 1 only, no timing events and a created stream; each
+    refusal happens before any CUDA call. Destroying NULL is a no-op; launching NULL is refused."""
+    from routed_long_context_b200 import _lib
+
+    layers = (_lib.LayerArgs * 1)()
+    a = _lib.InterleaveArgs()
+    a.n_layers, a.layers = 1, layers
+    g = ctypes.c_void_p(None)
+    a.fetch_mode = 0
+    assert lib.msa_interleave_graph_create(ctypes.byref(a), ctypes.c_void_p(256), ctypes.byref(g)) == 1
+    assert b"fetch_mode" in lib.msa_last_error() and not g.value
+    a.fetch_mode = 1
+    ev = (ctypes.c_void_p * 2)(256, 256)
+    a.route_events = ctypes.cast(ev, ctypes.c_void_p)
+    assert lib.msa_interleave_graph_create(ctypes.byref(a), ctypes.c_void_p(256), ctypes.byref(g)) == 1
+    assert b"route_events" in lib.msa_last_error()
+    a.route_events = None
+    assert lib.msa_interleave_graph_create(ctypes.byref(a), None, ctypes.byref(g)) == 1
+    assert b"stream" in lib.msa_last_error()
+    assert lib.msa_interleave_graph_create(None, ctypes.c_void_p(256), ctypes.byref(g)) == 1
+    assert lib.msa_interleave_graph_destroy(None) == 0
+    assert lib.msa_interleave_graph_launch(None, None) == 1

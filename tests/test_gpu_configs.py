@@ -411,3 +411,51 @@ def test_interleave_three_rounds(m):
                 assert _row_rel_err(_np(outs[l][r])[q], o) <= 2e-2, (l, r, q)
     del index
     _free()
+
+
+# ------------------------------------------------------------------------------------------ graphs
+@pytest.mark.parametrize("which", ["tiny", "1m"])
+def test_interleave_graph_replays_the_round_bitwise(m, which):
+    """A round captured into a CUDA graph (msa_interleave_graph_*) gives bit for bit the eager
+    round's selection and attention output; after the round's inputs are refilled in place, a replay
+    equals an eager run on the new inputs."""
+    from routed_long_context_b200.bank import BankLayout, encode_tokens, to_host_bank
+
+    w = workloads.tiny() if which == "tiny" else workloads.mem_1m()
+    lay = BankLayout.from_doc_lengths(w.doc_len, w.chunk)
+    cs = m.rope_table(4096, w.d, w.rope_base)
+    k, v, kr = (memory_tensor(w, 0, n) for n in ("k", "v", "kr"))
+    kvbar, index = encode_tokens(lay, k, v, kr, w.chunk, cs)
+    del k, v, kr
+    bank = to_host_bank(kvbar)
+    dv = small_tensors(w, 0)
+    local, outs, idx_host = alloc_round_buffers(w, 1)
+    r = run_round(m, w, lay, [dv], 0, cs, [index], [bank], local, outs, idx_host, fetch_mode=1)
+    eager_out, eager_idx = outs[0][0].clone(), idx_host[0][0].clone()
+
+    s = torch.cuda.Stream()
+    g = r.capture(s)
+    outs[0][0].zero_()
+    idx_host[0][0].fill_(-1)
+    g.launch(s)
+    s.synchronize()
+    assert m.device_status() == 0
+    assert torch.equal(idx_host[0][0], eager_idx)
+    assert torch.equal(outs[0][0], eager_out)
+
+    # new inputs in the same buffers: the replay reads them
+    dv2 = small_tensors(w, 1)
+    for n in ("qr", "q", "k_new", "v_new"):
+        dv[n].copy_(dv2[n])
+    torch.cuda.synchronize()
+    g.launch(s)
+    s.synchronize()
+    graph_out, graph_idx = outs[0][0].clone(), idx_host[0][0].clone()
+    r.run()
+    torch.cuda.synchronize()
+    assert torch.equal(idx_host[0][0], graph_idx)
+    assert torch.equal(outs[0][0], graph_out)
+    assert not torch.equal(graph_out, eager_out)
+    g.close()
+    assert m.device_status() == 0
+    _free()
