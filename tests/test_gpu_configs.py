@@ -353,8 +353,21 @@ def test_100m_two_layers_full_routing(m, fetch_mode):
     cs = m.rope_table(4096, w.d, w.rope_base)
     dvs = [small_tensors(w, l) for l in range(2)]
     local, outs, idx_host = alloc_round_buffers(w, 2)
-    run_round(m, w, lay, dvs, 0, cs, index, banks, local, outs, idx_host, fetch_mode)
+    r = run_round(m, w, lay, dvs, 0, cs, index, banks, local, outs, idx_host, fetch_mode)
     assert m.device_status() == 0
+    if fetch_mode == 1:
+        # the same two-layer round as a graph replay: every layer's selection and output bit for bit
+        eager = [(outs[l][0].clone(), idx_host[l][0].clone()) for l in range(2)]
+        s = torch.cuda.Stream()
+        g = r.capture(s)
+        for l in range(2):
+            outs[l][0].zero_()
+            idx_host[l][0].fill_(-1)
+        g.launch(s)
+        s.synchronize()
+        for l in range(2):
+            assert torch.equal(outs[l][0], eager[l][0]) and torch.equal(idx_host[l][0], eager[l][1])
+        g.close()
     for l in range(2):
         ds_gpu = _np(m.msa_route_scores(index[l], lay.chunk_doc, lay.n_docs, dvs[l]["qr"]))
         ref = oracle_route_prepooled(w, l, w.qr(l))

@@ -499,6 +499,37 @@ def test_sparse_attention_split_long_memory(m, impl, hq, hkv, T, mem_lens, q_sta
         np.testing.assert_allclose(_np(lse[qi]), ref_lse, atol=2e-3)
 
 
+@pytest.mark.parametrize("T,hq,hkv", [(64, 32, 8), (24, 32, 8), (100, 16, 8)])
+def test_sparse_attention_split_one_query_long_memory(m, T, hq, hkv):
+    """One query over a long memory (the fine stage's layout: 8 kv heads, 18 key ranges per head,
+    more than one co-resident cluster holds): the default plan against the oracle within the bf16
+    bound, and its log-sum-exp against the partials + combine path (impl 3)."""
+    n_q, d, dtype, q_start = 1, 128, "bf16", 3
+    mem_len = np.array([5000], dtype=np.int32)
+    max_mem = 5003
+    L = q_start + T
+    q = _gen(130, (n_q, T, hq, d), dtype)
+    mem = _gen(131, (n_q, max_mem, 2, hkv, d), dtype)
+    lk, lv = _gen(132, (n_q, L, hkv, d), dtype), _gen(133, (n_q, L, hkv, d), dtype)
+    args = (upload(q, dtype), upload(mem, dtype), torch.from_numpy(mem_len).cuda(), upload(lk, dtype),
+            upload(lv, dtype), L, q_start)
+    plan = m.api.sparse_attn_split_plan(n_q, T, hq, hkv, max_mem, L)
+    lse0 = torch.empty((n_q, T, hq), dtype=torch.float32, device="cuda")
+    out0 = m.msa_sparse_attn_split(*args, lse=lse0)
+    m.attn_set_impl(3)
+    try:
+        lse3 = torch.empty((n_q, T, hq), dtype=torch.float32, device="cuda")
+        out3 = m.msa_sparse_attn_split(*args, lse=lse3)
+    finally:
+        m.attn_set_impl(0)
+    _status(m)
+    assert plan["cluster"] == 0 or plan["key_ranges"] == plan["cluster"]
+    ref = O.sparse_attention(q[0], mem[0, :5000, 0], mem[0, :5000, 1], lk[0], lv[0], q_start, 1 / np.sqrt(d))
+    assert _row_rel_err(_np(out0)[0], ref) <= 2e-2
+    assert _row_rel_err(_np(out3)[0], ref) <= 2e-2
+    np.testing.assert_allclose(_np(lse0), _np(lse3), atol=1e-4)
+
+
 def test_sparse_attention_split_no_keys_gives_zero_and_rejects_fp32(m):
     q = upload(_gen(108, (2, 4, 32, 128), "bf16"), "bf16")
     mem = torch.zeros((2, 300, 2, 8, 128), dtype=torch.bfloat16, device="cuda")
