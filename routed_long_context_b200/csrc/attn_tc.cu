@@ -571,22 +571,33 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         for (int rr = rank * R + warp; rr < rr_end; rr += kThreads / 32) {
             const int row_g = r0 + rr;
             if (row_g >= n_rows) break;                   // rows only grow with rr
-            float M = ninf;
-            for (int s0 = 0; s0 < n_cl; ++s0) M = fmaxf(M, ld_cluster_f2(cluster_map(ml_base + rr * 8, s0)).x);
+            // every range's (max, sum) in one load per lane (lane s0 reads range s0) and every
+            // range's O piece in flight at once: the remote loads do not wait on one another
+            const float2 ml = lane < n_cl ? ld_cluster_f2(cluster_map(ml_base + rr * 8, (uint32_t)lane))
+                                          : make_float2(ninf, 0.f);
+            const uint32_t off = st_base + (uint32_t)(rr * kD * 4 + ((lane ^ (rr & 31)) << 4));
+            float4 o[16];
+#pragma unroll
+            for (int s0 = 0; s0 < 16; ++s0)
+                if (s0 < n_cl) o[s0] = ld_cluster_f4(cluster_map(off, (uint32_t)s0));
+            float M = ml.x;
+#pragma unroll
+            for (int sh = 16; sh >= 1; sh >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, sh));
+            // weights in range order; a range without keys (max -inf) staged no O and is skipped
+            const float wl = (ml.x == ninf) ? 0.f : exp2f(ml.x - M);
             float acc[4] = {0.f, 0.f, 0.f, 0.f}, L = 0.f;
-            if (M != ninf) {
-                const uint32_t off = st_base + (uint32_t)(rr * kD * 4 + ((lane ^ (rr & 31)) << 4));
-                for (int s0 = 0; s0 < n_cl; ++s0) {
-                    const float2 ml = ld_cluster_f2(cluster_map(ml_base + rr * 8, s0));
-                    if (ml.x == ninf) continue;
-                    const float w = exp2f(ml.x - M);
-                    const float4 o = ld_cluster_f4(cluster_map(off, s0));
-                    L = fmaf(w, ml.y, L);
-                    acc[0] = fmaf(w, o.x, acc[0]);
-                    acc[1] = fmaf(w, o.y, acc[1]);
-                    acc[2] = fmaf(w, o.z, acc[2]);
-                    acc[3] = fmaf(w, o.w, acc[3]);
-                }
+#pragma unroll
+            for (int s0 = 0; s0 < 16; ++s0) {
+                if (s0 >= n_cl) break;
+                const float w = __shfl_sync(0xffffffffu, wl, s0);
+                const float l_s = __shfl_sync(0xffffffffu, ml.y, s0);
+                const float m_s = __shfl_sync(0xffffffffu, ml.x, s0);
+                if (m_s == ninf) continue;
+                L = fmaf(w, l_s, L);
+                acc[0] = fmaf(w, o[s0].x, acc[0]);
+                acc[1] = fmaf(w, o[s0].y, acc[1]);
+                acc[2] = fmaf(w, o[s0].z, acc[2]);
+                acc[3] = fmaf(w, o[s0].w, acc[3]);
             }
             const float inv = L > 0.f ? 1.f / L : 0.f;
             const int64_t gr = ((int64_t)qi * a.T + row_g / G) * a.hq + g * G + row_g % G;

@@ -73,7 +73,7 @@ def run_round(m, w, lay, layers_dev, rnd, cs, index, banks, local, outs, idx_hos
                           fetch_mode=fetch_mode)
     r.run()
     torch.cuda.synchronize()
-    del keep
+    r.keep = keep          # the round holds raw pointers: the router-query slices live as long as it
     return r
 
 
@@ -471,4 +471,33 @@ def test_interleave_graph_replays_the_round_bitwise(m, which):
     assert not torch.equal(graph_out, eager_out)
     g.close()
     assert m.device_status() == 0
+    _free()
+
+
+def test_interleave_graph_of_a_later_round(m):
+    """Round 3 of a two-layer interleave (64 tokens already in the local caches, 32 appended, 128
+    routing tokens) captured after the eager rounds: a replay gives both layers' selections and
+    outputs bit for bit."""
+    w = workloads.interleave(layers=2, n_host_banks=2)
+    lay, index, banks = build_prepooled(m, w, 2)
+    cs = m.rope_table(4096, w.d, w.rope_base)
+    dvs = [small_tensors(w, l) for l in range(2)]
+    local, outs, idx_host = alloc_round_buffers(w, 2)
+    for r in range(w.rounds):
+        rnd = run_round(m, w, lay, dvs, r, cs, index, banks, local, outs, idx_host)
+    last = w.rounds - 1
+    assert w.round_tokens(last)[0] > 0
+    eager = [(outs[l][last].clone(), idx_host[l][last].clone()) for l in range(2)]
+    s = torch.cuda.Stream()
+    g = rnd.capture(s)
+    for l in range(2):
+        outs[l][last].zero_()
+        idx_host[l][last].fill_(-1)
+    g.launch(s)
+    s.synchronize()
+    assert m.device_status() == 0
+    for l in range(2):
+        assert torch.equal(idx_host[l][last], eager[l][1]) and torch.equal(outs[l][last], eager[l][0])
+    g.close()
+    del index
     _free()
